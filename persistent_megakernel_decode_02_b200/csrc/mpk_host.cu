@@ -1,0 +1,785 @@
+// Host side of the C ABI declared in include/mpk.h: tensor registry, graph
+// compiler (validation, task split, event assignment, workspace layout) and
+// the launch of the persistent kernel.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <vector>
+
+#include "../../include/mpk.h"
+#include "mpk_internal.h"
+
+namespace mpk {
+size_t kernel_smem_bytes();
+cudaError_t prepare_kernels();
+cudaError_t max_blocks_per_sm(int* n);
+cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream);
+cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, cudaStream_t stream);
+}  // namespace mpk
+
+using namespace mpk;
+
+namespace {
+
+struct Tensor {
+  void* ptr = nullptr;
+  mpk_dtype dtype = MPK_BF16;
+  std::vector<int64_t> dims;
+  bool owned = false;
+};
+
+size_t dtype_size(mpk_dtype t) {
+  switch (t) {
+    case MPK_BF16: return 2;
+    case MPK_FP32: return 4;
+    case MPK_INT32: return 4;
+    case MPK_INT64: return 8;
+  }
+  return 0;
+}
+
+const char* dtype_name(mpk_dtype t) {
+  switch (t) {
+    case MPK_BF16: return "bf16";
+    case MPK_FP32: return "fp32";
+    case MPK_INT32: return "int32";
+    case MPK_INT64: return "int64";
+  }
+  return "?";
+}
+
+std::string g_create_error;
+
+}  // namespace
+
+struct mpk_ctx {
+  int device = 0, sms = 0;
+  int num_workers = 0, num_local = 0, num_remote = 0;
+  std::map<std::string, Tensor> tensors;
+  bool compiled = false;
+  std::vector<OpDesc> ops;
+  OpDesc* ops_dev = nullptr;
+  Graph graph{};
+  std::vector<void*> allocs;      // library-owned device memory
+  void* sync_block = nullptr;     // per-run zeroed state
+  size_t sync_bytes = 0;
+  int32_t* abort_host = nullptr;  // mapped
+  Status* status_dev = nullptr;
+  int32_t R = 0, S_cache = 0, V = 0, H = 0, L = 0;
+  int32_t pred_S = 0;
+  std::string err, warnings;
+  int capture_iter = -1;
+  float* cap_logits = nullptr;
+  float* cap_hidden = nullptr;
+  mpk_options opts{};
+};
+
+namespace {
+
+int fail(mpk_ctx* c, int code, const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (c) c->err = buf;
+  else g_create_error = buf;
+  return code;
+}
+
+#define CUDA_OR_FAIL(ctx, call)                                                          \
+  do {                                                                                   \
+    cudaError_t e_ = (call);                                                             \
+    if (e_ != cudaSuccess)                                                               \
+      return fail(ctx, MPK_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));   \
+  } while (0)
+
+const Tensor* find(mpk_ctx* c, const char* name) {
+  if (!name) return nullptr;
+  auto it = c->tensors.find(name);
+  return it == c->tensors.end() ? nullptr : &it->second;
+}
+
+std::string dims_str(const std::vector<int64_t>& d) {
+  std::string s = "[";
+  for (size_t i = 0; i < d.size(); ++i) s += (i ? "," : "") + std::to_string(d[i]);
+  return s + "]";
+}
+
+// Fetch tensor `name`, check dtype and rank; fill *out.
+int need(mpk_ctx* c, int li, const char* role, const char* name, mpk_dtype dt, int ndim, const Tensor** out) {
+  if (!name) return fail(c, MPK_ERR_INVALID_ARG, "layer %d: %s name missing", li, role);
+  const Tensor* t = find(c, name);
+  if (!t) return fail(c, MPK_ERR_NOT_FOUND, "layer %d: %s tensor '%s' not registered", li, role, name);
+  if (t->dtype != dt)
+    return fail(c, MPK_ERR_DTYPE, "layer %d: %s '%s' is %s, expected %s", li, role, name, dtype_name(t->dtype),
+                dtype_name(dt));
+  if ((int)t->dims.size() != ndim)
+    return fail(c, MPK_ERR_SHAPE, "layer %d: %s '%s' has shape %s, expected rank %d", li, role, name,
+                dims_str(t->dims).c_str(), ndim);
+  *out = t;
+  return MPK_OK;
+}
+
+#define NEED(role, name, dt, nd, out)                       \
+  do {                                                      \
+    int rc_ = need(c, li, role, name, dt, nd, out);         \
+    if (rc_ != MPK_OK) return rc_;                          \
+  } while (0)
+
+#define SHAPE_CHECK(cond, ...)                              \
+  do {                                                      \
+    if (!(cond)) return fail(c, MPK_ERR_SHAPE, __VA_ARGS__); \
+  } while (0)
+
+// GEMV geometry: kw warps along K (EPL elements per lane), rw row groups,
+// rows per stage.
+int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats) {
+  const int K = o.K;
+  if (K % 256 != 0) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d is not a multiple of 256", li, K);
+  static const int supported[] = {8, 16, 24, 32, 48, 64};
+  int best_kw = 0, best_epl = 0;
+  for (int kw = MAX_KW; kw >= 1; kw >>= 1) {
+    if (o.nwarps % kw != 0 || K % (kw * 256) != 0) continue;
+    const int epl = K / (kw * 32);
+    bool ok = false;
+    for (int s : supported) ok |= (s == epl);
+    if (ok) { best_kw = kw; best_epl = epl; break; }
+  }
+  if (!best_kw)
+    return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: no warp split of K=%d over %d warps keeps 8..64 elements per lane",
+                li, K, o.nwarps);
+  o.kw = best_kw;
+  o.epl = best_epl;
+  o.rw = o.nwarps / best_kw;
+  const int row_bytes = K * 2 * (two_mats ? 2 : 1);
+  int rps = STAGE_BYTES / row_bytes;
+  if (rps < 1) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: one weight row (%d bytes) exceeds a stage", li, row_bytes);
+  if (rps > MAX_RPS) rps = MAX_RPS;
+  if (rps >= o.rw) rps -= rps % o.rw;
+  o.rps = rps;
+  return MPK_OK;
+}
+
+int check_grid(mpk_ctx* c, int li, const mpk_layer& Ly, int ntasks, int rows) {
+  if (ntasks < 1 || ntasks > 65535)
+    return fail(c, MPK_ERR_INVALID_ARG, "layer %d: grid_dim gives %d tasks (1..65535)", li, ntasks);
+  if (rows > 0 && ntasks > rows)
+    return fail(c, MPK_ERR_SHAPE, "layer %d: %d tasks for %d rows (at most one task per row)", li, ntasks, rows);
+  if (ntasks % c->num_workers != 0) {
+    char b[256];
+    snprintf(b, sizeof b, "layer %d: %d tasks is not a multiple of num_workers=%d (some workers idle in this phase)\n",
+             li, ntasks, c->num_workers);
+    c->warnings += b;
+  }
+  (void)Ly;
+  return MPK_OK;
+}
+
+template <typename T>
+int alloc(mpk_ctx* c, T** p, size_t bytes) {
+  void* q = nullptr;
+  CUDA_OR_FAIL(c, cudaMalloc(&q, bytes ? bytes : 16));
+  CUDA_OR_FAIL(c, cudaMemset(q, 0, bytes ? bytes : 16));
+  c->allocs.push_back(q);
+  *p = reinterpret_cast<T*>(q);
+  return MPK_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+int mpk_abi_version(void) { return MPK_ABI_VERSION; }
+int mpk_worker_threads(void) { return CONSUMER_THREADS; }
+
+int mpk_device_sm_count(void) {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MPK_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MPK_ERR_CUDA;
+  return n;
+}
+
+static int validate_split(int sms, int num_workers, int num_local_schedulers, int num_remote_schedulers) {
+  if (num_workers < 1 || num_local_schedulers < 0 || num_remote_schedulers < 0)
+    return fail(nullptr, MPK_ERR_INVALID_ARG, "counts must be positive (workers %d, local %d, remote %d)", num_workers,
+                num_local_schedulers, num_remote_schedulers);
+  const int sched = num_local_schedulers + num_remote_schedulers;
+  if (sched % 4 != 0)
+    return fail(nullptr, MPK_ERR_SM_FORMULA,
+                "num_local_schedulers + num_remote_schedulers = %d is not a multiple of 4", sched);
+  if (num_workers + sched / 4 != sms)
+    return fail(nullptr, MPK_ERR_SM_FORMULA,
+                "num_workers + (num_local_schedulers + num_remote_schedulers) / 4 = %d + %d = %d, but the GPU has %d SMs",
+                num_workers, sched / 4, num_workers + sched / 4, sms);
+  if (num_remote_schedulers != 0)
+    return fail(nullptr, MPK_ERR_UNSUPPORTED, "remote schedulers serve other GPUs; this build runs on one GPU");
+  if (num_local_schedulers == 0)
+    return fail(nullptr, MPK_ERR_INVALID_ARG, "at least one group of 4 local schedulers is required");
+  return MPK_OK;
+}
+
+int mpk_validate_split(int sm_count, int num_workers, int num_local_schedulers, int num_remote_schedulers) {
+  return validate_split(sm_count, num_workers, num_local_schedulers, num_remote_schedulers);
+}
+
+int mpk_create(int num_workers, int num_local_schedulers, int num_remote_schedulers, mpk_ctx** out) {
+  if (!out) return fail(nullptr, MPK_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  int dev = 0, sms = 0, major = 0, minor = 0, coop = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(nullptr, MPK_ERR_CUDA, "no CUDA device");
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+  const int rc_split = validate_split(sms, num_workers, num_local_schedulers, num_remote_schedulers);
+  if (rc_split != MPK_OK) return rc_split;
+  if (major != 10 || minor != 0)
+    return fail(nullptr, MPK_ERR_UNSUPPORTED, "device is sm_%d%d; this library is built for sm_100a", major, minor);
+  if (!coop) return fail(nullptr, MPK_ERR_UNSUPPORTED, "device lacks cooperative launch");
+  cudaError_t e = prepare_kernels();
+  if (e != cudaSuccess) return fail(nullptr, MPK_ERR_CUDA, "kernel setup failed: %s", cudaGetErrorString(e));
+  int per_sm = 0;
+  e = max_blocks_per_sm(&per_sm);
+  if (e != cudaSuccess || per_sm < 1)
+    return fail(nullptr, MPK_ERR_UNSUPPORTED, "persistent kernel cannot be resident (%d blocks/SM): %s", per_sm,
+                cudaGetErrorString(e));
+  mpk_ctx* c = new mpk_ctx();
+  c->device = dev;
+  c->sms = sms;
+  c->num_workers = num_workers;
+  c->num_local = num_local_schedulers;
+  c->num_remote = num_remote_schedulers;
+  if (cudaHostAlloc(reinterpret_cast<void**>(&c->abort_host), 64, cudaHostAllocMapped) != cudaSuccess) {
+    delete c;
+    return fail(nullptr, MPK_ERR_CUDA, "cudaHostAlloc of the abort flag failed");
+  }
+  *c->abort_host = 0;
+  *out = c;
+  return MPK_OK;
+}
+
+static int register_tensor(mpk_ctx* c, const char* name, void* ptr, mpk_dtype dtype, int ndim, const int64_t* dims,
+                           bool owned) {
+  if (!name || !*name) return fail(c, MPK_ERR_INVALID_ARG, "tensor name is empty");
+  if (c->compiled) return fail(c, MPK_ERR_STATE, "tensors cannot be added after compile");
+  if (ndim < 1 || ndim > 5 || !dims) return fail(c, MPK_ERR_INVALID_ARG, "'%s': rank must be 1..5", name);
+  if ((int)dtype < 0 || (int)dtype > 3) return fail(c, MPK_ERR_INVALID_ARG, "'%s': unknown dtype %d", name, (int)dtype);
+  if (c->tensors.count(name)) return fail(c, MPK_ERR_INVALID_ARG, "tensor '%s' already registered", name);
+  Tensor t;
+  for (int i = 0; i < ndim; ++i) {
+    if (dims[i] < 1) return fail(c, MPK_ERR_INVALID_ARG, "'%s': extent %lld < 1", name, (long long)dims[i]);
+    t.dims.push_back(dims[i]);
+  }
+  if (!owned) {
+    if (!ptr) return fail(c, MPK_ERR_INVALID_ARG, "'%s': device pointer is NULL", name);
+    if (reinterpret_cast<uintptr_t>(ptr) % 16 != 0)
+      return fail(c, MPK_ERR_INVALID_ARG, "'%s': pointer is not 16-byte aligned", name);
+  }
+  t.ptr = ptr;
+  t.dtype = dtype;
+  t.owned = owned;
+  c->tensors[name] = t;
+  return MPK_OK;
+}
+
+int mpk_attach_input(mpk_ctx* c, const char* name, void* dev_ptr, mpk_dtype dtype, int ndim, const int64_t* dims) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  return register_tensor(c, name, dev_ptr, dtype, ndim, dims, false);
+}
+
+int mpk_new_tensor(mpk_ctx* c, const char* name, mpk_dtype dtype, int ndim, const int64_t* dims, mpk_io io,
+                   void** dev_ptr_out) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  if (io == MPK_IO_NVSHMEM)
+    return fail(c, MPK_ERR_UNSUPPORTED, "'%s': nvshmem_tensor is for remote GPU access; this build runs on one GPU",
+                name ? name : "");
+  if (io != MPK_IO_CUDA) return fail(c, MPK_ERR_INVALID_ARG, "unknown io category %d", (int)io);
+  if ((int)dtype < 0 || (int)dtype > 3) return fail(c, MPK_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (ndim < 1 || ndim > 5 || !dims) return fail(c, MPK_ERR_INVALID_ARG, "rank must be 1..5");
+  int64_t n = 1;
+  for (int i = 0; i < ndim; ++i) {
+    if (dims[i] < 1) return fail(c, MPK_ERR_INVALID_ARG, "extent < 1");
+    n *= dims[i];
+  }
+  if (name && c->tensors.count(name)) return fail(c, MPK_ERR_INVALID_ARG, "tensor '%s' already registered", name);
+  if (c->compiled) return fail(c, MPK_ERR_STATE, "tensors cannot be added after compile");
+  void* p = nullptr;
+  int rc = alloc(c, &p, (size_t)n * dtype_size(dtype));
+  if (rc != MPK_OK) return rc;
+  rc = register_tensor(c, name, p, dtype, ndim, dims, true);
+  if (rc != MPK_OK) return rc;
+  if (dev_ptr_out) *dev_ptr_out = p;
+  return MPK_OK;
+}
+
+void* mpk_tensor_ptr(mpk_ctx* c, const char* name) {
+  if (!c) return nullptr;
+  const Tensor* t = find(c, name);
+  return t ? t->ptr : nullptr;
+}
+
+const char* mpk_warnings(mpk_ctx* c) { return c ? c->warnings.c_str() : ""; }
+
+int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_options* opts) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  if (c->compiled) return fail(c, MPK_ERR_STATE, "already compiled");
+  if (!layers || n_layers < 1) return fail(c, MPK_ERR_INVALID_ARG, "no layers");
+  if (n_layers > 65535) return fail(c, MPK_ERR_INVALID_ARG, "too many layers");
+  c->warnings.clear();
+  mpk_options o{};
+  if (opts) o = *opts;
+  if (o.sched_lookahead <= 0) o.sched_lookahead = 4;
+  if (o.timeout_s <= 0) o.timeout_s = 2.0;
+  if (o.max_timeline <= 0) o.max_timeline = 1 << 20;
+  c->opts = o;
+
+  std::vector<OpDesc> ops(n_layers);
+  int R = -1, H = -1, V = -1, L = -1, S = -1;
+  // attention workspace sizing
+  size_t part_floats = 0, merge_u32 = 0;
+  std::vector<std::pair<int, size_t>> merge_off(n_layers, {0, 0});
+  struct RopeKey { float theta; int d; int S; };
+  std::vector<RopeKey> rope_keys;
+  std::vector<int> rope_of(n_layers, -1);
+  int n_argmax = 0;
+
+  for (int li = 0; li < n_layers; ++li) {
+    const mpk_layer& Ly = layers[li];
+    OpDesc& op = ops[li];
+    memset(&op, 0, sizeof(op));
+    op.capture_slot = Ly.capture_slot;
+    op.eps = Ly.eps > 0 ? Ly.eps : 1e-6f;
+    const int64_t ntasks64 = (int64_t)Ly.grid_dim.x * (Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1) *
+                             (Ly.grid_dim.z > 0 ? Ly.grid_dim.z : 1);
+    if (Ly.grid_dim.x < 1 || ntasks64 > 65535)
+      return fail(c, MPK_ERR_INVALID_ARG, "layer %d: grid_dim must give 1..65535 tasks", li);
+    const int ntasks = (int)ntasks64;
+    const int64_t threads = (int64_t)(Ly.block_dim.x > 0 ? Ly.block_dim.x : CONSUMER_THREADS) *
+                            (Ly.block_dim.y > 0 ? Ly.block_dim.y : 1) * (Ly.block_dim.z > 0 ? Ly.block_dim.z : 1);
+    if (threads < 32 || threads > CONSUMER_THREADS || threads % 32 != 0)
+      return fail(c, MPK_ERR_INVALID_ARG, "layer %d: block_dim gives %lld threads (a multiple of 32, at most %d)", li,
+                  (long long)threads, CONSUMER_THREADS);
+    op.nwarps = (int)(threads / 32);
+    op.ntasks = ntasks;
+    const Tensor *x, *w0, *w1, *w2, *out;
+    switch (Ly.op) {
+      case MPK_OP_EMBED: {
+        op.kind = TK_EMBED;
+        NEED("weights[0] (embedding)", Ly.weights[0], MPK_BF16, 2, &w0);
+        NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32, 2, &out);
+        SHAPE_CHECK(out->dims[1] == w0->dims[1], "layer %d: x width %lld != embedding width %lld", li,
+                    (long long)out->dims[1], (long long)w0->dims[1]);
+        SHAPE_CHECK(out->dims[1] % 8 == 0, "layer %d: hidden size must be a multiple of 8", li);
+        if (R < 0) R = (int)out->dims[0];
+        SHAPE_CHECK(out->dims[0] == R, "layer %d: request count mismatch", li);
+        SHAPE_CHECK(ntasks == R, "layer %d: EMBED needs grid_dim = number of requests (%d)", li, R);
+        op.table = (const uint16_t*)w0->ptr;
+        op.x_out = (float*)out->ptr;
+        op.N = (int)out->dims[1];
+        if (V < 0) V = (int)w0->dims[0];
+        if (H < 0) H = op.N;
+        op.signal_per_task = 1;
+        op.out_trigger = ntasks;
+        break;
+      }
+      case MPK_OP_RMSNORM_LINEAR:
+      case MPK_OP_LINEAR_RESIDUAL:
+      case MPK_OP_RMSNORM_LINEAR_SILU_MUL:
+      case MPK_OP_RMSNORM_LMHEAD_ARGMAX: {
+        const bool resid = Ly.op == MPK_OP_LINEAR_RESIDUAL;
+        const bool silu = Ly.op == MPK_OP_RMSNORM_LINEAR_SILU_MUL;
+        const bool lmh = Ly.op == MPK_OP_RMSNORM_LMHEAD_ARGMAX;
+        op.kind = resid ? TK_GEMV_RESID : silu ? TK_NORM_GEMV_SILU : lmh ? TK_NORM_GEMV_ARGMAX : TK_NORM_GEMV;
+        if (resid) {
+          NEED("inputs[0] (a)", Ly.inputs[0], MPK_BF16, 2, &x);
+          op.a_in = (const uint16_t*)x->ptr;
+          op.K = (int)x->dims[1];
+          NEED("weights[0] (W)", Ly.weights[0], MPK_BF16, 2, &w0);
+          NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32, 2, &out);
+          SHAPE_CHECK(w0->dims[1] == op.K, "layer %d: W is %s but input has %d features", li,
+                      dims_str(w0->dims).c_str(), op.K);
+          SHAPE_CHECK(out->dims[1] == w0->dims[0] && out->dims[0] == x->dims[0],
+                      "layer %d: residual %s does not match W %s", li, dims_str(out->dims).c_str(),
+                      dims_str(w0->dims).c_str());
+          op.N = (int)w0->dims[0];
+          op.W[0] = (const uint16_t*)w0->ptr;
+          op.nseg = 1;
+          op.seg_row0[0] = 0;
+          op.seg_row0[1] = op.N;
+          op.x_out = (float*)out->ptr;
+          op.x = (const float*)out->ptr;
+        } else {
+          NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32, 2, &x);
+          op.x = (const float*)x->ptr;
+          op.K = (int)x->dims[1];
+          NEED("weights[0] (norm)", Ly.weights[0], MPK_BF16, 1, &w0);
+          SHAPE_CHECK(w0->dims[0] == op.K, "layer %d: norm weight %s, input width %d", li, dims_str(w0->dims).c_str(),
+                      op.K);
+          op.norm_w = (const uint16_t*)w0->ptr;
+          if (silu) {
+            NEED("weights[1] (gate)", Ly.weights[1], MPK_BF16, 2, &w1);
+            NEED("weights[2] (up)", Ly.weights[2], MPK_BF16, 2, &w2);
+            NEED("outputs[0] (a)", Ly.outputs[0], MPK_BF16, 2, &out);
+            SHAPE_CHECK(w1->dims == w2->dims && w1->dims[1] == op.K, "layer %d: gate %s / up %s vs K=%d", li,
+                        dims_str(w1->dims).c_str(), dims_str(w2->dims).c_str(), op.K);
+            SHAPE_CHECK(out->dims[1] == w1->dims[0] && out->dims[0] == x->dims[0], "layer %d: output %s", li,
+                        dims_str(out->dims).c_str());
+            op.N = (int)w1->dims[0];
+            op.W[0] = (const uint16_t*)w1->ptr;
+            op.W_up = (const uint16_t*)w2->ptr;
+            op.nseg = 1;
+            op.seg_row0[0] = 0;
+            op.seg_row0[1] = op.N;
+            op.a_out = (uint16_t*)out->ptr;
+          } else if (lmh) {
+            NEED("weights[1] (lm head)", Ly.weights[1], MPK_BF16, 2, &w1);
+            SHAPE_CHECK(w1->dims[1] == op.K, "layer %d: LM head %s vs K=%d", li, dims_str(w1->dims).c_str(), op.K);
+            op.N = (int)w1->dims[0];
+            op.W[0] = (const uint16_t*)w1->ptr;
+            op.nseg = 1;
+            op.seg_row0[0] = 0;
+            op.seg_row0[1] = op.N;
+            if (Ly.outputs[0]) {
+              NEED("outputs[0] (pred)", Ly.outputs[0], MPK_INT64, 2, &out);
+              op.pred = (int64_t*)out->ptr;
+              if (S < 0) S = (int)out->dims[1];
+            }
+            if (V < 0) V = op.N;
+            SHAPE_CHECK(op.N == V, "layer %d: LM head rows %d != vocabulary %d", li, op.N, V);
+            if (li != n_layers - 1)
+              return fail(c, MPK_ERR_INVALID_ARG, "layer %d: the LM-head/argmax operation must be last", li);
+            ++n_argmax;
+          } else {
+            op.nseg = 0;
+            int rows = 0;
+            for (int s = 0; s < MAX_SEG; ++s) {
+              if (!Ly.weights[1 + s]) break;
+              const Tensor *ws, *ys;
+              NEED("weights[1+i] (linear)", Ly.weights[1 + s], MPK_BF16, 2, &ws);
+              if (!Ly.outputs[s]) return fail(c, MPK_ERR_INVALID_ARG, "layer %d: outputs[%d] missing", li, s);
+              NEED("outputs[i]", Ly.outputs[s], MPK_FP32, 2, &ys);
+              SHAPE_CHECK(ws->dims[1] == op.K && ys->dims[1] == ws->dims[0] && ys->dims[0] == x->dims[0],
+                          "layer %d: linear %d W %s, y %s, K=%d", li, s, dims_str(ws->dims).c_str(),
+                          dims_str(ys->dims).c_str(), op.K);
+              op.W[s] = (const uint16_t*)ws->ptr;
+              op.y[s] = (float*)ys->ptr;
+              op.seg_row0[s] = rows;
+              rows += (int)ws->dims[0];
+              op.nseg = s + 1;
+            }
+            if (op.nseg == 0) return fail(c, MPK_ERR_INVALID_ARG, "layer %d: no linear weight", li);
+            op.seg_row0[op.nseg] = rows;
+            for (int s = op.nseg + 1; s <= MAX_SEG; ++s) op.seg_row0[s] = rows;
+            op.N = rows;
+          }
+        }
+        if (R < 0) R = (int)x->dims[0];
+        SHAPE_CHECK(x->dims[0] == R, "layer %d: %lld requests, graph has %d", li, (long long)x->dims[0], R);
+        if (R != 1)
+          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: projections with %d requests are not built yet (1 supported)",
+                      li, R);
+        int rc = gemv_geometry(c, li, op, silu);
+        if (rc != MPK_OK) return rc;
+        rc = check_grid(c, li, Ly, ntasks, op.N);
+        if (rc != MPK_OK) return rc;
+        op.signal_per_task = lmh ? 0 : 1;
+        op.out_trigger = lmh ? 1 : ntasks;
+        if (resid && H < 0) H = op.N;
+        break;
+      }
+      case MPK_OP_ATTENTION: {
+        op.kind = TK_ATTN;
+        const Tensor *q, *k, *v, *qn, *kn, *kc, *vc, *o;
+        NEED("inputs[0] (q)", Ly.inputs[0], MPK_FP32, 2, &q);
+        NEED("inputs[1] (k)", Ly.inputs[1], MPK_FP32, 2, &k);
+        NEED("inputs[2] (v)", Ly.inputs[2], MPK_FP32, 2, &v);
+        NEED("weights[0] (q_norm)", Ly.weights[0], MPK_BF16, 1, &qn);
+        NEED("weights[1] (k_norm)", Ly.weights[1], MPK_BF16, 1, &kn);
+        NEED("weights[2] (k_cache)", Ly.weights[2], MPK_BF16, 5, &kc);
+        NEED("weights[3] (v_cache)", Ly.weights[3], MPK_BF16, 5, &vc);
+        NEED("outputs[0] (o)", Ly.outputs[0], MPK_BF16, 2, &o);
+        SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
+        const int d = (int)kc->dims[4], Hkv = (int)kc->dims[2];
+        SHAPE_CHECK(qn->dims[0] == d && kn->dims[0] == d, "layer %d: norm weights must have head_dim %d", li, d);
+        SHAPE_CHECK(q->dims[1] % d == 0 && k->dims[1] == (int64_t)Hkv * d && v->dims[1] == k->dims[1],
+                    "layer %d: q %s k %s v %s vs Hkv=%d d=%d", li, dims_str(q->dims).c_str(), dims_str(k->dims).c_str(),
+                    dims_str(v->dims).c_str(), Hkv, d);
+        const int Hq = (int)(q->dims[1] / d);
+        SHAPE_CHECK(Hq % Hkv == 0, "layer %d: %d query heads not a multiple of %d kv heads", li, Hq, Hkv);
+        SHAPE_CHECK(o->dims[1] == q->dims[1], "layer %d: o %s vs q %s", li, dims_str(o->dims).c_str(),
+                    dims_str(q->dims).c_str());
+        if (R < 0) R = (int)q->dims[0];
+        SHAPE_CHECK(q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R && kc->dims[1] == R,
+                    "layer %d: request count mismatch (graph %d)", li, R);
+        SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range %lld", li, Ly.layer,
+                    (long long)kc->dims[0]);
+        const int G = Hq / Hkv;
+        const bool okGd = (d == 64 || d == 128) && (G == 1 || G == 2 || G == 4);
+        if (!okGd)
+          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: head_dim %d with %d query heads per kv head", li, d, G);
+        const int gx = Ly.grid_dim.x, gy = Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1, gz = Ly.grid_dim.z > 0 ? Ly.grid_dim.z : 1;
+        SHAPE_CHECK(gx == Hkv && gz == R, "layer %d: ATTENTION needs grid_dim = (kv_heads=%d, chunks, requests=%d)", li,
+                    Hkv, R);
+        op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = gy;
+        op.L = (int)kc->dims[0];
+        op.S = (int)kc->dims[3];
+        op.layer = Ly.layer;
+        op.q = (const float*)q->ptr; op.k = (const float*)k->ptr; op.v = (const float*)v->ptr;
+        op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
+        op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
+        op.a_out = (uint16_t*)o->ptr;
+        op.N = Hq * d;
+        if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
+        part_floats = std::max(part_floats, (size_t)R * Hq * gy * (d + 2));
+        merge_off[li] = {1, merge_u32};
+        merge_u32 += (size_t)R * Hkv;
+        const float theta = Ly.rope_theta > 0 ? Ly.rope_theta : 1.0e6f;
+        int ri = -1;
+        for (size_t i = 0; i < rope_keys.size(); ++i)
+          if (rope_keys[i].theta == theta && rope_keys[i].d == d && rope_keys[i].S == op.S) ri = (int)i;
+        if (ri < 0) { rope_keys.push_back({theta, d, op.S}); ri = (int)rope_keys.size() - 1; }
+        rope_of[li] = ri;
+        int rc = check_grid(c, li, Ly, ntasks, 0);
+        if (rc != MPK_OK) return rc;
+        op.signal_per_task = 0;
+        op.out_trigger = R * Hkv;
+        if (L < 0 || op.L > L) L = op.L;
+        break;
+      }
+      default:
+        return fail(c, MPK_ERR_INVALID_ARG, "layer %d: unknown op %d", li, Ly.op);
+    }
+  }
+  if (n_argmax != 1 || ops[n_layers - 1].kind != TK_NORM_GEMV_ARGMAX)
+    return fail(c, MPK_ERR_INVALID_ARG, "the graph must end with one RMSNORM_LMHEAD_ARGMAX operation");
+  if (ops[0].kind != TK_EMBED)
+    return fail(c, MPK_ERR_INVALID_ARG, "the graph must start with an EMBED operation");
+  if (H < 0) H = ops[0].N;
+
+  // events: op p signals event p; op p waits on event p-1 (op 0 on the last op,
+  // one iteration behind).
+  const int P = n_layers;
+  for (int p = 0; p < P; ++p) {
+    ops[p].out_event = p;
+    const int dp = (p + P - 1) % P;
+    ops[p].dep_event = dp;
+    ops[p].dep_trigger = ops[dp].out_trigger;
+    ops[p].dep_iter_offset = p == 0 ? 0 : 1;
+  }
+
+  // ---- workspace
+  // sync block (zeroed before every run): events | q_head | q_tail | ctl | status | keys | arrive | merge counters | timeline_n
+  const size_t line = EVENT_STRIDE * sizeof(uint32_t);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o2 = off; off += (bytes + 127) / 128 * 128; return o2; };
+  const size_t o_events = take(line * P);
+  const size_t o_qhead = take(line * c->num_workers);
+  const size_t o_qtail = take(line * c->num_workers);
+  const size_t o_ctl = take(sizeof(Control));
+  const size_t o_status = take(sizeof(Status));
+  const size_t o_keys = take(sizeof(unsigned long long) * (size_t)R);
+  const size_t o_arrive = take(line);
+  const size_t o_merge = take(sizeof(uint32_t) * (merge_u32 ? merge_u32 : 1));
+  const size_t o_tln = take(line);
+  c->sync_bytes = off;
+  uint8_t* sb = nullptr;
+  int rc = alloc(c, &sb, off);
+  if (rc != MPK_OK) return rc;
+  c->sync_block = sb;
+  unsigned long long* queue = nullptr;
+  rc = alloc(c, &queue, sizeof(unsigned long long) * QUEUE_CAP * c->num_workers);
+  if (rc != MPK_OK) return rc;
+  float* part = nullptr;
+  rc = alloc(c, &part, sizeof(float) * (part_floats ? part_floats : 1));
+  if (rc != MPK_OK) return rc;
+  std::vector<float2*> rope_dev(rope_keys.size(), nullptr);
+  for (size_t i = 0; i < rope_keys.size(); ++i) {
+    const RopeKey& k = rope_keys[i];
+    std::vector<float2> tab((size_t)k.S * (k.d / 2));
+    for (int s = 0; s < k.S; ++s)
+      for (int j = 0; j < k.d / 2; ++j) {
+        const double ang = (double)s * std::pow((double)k.theta, -2.0 * j / (double)k.d);
+        tab[(size_t)s * (k.d / 2) + j] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+      }
+    rc = alloc(c, &rope_dev[i], tab.size() * sizeof(float2));
+    if (rc != MPK_OK) return rc;
+    CUDA_OR_FAIL(c, cudaMemcpy(rope_dev[i], tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice));
+  }
+  unsigned long long* timeline = nullptr;
+  if (o.profiling) {
+    rc = alloc(c, &timeline, sizeof(unsigned long long) * 5 * (size_t)o.max_timeline);
+    if (rc != MPK_OK) return rc;
+  }
+  for (int p = 0; p < P; ++p) {
+    OpDesc& op = ops[p];
+    if (op.kind == TK_ATTN) {
+      op.part = part;
+      op.merge_cnt = reinterpret_cast<uint32_t*>(sb + o_merge) + merge_off[p].second;
+      op.rope = rope_dev[rope_of[p]];
+    }
+    if (op.kind == TK_NORM_GEMV_ARGMAX) {
+      op.keys = reinterpret_cast<unsigned long long*>(sb + o_keys);
+      op.arrive = reinterpret_cast<uint32_t*>(sb + o_arrive);
+    }
+  }
+  rc = alloc(c, &c->ops_dev, sizeof(OpDesc) * P);
+  if (rc != MPK_OK) return rc;
+  CUDA_OR_FAIL(c, cudaMemcpy(c->ops_dev, ops.data(), sizeof(OpDesc) * P, cudaMemcpyHostToDevice));
+
+  Graph& g = c->graph;
+  memset(&g, 0, sizeof(g));
+  g.ops = c->ops_dev;
+  g.nops = P;
+  g.R = R;
+  g.V = V;
+  g.H = H;
+  g.L = L < 0 ? 0 : L;
+  g.num_workers = c->num_workers;
+  g.num_sched = c->num_local;
+  g.sched_ctas = c->num_local / 4;
+  g.lookahead = o.sched_lookahead;
+  g.events = reinterpret_cast<uint32_t*>(sb + o_events);
+  g.queue = queue;
+  g.q_head = reinterpret_cast<uint32_t*>(sb + o_qhead);
+  g.q_tail = reinterpret_cast<uint32_t*>(sb + o_qtail);
+  g.ctl = reinterpret_cast<Control*>(sb + o_ctl);
+  g.status = reinterpret_cast<Status*>(sb + o_status);
+  uint32_t* abort_dev = nullptr;
+  CUDA_OR_FAIL(c, cudaHostGetDevicePointer(reinterpret_cast<void**>(&abort_dev), c->abort_host, 0));
+  g.abort_flag = reinterpret_cast<volatile int32_t*>(abort_dev);
+  g.timeout_ns = (uint64_t)(o.timeout_s * 1e9);
+  g.profiling = o.profiling;
+  g.max_timeline = o.max_timeline;
+  g.timeline = timeline;
+  g.timeline_n = reinterpret_cast<uint32_t*>(sb + o_tln);
+  c->status_dev = g.status;
+  c->R = R;
+  c->V = V;
+  c->H = H;
+  c->L = g.L;
+  c->pred_S = S;
+  c->ops = ops;
+  c->compiled = true;
+  return MPK_OK;
+}
+
+static int prepare_run(mpk_ctx* c, int32_t* step, int64_t* tokens, const int32_t* step_end, int64_t seq_len,
+                       cudaStream_t s) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  if (!c->compiled) return fail(c, MPK_ERR_STATE, "mpk_run before mpk_compile");
+  if (!step || !tokens) return fail(c, MPK_ERR_INVALID_ARG, "step and tokens are required");
+  if (seq_len < 2) return fail(c, MPK_ERR_INVALID_ARG, "seq_length %lld < 2", (long long)seq_len);
+  if (c->S_cache > 0 && seq_len - 1 > c->S_cache)
+    return fail(c, MPK_ERR_SHAPE, "seq_length %lld needs %lld cached positions, the KV cache holds %d",
+                (long long)seq_len, (long long)seq_len - 1, c->S_cache);
+  if (c->pred_S > 0 && c->pred_S != seq_len)
+    return fail(c, MPK_ERR_SHAPE, "pred has %d columns, tokens %lld", c->pred_S, (long long)seq_len);
+  Graph& g = c->graph;
+  g.step = step;
+  g.tokens = tokens;
+  g.step_end = step_end;
+  g.S = (int32_t)seq_len;
+  g.capture_iter = c->capture_iter;
+  g.cap_logits = c->cap_logits;
+  g.cap_hidden = c->cap_hidden;
+  CUDA_OR_FAIL(c, cudaMemsetAsync(c->sync_block, 0, c->sync_bytes, s));
+  return MPK_OK;
+}
+
+int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
+            const int32_t* step_end, void* stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (c && c->compiled && num_requests != c->R)
+    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->R);
+  int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
+  if (rc != MPK_OK) return rc;
+  *(volatile int32_t*)c->abort_host = 0;
+  CUDA_OR_FAIL(c, launch_persistent(c->graph, c->sms, s));
+  return MPK_OK;
+}
+
+int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
+                     const int32_t* step_end, void* stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (c && c->compiled && num_requests != c->R)
+    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->R);
+  int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
+  if (rc != MPK_OK) return rc;
+  // The host needs the iteration count: read step / step_end.
+  std::vector<int32_t> st(c->R), se(c->R, (int32_t)(seq_len - 1));
+  CUDA_OR_FAIL(c, cudaMemcpyAsync(st.data(), step, sizeof(int32_t) * c->R, cudaMemcpyDeviceToHost, s));
+  if (step_end)
+    CUDA_OR_FAIL(c, cudaMemcpyAsync(se.data(), step_end, sizeof(int32_t) * c->R, cudaMemcpyDeviceToHost, s));
+  CUDA_OR_FAIL(c, cudaStreamSynchronize(s));
+  int64_t n_iter = 0;
+  for (int r = 0; r < c->R; ++r) {
+    const int64_t end = std::min<int64_t>(se[r], seq_len - 1);
+    if (st[r] >= 0 && st[r] < end) n_iter = std::max<int64_t>(n_iter, end - st[r]);
+  }
+  for (int64_t it = 0; it < n_iter; ++it)
+    for (int p = 0; p < (int)c->ops.size(); ++p)
+      CUDA_OR_FAIL(c, launch_op(c->graph, p, c->ops[p].ntasks, (uint32_t)it, s));
+  return MPK_OK;
+}
+
+int mpk_set_capture(mpk_ctx* c, int iter, float* logits, float* hidden) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  c->capture_iter = iter;
+  c->cap_logits = logits;
+  c->cap_hidden = hidden;
+  return MPK_OK;
+}
+
+int mpk_status(mpk_ctx* c) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  if (!c->compiled) return MPK_OK;
+  Status st{};
+  cudaError_t e = cudaMemcpy(&st, c->status_dev, sizeof(st), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(c, MPK_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
+  if (st.code == 0) return MPK_OK;
+  static const char* where[] = {"?", "worker dependency wait", "producer queue wait", "weight ring wait",
+                                "task fifo wait", "scheduler gate wait", "scheduler queue space wait", "start",
+                                "embedding token check", "task dispatch"};
+  const char* w = (st.where >= 0 && st.where < 10) ? where[st.where] : "?";
+  fail(c, st.code, "device status %d at %s: op %d task %d worker %d iter %d observed %u expected %u", st.code, w, st.op,
+       st.task, st.worker, st.iter, st.observed, st.expected);
+  return st.code;
+}
+
+int mpk_request_abort(mpk_ctx* c) {
+  if (!c || !c->abort_host) return MPK_ERR_INVALID_ARG;
+  *(volatile int32_t*)c->abort_host = 1;
+  return MPK_OK;
+}
+
+int mpk_timeline(mpk_ctx* c, uint64_t* out, int cap) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  if (!c->compiled || !c->graph.timeline) return 0;
+  uint32_t n = 0;
+  CUDA_OR_FAIL(c, cudaMemcpy(&n, c->graph.timeline_n, sizeof(n), cudaMemcpyDeviceToHost));
+  if ((int)n > c->graph.max_timeline) n = (uint32_t)c->graph.max_timeline;
+  if (out && cap > 0) {
+    const size_t k = std::min<size_t>(n, (size_t)cap);
+    CUDA_OR_FAIL(c, cudaMemcpy(out, c->graph.timeline, k * 5 * sizeof(uint64_t), cudaMemcpyDeviceToHost));
+  }
+  return (int)n;
+}
+
+int mpk_destroy(mpk_ctx* c) {
+  if (!c) return MPK_ERR_INVALID_ARG;
+  for (void* p : c->allocs) cudaFree(p);
+  if (c->abort_host) cudaFreeHost(c->abort_host);
+  delete c;
+  return MPK_OK;
+}
+
+const char* mpk_last_error(mpk_ctx* c) { return c ? c->err.c_str() : g_create_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,126 @@
+// Internal layout shared by the host compiler and the device runtime.
+#pragma once
+#include <stdint.h>
+
+namespace mpk {
+
+// Worker block: one producer warp (weight stream) + CONSUMER_WARPS compute warps.
+constexpr int CONSUMER_WARPS = 8;
+constexpr int CONSUMER_THREADS = CONSUMER_WARPS * 32;
+constexpr int BLOCK_THREADS = CONSUMER_THREADS + 32;
+constexpr int STAGE_BYTES = 32768;          // one weight stage in shared memory
+constexpr int NSTAGES = 6;                  // weight ring depth
+constexpr int TASK_FIFO = 4;                // decoded task entries buffered per worker
+constexpr int QUEUE_CAP = 64;               // global task queue entries per worker
+constexpr int MAX_RPS = 64;                 // rows per stage upper bound
+constexpr int MAX_KW = 8;
+constexpr int MAX_SEG = 3;
+constexpr int MAX_G = 8;                    // query heads per kv head
+constexpr int MAX_D = 128;                  // head dim
+constexpr int SCHED_WARPS_PER_SM = 4;
+
+enum TaskKind : int32_t {
+  TK_EMBED = 1,
+  TK_NORM_GEMV = 2,
+  TK_ATTN = 3,
+  TK_GEMV_RESID = 4,
+  TK_NORM_GEMV_SILU = 5,
+  TK_NORM_GEMV_ARGMAX = 6,
+};
+
+// One operation of the compiled graph (device resident, read-only in the kernel).
+struct OpDesc {
+  int32_t kind;
+  int32_t ntasks;          // tasks per iteration
+  int32_t nwarps;          // consumer warps the task computes with (block_dim / 32)
+  int32_t N;               // output rows of the GEMV (gate/up: I); embed: H
+  int32_t K;               // reduction length
+  int32_t kw, rw;          // consumer warp grid: kw warps along K, rw row groups
+  int32_t epl;             // K elements per lane = K / (kw * 32)
+  int32_t rps;             // weight rows per stage (per matrix)
+  int32_t nseg;            // number of stacked weight matrices (RMSNORM_LINEAR)
+  int32_t seg_row0[MAX_SEG + 1];
+  const uint16_t* W[MAX_SEG];   // bf16 weights [rows, K]
+  float* y[MAX_SEG];            // fp32 outputs of RMSNORM_LINEAR
+  const uint16_t* W_up;         // SILU: up matrix (W[0] = gate)
+  const float* x;               // fp32 input (norm ops) / residual (RESID)
+  const uint16_t* a_in;         // bf16 input of RESID
+  const uint16_t* norm_w;       // bf16 [K]
+  float* x_out;                 // RESID: residual updated in place; EMBED: x
+  uint16_t* a_out;              // SILU / ATTN output bf16
+  float eps;
+  int32_t capture_slot;
+  // attention
+  int32_t layer, L, Hq, Hkv, d, G, C, S;
+  const float* q;
+  const float* k;
+  const float* v;
+  const uint16_t* qn_w;
+  const uint16_t* kn_w;
+  uint16_t* kc;
+  uint16_t* vc;
+  float* part;                  // [R][Hq][C][d + 2]
+  uint32_t* merge_cnt;          // [R][Hkv]
+  const float2* rope;           // [S][d/2] (cos, sin)
+  // embed / LM head
+  const uint16_t* table;        // EMBED: embedding table [V][H]
+  unsigned long long* keys;     // ARGMAX: per-request packed (value, index) maxima
+  uint32_t* arrive;             // ARGMAX: arrival counter
+  int64_t* pred;                // ARGMAX: optional [R][S]
+  // events
+  int32_t dep_event;            // event this op waits on
+  int32_t dep_trigger;          // increments of dep_event per iteration
+  int32_t dep_iter_offset;      // wait for (iter + offset) * trigger
+  int32_t out_event;            // event this op signals
+  int32_t out_trigger;          // increments of out_event per iteration
+  int32_t signal_per_task;      // 1: every task signals; 0: merges / finisher signal
+};
+
+struct Status {
+  int32_t code;      // 0 ok, else negative mpk_error
+  int32_t where;     // 1 worker dep, 2 producer queue, 3 producer ring, 4 consumer fifo, 5 scheduler gate, 6 scheduler space, 7 start
+  int32_t op, task, worker, iter;
+  uint32_t observed, expected;
+};
+
+struct Control {
+  uint32_t ready;
+  uint32_t n_iter;
+  uint32_t pad[30];
+};
+
+struct Graph {
+  const OpDesc* ops;
+  int32_t nops;
+  int32_t R, S, V, H, L;
+  int32_t num_workers, num_sched;   // scheduler warps
+  int32_t sched_ctas;
+  int32_t lookahead;
+  uint32_t* events;                 // [nops] (one 128-byte line each)
+  unsigned long long* queue;        // [num_workers][QUEUE_CAP]
+  uint32_t* q_head;                 // [num_workers] (one line each)
+  uint32_t* q_tail;
+  int32_t* step;
+  int64_t* tokens;
+  const int32_t* step_end;
+  Control* ctl;
+  Status* status;
+  volatile int32_t* abort_flag;     // host-mapped
+  uint64_t timeout_ns;
+  int32_t capture_iter;
+  float* cap_logits;
+  float* cap_hidden;
+  int32_t profiling;
+  int32_t max_timeline;
+  unsigned long long* timeline;     // [max_timeline][5]
+  uint32_t* timeline_n;
+};
+
+constexpr int EVENT_STRIDE = 32;    // uint32 per event / queue counter (128 bytes)
+constexpr unsigned long long QUEUE_TERMINATE = ~0ull;
+
+__host__ __device__ inline unsigned long long pack_entry(uint32_t iter, uint32_t op, uint32_t task) {
+  return ((unsigned long long)iter << 32) | ((unsigned long long)op << 16) | (unsigned long long)task;
+}
+
+}  // namespace mpk

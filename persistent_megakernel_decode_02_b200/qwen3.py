@@ -1,0 +1,119 @@
+"""Task graph of a Qwen3-style decoder built on the PersistentKernel API.
+
+The pages name Qwen3-8B as the demo model ("Mirage Persistent Kernel: Fusing
+Multi-GPU LLM Inference into One Kernel Launch", "Getting Started") and the
+fused rmsnorm_linear layer as the building block ("The API").  One decoding
+iteration is: embedding, then per layer [RMSNorm+QKV, QK-norm+RoPE+attention,
+o_proj+residual, RMSNorm+gate/up+SiLU*up, down_proj+residual], then final
+RMSNorm + LM head + greedy argmax, which advances `step` and writes `tokens`.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, List, Optional
+
+import torch
+
+from .kernel import PersistentKernel
+
+
+def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
+               block_dim: int = 256, tied: Optional[bool] = None) -> List[dict]:
+    """The fused-layer list (pure host logic, no GPU): one dict per operation with
+    the method name and its keyword arguments."""
+    s = shape
+    gt = gemv_tasks or num_workers
+    tied = s.tied if tied is None else tied
+    plan: List[dict] = [dict(method="embed_layer", embedding="embed_tokens", output="x", grid_dim=requests,
+                             block_dim=block_dim, capture_slot=0)]
+    for l in range(s.layers):
+        p = f"layers.{l}."
+        plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
+                         weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
+                         grid_dim=min(gt, s.q_dim + 2 * s.kv_dim), block_dim=block_dim, eps=s.eps))
+        plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm", k_norm=p + "k_norm",
+                         k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
+                         grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
+                         rope_theta=s.rope_theta))
+        plan.append(dict(method="linear_residual_layer", input="o", weight=p + "o_proj", residual="x",
+                         grid_dim=min(gt, s.hidden), block_dim=block_dim))
+        plan.append(dict(method="rmsnorm_linear_silu_mul_layer", input="x",
+                         weight_norm=p + "post_attention_layernorm", weight_gate=p + "gate_proj",
+                         weight_up=p + "up_proj", output="a", grid_dim=min(gt, s.intermediate), block_dim=block_dim,
+                         eps=s.eps))
+        plan.append(dict(method="linear_residual_layer", input="a", weight=p + "down_proj", residual="x",
+                         grid_dim=min(gt, s.hidden), block_dim=block_dim, capture_slot=l + 1))
+    plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
+                     weight_lm="embed_tokens" if tied else "lm_head", pred="pred", grid_dim=min(gt, s.vocab),
+                     block_dim=block_dim, eps=s.eps))
+    return plan
+
+
+def default_attn_chunks(shape, requests: int, num_workers: int, max_seq: int) -> int:
+    """Split-K chunks per (request, kv head): enough tasks to cover the workers for
+    long contexts, about 64 positions per chunk for short ones."""
+    by_workers = max(1, num_workers // (shape.kv_heads * requests))
+    by_length = max(1, -(-max_seq // 64))
+    return max(1, min(by_workers, by_length))
+
+
+@dataclass
+class Decoder:
+    """A compiled decoder: the kernel plus the tensors a caller reads or writes."""
+    kernel: PersistentKernel
+    shape: object
+    requests: int
+    max_seq: int
+    k_cache: torch.Tensor
+    v_cache: torch.Tensor
+    pred: torch.Tensor
+    buffers: Dict[str, torch.Tensor]
+
+    def run(self, step, tokens, step_end=None, stream=None):
+        self.kernel(step, tokens, step_end, stream)
+
+    def run_op_by_op(self, step, tokens, step_end=None, stream=None):
+        self.kernel.run_op_by_op(step, tokens, step_end, stream)
+
+
+def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_seq: int,
+                  num_workers: Optional[int] = None, num_local_schedulers: int = 16,
+                  attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 256,
+                  k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
+                  profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0) -> Decoder:
+    """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
+    activations and compile the task graph.  max_seq = KV-cache positions = the
+    tokens' row length (seq_length)."""
+    from . import _lib
+
+    s = shape
+    if num_workers is None:
+        num_workers = _lib.load().mpk_device_sm_count() - num_local_schedulers // 4
+    mk = PersistentKernel(num_workers, num_local_schedulers, 0)
+    for name, t in weights.items():
+        mk.attach_input(t, name)
+    dev = next(iter(weights.values())).device
+    kv_shape = (s.layers, requests, s.kv_heads, max_seq, s.head_dim)
+    if k_cache is None:
+        k_cache = torch.zeros(kv_shape, dtype=torch.bfloat16, device=dev)
+    if v_cache is None:
+        v_cache = torch.zeros(kv_shape, dtype=torch.bfloat16, device=dev)
+    mk.attach_input(k_cache, "k_cache")
+    mk.attach_input(v_cache, "v_cache")
+    pred = torch.full((requests, max_seq), -1, dtype=torch.int64, device=dev)
+    mk.attach_input(pred, "pred")
+    bufs = {
+        "x": mk.new_tensor((requests, s.hidden), torch.float32, "x"),
+        "q": mk.new_tensor((requests, s.q_dim), torch.float32, "q"),
+        "k": mk.new_tensor((requests, s.kv_dim), torch.float32, "k"),
+        "v": mk.new_tensor((requests, s.kv_dim), torch.float32, "v"),
+        "o": mk.new_tensor((requests, s.q_dim), torch.bfloat16, "o"),
+        "a": mk.new_tensor((requests, s.intermediate), torch.bfloat16, "a"),
+    }
+    if attn_chunks is None:
+        attn_chunks = default_attn_chunks(s, requests, num_workers, max_seq)
+    for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim):
+        op = dict(op)
+        getattr(mk, op.pop("method"))(**op)
+    mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s)
+    return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)

@@ -1,0 +1,72 @@
+"""Host-only checks of the C ABI (no GPU needed): the library loads, exports every
+symbol the header declares, and validates the worker/scheduler split."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+
+from persistent_megakernel_decode_02_b200 import _lib, layer_plan, default_attn_chunks
+from synth import qwen3 as sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    txt = open(os.path.join(ROOT, "include", "mpk.h")).read()
+    return sorted(set(re.findall(r"^MPK_API [^(]*?\b(mpk_\w+)\(", txt, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _header_functions()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks {n}"
+    assert lib.mpk_abi_version() == 1
+    assert lib.mpk_worker_threads() == 256
+
+
+GOLDEN = json.load(open(os.path.join(ROOT, "tests", "golden", "sm_split.json")))
+
+
+@pytest.mark.parametrize("case", GOLDEN["cases"], ids=lambda c: c["id"])
+def test_sm_formula_cases(case):
+    lib = _lib.load()
+    rc = lib.mpk_validate_split(case["sms"], case["workers"], case["local"], case["remote"])
+    assert _lib.ERRORS.get(rc, "OK") == case["expect"], lib.mpk_last_error(None)
+
+
+def test_create_without_device_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host without a GPU only")
+    lib = _lib.load()
+    ctx = ctypes.c_void_p()
+    rc = lib.mpk_create(144, 16, 0, ctypes.byref(ctx))
+    assert _lib.ERRORS[rc] == "CUDA" and not ctx.value
+
+
+def test_layer_plan_structure():
+    s = sq.QWEN3_8B
+    plan = layer_plan(s, requests=1, num_workers=144, attn_chunks=9)
+    assert plan[0]["method"] == "embed_layer" and plan[-1]["method"] == "rmsnorm_lmhead_argmax_layer"
+    assert len(plan) == 2 + 5 * s.layers
+    kinds = [p["method"] for p in plan[1:6]]
+    assert kinds == ["rmsnorm_linear_layer", "attention_layer", "linear_residual_layer",
+                     "rmsnorm_linear_silu_mul_layer", "linear_residual_layer"]
+    assert plan[2]["grid_dim"] == (8, 9, 1)
+    assert all(p["grid_dim"] == 144 for p in plan[1:-1] if p["method"] != "attention_layer")
+    assert plan[-1]["weight_lm"] == "lm_head"
+    assert layer_plan(sq.QWEN3_0_6B, 1, 144, 4)[-1]["weight_lm"] == "embed_tokens"
+    # the down projection of layer l captures residual slot l+1
+    assert [p.get("capture_slot") for p in plan if p.get("weight", "").endswith("down_proj")] == \
+        list(range(1, s.layers + 1))
+
+
+def test_default_attention_chunks():
+    assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 551) == 9
+    assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 32897) == 18
+    assert default_attn_chunks(sq.TINY, 1, 144, 24) == 1
