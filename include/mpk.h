@@ -132,6 +132,8 @@ typedef struct {
     int32_t sched_lookahead;/* scheduler dispatch window in operations (<=0: default 4)   */
     double timeout_s;       /* limit of every device-side wait (<=0: default 2 s)        */
     int32_t max_timeline;   /* timeline entries kept when profiling (<=0: 1<<20)         */
+    int32_t prefetch_kb;    /* L2 prefetch distance per worker ahead of the shared-memory
+                               weight ring, KiB (<=0: off)                                 */
 } mpk_options;
 
 /* Library build facts. */
@@ -237,8 +239,10 @@ MPK_API int mpk_status(mpk_ctx *ctx);
 MPK_API int mpk_request_abort(mpk_ctx *ctx);
 
 /* Number of timeline records of the last profiled run, and a copy of up to
- * `cap` of them into host memory `out` (5 x uint64 each: packed task id
- * (iter<<32 | op<<16 | task), worker, start ns, dependency-ready ns, end ns). */
+ * `cap` of them into host memory `out` (8 x uint64 each, %globaltimer ns):
+ * packed task id (iter<<32 | op<<16 | task), worker, task popped, dependency
+ * met, task done, prologue done (0 if none), first weight stage ready (0 if
+ * none), first weight stage issued by the producer (0 if none). */
 MPK_API int mpk_timeline(mpk_ctx *ctx, uint64_t *out, int cap);
 
 /* Free the context and every library-owned allocation. */

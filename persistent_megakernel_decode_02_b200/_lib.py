@@ -51,6 +51,7 @@ class Options(ctypes.Structure):
         ("sched_lookahead", ctypes.c_int32),
         ("timeout_s", ctypes.c_double),
         ("max_timeline", ctypes.c_int32),
+        ("prefetch_kb", ctypes.c_int32),
     ]
 
 
@@ -88,12 +89,14 @@ _lib = None
 
 
 def load():
-    """Load libmpk.so (built by build.py / __graft_entry__.build())."""
+    """Load libmpk.so (built by build.py / __graft_entry__.build()).  MPK_LIBRARY
+    may name another build of the same library (e.g. a ring-depth variant)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(SO_PATH):
-            raise ImportError(f"libmpk.so not found at {SO_PATH}: run persistent_megakernel_decode_02_b200/build.py")
-        lib = ctypes.CDLL(SO_PATH)
+        path = os.environ.get("MPK_LIBRARY", SO_PATH)
+        if not os.path.exists(path):
+            raise ImportError(f"libmpk.so not found at {path}: run persistent_megakernel_decode_02_b200/build.py")
+        lib = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(lib, name)
             fn.restype = res

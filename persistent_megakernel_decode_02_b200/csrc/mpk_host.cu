@@ -137,31 +137,18 @@ int need(mpk_ctx* c, int li, const char* role, const char* name, mpk_dtype dt, i
     if (!(cond)) return fail(c, MPK_ERR_SHAPE, __VA_ARGS__); \
   } while (0)
 
-// GEMV geometry: kw warps along K (EPL elements per lane), rw row groups,
-// rows per stage.
-int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats) {
+// GEMV geometry: rows per shared-memory stage (each consumer warp owns whole
+// rows, so any K that is a multiple of 256 and fits the input buffer works).
+int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats, bool norm) {
   const int K = o.K;
   if (K % 256 != 0) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d is not a multiple of 256", li, K);
-  static const int supported[] = {8, 16, 24, 32, 48, 64};
-  int best_kw = 0, best_epl = 0;
-  for (int kw = MAX_KW; kw >= 1; kw >>= 1) {
-    if (o.nwarps % kw != 0 || K % (kw * 256) != 0) continue;
-    const int epl = K / (kw * 32);
-    bool ok = false;
-    for (int s : supported) ok |= (s == epl);
-    if (ok) { best_kw = kw; best_epl = epl; break; }
-  }
-  if (!best_kw)
-    return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: no warp split of K=%d over %d warps keeps 8..64 elements per lane",
-                li, K, o.nwarps);
-  o.kw = best_kw;
-  o.epl = best_epl;
-  o.rw = o.nwarps / best_kw;
+  if (K > MAX_K) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d exceeds %d", li, K, MAX_K);
+  if (norm && K > MAX_NORM_K)
+    return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: RMSNorm width %d exceeds %d", li, K, MAX_NORM_K);
   const int row_bytes = K * 2 * (two_mats ? 2 : 1);
   int rps = STAGE_BYTES / row_bytes;
   if (rps < 1) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: one weight row (%d bytes) exceeds a stage", li, row_bytes);
   if (rps > MAX_RPS) rps = MAX_RPS;
-  if (rps >= o.rw) rps -= rps % o.rw;
   o.rps = rps;
   return MPK_OK;
 }
@@ -338,6 +325,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (o.sched_lookahead <= 0) o.sched_lookahead = 4;
   if (o.timeout_s <= 0) o.timeout_s = 2.0;
   if (o.max_timeline <= 0) o.max_timeline = 1 << 20;
+  if (o.prefetch_kb == 0) o.prefetch_kb = -1;
   c->opts = o;
 
   std::vector<OpDesc> ops(n_layers);
@@ -485,7 +473,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         if (R != 1)
           return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: projections with %d requests are not built yet (1 supported)",
                       li, R);
-        int rc = gemv_geometry(c, li, op, silu);
+        int rc = gemv_geometry(c, li, op, silu, !resid);
         if (rc != MPK_OK) return rc;
         rc = check_grid(c, li, Ly, ntasks, op.N);
         if (rc != MPK_OK) return rc;
@@ -614,7 +602,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   }
   unsigned long long* timeline = nullptr;
   if (o.profiling) {
-    rc = alloc(c, &timeline, sizeof(unsigned long long) * 5 * (size_t)o.max_timeline);
+    rc = alloc(c, &timeline, sizeof(unsigned long long) * TIMELINE_FIELDS * (size_t)o.max_timeline);
     if (rc != MPK_OK) return rc;
   }
   for (int p = 0; p < P; ++p) {
@@ -645,6 +633,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   g.num_sched = c->num_local;
   g.sched_ctas = c->num_local / 4;
   g.lookahead = o.sched_lookahead;
+  g.prefetch_bytes = o.prefetch_kb > 0 ? (uint32_t)o.prefetch_kb * 1024u : 0u;
   g.events = reinterpret_cast<uint32_t*>(sb + o_events);
   g.queue = queue;
   g.q_head = reinterpret_cast<uint32_t*>(sb + o_qhead);
@@ -767,7 +756,7 @@ int mpk_timeline(mpk_ctx* c, uint64_t* out, int cap) {
   if ((int)n > c->graph.max_timeline) n = (uint32_t)c->graph.max_timeline;
   if (out && cap > 0) {
     const size_t k = std::min<size_t>(n, (size_t)cap);
-    CUDA_OR_FAIL(c, cudaMemcpy(out, c->graph.timeline, k * 5 * sizeof(uint64_t), cudaMemcpyDeviceToHost));
+    CUDA_OR_FAIL(c, cudaMemcpy(out, c->graph.timeline, k * TIMELINE_FIELDS * sizeof(uint64_t), cudaMemcpyDeviceToHost));
   }
   return (int)n;
 }

@@ -8,12 +8,20 @@ namespace mpk {
 constexpr int CONSUMER_WARPS = 8;
 constexpr int CONSUMER_THREADS = CONSUMER_WARPS * 32;
 constexpr int BLOCK_THREADS = CONSUMER_THREADS + 32;
-constexpr int STAGE_BYTES = 32768;          // one weight stage in shared memory
-constexpr int NSTAGES = 6;                  // weight ring depth
+#ifndef MPK_STAGE_BYTES
+#define MPK_STAGE_BYTES 32768
+#endif
+#ifndef MPK_NSTAGES
+#define MPK_NSTAGES 6
+#endif
+constexpr int STAGE_BYTES = MPK_STAGE_BYTES;  // one weight stage in shared memory
+constexpr int NSTAGES = MPK_NSTAGES;          // weight ring depth
 constexpr int TASK_FIFO = 4;                // decoded task entries buffered per worker
 constexpr int QUEUE_CAP = 64;               // global task queue entries per worker
 constexpr int MAX_RPS = 64;                 // rows per stage upper bound
-constexpr int MAX_KW = 8;
+constexpr int MAX_K = 12288;                // longest GEMV input kept in shared memory (bf16)
+constexpr int MAX_NORM_K = 4096;            // longest RMSNorm input (held in registers)
+constexpr int MAX_XS = 1024;                // residual rows of a task preloaded to shared memory
 constexpr int MAX_SEG = 3;
 constexpr int MAX_G = 8;                    // query heads per kv head
 constexpr int MAX_D = 128;                  // head dim
@@ -35,8 +43,6 @@ struct OpDesc {
   int32_t nwarps;          // consumer warps the task computes with (block_dim / 32)
   int32_t N;               // output rows of the GEMV (gate/up: I); embed: H
   int32_t K;               // reduction length
-  int32_t kw, rw;          // consumer warp grid: kw warps along K, rw row groups
-  int32_t epl;             // K elements per lane = K / (kw * 32)
   int32_t rps;             // weight rows per stage (per matrix)
   int32_t nseg;            // number of stacked weight matrices (RMSNORM_LINEAR)
   int32_t seg_row0[MAX_SEG + 1];
@@ -96,6 +102,7 @@ struct Graph {
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;
   int32_t lookahead;
+  uint32_t prefetch_bytes;          // L2 prefetch distance per worker (0 = off)
   uint32_t* events;                 // [nops] (one 128-byte line each)
   unsigned long long* queue;        // [num_workers][QUEUE_CAP]
   uint32_t* q_head;                 // [num_workers] (one line each)
@@ -112,10 +119,11 @@ struct Graph {
   float* cap_hidden;
   int32_t profiling;
   int32_t max_timeline;
-  unsigned long long* timeline;     // [max_timeline][5]
+  unsigned long long* timeline;     // [max_timeline][TIMELINE_FIELDS]
   uint32_t* timeline_n;
 };
 
+constexpr int TIMELINE_FIELDS = 8;  // entry, worker, popped, dependency met, end, prologue done, first stage ready, first stage issued
 constexpr int EVENT_STRIDE = 32;    // uint32 per event / queue counter (128 bytes)
 constexpr unsigned long long QUEUE_TERMINATE = ~0ull;
 

@@ -45,15 +45,14 @@ struct AttnScratch {
 };
 static_assert(MAX_G * MAX_D / 2 >= 512, "attention scratch");
 
-struct GemvScratch {
-  float red[2][MAX_RPS][MAX_KW][2];              // per-row partial dots [parity][row][k-warp][gate/up]
-};
-
 struct __align__(128) Smem {
   uint8_t ring[NSTAGES][STAGE_BYTES];
   union {
     AttnScratch a;
-    GemvScratch g;
+    struct {
+      uint16_t hs[MAX_K];                        // GEMV input vector (bf16)
+      float xs[MAX_XS];                          // residual rows of the task
+    } g;
   } u;
   float ss[CONSUMER_WARPS];
   unsigned long long bestk[CONSUMER_WARPS];
@@ -63,6 +62,8 @@ struct __align__(128) Smem {
   uint64_t fifo_full[TASK_FIFO];
   uint64_t fifo_empty[TASK_FIFO];
   unsigned long long cur_entry;
+  unsigned long long fifo_t[TASK_FIFO];          // profiling: first weight stage issued
+  unsigned long long t_pro, t_data;              // profiling: prologue done, first stage ready
   int32_t last;     // last-arrival flag
 };
 
@@ -72,18 +73,23 @@ __device__ __forceinline__ bool aborted(const Graph& g) {
   return false;
 }
 
-__device__ __noinline__ void record_error(const Graph& g, int code, int where, int op, int task,
-                                          int worker, int iter, uint32_t observed, uint32_t expected) {
-  if (atomicCAS(&g.status->code, 0, code) == 0) {
-    g.status->where = where;
-    g.status->op = op;
-    g.status->task = task;
-    g.status->worker = worker;
-    g.status->iter = iter;
-    g.status->observed = observed;
-    g.status->expected = expected;
+__device__ __noinline__ void record_error_at(Status* st, int code, int where, int op, int task, int worker,
+                                             int iter, uint32_t observed, uint32_t expected) {
+  if (atomicCAS(&st->code, 0, code) == 0) {
+    st->where = where;
+    st->op = op;
+    st->task = task;
+    st->worker = worker;
+    st->iter = iter;
+    st->observed = observed;
+    st->expected = expected;
     __threadfence();
   }
+}
+
+__device__ __forceinline__ void record_error(const Graph& g, int code, int where, int op, int task, int worker,
+                                             int iter, uint32_t observed, uint32_t expected) {
+  record_error_at(g.status, code, where, op, task, worker, iter, observed, expected);
 }
 
 // Polls the host abort flag (mapped memory, slow) only now and then.
@@ -174,6 +180,39 @@ __device__ void issue_stage(const OpDesc& op, int r, int n, uint8_t* dst, uint64
   }
 }
 
+// Prefetch rows [r, r+n) of a GEMV operation's weights into L2.
+__device__ void prefetch_rows(const OpDesc& op, int r, int n) {
+  const uint32_t row_bytes = (uint32_t)op.K * 2u;
+  if (op.kind == TK_NORM_GEMV_SILU) {
+    prefetch_l2(op.W[0] + (size_t)r * op.K, row_bytes * n);
+    prefetch_l2(op.W_up + (size_t)r * op.K, row_bytes * n);
+    return;
+  }
+  while (n > 0) {
+    const int s = seg_of(op, r);
+    const int cnt = min(n, op.seg_row0[s + 1] - r);
+    prefetch_l2(op.W[s] + (size_t)(r - op.seg_row0[s]) * op.K, row_bytes * cnt);
+    r += cnt;
+    n -= cnt;
+  }
+}
+
+// The producer keeps a second cursor over the same task sequence that issues
+// L2 prefetches for the weight bytes just beyond what the shared-memory ring
+// will hold: [loaded + ring, loaded + ring + prefetch_bytes).  It peeks at
+// queued entries without popping them (the scheduler never overwrites an entry
+// that has not been popped), so HBM keeps streaming the next operations'
+// weights while this worker waits on a dependency; bytes the ring itself is
+// about to load are never requested twice.
+struct PrefetchCursor {
+  uint32_t q;              // queue index of the task the cursor is in
+  int row;                 // next row of that task (-1: not started)
+  bool done;               // reached the end of the queue
+  bool have;               // e holds entry q (already popped, so not re-read)
+  unsigned long long e;
+  uint64_t pos;            // stream byte offset of (q, row)
+};
+
 template <bool kStandalone>
 __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
   const uint64_t pol = policy_evict_first();
@@ -181,19 +220,74 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
   bool ok = true;
   uint32_t* qtail = g.q_tail + (size_t)worker * EVENT_STRIDE;
   uint32_t* qhead = g.q_head + (size_t)worker * EVENT_STRIDE;
+  const unsigned long long* queue = g.queue + (size_t)worker * QUEUE_CAP;
+  uint32_t tail_seen = 0;
+  uint64_t ld_bytes = 0;
+  PrefetchCursor pf{0u, -1, false, false, 0ull, 0ull};
+  const uint64_t pf_dist = kStandalone ? 0ull : (uint64_t)g.prefetch_bytes;
+  constexpr uint64_t RING = (uint64_t)NSTAGES * STAGE_BYTES;
+
+  auto prefetch_some = [&]() {
+    const uint64_t lo = ld_bytes + RING, hi = lo + pf_dist;
+    while (!pf.done && pf.pos < hi) {
+      if (!pf.have) {
+        // entries at or after the pop position are never overwritten
+        if (pf.q >= tail_seen) {
+          tail_seen = ld_acquire(qtail);
+          if (pf.q >= tail_seen) return;
+        }
+        pf.e = __ldcg(queue + (pf.q % QUEUE_CAP));
+        pf.have = true;
+      }
+      if (pf.e == QUEUE_TERMINATE) {
+        pf.done = true;
+        return;
+      }
+      const OpDesc& op = g.ops[(int)((pf.e >> 16) & 0xFFFFu)];
+      int r0 = 0, r1 = 0;
+      if (is_gemv(op.kind)) task_rows(op, (int)(pf.e & 0xFFFFu), r0, r1);
+      if (pf.row < 0) pf.row = r0;
+      if (pf.row >= r1) {
+        ++pf.q;
+        pf.row = -1;
+        pf.have = false;
+        continue;
+      }
+      const uint32_t rb = (uint32_t)op.K * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
+      const int n = min(r1 - pf.row, max(1, (int)(65536u / rb)));
+      if (pf.pos + (uint64_t)rb * n > lo) prefetch_rows(op, pf.row, n);
+      pf.row += n;
+      pf.pos += (uint64_t)rb * n;
+    }
+  };
+
   while (true) {
     unsigned long long entry;
     if (kStandalone) {
       entry = (fpos == 0) ? pack_entry(sa_iter, (uint32_t)sa_op, blockIdx.x) : QUEUE_TERMINATE;
     } else {
       if (!wait_counter(g, qtail, qpos + 1, 2, -1, -1, worker, -1)) { ok = false; break; }
-      entry = __ldcg(g.queue + (size_t)worker * QUEUE_CAP + (qpos % QUEUE_CAP));
+      entry = __ldcg(queue + (qpos % QUEUE_CAP));
+      // a prefetch cursor that has not passed this task restarts at its first row
+      if (pf.q < qpos || (pf.q == qpos && !pf.have)) {
+        // the cursor is behind: restart it at this task (the stream offset of
+        // its first row is the current load offset)
+        pf.q = qpos;
+        pf.row = -1;
+        pf.have = true;
+        pf.e = entry;
+        pf.pos = ld_bytes;
+      }
       ++qpos;
       st_release(qhead, qpos);
     }
     const uint32_t f = fpos % TASK_FIFO;
     if (!wait_mbar(g, &sm.fifo_empty[f], ((fpos / TASK_FIFO) & 1u) ^ 1u, 4, worker)) { ok = false; break; }
     sm.fifo[f] = entry;
+    // profiling: the issue time of this task's first stage is stored before
+    // the slot is published; it is overwritten below once the stage is issued
+    // (the consumer reads it only at the end of the task).
+    if (g.profiling) sm.fifo_t[f] = 0ull;
     mbar_arrive(&sm.fifo_full[f]);
     ++fpos;
     if (entry == QUEUE_TERMINATE) break;
@@ -208,10 +302,22 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     for (int r = row0; r < row1; r += op.rps) {
       const int n = min(op.rps, row1 - r);
       const uint32_t slot = pstage % NSTAGES;
-      if (!wait_mbar(g, &sm.empty[slot], ((pstage / NSTAGES) & 1u) ^ 1u, 3, worker)) { ok = false; break; }
+      const uint32_t par = ((pstage / NSTAGES) & 1u) ^ 1u;
+      if (!mbar_try_wait(&sm.empty[slot], par)) {
+        const uint64_t t0 = globaltimer();
+        for (uint32_t it = 0;; ++it) {
+          if (pf_dist) prefetch_some();
+          if (mbar_try_wait(&sm.empty[slot], par)) break;
+          if (check_stop(g, t0, it, 3, opi, task, worker, -1, par, 0)) { ok = false; break; }
+        }
+        if (!ok) break;
+      }
+      if (g.profiling && r == row0) atomicExch(&sm.fifo_t[f], (unsigned long long)globaltimer());
       mbar_arrive_expect_tx(&sm.full[slot], bytes_row * (uint32_t)n);
       issue_stage(op, r, n, sm.ring[slot], &sm.full[slot], pol);
+      ld_bytes += (uint64_t)bytes_row * n;
       ++pstage;
+      if (pf_dist) prefetch_some();
     }
     if (!ok) break;
   }
@@ -229,71 +335,123 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
 }
 
 // ------------------------------------------------------------------ consumer helpers
-// Elected-thread wait for a ring stage.  Returns true on failure (thread 0
-// only); the caller shares the outcome through consumer_sync_or.
-__device__ __forceinline__ bool stage_wait_elected(Smem& sm, const Graph& g, uint32_t cstage, int ctid,
-                                                   int worker) {
-  if (ctid != 0) return false;
-  const uint32_t slot = cstage % NSTAGES;
-  return !wait_mbar(g, &sm.full[slot], (cstage / NSTAGES) & 1u, 3, worker);
+// Dot product of one bf16 weight row with the bf16 input vector, both in shared
+// memory; lane l covers elements [8l + 256j, 8l + 256j + 8).
+__device__ __forceinline__ float dot_row(const uint16_t* w, const uint16_t* h, int K, int lane) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+  for (int e = lane * 8; e < K; e += 256) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
+    const uint4 hv = *reinterpret_cast<const uint4*>(h + e);
+    a0 = fmaf(bf16_lo(wv.x), bf16_lo(hv.x), a0);
+    a1 = fmaf(bf16_hi(wv.x), bf16_hi(hv.x), a1);
+    a2 = fmaf(bf16_lo(wv.y), bf16_lo(hv.y), a2);
+    a3 = fmaf(bf16_hi(wv.y), bf16_hi(hv.y), a3);
+    a0 = fmaf(bf16_lo(wv.z), bf16_lo(hv.z), a0);
+    a1 = fmaf(bf16_hi(wv.z), bf16_hi(hv.z), a1);
+    a2 = fmaf(bf16_lo(wv.w), bf16_lo(hv.w), a2);
+    a3 = fmaf(bf16_hi(wv.w), bf16_hi(hv.w), a3);
+  }
+  return (a0 + a1) + (a2 + a3);
 }
 
-template <int EPL>
-__device__ __forceinline__ float dot_slice(const uint16_t* w, const float (&h)[EPL], int lane) {
-  float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-  for (int j = 0; j < EPL / 8; ++j) {
-    const uint4 v = *reinterpret_cast<const uint4*>(w + j * 256 + lane * 8);
-    a0 = fmaf(bf16_lo(v.x), h[j * 8 + 0], a0);
-    a1 = fmaf(bf16_hi(v.x), h[j * 8 + 1], a1);
-    a0 = fmaf(bf16_lo(v.y), h[j * 8 + 2], a0);
-    a1 = fmaf(bf16_hi(v.y), h[j * 8 + 3], a1);
-    a0 = fmaf(bf16_lo(v.z), h[j * 8 + 4], a0);
-    a1 = fmaf(bf16_hi(v.z), h[j * 8 + 5], a1);
-    a0 = fmaf(bf16_lo(v.w), h[j * 8 + 6], a0);
-    a1 = fmaf(bf16_hi(v.w), h[j * 8 + 7], a1);
+// Two rows (gate and up) against the same input: one pass over h.
+__device__ __forceinline__ void dot_row2(const uint16_t* w, const uint16_t* u, const uint16_t* h, int K, int lane,
+                                         float& dw, float& du) {
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll 2
+  for (int e = lane * 8; e < K; e += 256) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
+    const uint4 uv = *reinterpret_cast<const uint4*>(u + e);
+    const uint4 hv = *reinterpret_cast<const uint4*>(h + e);
+    const float h0 = bf16_lo(hv.x), h1 = bf16_hi(hv.x), h2 = bf16_lo(hv.y), h3 = bf16_hi(hv.y);
+    const float h4 = bf16_lo(hv.z), h5 = bf16_hi(hv.z), h6 = bf16_lo(hv.w), h7 = bf16_hi(hv.w);
+    a0 = fmaf(bf16_lo(wv.x), h0, a0); a1 = fmaf(bf16_hi(wv.x), h1, a1);
+    a0 = fmaf(bf16_lo(wv.y), h2, a0); a1 = fmaf(bf16_hi(wv.y), h3, a1);
+    a0 = fmaf(bf16_lo(wv.z), h4, a0); a1 = fmaf(bf16_hi(wv.z), h5, a1);
+    a0 = fmaf(bf16_lo(wv.w), h6, a0); a1 = fmaf(bf16_hi(wv.w), h7, a1);
+    b0 = fmaf(bf16_lo(uv.x), h0, b0); b1 = fmaf(bf16_hi(uv.x), h1, b1);
+    b0 = fmaf(bf16_lo(uv.y), h2, b0); b1 = fmaf(bf16_hi(uv.y), h3, b1);
+    b0 = fmaf(bf16_lo(uv.z), h4, b0); b1 = fmaf(bf16_hi(uv.z), h5, b1);
+    b0 = fmaf(bf16_lo(uv.w), h6, b0); b1 = fmaf(bf16_hi(uv.w), h7, b1);
   }
-  return a0 + a1;
+  dw = a0 + a1;
+  du = b0 + b1;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)f32_to_bf16_rn(lo) | ((uint32_t)f32_to_bf16_rn(hi) << 16);
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
 // ------------------------------------------------------------------ GEMV tasks
-// Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector.
-// Consumer warp cw covers K slice kwi = cw % kw for rows i = grp (mod rw),
-// grp = cw / kw; each lane holds EPL elements of h in registers.  Per stage
-// every warp writes its per-row partial dot into shared memory; after the
-// stage barrier the first n threads sum the kw partials in fixed order and run
-// the operation's epilogue.
-template <int KIND, int EPL>
+// Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector h
+// held in shared memory as bf16.  Each consumer warp owns whole rows (task
+// row j goes to warp j % nwarps) and runs the operation's epilogue for them
+// itself, so the weight stages need no block-wide barrier: every warp waits
+// for each stage, computes its rows in it and releases the stage.
+template <int KIND>
 __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
                           uint32_t& cstage, int cw, int lane, int worker) {
   const int ctid = cw * 32 + lane;
-  const int K = op.K, kw = op.kw, rw = op.rw, rps = op.rps;
-  const bool computes = cw < op.nwarps;
-  const int kwi = cw % kw, grp = cw / kw;
-  const int kbase = kwi * (K / kw);
+  const int K = op.K, rps = op.rps, nw = op.nwarps;
   int row0, row1;
   task_rows(op, task, row0, row1);
+  uint16_t* hs = sm.u.g.hs;
 
-  // ---- prologue: the input vector slice of this warp, rounded to bf16
-  float h[EPL];
+  // ---- prologue: the input vector, bf16, in shared memory.  Every global
+  // load of the prologue is issued before the first use (one L2 round trip).
+  const int nrows = row1 - row0;
+  const bool xs_ok = KIND == TK_GEMV_RESID && nrows <= MAX_XS;
   if (KIND == TK_GEMV_RESID) {
+    constexpr int NA = MAX_K / (CONSUMER_THREADS * 8);
+    uint4 av[NA];
 #pragma unroll
-    for (int j = 0; j < EPL / 8; ++j) {
-      const uint4 a = ldcg_u4(op.a_in + kbase + j * 256 + lane * 8);
-      h[j * 8 + 0] = bf16_lo(a.x); h[j * 8 + 1] = bf16_hi(a.x);
-      h[j * 8 + 2] = bf16_lo(a.y); h[j * 8 + 3] = bf16_hi(a.y);
-      h[j * 8 + 4] = bf16_lo(a.z); h[j * 8 + 5] = bf16_hi(a.z);
-      h[j * 8 + 6] = bf16_lo(a.w); h[j * 8 + 7] = bf16_hi(a.w);
+    for (int c = 0; c < NA; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) av[c] = ldcg_u4(op.a_in + k);
+    }
+    float xv[MAX_XS / CONSUMER_THREADS];
+#pragma unroll
+    for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
+      const int j = c * CONSUMER_THREADS + ctid;
+      if (xs_ok && j < nrows) xv[c] = __ldcg(op.x_out + row0 + j);
+    }
+#pragma unroll
+    for (int c = 0; c < NA; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) *reinterpret_cast<uint4*>(hs + k) = av[c];
+    }
+#pragma unroll
+    for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
+      const int j = c * CONSUMER_THREADS + ctid;
+      if (xs_ok && j < nrows) sm.u.g.xs[j] = xv[c];
     }
   } else {
-    // RMSNorm statistics over the whole input (fixed reduction order).
+    // RMSNorm: x and the norm weight are read once into registers, the
+    // statistics are reduced in a fixed order.
+    constexpr int NCH = MAX_NORM_K / (CONSUMER_THREADS * 8);
+    float xr[NCH][8];
+    uint4 wr[NCH];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) {
+        const float4 x0 = ldcg_f4(op.x + k), x1 = ldcg_f4(op.x + k + 4);
+        wr[c] = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
+        xr[c][0] = x0.x; xr[c][1] = x0.y; xr[c][2] = x0.z; xr[c][3] = x0.w;
+        xr[c][4] = x1.x; xr[c][5] = x1.y; xr[c][6] = x1.z; xr[c][7] = x1.w;
+      }
+    }
     float ss = 0.f;
-    for (int k = ctid * 4; k < K; k += CONSUMER_THREADS * 4) {
-      const float4 v = ldcg_f4(op.x + k);
-      ss = fmaf(v.x, v.x, ss); ss = fmaf(v.y, v.y, ss);
-      ss = fmaf(v.z, v.z, ss); ss = fmaf(v.w, v.w, ss);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(xr[c][e], xr[c][e], ss);
+      }
     }
     ss = warp_sum(ss);
     if (lane == 0) sm.ss[cw] = ss;
@@ -303,105 +461,88 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     for (int w = 0; w < CONSUMER_WARPS; ++w) tot += sm.ss[w];
     const float rinv = 1.0f / sqrtf(tot / (float)K + op.eps);
 #pragma unroll
-    for (int j = 0; j < EPL / 8; ++j) {
-      const int k = kbase + j * 256 + lane * 8;
-      const float4 x0 = ldcg_f4(op.x + k), x1 = ldcg_f4(op.x + k + 4);
-      const uint4 w = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
-      h[j * 8 + 0] = round_bf16(x0.x * rinv * bf16_lo(w.x));
-      h[j * 8 + 1] = round_bf16(x0.y * rinv * bf16_hi(w.x));
-      h[j * 8 + 2] = round_bf16(x0.z * rinv * bf16_lo(w.y));
-      h[j * 8 + 3] = round_bf16(x0.w * rinv * bf16_hi(w.y));
-      h[j * 8 + 4] = round_bf16(x1.x * rinv * bf16_lo(w.z));
-      h[j * 8 + 5] = round_bf16(x1.y * rinv * bf16_hi(w.z));
-      h[j * 8 + 6] = round_bf16(x1.z * rinv * bf16_lo(w.w));
-      h[j * 8 + 7] = round_bf16(x1.w * rinv * bf16_hi(w.w));
+    for (int c = 0; c < NCH; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) {
+        const uint4 w = wr[c];
+        uint4 hv;
+        hv.x = pack_bf16x2(xr[c][0] * rinv * bf16_lo(w.x), xr[c][1] * rinv * bf16_hi(w.x));
+        hv.y = pack_bf16x2(xr[c][2] * rinv * bf16_lo(w.y), xr[c][3] * rinv * bf16_hi(w.y));
+        hv.z = pack_bf16x2(xr[c][4] * rinv * bf16_lo(w.z), xr[c][5] * rinv * bf16_hi(w.z));
+        hv.w = pack_bf16x2(xr[c][6] * rinv * bf16_lo(w.w), xr[c][7] * rinv * bf16_hi(w.w));
+        *reinterpret_cast<uint4*>(hs + k) = hv;
+      }
     }
   }
+  consumer_sync();
+  if (g.profiling && ctid == 0) sm.t_pro = globaltimer();
 
-  unsigned long long best = 0ull;
   const bool capture = (g.capture_iter == (int)iter);
-  int par = 0;
-  // first stage
-  if (row0 < row1 && consumer_sync_or(stage_wait_elected(sm, g, cstage, ctid, worker))) return false;
-  for (int r = row0; r < row1; r += rps) {
-    const int n = min(rps, row1 - r);
+  unsigned long long best = 0ull;
+  bool fail = false;
+
+  // Epilogue of task-local row j with its full dot product(s).
+  auto finish = [&](int j, float v, float u) {
+    const int row = row0 + j;
+    if (KIND == TK_NORM_GEMV) {
+      const int sg = seg_of(op, row);
+      op.y[sg][row - op.seg_row0[sg]] = v;
+    } else if (KIND == TK_GEMV_RESID) {
+      const float nx = (xs_ok ? sm.u.g.xs[j] : __ldcg(op.x_out + row)) + v;
+      op.x_out[row] = nx;
+      if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
+        g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
+    } else if (KIND == TK_NORM_GEMV_SILU) {
+      op.a_out[row] = f32_to_bf16_rn(silu_f(v) * u);
+    } else {  // LM head
+      const unsigned long long key = argmax_key(v, (uint32_t)row);
+      best = key > best ? key : best;
+      if (capture && g.cap_logits != nullptr) g.cap_logits[row] = v;
+    }
+  };
+
+
+  int jn = cw;  // next task-local row of this warp
+  for (int base = 0; base < nrows; base += rps) {
+    const int n = min(rps, nrows - base);
     const uint32_t slot = cstage % NSTAGES;
+    bool ok = true;
+    if (lane == 0) ok = wait_mbar(g, &sm.full[slot], (cstage / NSTAGES) & 1u, 3, worker);
+    ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+    if (!ok) {
+      fail = true;
+      break;
+    }
+    if (g.profiling && ctid == 0 && base == 0) sm.t_data = globaltimer();
     const uint8_t* stage = sm.ring[slot];
-    if (computes) {
-      for (int i0 = grp; i0 < n; i0 += 4 * rw) {
-        float acc[4], accu[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int i = i0 + q * rw;
-          acc[q] = 0.f;
-          accu[q] = 0.f;
-          if (i < n) {
-            const uint16_t* wrow = reinterpret_cast<const uint16_t*>(stage + (size_t)i * K * 2) + kbase;
-            acc[q] = dot_slice<EPL>(wrow, h, lane);
-            if (KIND == TK_NORM_GEMV_SILU) {
-              const uint16_t* urow =
-                  reinterpret_cast<const uint16_t*>(stage + (size_t)(rps + i) * K * 2) + kbase;
-              accu[q] = dot_slice<EPL>(urow, h, lane);
-            }
-          }
+    if (cw < nw) {
+      int j = jn;
+      for (; j < base + n; j += nw) {
+        const int i = j - base;
+        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(stage + (size_t)i * K * 2);
+        float v, u = 0.f;
+        if (KIND == TK_NORM_GEMV_SILU) {
+          const uint16_t* urow = reinterpret_cast<const uint16_t*>(stage + (size_t)(rps + i) * K * 2);
+          dot_row2(wrow, urow, hs, K, lane, v, u);
+          u = warp_sum(u);
+        } else {
+          v = dot_row(wrow, hs, K, lane);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          acc[q] = warp_sum(acc[q]);
-          if (KIND == TK_NORM_GEMV_SILU) accu[q] = warp_sum(accu[q]);
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = i0 + q * rw;
-            if (i < n) {
-              sm.u.g.red[par][i][kwi][0] = acc[q];
-              if (KIND == TK_NORM_GEMV_SILU) sm.u.g.red[par][i][kwi][1] = accu[q];
-            }
-          }
-        }
+        v = warp_sum(v);
+        if (lane == 0) finish(j, v, u);
       }
+      jn = j;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
     ++cstage;
-    // Wait for the next stage of this task while the others reach the barrier.
-    const bool fail = (r + rps < row1) && stage_wait_elected(sm, g, cstage, ctid, worker);
-    const bool stop = consumer_sync_or(fail);
-    // ---- epilogue of this stage
-    if (ctid < n) {
-      float v = 0.f, u = 0.f;
-      for (int kk = 0; kk < kw; ++kk) {
-        v += sm.u.g.red[par][ctid][kk][0];
-        if (KIND == TK_NORM_GEMV_SILU) u += sm.u.g.red[par][ctid][kk][1];
-      }
-      const int row = r + ctid;
-      if (KIND == TK_NORM_GEMV) {
-        const int s = seg_of(op, row);
-        op.y[s][row - op.seg_row0[s]] = v;
-      } else if (KIND == TK_GEMV_RESID) {
-        const float nx = __ldcg(op.x_out + row) + v;
-        op.x_out[row] = nx;
-        if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
-          g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
-      } else if (KIND == TK_NORM_GEMV_SILU) {
-        op.a_out[row] = f32_to_bf16_rn(silu_f(v) * u);
-      } else {  // LM head
-        const unsigned long long key = argmax_key(v, (uint32_t)row);
-        best = key > best ? key : best;
-        if (capture && g.cap_logits != nullptr) g.cap_logits[row] = v;
-      }
-    }
-    par ^= 1;
-    if (stop) return false;
   }
+  if (KIND == TK_NORM_GEMV_ARGMAX && lane == 0) sm.bestk[cw] = best;
+  if (consumer_sync_or(fail)) return false;
 
   if (KIND == TK_NORM_GEMV_ARGMAX) {
     // Per-task maximum -> one 64-bit atomicMax; the last task to arrive
     // finishes the iteration.
-    best = warp_max_u64(best);
-    if (lane == 0) sm.bestk[cw] = best;
-    consumer_sync();
     if (ctid == 0) {
       unsigned long long b = 0ull;
       for (int w = 0; w < CONSUMER_WARPS; ++w) b = sm.bestk[w] > b ? sm.bestk[w] : b;
@@ -427,10 +568,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
         op.keys[rq] = 0ull;
       }
       consumer_sync();
-      if (ctid == 0) {
-        __threadfence();
-        red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
-      }
+      if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
     }
   }
   return true;
@@ -444,8 +582,10 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // query head.  Partials (max, sum, unnormalised output) go to global memory;
 // the last chunk task of (r, j) to arrive merges them in chunk order and
 // writes o = bf16(output).
+// Not inlined: it has its own register allocation, so its per-head arrays
+// never push the GEMV loops into spills.
 template <int G, int D>
-__device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, int cw, int lane) {
+__device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, int cw, int lane) {
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
   constexpr float LOG2E = 1.4426950408889634f;
@@ -454,42 +594,50 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   const int j = task % Hkv;
   const int c = (task / Hkv) % C;
   const int r = task / (Hkv * C);
-  int s;
-  const bool active = request_active(g, r, s);
   AttnScratch& A = sm.u.a;
   const size_t kvbase = ((((size_t)op.layer * g.R + r) * Hkv + j) * (size_t)op.S) * D;
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * C) * (D + 2);
+  // Prologue rows: warp cw < G takes query head cw of the group, warp G the
+  // key, warp G+1 the value.  Their loads do not depend on the step, so they
+  // are issued before it is read.
+  constexpr int EL = D / 32;  // elements per lane
+  const int prow = cw;
+  float x[EL];
+  if (prow < G + 2) {
+    const float* src = prow < G ? op.q + (size_t)r * op.Hq * D + (size_t)(j * G + prow) * D
+                     : prow == G ? op.k + (size_t)r * Hkv * D + (size_t)j * D
+                                 : op.v + (size_t)r * Hkv * D + (size_t)j * D;
+#pragma unroll
+    for (int e = 0; e < EL; ++e) x[e] = __ldcg(src + lane + 32 * e);
+  }
+  int s;
+  const bool active = request_active(g, r, s);
 
   if (active) {
     const int npos = s + 1;
     const int lo = (int)(((long long)c * npos) / C);
     const int hi = (int)(((long long)(c + 1) * npos) / C);
-    // ---- prologue: rows 0..G-1 = query heads, G = k, G+1 = v
-    for (int row = cw; row < G + 2; row += CONSUMER_WARPS) {
-      constexpr int EL = D / 32;  // elements per lane
-      float x[EL];
-      const float* src = row < G ? op.q + (size_t)r * op.Hq * D + (size_t)(j * G + row) * D
-                       : row == G ? op.k + (size_t)r * Hkv * D + (size_t)j * D
-                                  : op.v + (size_t)r * Hkv * D + (size_t)j * D;
+    if (prow < G + 2) {
+      if (prow <= G) {
+        float2 rc[EL / 2];
+        const float2* cs = op.rope + (size_t)s * (D / 2);
 #pragma unroll
-      for (int e = 0; e < EL; ++e) x[e] = __ldcg(src + lane + 32 * e);
-      if (row <= G) {
+        for (int e = 0; e < EL / 2; ++e) rc[e] = __ldg(cs + lane + 32 * e);
+        const uint16_t* wn = prow < G ? op.qn_w : op.kn_w;
+        uint16_t wb[EL];
+#pragma unroll
+        for (int e = 0; e < EL; ++e) wb[e] = __ldg(wn + lane + 32 * e);
         float ss = 0.f;
 #pragma unroll
         for (int e = 0; e < EL; ++e) ss = fmaf(x[e], x[e], ss);
         ss = warp_sum(ss);
         const float rinv = 1.0f / sqrtf(ss / (float)D + op.eps);
-        const uint16_t* wn = row < G ? op.qn_w : op.kn_w;
 #pragma unroll
-        for (int e = 0; e < EL; ++e) {
-          const uint16_t wb = __ldg(wn + lane + 32 * e);
-          x[e] = x[e] * rinv * __uint_as_float((uint32_t)wb << 16);
-        }
+        for (int e = 0; e < EL; ++e) x[e] = x[e] * rinv * __uint_as_float((uint32_t)wb[e] << 16);
         // rotate-half RoPE: element i pairs with i + D/2 (same lane, e + EL/2)
-        const float2* cs = op.rope + (size_t)s * (D / 2);
 #pragma unroll
         for (int e = 0; e < EL / 2; ++e) {
-          const float2 t = __ldg(cs + lane + 32 * e);
+          const float2 t = rc[e];
           const float a = x[e], b = x[e + EL / 2];
           x[e] = a * t.x - b * t.y;
           x[e + EL / 2] = b * t.x + a * t.y;
@@ -498,8 +646,8 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 #pragma unroll
       for (int e = 0; e < EL; ++e) {
         const int i = lane + 32 * e;
-        if (row < G) A.qs[row * D + i] = x[e];
-        else if (row == G) A.ks[i] = f32_to_bf16_rn(x[e]);
+        if (prow < G) A.qs[prow * D + i] = x[e] * (LOG2E / sqrtf((float)D));
+        else if (prow == G) A.ks[i] = f32_to_bf16_rn(x[e]);
         else A.vs[i] = f32_to_bf16_rn(x[e]);
       }
     }
@@ -515,17 +663,13 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 
     // ---- main loop
     const int grp = lane / LP, sub = lane % LP;
-    const float qscale = LOG2E / sqrtf((float)D);
-    float qr[G][8], acc[G][8], m[G], l[G];
+    float acc[G][8], m[G], l[G];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) {
       m[hh] = -INFINITY;
       l[hh] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        qr[hh][e] = A.qs[hh * D + sub * 8 + e] * qscale;
-        acc[hh][e] = 0.f;
-      }
+      for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
     }
     const uint16_t* kg = op.kc + kvbase + sub * 8;
     const uint16_t* vg = op.vc + kvbase + sub * 8;
@@ -547,9 +691,11 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       float sc[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaf(qr[hh][e], kf[e], a);
+        const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
+        const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
+        float a = q0.x * kf[0];
+        a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+        a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
 #pragma unroll
         for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
         sc[hh] = a;
@@ -631,26 +777,32 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   if (sm.last) {
     if (active) {
       __threadfence();
+      // one pass over the chunk partials, in chunk order (online rescaling)
       for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
         const int hh = idx / D, i = idx % D;
         const float* p = pbase + (size_t)hh * C * (D + 2);
-        float M = -INFINITY;
-        for (int cc = 0; cc < C; ++cc) M = fmaxf(M, __ldcg(p + (size_t)cc * (D + 2)));
-        float Ls = 0.f, Os = 0.f;
+        float M = -INFINITY, Ls = 0.f, Os = 0.f;
+#pragma unroll 4
         for (int cc = 0; cc < C; ++cc) {
           const float mc = __ldcg(p + (size_t)cc * (D + 2));
-          const float f = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-          Ls = fmaf(__ldcg(p + (size_t)cc * (D + 2) + 1), f, Ls);
-          Os = fmaf(__ldcg(p + (size_t)cc * (D + 2) + 2 + i), f, Os);
+          const float lc = __ldcg(p + (size_t)cc * (D + 2) + 1);
+          const float oc = __ldcg(p + (size_t)cc * (D + 2) + 2 + i);
+          if (mc == -INFINITY) continue;
+          if (mc > M) {
+            const float sc = exp2f(M - mc);  // M = -inf -> 0
+            Ls *= sc;
+            Os *= sc;
+            M = mc;
+          }
+          const float f = exp2f(mc - M);
+          Ls = fmaf(lc, f, Ls);
+          Os = fmaf(oc, f, Os);
         }
         op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = f32_to_bf16_rn(Os / Ls);
       }
     }
     consumer_sync();
-    if (ctid == 0) {
-      __threadfence();
-      red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
-    }
+    if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
   }
   return true;
 }
@@ -685,20 +837,6 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 }
 
 // ------------------------------------------------------------------ dispatch
-template <int KIND>
-__device__ bool gemv_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
-                              uint32_t& cstage, int cw, int lane, int worker) {
-  switch (op.epl) {
-    case 8: return gemv_task<KIND, 8>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    case 16: return gemv_task<KIND, 16>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    case 24: return gemv_task<KIND, 24>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    case 32: return gemv_task<KIND, 32>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    case 48: return gemv_task<KIND, 48>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    case 64: return gemv_task<KIND, 64>(sm, g, op, task, iter, cstage, cw, lane, worker);
-    default: return false;
-  }
-}
-
 __device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int task, int cw, int lane) {
   const int key = op.G * 1000 + op.d;
   switch (key) {
@@ -738,7 +876,11 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     const OpDesc& op = g.ops[opi];
 
     uint64_t t_start = 0, t_ready = 0;
-    if (g.profiling && ctid == 0) t_start = globaltimer();
+    if (g.profiling && ctid == 0) {
+      t_start = globaltimer();
+      sm.t_pro = 0ull;
+      sm.t_data = 0ull;
+    }
     // dependency: the event of the op this one follows
     if (!kStandalone && ctid == 0) {
       const uint32_t target = (iter + (uint32_t)op.dep_iter_offset) * (uint32_t)op.dep_trigger;
@@ -752,13 +894,13 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     bool ok = true;
     switch (op.kind) {
       case TK_EMBED: ok = embed_task(g, op, task, iter, ctid); break;
-      case TK_NORM_GEMV: ok = gemv_dispatch<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
-      case TK_GEMV_RESID: ok = gemv_dispatch<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
+      case TK_NORM_GEMV: ok = gemv_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
+      case TK_GEMV_RESID: ok = gemv_task<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       case TK_NORM_GEMV_SILU:
-        ok = gemv_dispatch<TK_NORM_GEMV_SILU>(sm, g, op, task, iter, cstage, cw, lane, worker);
+        ok = gemv_task<TK_NORM_GEMV_SILU>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
       case TK_NORM_GEMV_ARGMAX:
-        ok = gemv_dispatch<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
+        ok = gemv_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
       case TK_ATTN: ok = attn_dispatch(sm, g, op, task, cw, lane); break;
       default: ok = false;
@@ -769,19 +911,19 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     }
     consumer_sync();
     if (ctid == 0) {
-      if (op.signal_per_task) {
-        __threadfence();
-        red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
-      }
+      if (op.signal_per_task) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
       if (g.profiling) {
         const uint32_t k = atomicAdd(g.timeline_n, 1u);
         if (k < (uint32_t)g.max_timeline) {
-          unsigned long long* rec = g.timeline + (size_t)k * 5;
+          unsigned long long* rec = g.timeline + (size_t)k * TIMELINE_FIELDS;
           rec[0] = entry;
           rec[1] = (unsigned long long)worker;
           rec[2] = t_start;
           rec[3] = t_ready;
           rec[4] = globaltimer();
+          rec[5] = sm.t_pro;
+          rec[6] = sm.t_data;
+          rec[7] = atomicAdd(&sm.fifo_t[(fpos - 1) % TASK_FIFO], 0ull);
         }
       }
     }

@@ -165,9 +165,10 @@ class PersistentKernel:
 
     # ------------------------------------------------------------------ compile / run
     def compile(self, profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
-                max_timeline: int = 0) -> str:
+                max_timeline: int = 0, prefetch_kb: int = 0) -> str:
         arr = (_lib.Layer * len(self._layers))(*self._layers)
-        opts = _lib.Options(int(profiling), int(sched_lookahead), float(timeout_s), int(max_timeline))
+        opts = _lib.Options(int(profiling), int(sched_lookahead), float(timeout_s), int(max_timeline),
+                            int(prefetch_kb))
         check(self._lib.mpk_compile(self._ctx, arr, len(self._layers), ctypes.byref(opts)), self._ctx)
         self._keep.append(arr)
         self.compiled = True
@@ -235,10 +236,12 @@ class PersistentKernel:
     def request_abort(self) -> None:
         check(self._lib.mpk_request_abort(self._ctx), self._ctx)
 
+    TIMELINE_FIELDS = ("entry", "worker", "popped", "ready", "end", "prologue", "first_data", "first_issue")
+
     def timeline(self) -> torch.Tensor:
-        """[n, 5] uint64 records (iter<<32|op<<16|task, worker, start, ready, end) in ns."""
+        """[n, 8] records (see TIMELINE_FIELDS; times in %globaltimer ns)."""
         n = int(self._lib.mpk_timeline(self._ctx, None, 0))
-        out = torch.zeros((max(n, 0), 5), dtype=torch.int64)
+        out = torch.zeros((max(n, 0), len(self.TIMELINE_FIELDS)), dtype=torch.int64)
         if n > 0:
             self._lib.mpk_timeline(self._ctx, ctypes.c_void_p(out.data_ptr()), n)
         return out

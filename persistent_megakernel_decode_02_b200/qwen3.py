@@ -80,7 +80,8 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   num_workers: Optional[int] = None, num_local_schedulers: int = 16,
                   attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 256,
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
-                  profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0) -> Decoder:
+                  profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
+                  prefetch_kb: int = 0) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length)."""
@@ -115,5 +116,5 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim):
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
-    mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s)
+    mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb)
     return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)
