@@ -57,7 +57,8 @@ def parse():
     p.add_argument("--profiling", action="store_true", help="record the task timeline of the timed run")
     p.add_argument("--timeline-out", default="")
     p.add_argument("--cpu-budget-s", type=float, default=20.0)
-    p.add_argument("--prefetch-kb", type=int, default=0, help="L2 prefetch distance per worker (0 default, <0 off)")
+    p.add_argument("--prefetch-kb", type=int, default=0, help="L2 prefetch distance per worker (<=0 off)")
+    p.add_argument("--attention", choices=["auto", "fused", "split"], default="auto")
     p.add_argument("--layers", type=int, default=0, help="override the layer count (profiling cases)")
     p.add_argument("--vocab", type=int, default=0, help="override the vocabulary (profiling cases)")
     return p.parse_args()
@@ -302,7 +303,8 @@ def main():
     W = args.workers or (load().mpk_device_sm_count() - ls // 4)
     dec = build_decoder(shape, w, requests=1, max_seq=S, num_workers=W, num_local_schedulers=ls,
                         attn_chunks=args.attn_chunks or None, sched_lookahead=args.lookahead,
-                        profiling=args.profiling, prefetch_kb=args.prefetch_kb)
+                        profiling=args.profiling, prefetch_kb=args.prefetch_kb,
+                        fused_attention={"auto": None, "fused": True, "split": False}[args.attention])
     stream = torch.cuda.current_stream(dev)
     tok = tokens_cpu.to(dev)
     step = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -345,6 +347,7 @@ def main():
         tl = dec.kernel.timeline()
         if args.timeline_out:
             write_chrome_trace(tl, dec, args.timeline_out)
+        op_kind.per_layer = (dec.kernel.num_ops() - 2) // shape.layers
         timeline_stats = timeline_summary(tl, shape)
 
     op_ms = None
@@ -420,12 +423,18 @@ def main():
 
 
 def op_kind(op: int, shape) -> str:
-    last = 1 + 5 * shape.layers
+    last = 1 + op_kind.per_layer * shape.layers
     if op == 0:
         return "embed"
     if op == last:
         return "lmhead_argmax"
-    return ["rmsnorm_qkv", "attention", "o_proj_resid", "rmsnorm_gateup_silu", "down_resid"][(op - 1) % 5]
+    per = 5 if op_kind.per_layer == 5 else 4
+    names = (["rmsnorm_qkv", "attention", "o_proj_resid", "rmsnorm_gateup_silu", "down_resid"] if per == 5 else
+             ["rmsnorm_qkv_attention", "o_proj_resid", "rmsnorm_gateup_silu", "down_resid"])
+    return names[(op - 1) % per]
+
+
+op_kind.per_layer = 5
 
 
 def timeline_summary(tl, shape) -> dict:

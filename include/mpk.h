@@ -102,12 +102,23 @@ typedef enum {
      * the runtime advances `step` after every iteration).  inputs[0] = x;
      * weights = w_norm [K], W_lm [V,K]; outputs[0] (optional, may be NULL) =
      * pred int64 [R,S].  Must be the last operation of the graph. */
-    MPK_OP_RMSNORM_LMHEAD_ARGMAX = 6
+    MPK_OP_RMSNORM_LMHEAD_ARGMAX = 6,
+    /* RMSNORM_LINEAR for the stacked q/k/v projections fused with ATTENTION:
+     * the projection rows are split per kv head j (its G query heads, its key
+     * and its value: G*d + 2d rows) into grid_dim.x tasks per head, and the
+     * last of those tasks to finish computes head j's attention directly (one
+     * pass over positions 0..s, no split-K).  inputs[0] = x fp32 [R,K];
+     * weights = w_norm [K], Wq [Hq*d,K], Wk [Hkv*d,K], Wv [Hkv*d,K], q_norm [d],
+     * k_norm [d], k_cache, v_cache [L,R,Hkv,S,d]; outputs = q [R,Hq*d],
+     * k, v [R,Hkv*d] (fp32 scratch), o bf16 [R,Hq*d].
+     * grid_dim = (tasks per kv head, Hkv, R).  Meant for short contexts; long
+     * ones use RMSNORM_LINEAR followed by ATTENTION with split-K. */
+    MPK_OP_RMSNORM_QKV_ATTENTION = 7
 } mpk_op;
 
 typedef struct { int32_t x, y, z; } mpk_dim3;
 
-#define MPK_MAX_IO 4
+#define MPK_MAX_IO 8
 
 /* One fused operation.  Unused name slots are NULL.  grid_dim gives the number
  * of tasks (thread blocks) x*y*z; block_dim the threads per task (a multiple

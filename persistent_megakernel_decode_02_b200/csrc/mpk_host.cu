@@ -342,6 +342,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     const mpk_layer& Ly = layers[li];
     OpDesc& op = ops[li];
     memset(&op, 0, sizeof(op));
+    op.groups = 1;
     op.capture_slot = Ly.capture_slot;
     op.eps = Ly.eps > 0 ? Ly.eps : 1e-6f;
     const int64_t ntasks64 = (int64_t)Ly.grid_dim.x * (Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1) *
@@ -465,6 +466,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
             if (op.nseg == 0) return fail(c, MPK_ERR_INVALID_ARG, "layer %d: no linear weight", li);
             op.seg_row0[op.nseg] = rows;
             for (int s = op.nseg + 1; s <= MAX_SEG; ++s) op.seg_row0[s] = rows;
+            for (int s = 0; s < op.nseg; ++s) op.grp_rows[s] = op.seg_row0[s + 1] - op.seg_row0[s];
             op.N = rows;
           }
         }
@@ -541,6 +543,100 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         if (L < 0 || op.L > L) L = op.L;
         break;
       }
+      case MPK_OP_RMSNORM_QKV_ATTENTION: {
+        op.kind = TK_QKV_ATTN;
+        const Tensor *x, *wn, *wq, *wk, *wv, *qn, *kn, *kc, *vc, *q, *k, *v, *o;
+        NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32, 2, &x);
+        NEED("weights[0] (norm)", Ly.weights[0], MPK_BF16, 1, &wn);
+        NEED("weights[1] (Wq)", Ly.weights[1], MPK_BF16, 2, &wq);
+        NEED("weights[2] (Wk)", Ly.weights[2], MPK_BF16, 2, &wk);
+        NEED("weights[3] (Wv)", Ly.weights[3], MPK_BF16, 2, &wv);
+        NEED("weights[4] (q_norm)", Ly.weights[4], MPK_BF16, 1, &qn);
+        NEED("weights[5] (k_norm)", Ly.weights[5], MPK_BF16, 1, &kn);
+        NEED("weights[6] (k_cache)", Ly.weights[6], MPK_BF16, 5, &kc);
+        NEED("weights[7] (v_cache)", Ly.weights[7], MPK_BF16, 5, &vc);
+        NEED("outputs[0] (q)", Ly.outputs[0], MPK_FP32, 2, &q);
+        NEED("outputs[1] (k)", Ly.outputs[1], MPK_FP32, 2, &k);
+        NEED("outputs[2] (v)", Ly.outputs[2], MPK_FP32, 2, &v);
+        NEED("outputs[3] (o)", Ly.outputs[3], MPK_BF16, 2, &o);
+        op.K = (int)x->dims[1];
+        SHAPE_CHECK(wn->dims[0] == op.K, "layer %d: norm weight %s, input width %d", li, dims_str(wn->dims).c_str(), op.K);
+        SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
+        const int d = (int)kc->dims[4], Hkv = (int)kc->dims[2];
+        SHAPE_CHECK(wq->dims[0] % d == 0, "layer %d: Wq rows %lld not a multiple of head_dim %d", li,
+                    (long long)wq->dims[0], d);
+        const int Hq = (int)(wq->dims[0] / d);
+        SHAPE_CHECK(Hq % Hkv == 0, "layer %d: %d query heads not a multiple of %d kv heads", li, Hq, Hkv);
+        SHAPE_CHECK(wq->dims[1] == op.K && wk->dims[1] == op.K && wv->dims[1] == op.K &&
+                        wk->dims[0] == (int64_t)Hkv * d && wv->dims[0] == (int64_t)Hkv * d,
+                    "layer %d: Wq %s Wk %s Wv %s vs K=%d, Hkv=%d, d=%d", li, dims_str(wq->dims).c_str(),
+                    dims_str(wk->dims).c_str(), dims_str(wv->dims).c_str(), op.K, Hkv, d);
+        SHAPE_CHECK(qn->dims[0] == d && kn->dims[0] == d, "layer %d: norm weights must have head_dim %d", li, d);
+        if (R < 0) R = (int)x->dims[0];
+        SHAPE_CHECK(x->dims[0] == R && q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R &&
+                        kc->dims[1] == R,
+                    "layer %d: request count mismatch (graph %d)", li, R);
+        SHAPE_CHECK(q->dims[1] == (int64_t)Hq * d && k->dims[1] == (int64_t)Hkv * d && v->dims[1] == k->dims[1] &&
+                        o->dims[1] == q->dims[1],
+                    "layer %d: q %s k %s v %s o %s", li, dims_str(q->dims).c_str(), dims_str(k->dims).c_str(),
+                    dims_str(v->dims).c_str(), dims_str(o->dims).c_str());
+        SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range", li, Ly.layer);
+        if (R != 1)
+          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: projections with %d requests are not built yet (1 supported)",
+                      li, R);
+        const int G = Hq / Hkv;
+        if (!((d == 64 || d == 128) && (G == 1 || G == 2 || G == 4)))
+          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: head_dim %d with %d query heads per kv head", li, d, G);
+        const int gx = Ly.grid_dim.x, gy = Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1,
+                  gz = Ly.grid_dim.z > 0 ? Ly.grid_dim.z : 1;
+        SHAPE_CHECK(gy == Hkv && gz == R,
+                    "layer %d: RMSNORM_QKV_ATTENTION needs grid_dim = (tasks per kv head, kv_heads=%d, requests=%d)",
+                    li, Hkv, R);
+        op.groups = Hkv;
+        op.N = G * d + 2 * d;
+        SHAPE_CHECK(gx <= op.N, "layer %d: %d tasks per kv head for %d rows", li, gx, op.N);
+        op.nseg = 3;
+        op.seg_row0[0] = 0;
+        op.seg_row0[1] = G * d;
+        op.seg_row0[2] = G * d + d;
+        op.seg_row0[3] = G * d + 2 * d;
+        op.grp_rows[0] = G * d;
+        op.grp_rows[1] = d;
+        op.grp_rows[2] = d;
+        op.W[0] = (const uint16_t*)wq->ptr;
+        op.W[1] = (const uint16_t*)wk->ptr;
+        op.W[2] = (const uint16_t*)wv->ptr;
+        op.y[0] = (float*)q->ptr;
+        op.y[1] = (float*)k->ptr;
+        op.y[2] = (float*)v->ptr;
+        op.x = (const float*)x->ptr;
+        op.norm_w = (const uint16_t*)wn->ptr;
+        op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = 1;
+        op.L = (int)kc->dims[0];
+        op.S = (int)kc->dims[3];
+        op.layer = Ly.layer;
+        op.q = op.y[0]; op.k = op.y[1]; op.v = op.y[2];
+        op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
+        op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
+        op.a_out = (uint16_t*)o->ptr;
+        if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
+        merge_off[li] = {1, merge_u32};
+        merge_u32 += (size_t)R * Hkv;
+        const float theta = Ly.rope_theta > 0 ? Ly.rope_theta : 1.0e6f;
+        int ri = -1;
+        for (size_t i = 0; i < rope_keys.size(); ++i)
+          if (rope_keys[i].theta == theta && rope_keys[i].d == d && rope_keys[i].S == op.S) ri = (int)i;
+        if (ri < 0) { rope_keys.push_back({theta, d, op.S}); ri = (int)rope_keys.size() - 1; }
+        rope_of[li] = ri;
+        int rc = gemv_geometry(c, li, op, false, true);
+        if (rc != MPK_OK) return rc;
+        rc = check_grid(c, li, Ly, ntasks, 0);
+        if (rc != MPK_OK) return rc;
+        op.signal_per_task = 0;
+        op.out_trigger = R * Hkv;
+        if (L < 0 || op.L > L) L = op.L;
+        break;
+      }
       default:
         return fail(c, MPK_ERR_INVALID_ARG, "layer %d: unknown op %d", li, Ly.op);
     }
@@ -610,6 +706,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     if (op.kind == TK_ATTN) {
       op.part = part;
       op.merge_cnt = reinterpret_cast<uint32_t*>(sb + o_merge) + merge_off[p].second;
+      op.rope = rope_dev[rope_of[p]];
+    }
+    if (op.kind == TK_QKV_ATTN) {
+      op.grp_cnt = reinterpret_cast<uint32_t*>(sb + o_merge) + merge_off[p].second;
       op.rope = rope_dev[rope_of[p]];
     }
     if (op.kind == TK_NORM_GEMV_ARGMAX) {

@@ -34,6 +34,7 @@ enum TaskKind : int32_t {
   TK_GEMV_RESID = 4,
   TK_NORM_GEMV_SILU = 5,
   TK_NORM_GEMV_ARGMAX = 6,
+  TK_QKV_ATTN = 7,
 };
 
 // One operation of the compiled graph (device resident, read-only in the kernel).
@@ -45,7 +46,10 @@ struct OpDesc {
   int32_t K;               // reduction length
   int32_t rps;             // weight rows per stage (per matrix)
   int32_t nseg;            // number of stacked weight matrices (RMSNORM_LINEAR)
-  int32_t seg_row0[MAX_SEG + 1];
+  int32_t seg_row0[MAX_SEG + 1];  // segment offsets within one group's rows
+  int32_t groups;          // row groups (QKV+attention: kv heads; else 1); N = rows per group
+  int32_t grp_rows[MAX_SEG];      // rows of segment s per group (matrix row = g * grp_rows + local)
+  uint32_t* grp_cnt;       // QKV+attention: finished tasks per (request, group)
   const uint16_t* W[MAX_SEG];   // bf16 weights [rows, K]
   float* y[MAX_SEG];            // fp32 outputs of RMSNORM_LINEAR
   const uint16_t* W_up;         // SILU: up matrix (W[0] = gate)

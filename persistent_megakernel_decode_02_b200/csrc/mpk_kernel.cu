@@ -131,14 +131,19 @@ __device__ bool wait_mbar(const Graph& g, uint64_t* bar, uint32_t parity, int wh
 }
 
 // ------------------------------------------------------------------ task geometry
-__device__ __forceinline__ void task_rows(const OpDesc& op, int task, int& row0, int& row1) {
-  row0 = (int)(((long long)task * op.N) / op.ntasks);
-  row1 = (int)(((long long)(task + 1) * op.N) / op.ntasks);
+// Rows [row0, row1) of group g that task `task` computes (groups split the
+// tasks evenly; N is the row count of one group).
+__device__ __forceinline__ void task_rows(const OpDesc& op, int task, int& g, int& row0, int& row1) {
+  const int tpg = op.ntasks / op.groups;
+  g = task / tpg;
+  const int t = task - g * tpg;
+  row0 = (int)(((long long)t * op.N) / tpg);
+  row1 = (int)(((long long)(t + 1) * op.N) / tpg);
 }
 
 __device__ __forceinline__ bool is_gemv(int kind) {
   return kind == TK_NORM_GEMV || kind == TK_GEMV_RESID || kind == TK_NORM_GEMV_SILU ||
-         kind == TK_NORM_GEMV_ARGMAX;
+         kind == TK_NORM_GEMV_ARGMAX || kind == TK_QKV_ATTN;
 }
 
 __device__ __forceinline__ bool request_active(const Graph& g, int r, int& s) {
@@ -160,9 +165,14 @@ __device__ __forceinline__ int seg_of(const OpDesc& op, int row) {
   return s;
 }
 
+// Matrix row of group-local row `row` that lies in segment s.
+__device__ __forceinline__ size_t seg_row(const OpDesc& op, int g, int s, int row) {
+  return (size_t)g * op.grp_rows[s] + (size_t)(row - op.seg_row0[s]);
+}
+
 // ------------------------------------------------------------------ producer
 // Issue the bulk copies of one stage: rows [r, r+n) of the op's row space.
-__device__ void issue_stage(const OpDesc& op, int r, int n, uint8_t* dst, uint64_t* bar, uint64_t pol) {
+__device__ void issue_stage(const OpDesc& op, int g, int r, int n, uint8_t* dst, uint64_t* bar, uint64_t pol) {
   const uint32_t row_bytes = (uint32_t)op.K * 2u;
   if (op.kind == TK_NORM_GEMV_SILU) {
     bulk_g2s(dst, op.W[0] + (size_t)r * op.K, row_bytes * n, bar, pol);
@@ -173,7 +183,7 @@ __device__ void issue_stage(const OpDesc& op, int r, int n, uint8_t* dst, uint64
     const int s = seg_of(op, r);
     const int seg_end = op.seg_row0[s + 1];
     const int cnt = min(n, seg_end - r);
-    bulk_g2s(dst, op.W[s] + (size_t)(r - op.seg_row0[s]) * op.K, row_bytes * cnt, bar, pol);
+    bulk_g2s(dst, op.W[s] + seg_row(op, g, s, r) * op.K, row_bytes * cnt, bar, pol);
     dst += (size_t)cnt * row_bytes;
     r += cnt;
     n -= cnt;
@@ -181,7 +191,7 @@ __device__ void issue_stage(const OpDesc& op, int r, int n, uint8_t* dst, uint64
 }
 
 // Prefetch rows [r, r+n) of a GEMV operation's weights into L2.
-__device__ void prefetch_rows(const OpDesc& op, int r, int n) {
+__device__ void prefetch_rows(const OpDesc& op, int g, int r, int n) {
   const uint32_t row_bytes = (uint32_t)op.K * 2u;
   if (op.kind == TK_NORM_GEMV_SILU) {
     prefetch_l2(op.W[0] + (size_t)r * op.K, row_bytes * n);
@@ -191,7 +201,7 @@ __device__ void prefetch_rows(const OpDesc& op, int r, int n) {
   while (n > 0) {
     const int s = seg_of(op, r);
     const int cnt = min(n, op.seg_row0[s + 1] - r);
-    prefetch_l2(op.W[s] + (size_t)(r - op.seg_row0[s]) * op.K, row_bytes * cnt);
+    prefetch_l2(op.W[s] + seg_row(op, g, s, r) * op.K, row_bytes * cnt);
     r += cnt;
     n -= cnt;
   }
@@ -244,8 +254,8 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
         return;
       }
       const OpDesc& op = g.ops[(int)((pf.e >> 16) & 0xFFFFu)];
-      int r0 = 0, r1 = 0;
-      if (is_gemv(op.kind)) task_rows(op, (int)(pf.e & 0xFFFFu), r0, r1);
+      int r0 = 0, r1 = 0, pg = 0;
+      if (is_gemv(op.kind)) task_rows(op, (int)(pf.e & 0xFFFFu), pg, r0, r1);
       if (pf.row < 0) pf.row = r0;
       if (pf.row >= r1) {
         ++pf.q;
@@ -255,7 +265,7 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
       }
       const uint32_t rb = (uint32_t)op.K * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
       const int n = min(r1 - pf.row, max(1, (int)(65536u / rb)));
-      if (pf.pos + (uint64_t)rb * n > lo) prefetch_rows(op, pf.row, n);
+      if (pf.pos + (uint64_t)rb * n > lo) prefetch_rows(op, pg, pf.row, n);
       pf.row += n;
       pf.pos += (uint64_t)rb * n;
     }
@@ -296,8 +306,8 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     const int task = (int)(entry & 0xFFFFu);
     const OpDesc& op = g.ops[opi];
     if (!is_gemv(op.kind)) continue;
-    int row0, row1;
-    task_rows(op, task, row0, row1);
+    int grp, row0, row1;
+    task_rows(op, task, grp, row0, row1);
     const uint32_t bytes_row = (uint32_t)op.K * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
     for (int r = row0; r < row1; r += op.rps) {
       const int n = min(op.rps, row1 - r);
@@ -314,7 +324,7 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
       }
       if (g.profiling && r == row0) atomicExch(&sm.fifo_t[f], (unsigned long long)globaltimer());
       mbar_arrive_expect_tx(&sm.full[slot], bytes_row * (uint32_t)n);
-      issue_stage(op, r, n, sm.ring[slot], &sm.full[slot], pol);
+      issue_stage(op, grp, r, n, sm.ring[slot], &sm.full[slot], pol);
       ld_bytes += (uint64_t)bytes_row * n;
       ++pstage;
       if (pf_dist) prefetch_some();
@@ -385,6 +395,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
+__device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
+                              int cw, int lane);
+
 // ------------------------------------------------------------------ GEMV tasks
 // Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector h
 // held in shared memory as bf16.  Each consumer warp owns whole rows (task
@@ -396,8 +409,8 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
                           uint32_t& cstage, int cw, int lane, int worker) {
   const int ctid = cw * 32 + lane;
   const int K = op.K, rps = op.rps, nw = op.nwarps;
-  int row0, row1;
-  task_rows(op, task, row0, row1);
+  int grp, row0, row1;
+  task_rows(op, task, grp, row0, row1);
   uint16_t* hs = sm.u.g.hs;
 
   // ---- prologue: the input vector, bf16, in shared memory.  Every global
@@ -484,9 +497,9 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   // Epilogue of task-local row j with its full dot product(s).
   auto finish = [&](int j, float v, float u) {
     const int row = row0 + j;
-    if (KIND == TK_NORM_GEMV) {
+    if (KIND == TK_NORM_GEMV || KIND == TK_QKV_ATTN) {
       const int sg = seg_of(op, row);
-      op.y[sg][row - op.seg_row0[sg]] = v;
+      op.y[sg][seg_row(op, grp, sg, row)] = v;
     } else if (KIND == TK_GEMV_RESID) {
       const float nx = (xs_ok ? sm.u.g.xs[j] : __ldcg(op.x_out + row)) + v;
       op.x_out[row] = nx;
@@ -540,6 +553,22 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   if (KIND == TK_NORM_GEMV_ARGMAX && lane == 0) sm.bestk[cw] = best;
   if (consumer_sync_or(fail)) return false;
 
+  if (KIND == TK_QKV_ATTN) {
+    // The last projection task of this kv head's group runs its attention.
+    if (ctid == 0) {
+      __threadfence();
+      const uint32_t old = atomicAdd(op.grp_cnt + grp, 1u);
+      sm.last = ((old + 1u) % (uint32_t)(op.ntasks / op.groups)) == 0u;
+    }
+    consumer_sync();
+    if (sm.last) {
+      __threadfence();
+      if (!attn_dispatch(sm, g, op, grp, 0, 1, 0, true, cw, lane)) return false;
+      consumer_sync();
+      if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+    }
+  }
+
   if (KIND == TK_NORM_GEMV_ARGMAX) {
     // Per-task maximum -> one 64-bit atomicMax; the last task to arrive
     // finishes the iteration.
@@ -575,25 +604,25 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 }
 
 // ------------------------------------------------------------------ attention task
-// Task (kv head j, chunk c, request r).  Prologue: RMSNorm over the head dim and
-// rotate-half RoPE of the G query heads of the group and of k; the last chunk
-// appends bf16 k, v at position s.  Main loop: LP = D/8 lanes per position (8
-// dims per lane), 32/LP positions per warp step, online softmax in base 2 per
-// query head.  Partials (max, sum, unnormalised output) go to global memory;
-// the last chunk task of (r, j) to arrive merges them in chunk order and
-// writes o = bf16(output).
-// Not inlined: it has its own register allocation, so its per-head arrays
-// never push the GEMV loops into spills.
+// Attention of kv head j for request r at position s = step[r], over the
+// positions of chunk c of C (split-K) or over all of 0..s (direct).
+// Prologue: RMSNorm over the head dim and rotate-half RoPE of the G query
+// heads of the group and of k; the chunk holding s appends bf16 k, v at
+// position s.  Main loop: LP = D/8 lanes per position (8 dims per lane),
+// 32/LP positions per warp step, NSTEP steps' K/V loads issued before any is
+// used, online softmax in base 2 per query head.  Direct: o = bf16(output)
+// is written here.  Split-K: (max, sum, unnormalised output) partials go to
+// global memory and the last chunk task of (r, j) to arrive merges them in
+// chunk order and signals the operation's event.
 template <int G, int D>
-__device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int task, int cw, int lane) {
+__device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
+                          int cw, int lane) {
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
+  constexpr int NSTEP = 4;           // warp steps whose loads are in flight together
   constexpr float LOG2E = 1.4426950408889634f;
   const int ctid = cw * 32 + lane;
-  const int Hkv = op.Hkv, C = op.C;
-  const int j = task % Hkv;
-  const int c = (task / Hkv) % C;
-  const int r = task / (Hkv * C);
+  const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
   const size_t kvbase = ((((size_t)op.layer * g.R + r) * Hkv + j) * (size_t)op.S) * D;
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * C) * (D + 2);
@@ -652,7 +681,7 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
       }
     }
     consumer_sync();
-    if (c == C - 1 && ctid < D / 4) {
+    if (hi == npos && ctid < D / 4) {
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
@@ -673,45 +702,53 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
     }
     const uint16_t* kg = op.kc + kvbase + sub * 8;
     const uint16_t* vg = op.vc + kvbase + sub * 8;
-    for (int base = lo + cw * PPW; base < hi; base += CONSUMER_WARPS * PPW) {
-      const int t = base + grp;
-      const bool valid = t < hi;
-      uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-      if (valid) {
-        if (t == s) {
-          kv = *reinterpret_cast<const uint4*>(A.ks + sub * 8);
-          vv = *reinterpret_cast<const uint4*>(A.vs + sub * 8);
-        } else {
-          kv = ldcg_u4(kg + (size_t)t * D);
-          vv = ldcg_u4(vg + (size_t)t * D);
+    for (int base = lo + cw * PPW; base < hi; base += NSTEP * CONSUMER_WARPS * PPW) {
+      uint4 kv[NSTEP], vv[NSTEP];
+#pragma unroll
+      for (int u = 0; u < NSTEP; ++u) {
+        const int t = base + u * CONSUMER_WARPS * PPW + grp;
+        kv[u] = make_uint4(0, 0, 0, 0);
+        vv[u] = make_uint4(0, 0, 0, 0);
+        if (t < hi) {
+          if (t == s) {
+            kv[u] = *reinterpret_cast<const uint4*>(A.ks + sub * 8);
+            vv[u] = *reinterpret_cast<const uint4*>(A.vs + sub * 8);
+          } else {
+            kv[u] = ldcg_u4(kg + (size_t)t * D);
+            vv[u] = ldcg_u4(vg + (size_t)t * D);
+          }
         }
       }
-      const float kf[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
-                           bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
-      float sc[G];
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
-        const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
-        float a = q0.x * kf[0];
-        a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
-        a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
-#pragma unroll
-        for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        sc[hh] = a;
-      }
-      if (valid) {
-        const float vf[8] = {bf16_lo(vv.x), bf16_hi(vv.x), bf16_lo(vv.y), bf16_hi(vv.y),
-                             bf16_lo(vv.z), bf16_hi(vv.z), bf16_lo(vv.w), bf16_hi(vv.w)};
+      for (int u = 0; u < NSTEP; ++u) {
+        const bool valid = base + u * CONSUMER_WARPS * PPW + grp < hi;
+        const float kf[8] = {bf16_lo(kv[u].x), bf16_hi(kv[u].x), bf16_lo(kv[u].y), bf16_hi(kv[u].y),
+                             bf16_lo(kv[u].z), bf16_hi(kv[u].z), bf16_lo(kv[u].w), bf16_hi(kv[u].w)};
+        float sc[G];
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          const float mn = fmaxf(m[hh], sc[hh]);
-          const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
-          const float p = exp2f(sc[hh] - mn);
-          l[hh] = l[hh] * al + p;
+          const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
+          const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
+          float a = q0.x * kf[0];
+          a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+          a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
-          m[hh] = mn;
+          for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          sc[hh] = a;
+        }
+        if (valid) {
+          const float vf[8] = {bf16_lo(vv[u].x), bf16_hi(vv[u].x), bf16_lo(vv[u].y), bf16_hi(vv[u].y),
+                               bf16_lo(vv[u].z), bf16_hi(vv[u].z), bf16_lo(vv[u].w), bf16_hi(vv[u].w)};
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float mn = fmaxf(m[hh], sc[hh]);
+            const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
+            const float p = exp2f(sc[hh] - mn);
+            l[hh] = l[hh] * al + p;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
+            m[hh] = mn;
+          }
         }
       }
     }
@@ -746,7 +783,7 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
       }
     }
     consumer_sync();
-    // merge the warps in fixed order -> this chunk's partial
+    // merge the warps in fixed order -> the output (direct) or this chunk's partial
     for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
       const int hh = idx / D, i = idx % D;
       float M = -INFINITY;
@@ -759,14 +796,19 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
           Os = fmaf(A.wacc[w][hh * D + i], f, Os);
         }
       }
-      float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
-      p[2 + i] = Os;
-      if (i == 0) {
-        p[0] = M;
-        p[1] = Ls;
+      if (direct) {
+        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = f32_to_bf16_rn(Os / Ls);
+      } else {
+        float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
+        p[2 + i] = Os;
+        if (i == 0) {
+          p[0] = M;
+          p[1] = Ls;
+        }
       }
     }
   }
+  if (direct) return true;
   consumer_sync();
   if (ctid == 0) {
     __threadfence();
@@ -837,15 +879,18 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 }
 
 // ------------------------------------------------------------------ dispatch
-__device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int task, int cw, int lane) {
+// Not inlined: attention gets its own register allocation, so its per-head
+// arrays never push the GEMV loops into spills.
+__device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                           bool direct, int cw, int lane) {
   const int key = op.G * 1000 + op.d;
   switch (key) {
-    case 1000 + 64: return attn_task<1, 64>(sm, g, op, task, cw, lane);
-    case 2000 + 64: return attn_task<2, 64>(sm, g, op, task, cw, lane);
-    case 4000 + 64: return attn_task<4, 64>(sm, g, op, task, cw, lane);
-    case 1000 + 128: return attn_task<1, 128>(sm, g, op, task, cw, lane);
-    case 2000 + 128: return attn_task<2, 128>(sm, g, op, task, cw, lane);
-    case 4000 + 128: return attn_task<4, 128>(sm, g, op, task, cw, lane);
+    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
     default: return false;
   }
 }
@@ -902,7 +947,11 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
       case TK_NORM_GEMV_ARGMAX:
         ok = gemv_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
-      case TK_ATTN: ok = attn_dispatch(sm, g, op, task, cw, lane); break;
+      case TK_ATTN:
+        ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C), false, cw,
+                           lane);
+        break;
+      case TK_QKV_ATTN: ok = gemv_task<TK_QKV_ATTN>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       default: ok = false;
     }
     if (!ok) {

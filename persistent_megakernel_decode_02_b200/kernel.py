@@ -148,6 +148,14 @@ class PersistentKernel:
         self._add(_lib.OP_ATTENTION, (q, k, v), (q_norm, k_norm, k_cache, v_cache), (output,), grid_dim,
                   block_dim, layer=layer, eps=eps, rope_theta=rope_theta)
 
+    def rmsnorm_qkv_attention_layer(self, input: Name, weight_norm: Name, wq: Name, wk: Name, wv: Name,
+                                    q_norm: Name, k_norm: Name, k_cache: Name, v_cache: Name, q: Name, k: Name,
+                                    v: Name, output: Name, layer: int, grid_dim, block_dim=256, eps: float = 1e-6,
+                                    rope_theta: float = 1e6):
+        self._add(_lib.OP_RMSNORM_QKV_ATTENTION, (input,),
+                  (weight_norm, wq, wk, wv, q_norm, k_norm, k_cache, v_cache), (q, k, v, output), grid_dim,
+                  block_dim, layer=layer, eps=eps, rope_theta=rope_theta)
+
     def linear_residual_layer(self, input: Name, weight: Name, residual: Name, grid_dim, block_dim=256,
                               capture_slot: int = -1):
         self._add(_lib.OP_LINEAR_RESIDUAL, (input,), (weight,), (residual,), grid_dim, block_dim,
@@ -173,6 +181,9 @@ class PersistentKernel:
         self._keep.append(arr)
         self.compiled = True
         return self.warnings()
+
+    def num_ops(self) -> int:
+        return len(self._layers)
 
     def warnings(self) -> str:
         w = self._lib.mpk_warnings(self._ctx)

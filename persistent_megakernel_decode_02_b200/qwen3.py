@@ -17,24 +17,39 @@ import torch
 from .kernel import PersistentKernel
 
 
+FUSED_ATTENTION_MAX_SEQ = 4096
+
+
 def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
-               block_dim: int = 256, tied: Optional[bool] = None) -> List[dict]:
+               block_dim: int = 256, tied: Optional[bool] = None, fused_attention: bool = False) -> List[dict]:
     """The fused-layer list (pure host logic, no GPU): one dict per operation with
-    the method name and its keyword arguments."""
+    the method name and its keyword arguments.  With ``fused_attention`` the q/k/v
+    projections and the attention are one operation (tasks grouped per kv head,
+    the last task of a group runs its attention); otherwise attention is its own
+    split-K operation with ``attn_chunks`` chunks."""
     s = shape
     gt = gemv_tasks or num_workers
     tied = s.tied if tied is None else tied
     plan: List[dict] = [dict(method="embed_layer", embedding="embed_tokens", output="x", grid_dim=requests,
                              block_dim=block_dim, capture_slot=0)]
+    rows_per_group = (s.q_heads // s.kv_heads + 2) * s.head_dim
     for l in range(s.layers):
         p = f"layers.{l}."
-        plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
-                         weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
-                         grid_dim=min(gt, s.q_dim + 2 * s.kv_dim), block_dim=block_dim, eps=s.eps))
-        plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm", k_norm=p + "k_norm",
-                         k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
-                         grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
-                         rope_theta=s.rope_theta))
+        if fused_attention:
+            tpg = max(1, min(rows_per_group, gt // (s.kv_heads * requests)))
+            plan.append(dict(method="rmsnorm_qkv_attention_layer", input="x", weight_norm=p + "input_layernorm",
+                             wq=p + "q_proj", wk=p + "k_proj", wv=p + "v_proj", q_norm=p + "q_norm",
+                             k_norm=p + "k_norm", k_cache="k_cache", v_cache="v_cache", q="q", k="k", v="v",
+                             output="o", layer=l, grid_dim=(tpg, s.kv_heads, requests), block_dim=block_dim,
+                             eps=s.eps, rope_theta=s.rope_theta))
+        else:
+            plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
+                             weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
+                             grid_dim=min(gt, s.q_dim + 2 * s.kv_dim), block_dim=block_dim, eps=s.eps))
+            plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm",
+                             k_norm=p + "k_norm", k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
+                             grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
+                             rope_theta=s.rope_theta))
         plan.append(dict(method="linear_residual_layer", input="o", weight=p + "o_proj", residual="x",
                          grid_dim=min(gt, s.hidden), block_dim=block_dim))
         plan.append(dict(method="rmsnorm_linear_silu_mul_layer", input="x",
@@ -81,10 +96,12 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 256,
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
-                  prefetch_kb: int = 0) -> Decoder:
+                  prefetch_kb: int = 0, fused_attention: Optional[bool] = None) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
-    tokens' row length (seq_length)."""
+    tokens' row length (seq_length).  fused_attention: None picks the fused
+    projection+attention operation for one request with up to
+    FUSED_ATTENTION_MAX_SEQ positions, split-K attention otherwise."""
     from . import _lib
 
     s = shape
@@ -113,7 +130,10 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     }
     if attn_chunks is None:
         attn_chunks = default_attn_chunks(s, requests, num_workers, max_seq)
-    for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim):
+    if fused_attention is None:
+        fused_attention = requests == 1 and max_seq <= FUSED_ATTENTION_MAX_SEQ
+    for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim,
+                         fused_attention=fused_attention):
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
     mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb)

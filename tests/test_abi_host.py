@@ -66,6 +66,17 @@ def test_layer_plan_structure():
         list(range(1, s.layers + 1))
 
 
+def test_layer_plan_fused_attention():
+    s = sq.QWEN3_8B
+    plan = layer_plan(s, requests=1, num_workers=144, attn_chunks=9, fused_attention=True)
+    assert len(plan) == 2 + 4 * s.layers
+    op = plan[1]
+    assert op["method"] == "rmsnorm_qkv_attention_layer"
+    assert op["grid_dim"] == (18, 8, 1)      # 18 tasks per kv head, 8 kv heads
+    assert [p["method"] for p in plan[1:5]] == ["rmsnorm_qkv_attention_layer", "linear_residual_layer",
+                                                "rmsnorm_linear_silu_mul_layer", "linear_residual_layer"]
+
+
 def test_default_attention_chunks():
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 551) == 9
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 32897) == 18

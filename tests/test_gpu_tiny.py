@@ -39,12 +39,13 @@ def _greedy(dec, tokens_cpu, step0=0):
     return tok.cpu(), step.cpu()
 
 
-def test_greedy_tokens_bit_identical_to_oracle(weights):
-    """The tiny config's greedy tokens must match the oracle exactly (north-star
-    contract); the oracle's top-2 margins show how far each choice is from a tie."""
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-attention", "split-attention"])
+def test_greedy_tokens_bit_identical_to_oracle(weights, fused):
+    """The tiny config's greedy tokens must match the oracle exactly; the oracle's
+    top-2 margins show how far each choice is from a tie."""
     w_cpu, w = weights
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=0)
-    dec = _build(w)
+    dec = _build(w, fused_attention=fused)
     got, step = _greedy(dec, tokens)
     ref = oracle.Decoder(SHAPE, w_cpu)
     toks = tokens.numpy().copy()
@@ -73,10 +74,11 @@ def test_greedy_tokens_bit_identical_to_oracle(weights):
     dec.kernel.close()
 
 
-def test_teacher_forced_logits_and_hidden_states(weights):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-attention", "split-attention"])
+def test_teacher_forced_logits_and_hidden_states(weights, fused):
     w_cpu, w = weights
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=1, teacher_forced=True)
-    dec = _build(w)
+    dec = _build(w, fused_attention=fused)
     gpu, gtok, _ = gpu_teacher_forced(dec, tokens, S - 1)
     ref, rtok, _, _ = oracle_teacher_forced(SHAPE, w_cpu, tokens, S - 1)
     wl, wh = compare_captures(gpu, ref)
@@ -86,12 +88,13 @@ def test_teacher_forced_logits_and_hidden_states(weights):
     dec.kernel.close()
 
 
-def test_op_by_op_is_bit_identical_to_persistent(weights):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-attention", "split-attention"])
+def test_op_by_op_is_bit_identical_to_persistent(weights, fused):
     _, w = weights
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=2)
     outs = []
     for mode in ("persistent", "op_by_op"):
-        dec = _build(w)
+        dec = _build(w, fused_attention=fused)
         lg = torch.zeros((1, SHAPE.vocab), device="cuda")
         hd = torch.zeros((SHAPE.layers + 1, 1, SHAPE.hidden), device="cuda")
         dec.kernel.set_capture(S - 3, lg, hd)
@@ -116,7 +119,8 @@ def test_worker_scheduler_split_invariance(weights, split):
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=3)
     res = []
     for W, Ls in ((sms - 4, 16), (sms - split[1] // 4, split[1])):
-        dec = _build(w, num_workers=W, num_local_schedulers=Ls, gemv_tasks=144, attn_chunks=5)
+        dec = _build(w, num_workers=W, num_local_schedulers=Ls, gemv_tasks=144, attn_chunks=5,
+                     fused_attention=split[0] % 2 == 0)
         lg = torch.zeros((1, SHAPE.vocab), device="cuda")
         dec.kernel.set_capture(S - 2, lg, None)
         got, _ = _greedy(dec, tokens)
@@ -153,7 +157,7 @@ def test_attention_chunking_ragged(weights, chunks):
     sizes and a single chunk all agree with the oracle."""
     w_cpu, w = weights
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=5, teacher_forced=True)
-    dec = _build(w, attn_chunks=chunks)
+    dec = _build(w, attn_chunks=chunks, fused_attention=False)
     gpu, _, _ = gpu_teacher_forced(dec, tokens, 12)
     ref, _, _, _ = oracle_teacher_forced(SHAPE, w_cpu, tokens, 12)
     compare_captures(gpu, ref)
@@ -161,12 +165,13 @@ def test_attention_chunking_ragged(weights, chunks):
 
 
 @pytest.mark.parametrize("tasks", [1, 7, 100, 288])
-def test_ragged_task_splits(weights, tasks):
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-attention", "split-attention"])
+def test_ragged_task_splits(weights, tasks, fused):
     """Row splits that are not multiples of the worker count (warning only), one
-    task for a whole matrix, and more tasks than workers."""
+    task for a whole matrix (or kv-head group), and more tasks than workers."""
     w_cpu, w = weights
     tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=6, teacher_forced=True)
-    dec = _build(w, gemv_tasks=tasks)
+    dec = _build(w, gemv_tasks=tasks, fused_attention=fused)
     gpu, _, _ = gpu_teacher_forced(dec, tokens, 6)
     ref, _, _, _ = oracle_teacher_forced(SHAPE, w_cpu, tokens, 6)
     compare_captures(gpu, ref)
