@@ -11,7 +11,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/mpk.h"
+#include "mpk.h"
 #include "mpk_internal.h"
 
 namespace mpk {

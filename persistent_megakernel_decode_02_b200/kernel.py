@@ -50,6 +50,9 @@ def _dim3(v) -> _lib.Dim3:
 
 
 class PersistentKernel:
+    """block_dim 0 (the default of every layer method) means all worker threads
+    (mpk_worker_threads())."""
+
     def __init__(self, num_workers: int, num_local_schedulers: int, num_remote_schedulers: int = 0,
                  world_size: int = 1, mpi_rank: int = 0):
         self._lib = _lib.load()
@@ -112,7 +115,7 @@ class PersistentKernel:
 
     # ------------------------------------------------------------------ layers
     def _add(self, op: int, inputs: Iterable[Optional[Name]] = (), weights: Iterable[Optional[Name]] = (),
-             outputs: Iterable[Optional[Name]] = (), grid_dim=1, block_dim=256, layer: int = 0,
+             outputs: Iterable[Optional[Name]] = (), grid_dim=1, block_dim=0, layer: int = 0,
              capture_slot: int = -1, eps: float = 1e-6, rope_theta: float = 1e6) -> None:
         L = _lib.Layer()
         L.op = op
@@ -133,41 +136,41 @@ class PersistentKernel:
         L.rope_theta = rope_theta
         self._layers.append(L)
 
-    def embed_layer(self, embedding: Name, output: Name, grid_dim, block_dim=256, capture_slot: int = -1):
+    def embed_layer(self, embedding: Name, output: Name, grid_dim, block_dim=0, capture_slot: int = -1):
         self._add(_lib.OP_EMBED, (), (embedding,), (output,), grid_dim, block_dim, capture_slot=capture_slot)
 
     def rmsnorm_linear_layer(self, input: Name, weight_norm: Name, weight_linear, output, grid_dim,
-                             block_dim=256, eps: float = 1e-6):
+                             block_dim=0, eps: float = 1e-6):
         wl = weight_linear if isinstance(weight_linear, (list, tuple)) else [weight_linear]
         out = output if isinstance(output, (list, tuple)) else [output]
         self._add(_lib.OP_RMSNORM_LINEAR, (input,), [weight_norm, *wl], out, grid_dim, block_dim, eps=eps)
 
     def attention_layer(self, q: Name, k: Name, v: Name, q_norm: Name, k_norm: Name, k_cache: Name,
-                        v_cache: Name, output: Name, layer: int, grid_dim, block_dim=256, eps: float = 1e-6,
+                        v_cache: Name, output: Name, layer: int, grid_dim, block_dim=0, eps: float = 1e-6,
                         rope_theta: float = 1e6):
         self._add(_lib.OP_ATTENTION, (q, k, v), (q_norm, k_norm, k_cache, v_cache), (output,), grid_dim,
                   block_dim, layer=layer, eps=eps, rope_theta=rope_theta)
 
     def rmsnorm_qkv_attention_layer(self, input: Name, weight_norm: Name, wq: Name, wk: Name, wv: Name,
                                     q_norm: Name, k_norm: Name, k_cache: Name, v_cache: Name, q: Name, k: Name,
-                                    v: Name, output: Name, layer: int, grid_dim, block_dim=256, eps: float = 1e-6,
+                                    v: Name, output: Name, layer: int, grid_dim, block_dim=0, eps: float = 1e-6,
                                     rope_theta: float = 1e6):
         self._add(_lib.OP_RMSNORM_QKV_ATTENTION, (input,),
                   (weight_norm, wq, wk, wv, q_norm, k_norm, k_cache, v_cache), (q, k, v, output), grid_dim,
                   block_dim, layer=layer, eps=eps, rope_theta=rope_theta)
 
-    def linear_residual_layer(self, input: Name, weight: Name, residual: Name, grid_dim, block_dim=256,
+    def linear_residual_layer(self, input: Name, weight: Name, residual: Name, grid_dim, block_dim=0,
                               capture_slot: int = -1):
         self._add(_lib.OP_LINEAR_RESIDUAL, (input,), (weight,), (residual,), grid_dim, block_dim,
                   capture_slot=capture_slot)
 
     def rmsnorm_linear_silu_mul_layer(self, input: Name, weight_norm: Name, weight_gate: Name, weight_up: Name,
-                                      output: Name, grid_dim, block_dim=256, eps: float = 1e-6):
+                                      output: Name, grid_dim, block_dim=0, eps: float = 1e-6):
         self._add(_lib.OP_RMSNORM_LINEAR_SILU_MUL, (input,), (weight_norm, weight_gate, weight_up), (output,),
                   grid_dim, block_dim, eps=eps)
 
     def rmsnorm_lmhead_argmax_layer(self, input: Name, weight_norm: Name, weight_lm: Name,
-                                    pred: Optional[Name] = None, grid_dim=1, block_dim=256, eps: float = 1e-6):
+                                    pred: Optional[Name] = None, grid_dim=1, block_dim=0, eps: float = 1e-6):
         self._add(_lib.OP_RMSNORM_LMHEAD_ARGMAX, (input,), (weight_norm, weight_lm), (pred,), grid_dim, block_dim,
                   eps=eps)
 

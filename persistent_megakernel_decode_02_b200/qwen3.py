@@ -21,7 +21,7 @@ FUSED_ATTENTION_MAX_SEQ = 4096
 
 
 def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
-               block_dim: int = 256, tied: Optional[bool] = None, fused_attention: bool = False) -> List[dict]:
+               block_dim: int = 0, tied: Optional[bool] = None, fused_attention: bool = False) -> List[dict]:
     """The fused-layer list (pure host logic, no GPU): one dict per operation with
     the method name and its keyword arguments.  With ``fused_attention`` the q/k/v
     projections and the attention are one operation (tasks grouped per kv head,
@@ -93,7 +93,7 @@ class Decoder:
 
 def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_seq: int,
                   num_workers: Optional[int] = None, num_local_schedulers: int = 16,
-                  attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 256,
+                  attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 0,
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None) -> Decoder:
