@@ -256,6 +256,44 @@ MPK_API int mpk_request_abort(mpk_ctx *ctx);
  * none), first weight stage issued by the producer (0 if none). */
 MPK_API int mpk_timeline(mpk_ctx *ctx, uint64_t *out, int cap);
 
+/*
+ * Final RMSNorm + LM head + greedy argmax that allocates nothing.  The MPK
+ * pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory (for example a serving framework whose memory pool
+ * owns all device memory and forbids cudaMalloc / cudaFree, which would also
+ * synchronise the device, on its decode path).
+ *
+ * For each request r < num_requests: h = bf16(x[r] / sqrt(mean(x[r]^2) + eps)
+ * * norm_w), z = w_lm h in fp32, tokens_out[r] = argmax z (lowest index on
+ * ties), and logits_out[r, :] = z when logits_out is not NULL.
+ *   x          device fp32 [num_requests, K]
+ *   norm_w     device bf16 [K]
+ *   w_lm       device bf16 [V, K] (16-byte aligned)
+ *   tokens_out device int64 [num_requests]
+ *   logits_out device fp32 [num_requests, V] or NULL
+ *   stream     cudaStream_t (NULL: legacy default stream); asynchronous.
+ * Limits: 1 <= num_requests <= MPK_NOALLOC_MAX_REQUESTS, K a multiple of 8 up
+ * to MPK_NOALLOC_MAX_K; larger sizes return MPK_ERR_INVALID_ARG / MPK_ERR_SHAPE
+ * (message in mpk_noalloc_last_error()).
+ * Scratch: a fixed __device__ array of 2 * MPK_NOALLOC_MAX_REQUESTS 64-bit
+ * words (1 KiB) inside this library; every GPU that loads the library holds it
+ * until the process exits.  Each call clears it on `stream` before use.  All
+ * calls share it, so calls that overlap on the GPU (on different streams, or
+ * from different threads) race and must be serialised by the caller.  The
+ * first call on a device looks up the array's device address (set-up done once
+ * per device, with that device current); make that first call before any
+ * stream capture.  No cudaMalloc, cudaFree or allocating library routine is
+ * called.
+ */
+#define MPK_NOALLOC_MAX_REQUESTS 64
+#define MPK_NOALLOC_MAX_K 16384
+MPK_API int mpk_lmhead_argmax_noalloc(const float *x, const uint16_t *norm_w, const uint16_t *w_lm,
+                                      int num_requests, int K, int V, float eps, int64_t *tokens_out,
+                                      float *logits_out, void *stream);
+
+/* Message of the last failed mpk_lmhead_argmax_noalloc call ("" if none). */
+MPK_API const char *mpk_noalloc_last_error(void);
+
 /* Free the context and every library-owned allocation. */
 MPK_API int mpk_destroy(mpk_ctx *ctx);
 

@@ -83,6 +83,8 @@ SIGNATURES = {
     "mpk_timeline": (_I, [_VP, _VP, _I]),
     "mpk_destroy": (_I, [_VP]),
     "mpk_last_error": (_CP, [_VP]),
+    "mpk_lmhead_argmax_noalloc": (_I, [_VP, _VP, _VP, _I, _I, _I, ctypes.c_float, _VP, _VP, _VP]),
+    "mpk_noalloc_last_error": (_CP, []),
 }
 
 _lib = None
