@@ -122,6 +122,33 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def kernel_source_digest() -> str:
+    import hashlib
+    csrc = os.path.join(ROOT, "persistent_megakernel_decode_02_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("mpk_kernel.cu", "mpk_internal.h", "mpk_ptx.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_ratio():
+    """DRAM bytes per algorithmic byte from the committed ncu summary, when it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "mpk_persistent_kernel_dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    kv = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != kernel_source_digest():
+        return None
+    return float(kv["dram_bytes_per_algorithmic_byte"])
+
+
 def algorithmic_bytes(shape, first_pos: int, iters: int) -> int:
     """Bytes one decode iteration must move, summed over iterations at positions
     first_pos .. first_pos+iters-1: every streamed weight byte once, the K/V of
@@ -405,7 +432,9 @@ def main():
             "tokens_per_s": 1e3 * args.steps * world / ms_max,
             "hbm_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "peak_kind": peak_kind,
+                         "traffic": (None if traffic_ratio() is None else traffic_ratio() * bytes_launch),
+                         "traffic_source": "ncu dram bytes of a 4-layer case scaled by algorithmic bytes",
+                         "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_launch,
                          "kernel": "mpk_persistent_kernel"},
             "cpu_baseline": cpu,
