@@ -184,6 +184,14 @@ def max_over_ranks(pg, value: float, device=None) -> float:
     return float(t.item())
 
 
+def whole_job(ms_max: float, steps: int, world: int):
+    """Replicas: each of `world` ranks decodes `steps` tokens of its own request;
+    the job took the slowest rank's `ms_max`.  Returns (ms per generated token
+    of the whole job, whole-job tokens/s)."""
+    tokens = steps * world
+    return ms_max / tokens, 1e3 * tokens / ms_max
+
+
 def barrier(pg, device=None):
     if pg is None:
         return
@@ -218,7 +226,7 @@ def time_oracle(shape, w_cpu, tokens_cpu, budget_s: float, max_iters: int = 64, 
     t_start = time.perf_counter()
     while len(times) < max_iters:
         t0 = time.perf_counter()
-        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_BF16, None, None)
+        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_NONE, None, None)
         times.append(time.perf_counter() - t0)
         if time.perf_counter() - t_start > budget_s:
             break
@@ -265,10 +273,10 @@ def run_reference(args):
     kc, vc = dec.new_cache(1, S)
     step = np.zeros(1, np.int32)
     for _ in range(args.warmup):
-        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_BF16, None, None)
+        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_NONE, None, None)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_BF16, None, None)
+        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_NONE, None, None)
     el = time.perf_counter() - t0
     ms = 1e3 * el / max(args.steps, 1) / frac
     sample = (f"each step: one oracle decode iteration over the first {layers} of {shape.layers} layers + LM head, "
@@ -363,7 +371,7 @@ def main():
     gen = tok[0, PROMPT:PROMPT + args.steps].cpu()
     assert bool((gen >= 0).all()), "some timed tokens were not generated"
     ms_max = max_over_ranks(pg, ms_launch, dev)
-    value = ms_max / (args.steps * world)          # whole-job ms per generated token
+    value, tokens_per_s = whole_job(ms_max, args.steps, world)
     ms_per_step = ms_max / args.steps
     bytes_launch = algorithmic_bytes(shape, PROMPT - 1, args.steps)
     gbs = bytes_launch / (ms_launch * 1e-3) / 1e9
@@ -413,7 +421,7 @@ def main():
         assert torch.equal(out_tok[0, PROMPT:PROMPT + args.steps], gen), "e2e tokens differ from the timed run"
         h2d = host_tok.numel() * 8 + 4 + 4
         d2h = out_tok.numel() * 8
-        e2e = {"value": e2e_ms / (args.steps * world), "unit": UNIT,
+        e2e = {"value": whole_job(e2e_ms, args.steps, world)[0], "unit": UNIT,
                "h2d_bytes_per_step": h2d / args.steps, "d2h_bytes_per_step": d2h / args.steps,
                "includes": f"H2D of tokens/step/step_end, {PROMPT - 1} prompt iterations + {args.steps} decode "
                            f"iterations in one launch, D2H of tokens"}
@@ -429,7 +437,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": value / A100_MPK_MS, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(shape, args, dec),
-            "tokens_per_s": 1e3 * args.steps * world / ms_max,
+            "tokens_per_s": tokens_per_s,
             "hbm_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                          "traffic": (None if traffic_ratio() is None else traffic_ratio() * bytes_launch),

@@ -68,13 +68,16 @@ typedef enum { MPK_BF16 = 0, MPK_FP32 = 1, MPK_INT32 = 2, MPK_INT64 = 3 } mpk_dt
 typedef enum { MPK_IO_CUDA = 0, MPK_IO_NVSHMEM = 1 } mpk_io;
 
 /* Fused operations of the task graph ([EN] "The API": operations are chained
- * to build the graph; rmsnorm_linear_layer is the one the pages name). */
+ * to build the graph; rmsnorm_linear_layer is the one the pages name).
+ * Number format: weights and the KV cache are bf16; every activation (the
+ * residual stream x, normed inputs h, q/k/v, the attention output o, the MLP
+ * product a, logits) is fp32; dot products accumulate in fp32. */
 typedef enum {
     /* x[r,:] = fp32(E[tokens[r, step[r]], :]).
      * weights[0] = E bf16 [V,H]; outputs[0] = x fp32 [R,H].  grid_dim = R tasks. */
     MPK_OP_EMBED = 1,
     /* RMSNorm feeding one or more linear layers stacked by rows:
-     * h = bf16(x / sqrt(mean(x^2) + eps) * w_norm); y_i = W_i h.
+     * h = x / sqrt(mean(x^2) + eps) * w_norm; y_i = W_i h.
      * inputs[0] = x fp32 [R,K]; weights[0] = w_norm bf16 [K];
      * weights[1..3] = W_i bf16 [N_i,K]; outputs[0..2] = y_i fp32 [R,N_i]
      * (output i belongs to weight i+1).  grid_dim = row-block tasks. */
@@ -83,20 +86,20 @@ typedef enum {
      * head dim and rotate-half RoPE of q (its query-head group) and k, append
      * bf16 k and v at position s of the cache, causal grouped-query attention
      * over positions 0..s (split into grid_dim.y chunks, merged by
-     * log-sum-exp), o = bf16(attention output).
+     * log-sum-exp), o = attention output.
      * inputs = q fp32 [R,Hq*d], k fp32 [R,Hkv*d], v fp32 [R,Hkv*d];
      * weights = q_norm bf16 [d], k_norm bf16 [d], k_cache, v_cache bf16
-     * [L,R,Hkv,S,d]; outputs[0] = o bf16 [R,Hq*d].  layer selects the cache
+     * [L,R,Hkv,S,d]; outputs[0] = o fp32 [R,Hq*d].  layer selects the cache
      * slice; rope_theta the RoPE base.  grid_dim = (Hkv, chunks, R). */
     MPK_OP_ATTENTION = 3,
-    /* x += W a.  inputs[0] = a bf16 [R,K]; weights[0] = W bf16 [N,K];
+    /* x += W a.  inputs[0] = a fp32 [R,K]; weights[0] = W bf16 [N,K];
      * outputs[0] = x fp32 [R,N] (read and written in place). */
     MPK_OP_LINEAR_RESIDUAL = 4,
-    /* h = bf16(rmsnorm(x) * w_norm); a = bf16(silu(W_gate h) * (W_up h)).
+    /* h = rmsnorm(x) * w_norm; a = silu(W_gate h) * (W_up h).
      * inputs[0] = x fp32 [R,K]; weights = w_norm [K], W_gate [I,K], W_up [I,K];
-     * outputs[0] = a bf16 [R,I]. */
+     * outputs[0] = a fp32 [R,I]. */
     MPK_OP_RMSNORM_LINEAR_SILU_MUL = 5,
-    /* z = W_lm bf16(rmsnorm(x) * w_norm) in fp32; greedy argmax (lowest index on
+    /* z = W_lm (rmsnorm(x) * w_norm) in fp32; greedy argmax (lowest index on
      * ties); then, per active request: tokens[r, s+1] = argmax if that slot
      * holds -1, pred[r, s+1] = argmax, step[r] = s + 1 ([EN] "How MPK Works":
      * the runtime advances `step` after every iteration).  inputs[0] = x;
@@ -110,7 +113,7 @@ typedef enum {
      * pass over positions 0..s, no split-K).  inputs[0] = x fp32 [R,K];
      * weights = w_norm [K], Wq [Hq*d,K], Wk [Hkv*d,K], Wv [Hkv*d,K], q_norm [d],
      * k_norm [d], k_cache, v_cache [L,R,Hkv,S,d]; outputs = q [R,Hq*d],
-     * k, v [R,Hkv*d] (fp32 scratch), o bf16 [R,Hq*d].
+     * k, v [R,Hkv*d] (fp32 scratch), o fp32 [R,Hq*d].
      * grid_dim = (tasks per kv head, Hkv, R).  Meant for short contexts; long
      * ones use RMSNORM_LINEAR followed by ATTENTION with split-K. */
     MPK_OP_RMSNORM_QKV_ATTENTION = 7
@@ -145,6 +148,10 @@ typedef struct {
     int32_t max_timeline;   /* timeline entries kept when profiling (<=0: 1<<20)         */
     int32_t prefetch_kb;    /* L2 prefetch distance per worker ahead of the shared-memory
                                weight ring, KiB (<=0: off)                                 */
+    int32_t debug_stall_op; /* fault injection for tests: k > 0 makes operation k-1 wait
+                               for one more completion per iteration than its dependency
+                               delivers, so that wait runs out and the run ends with
+                               MPK_ERR_TIMEOUT (0: off)                                    */
 } mpk_options;
 
 /* Library build facts. */
@@ -245,8 +252,11 @@ MPK_API int mpk_set_capture(mpk_ctx *ctx, int iter, float *logits, float *hidden
  * MPK_ERR_DEVICE; details in mpk_last_error. */
 MPK_API int mpk_status(mpk_ctx *ctx);
 
-/* Ask a running kernel to stop at its next wait (host-mapped flag; safe while
- * the kernel runs).  The run then reports MPK_ERR_ABORTED. */
+/* Ask a running kernel to stop (host-mapped flag, safe while the kernel runs).
+ * The scheduler warps read it at every iteration boundary and long waits read
+ * it now and then; the run then reports MPK_ERR_ABORTED.  `step`, `tokens` and
+ * the KV cache stay consistent: a later mpk_run resumes from `step` and
+ * produces what an uninterrupted run would have. */
 MPK_API int mpk_request_abort(mpk_ctx *ctx);
 
 /* Number of timeline records of the last profiled run, and a copy of up to
@@ -263,8 +273,8 @@ MPK_API int mpk_timeline(mpk_ctx *ctx, uint64_t *out, int cap);
  * owns all device memory and forbids cudaMalloc / cudaFree, which would also
  * synchronise the device, on its decode path).
  *
- * For each request r < num_requests: h = bf16(x[r] / sqrt(mean(x[r]^2) + eps)
- * * norm_w), z = w_lm h in fp32, tokens_out[r] = argmax z (lowest index on
+ * For each request r < num_requests: h = x[r] / sqrt(mean(x[r]^2) + eps)
+ * * norm_w (fp32), z = w_lm h in fp32, tokens_out[r] = argmax z (lowest index on
  * ties), and logits_out[r, :] = z when logits_out is not NULL.
  *   x          device fp32 [num_requests, K]
  *   norm_w     device bf16 [K]

@@ -192,7 +192,7 @@ class Decoder:
         return np.zeros(shp, dtype=np.uint16), np.zeros(shp, dtype=np.uint16)
 
     def iteration(self, kc: np.ndarray, vc: np.ndarray, step: np.ndarray, tokens: np.ndarray,
-                  step_end: Optional[np.ndarray] = None, round_mode: int = ROUND_BF16,
+                  step_end: Optional[np.ndarray] = None, round_mode: int = ROUND_NONE,
                   logits: Optional[np.ndarray] = None, hidden: Optional[np.ndarray] = None,
                   pred: Optional[np.ndarray] = None) -> int:
         """One decoding iteration in place (see ``orc_decode_iteration``)."""
@@ -214,7 +214,7 @@ class Decoder:
             None if pred is None else pred.ctypes.data)
 
     def generate(self, tokens: np.ndarray, step: np.ndarray, step_end: np.ndarray,
-                 kc=None, vc=None, round_mode: int = ROUND_BF16, capture: bool = False):
+                 kc=None, vc=None, round_mode: int = ROUND_NONE, capture: bool = False):
         """Iterate until no request is active.  Returns (tokens, step, kc, vc, captures)
         where captures is a list of (logits, hidden) per iteration when ``capture``."""
         tokens = np.array(tokens, dtype=np.int64, copy=True)

@@ -22,13 +22,13 @@
  * grouped-query attention with softmax, output projection with residual,
  * RMSNorm, SwiGLU MLP with residual, final RMSNorm, LM head, argmax.
  *
- * Arithmetic: double throughout.  Weights and the KV cache are bf16.  With
- * round_mode = ORC_ROUND_BF16 the inputs of every projection (the normed hidden
- * state, the attention output, the SiLU*up product and the final normed state)
- * are rounded to bf16, the rounding points of the GPU path's number format;
- * ORC_ROUND_NONE keeps them in double.  The greedy choice is taken on the
- * logits rounded to fp32 (the precision the GPU path decides in), lowest index
- * on ties.
+ * Arithmetic: double throughout.  Weights and the KV cache are bf16 (the
+ * stored state).  ORC_ROUND_NONE, the plain reading, keeps every activation in
+ * double.  ORC_ROUND_BF16 models a deployment that also stores activations in
+ * bf16: the inputs of every projection (the normed hidden state, the attention
+ * output, the SiLU*up product and the final normed state) are rounded to bf16.
+ * The greedy choice is taken on the logits rounded to fp32, lowest index on
+ * ties.
  */
 #include <math.h>
 #include <stdint.h>

@@ -387,8 +387,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         const bool lmh = Ly.op == MPK_OP_RMSNORM_LMHEAD_ARGMAX;
         op.kind = resid ? TK_GEMV_RESID : silu ? TK_NORM_GEMV_SILU : lmh ? TK_NORM_GEMV_ARGMAX : TK_NORM_GEMV;
         if (resid) {
-          NEED("inputs[0] (a)", Ly.inputs[0], MPK_BF16, 2, &x);
-          op.a_in = (const uint16_t*)x->ptr;
+          NEED("inputs[0] (a)", Ly.inputs[0], MPK_FP32, 2, &x);
+          op.a_in = (const float*)x->ptr;
           op.K = (int)x->dims[1];
           NEED("weights[0] (W)", Ly.weights[0], MPK_BF16, 2, &w0);
           NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32, 2, &out);
@@ -415,7 +415,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
           if (silu) {
             NEED("weights[1] (gate)", Ly.weights[1], MPK_BF16, 2, &w1);
             NEED("weights[2] (up)", Ly.weights[2], MPK_BF16, 2, &w2);
-            NEED("outputs[0] (a)", Ly.outputs[0], MPK_BF16, 2, &out);
+            NEED("outputs[0] (a)", Ly.outputs[0], MPK_FP32, 2, &out);
             SHAPE_CHECK(w1->dims == w2->dims && w1->dims[1] == op.K, "layer %d: gate %s / up %s vs K=%d", li,
                         dims_str(w1->dims).c_str(), dims_str(w2->dims).c_str(), op.K);
             SHAPE_CHECK(out->dims[1] == w1->dims[0] && out->dims[0] == x->dims[0], "layer %d: output %s", li,
@@ -426,7 +426,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
             op.nseg = 1;
             op.seg_row0[0] = 0;
             op.seg_row0[1] = op.N;
-            op.a_out = (uint16_t*)out->ptr;
+            op.a_out = (float*)out->ptr;
           } else if (lmh) {
             NEED("weights[1] (lm head)", Ly.weights[1], MPK_BF16, 2, &w1);
             SHAPE_CHECK(w1->dims[1] == op.K, "layer %d: LM head %s vs K=%d", li, dims_str(w1->dims).c_str(), op.K);
@@ -494,7 +494,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         NEED("weights[1] (k_norm)", Ly.weights[1], MPK_BF16, 1, &kn);
         NEED("weights[2] (k_cache)", Ly.weights[2], MPK_BF16, 5, &kc);
         NEED("weights[3] (v_cache)", Ly.weights[3], MPK_BF16, 5, &vc);
-        NEED("outputs[0] (o)", Ly.outputs[0], MPK_BF16, 2, &o);
+        NEED("outputs[0] (o)", Ly.outputs[0], MPK_FP32, 2, &o);
         SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
         const int d = (int)kc->dims[4], Hkv = (int)kc->dims[2];
         SHAPE_CHECK(qn->dims[0] == d && kn->dims[0] == d, "layer %d: norm weights must have head_dim %d", li, d);
@@ -524,7 +524,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.q = (const float*)q->ptr; op.k = (const float*)k->ptr; op.v = (const float*)v->ptr;
         op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
         op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
-        op.a_out = (uint16_t*)o->ptr;
+        op.a_out = (float*)o->ptr;
         op.N = Hq * d;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
         part_floats = std::max(part_floats, (size_t)R * Hq * gy * (d + 2));
@@ -558,7 +558,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         NEED("outputs[0] (q)", Ly.outputs[0], MPK_FP32, 2, &q);
         NEED("outputs[1] (k)", Ly.outputs[1], MPK_FP32, 2, &k);
         NEED("outputs[2] (v)", Ly.outputs[2], MPK_FP32, 2, &v);
-        NEED("outputs[3] (o)", Ly.outputs[3], MPK_BF16, 2, &o);
+        NEED("outputs[3] (o)", Ly.outputs[3], MPK_FP32, 2, &o);
         op.K = (int)x->dims[1];
         SHAPE_CHECK(wn->dims[0] == op.K, "layer %d: norm weight %s, input width %d", li, dims_str(wn->dims).c_str(), op.K);
         SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
@@ -618,7 +618,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.q = op.y[0]; op.k = op.y[1]; op.v = op.y[2];
         op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
         op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
-        op.a_out = (uint16_t*)o->ptr;
+        op.a_out = (float*)o->ptr;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
         merge_off[li] = {1, merge_u32};
         merge_u32 += (size_t)R * Hkv;
@@ -656,6 +656,14 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     ops[p].dep_event = dp;
     ops[p].dep_trigger = ops[dp].out_trigger;
     ops[p].dep_iter_offset = p == 0 ? 0 : 1;
+  }
+  if (o.debug_stall_op > 0) {
+    const int p = o.debug_stall_op - 1;
+    if (p >= P)
+      return fail(c, MPK_ERR_INVALID_ARG, "debug_stall_op %d beyond the %d operations", o.debug_stall_op, P);
+    // one more completion per iteration than the dependency ever delivers
+    ops[p].dep_trigger += 1;
+    ops[p].dep_iter_offset = 1;
   }
 
   // ---- workspace
@@ -835,8 +843,8 @@ int mpk_status(mpk_ctx* c) {
   if (st.code == 0) return MPK_OK;
   static const char* where[] = {"?", "worker dependency wait", "producer queue wait", "weight ring wait",
                                 "task fifo wait", "scheduler gate wait", "scheduler queue space wait", "start",
-                                "embedding token check", "task dispatch"};
-  const char* w = (st.where >= 0 && st.where < 10) ? where[st.where] : "?";
+                                "embedding token check", "task dispatch", "iteration boundary"};
+  const char* w = (st.where >= 0 && st.where < 11) ? where[st.where] : "?";
   fail(c, st.code, "device status %d at %s: op %d task %d worker %d iter %d observed %u expected %u", st.code, w, st.op,
        st.task, st.worker, st.iter, st.observed, st.expected);
   return st.code;

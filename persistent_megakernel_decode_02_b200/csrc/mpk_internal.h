@@ -12,14 +12,14 @@ constexpr int BLOCK_THREADS = CONSUMER_THREADS + 32;
 #define MPK_STAGE_BYTES 32768
 #endif
 #ifndef MPK_NSTAGES
-#define MPK_NSTAGES 6
+#define MPK_NSTAGES 5
 #endif
 constexpr int STAGE_BYTES = MPK_STAGE_BYTES;  // one weight stage in shared memory
 constexpr int NSTAGES = MPK_NSTAGES;          // weight ring depth
 constexpr int TASK_FIFO = 4;                // decoded task entries buffered per worker
 constexpr int QUEUE_CAP = 64;               // global task queue entries per worker
 constexpr int MAX_RPS = 64;                 // rows per stage upper bound
-constexpr int MAX_K = 12288;                // longest GEMV input kept in shared memory (bf16)
+constexpr int MAX_K = 12288;                // longest GEMV input kept in shared memory (fp32)
 constexpr int MAX_NORM_K = 4096;            // longest RMSNorm input (held in registers)
 constexpr int MAX_XS = 1024;                // residual rows of a task preloaded to shared memory
 constexpr int MAX_SEG = 3;
@@ -54,10 +54,10 @@ struct OpDesc {
   float* y[MAX_SEG];            // fp32 outputs of RMSNORM_LINEAR
   const uint16_t* W_up;         // SILU: up matrix (W[0] = gate)
   const float* x;               // fp32 input (norm ops) / residual (RESID)
-  const uint16_t* a_in;         // bf16 input of RESID
+  const float* a_in;            // fp32 input of RESID
   const uint16_t* norm_w;       // bf16 [K]
   float* x_out;                 // RESID: residual updated in place; EMBED: x
-  uint16_t* a_out;              // SILU / ATTN output bf16
+  float* a_out;                 // SILU / ATTN output (fp32)
   float eps;
   int32_t capture_slot;
   // attention

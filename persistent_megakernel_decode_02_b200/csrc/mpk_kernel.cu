@@ -50,7 +50,7 @@ struct __align__(128) Smem {
   union {
     AttnScratch a;
     struct {
-      uint16_t hs[MAX_K];                        // GEMV input vector (bf16)
+      float hs[MAX_K];                           // GEMV input vector (fp32)
       float xs[MAX_XS];                          // residual rows of the task
     } g;
   } u;
@@ -331,7 +331,7 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     }
     if (!ok) break;
   }
-  if (!ok) {
+  if (!ok || aborted(g)) {
     // Never leave the block with bulk copies in flight: wait (bounded) for the
     // most recent stages to land before returning.
     const uint32_t first = pstage > (uint32_t)NSTAGES ? pstage - NSTAGES : 0u;
@@ -345,52 +345,48 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
 }
 
 // ------------------------------------------------------------------ consumer helpers
-// Dot product of one bf16 weight row with the bf16 input vector, both in shared
-// memory; lane l covers elements [8l + 256j, 8l + 256j + 8).
-__device__ __forceinline__ float dot_row(const uint16_t* w, const uint16_t* h, int K, int lane) {
+// Dot product of one bf16 weight row with the fp32 input vector, both in
+// shared memory; lane l covers elements [8l + 256j, 8l + 256j + 8).
+__device__ __forceinline__ float dot_row(const uint16_t* w, const float* h, int K, int lane) {
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll 4
   for (int e = lane * 8; e < K; e += 256) {
     const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
-    const uint4 hv = *reinterpret_cast<const uint4*>(h + e);
-    a0 = fmaf(bf16_lo(wv.x), bf16_lo(hv.x), a0);
-    a1 = fmaf(bf16_hi(wv.x), bf16_hi(hv.x), a1);
-    a2 = fmaf(bf16_lo(wv.y), bf16_lo(hv.y), a2);
-    a3 = fmaf(bf16_hi(wv.y), bf16_hi(hv.y), a3);
-    a0 = fmaf(bf16_lo(wv.z), bf16_lo(hv.z), a0);
-    a1 = fmaf(bf16_hi(wv.z), bf16_hi(hv.z), a1);
-    a2 = fmaf(bf16_lo(wv.w), bf16_lo(hv.w), a2);
-    a3 = fmaf(bf16_hi(wv.w), bf16_hi(hv.w), a3);
+    const float4 h0 = *reinterpret_cast<const float4*>(h + e);
+    const float4 h1 = *reinterpret_cast<const float4*>(h + e + 4);
+    a0 = fmaf(bf16_lo(wv.x), h0.x, a0);
+    a1 = fmaf(bf16_hi(wv.x), h0.y, a1);
+    a2 = fmaf(bf16_lo(wv.y), h0.z, a2);
+    a3 = fmaf(bf16_hi(wv.y), h0.w, a3);
+    a0 = fmaf(bf16_lo(wv.z), h1.x, a0);
+    a1 = fmaf(bf16_hi(wv.z), h1.y, a1);
+    a2 = fmaf(bf16_lo(wv.w), h1.z, a2);
+    a3 = fmaf(bf16_hi(wv.w), h1.w, a3);
   }
   return (a0 + a1) + (a2 + a3);
 }
 
-// Two rows (gate and up) against the same input: one pass over h.
-__device__ __forceinline__ void dot_row2(const uint16_t* w, const uint16_t* u, const uint16_t* h, int K, int lane,
+// Two rows against the same input: one pass over h serves both.
+__device__ __forceinline__ void dot_row2(const uint16_t* w, const uint16_t* u, const float* h, int K, int lane,
                                          float& dw, float& du) {
   float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll 2
   for (int e = lane * 8; e < K; e += 256) {
     const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
     const uint4 uv = *reinterpret_cast<const uint4*>(u + e);
-    const uint4 hv = *reinterpret_cast<const uint4*>(h + e);
-    const float h0 = bf16_lo(hv.x), h1 = bf16_hi(hv.x), h2 = bf16_lo(hv.y), h3 = bf16_hi(hv.y);
-    const float h4 = bf16_lo(hv.z), h5 = bf16_hi(hv.z), h6 = bf16_lo(hv.w), h7 = bf16_hi(hv.w);
-    a0 = fmaf(bf16_lo(wv.x), h0, a0); a1 = fmaf(bf16_hi(wv.x), h1, a1);
-    a0 = fmaf(bf16_lo(wv.y), h2, a0); a1 = fmaf(bf16_hi(wv.y), h3, a1);
-    a0 = fmaf(bf16_lo(wv.z), h4, a0); a1 = fmaf(bf16_hi(wv.z), h5, a1);
-    a0 = fmaf(bf16_lo(wv.w), h6, a0); a1 = fmaf(bf16_hi(wv.w), h7, a1);
-    b0 = fmaf(bf16_lo(uv.x), h0, b0); b1 = fmaf(bf16_hi(uv.x), h1, b1);
-    b0 = fmaf(bf16_lo(uv.y), h2, b0); b1 = fmaf(bf16_hi(uv.y), h3, b1);
-    b0 = fmaf(bf16_lo(uv.z), h4, b0); b1 = fmaf(bf16_hi(uv.z), h5, b1);
-    b0 = fmaf(bf16_lo(uv.w), h6, b0); b1 = fmaf(bf16_hi(uv.w), h7, b1);
+    const float4 hA = *reinterpret_cast<const float4*>(h + e);
+    const float4 hB = *reinterpret_cast<const float4*>(h + e + 4);
+    a0 = fmaf(bf16_lo(wv.x), hA.x, a0); a1 = fmaf(bf16_hi(wv.x), hA.y, a1);
+    a0 = fmaf(bf16_lo(wv.y), hA.z, a0); a1 = fmaf(bf16_hi(wv.y), hA.w, a1);
+    a0 = fmaf(bf16_lo(wv.z), hB.x, a0); a1 = fmaf(bf16_hi(wv.z), hB.y, a1);
+    a0 = fmaf(bf16_lo(wv.w), hB.z, a0); a1 = fmaf(bf16_hi(wv.w), hB.w, a1);
+    b0 = fmaf(bf16_lo(uv.x), hA.x, b0); b1 = fmaf(bf16_hi(uv.x), hA.y, b1);
+    b0 = fmaf(bf16_lo(uv.y), hA.z, b0); b1 = fmaf(bf16_hi(uv.y), hA.w, b1);
+    b0 = fmaf(bf16_lo(uv.z), hB.x, b0); b1 = fmaf(bf16_hi(uv.z), hB.y, b1);
+    b0 = fmaf(bf16_lo(uv.w), hB.z, b0); b1 = fmaf(bf16_hi(uv.w), hB.w, b1);
   }
   dw = a0 + a1;
   du = b0 + b1;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  return (uint32_t)f32_to_bf16_rn(lo) | ((uint32_t)f32_to_bf16_rn(hi) << 16);
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
@@ -400,7 +396,7 @@ __device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j,
 
 // ------------------------------------------------------------------ GEMV tasks
 // Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector h
-// held in shared memory as bf16.  Each consumer warp owns whole rows (task
+// held in shared memory as fp32.  Each consumer warp owns whole rows (task
 // row j goes to warp j % nwarps) and runs the operation's epilogue for them
 // itself, so the weight stages need no block-wide barrier: every warp waits
 // for each stage, computes its rows in it and releases the stage.
@@ -411,20 +407,16 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   const int K = op.K, rps = op.rps, nw = op.nwarps;
   int grp, row0, row1;
   task_rows(op, task, grp, row0, row1);
-  uint16_t* hs = sm.u.g.hs;
+  float* hs = sm.u.g.hs;
 
-  // ---- prologue: the input vector, bf16, in shared memory.  Every global
+  // ---- prologue: the input vector, fp32, in shared memory.  Every global
   // load of the prologue is issued before the first use (one L2 round trip).
   const int nrows = row1 - row0;
   const bool xs_ok = KIND == TK_GEMV_RESID && nrows <= MAX_XS;
   if (KIND == TK_GEMV_RESID) {
-    constexpr int NA = MAX_K / (CONSUMER_THREADS * 8);
-    uint4 av[NA];
-#pragma unroll
-    for (int c = 0; c < NA; ++c) {
-      const int k = (c * CONSUMER_THREADS + ctid) * 8;
-      if (k < K) av[c] = ldcg_u4(op.a_in + k);
-    }
+    // the input goes straight to shared memory (cp.async through L2), the
+    // task's residual rows through registers
+    for (int k = ctid * 4; k < K; k += CONSUMER_THREADS * 4) cp_async16(hs + k, op.a_in + k);
     float xv[MAX_XS / CONSUMER_THREADS];
 #pragma unroll
     for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
@@ -432,15 +424,11 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       if (xs_ok && j < nrows) xv[c] = __ldcg(op.x_out + row0 + j);
     }
 #pragma unroll
-    for (int c = 0; c < NA; ++c) {
-      const int k = (c * CONSUMER_THREADS + ctid) * 8;
-      if (k < K) *reinterpret_cast<uint4*>(hs + k) = av[c];
-    }
-#pragma unroll
     for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
       const int j = c * CONSUMER_THREADS + ctid;
       if (xs_ok && j < nrows) sm.u.g.xs[j] = xv[c];
     }
+    cp_async_wait_all();
   } else {
     // RMSNorm: x and the norm weight are read once into registers, the
     // statistics are reduced in a fixed order.
@@ -478,12 +466,13 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       const int k = (c * CONSUMER_THREADS + ctid) * 8;
       if (k < K) {
         const uint4 w = wr[c];
-        uint4 hv;
-        hv.x = pack_bf16x2(xr[c][0] * rinv * bf16_lo(w.x), xr[c][1] * rinv * bf16_hi(w.x));
-        hv.y = pack_bf16x2(xr[c][2] * rinv * bf16_lo(w.y), xr[c][3] * rinv * bf16_hi(w.y));
-        hv.z = pack_bf16x2(xr[c][4] * rinv * bf16_lo(w.z), xr[c][5] * rinv * bf16_hi(w.z));
-        hv.w = pack_bf16x2(xr[c][6] * rinv * bf16_lo(w.w), xr[c][7] * rinv * bf16_hi(w.w));
-        *reinterpret_cast<uint4*>(hs + k) = hv;
+        float4 h0, h1;
+        h0.x = xr[c][0] * rinv * bf16_lo(w.x); h0.y = xr[c][1] * rinv * bf16_hi(w.x);
+        h0.z = xr[c][2] * rinv * bf16_lo(w.y); h0.w = xr[c][3] * rinv * bf16_hi(w.y);
+        h1.x = xr[c][4] * rinv * bf16_lo(w.z); h1.y = xr[c][5] * rinv * bf16_hi(w.z);
+        h1.z = xr[c][6] * rinv * bf16_lo(w.w); h1.w = xr[c][7] * rinv * bf16_hi(w.w);
+        *reinterpret_cast<float4*>(hs + k) = h0;
+        *reinterpret_cast<float4*>(hs + k + 4) = h1;
       }
     }
   }
@@ -506,7 +495,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
         g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
     } else if (KIND == TK_NORM_GEMV_SILU) {
-      op.a_out[row] = f32_to_bf16_rn(silu_f(v) * u);
+      op.a_out[row] = silu_f(v) * u;
     } else {  // LM head
       const unsigned long long key = argmax_key(v, (uint32_t)row);
       best = key > best ? key : best;
@@ -797,7 +786,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         }
       }
       if (direct) {
-        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = f32_to_bf16_rn(Os / Ls);
+        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = Os / Ls;
       } else {
         float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
         p[2 + i] = Os;
@@ -840,7 +829,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
           Ls = fmaf(lc, f, Ls);
           Os = fmaf(oc, f, Os);
         }
-        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = f32_to_bf16_rn(Os / Ls);
+        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = Os / Ls;
       }
     }
     consumer_sync();
@@ -1004,6 +993,13 @@ __device__ void scheduler_lane(const Graph& g, int si, int lane) {
 
   uint32_t off = 0;  // rotating task offset: op p's task t goes to worker (t + off) % W
   for (uint32_t n = 0; n < n_iter; ++n) {
+    // host abort request, read once per iteration; the scheduler is ahead of
+    // the workers by the dispatch window, so this read is off their path
+    if (g.abort_flag != nullptr && *g.abort_flag != 0) {
+      record_error(g, -10 /*ABORTED*/, 10, -1, -1, wk, (int)n, 0, 0);
+      return;
+    }
+    if (aborted(g)) return;
     for (int p = 0; p < P; ++p) {
       const long long gidx = (long long)n * P + p - g.lookahead;
       if (g.lookahead > 0 && gidx >= 0) {

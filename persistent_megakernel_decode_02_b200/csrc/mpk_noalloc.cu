@@ -29,11 +29,6 @@ unsigned long long* g_scratch_addr[kMaxDevices] = {};
 std::mutex g_scratch_mu;
 
 __device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ uint16_t to_bf16(float f) {
-  uint16_t r;
-  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
-  return r;
-}
 __device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 __device__ __forceinline__ unsigned long long key_of(float v, uint32_t idx) {
@@ -48,14 +43,14 @@ __device__ __forceinline__ unsigned long long key_of(float v, uint32_t idx) {
 __global__ void __launch_bounds__(kThreads) lmhead_argmax_noalloc_kernel(
     const float* __restrict__ x, const uint16_t* __restrict__ nw, const uint16_t* __restrict__ W, int K, int V,
     float eps, unsigned long long* scratch, int64_t* tok, float* logits) {
-  extern __shared__ __align__(16) uint16_t hsm[];
+  extern __shared__ __align__(16) float hsm[];
   __shared__ float ss_w[kThreads / 32];
   __shared__ unsigned long long best_w[kThreads / 32];
   __shared__ int last;
   const int r = blockIdx.y, nb = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* xr = x + (size_t)r * K;
-  // RMSNorm statistics in a fixed order, then h = bf16(x * rinv * w).
+  // RMSNorm statistics in a fixed order, then h = x * rinv * w (fp32).
   float ss = 0.f;
   for (int k = threadIdx.x; k < K; k += kThreads) ss = fmaf(xr[k], xr[k], ss);
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -66,7 +61,7 @@ __global__ void __launch_bounds__(kThreads) lmhead_argmax_noalloc_kernel(
   const float rinv = 1.0f / sqrtf(tot / (float)K + eps);
   for (int k = threadIdx.x; k < K; k += kThreads) {
     const float wv = __uint_as_float((uint32_t)nw[k] << 16);
-    hsm[k] = to_bf16(xr[k] * rinv * wv);
+    hsm[k] = xr[k] * rinv * wv;
   }
   __syncthreads();
 
@@ -77,11 +72,12 @@ __global__ void __launch_bounds__(kThreads) lmhead_argmax_noalloc_kernel(
     float a0 = 0.f, a1 = 0.f;
     for (int e = lane * 8; e < K; e += 256) {
       const uint4 wv = __ldg(reinterpret_cast<const uint4*>(wr + e));
-      const uint4 hv = *reinterpret_cast<const uint4*>(hsm + e);
-      a0 = fmaf(lo16(wv.x), lo16(hv.x), a0); a1 = fmaf(hi16(wv.x), hi16(hv.x), a1);
-      a0 = fmaf(lo16(wv.y), lo16(hv.y), a0); a1 = fmaf(hi16(wv.y), hi16(hv.y), a1);
-      a0 = fmaf(lo16(wv.z), lo16(hv.z), a0); a1 = fmaf(hi16(wv.z), hi16(hv.z), a1);
-      a0 = fmaf(lo16(wv.w), lo16(hv.w), a0); a1 = fmaf(hi16(wv.w), hi16(hv.w), a1);
+      const float4 h0 = *reinterpret_cast<const float4*>(hsm + e);
+      const float4 h1 = *reinterpret_cast<const float4*>(hsm + e + 4);
+      a0 = fmaf(lo16(wv.x), h0.x, a0); a1 = fmaf(hi16(wv.x), h0.y, a1);
+      a0 = fmaf(lo16(wv.y), h0.z, a0); a1 = fmaf(hi16(wv.y), h0.w, a1);
+      a0 = fmaf(lo16(wv.z), h1.x, a0); a1 = fmaf(hi16(wv.z), h1.y, a1);
+      a0 = fmaf(lo16(wv.w), h1.z, a0); a1 = fmaf(hi16(wv.w), h1.w, a1);
     }
     float v = a0 + a1;
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -162,7 +158,7 @@ MPK_API int mpk_lmhead_argmax_noalloc(const float* x, const uint16_t* norm_w, co
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nb = V < 2 * sms ? V : 2 * sms;
-  const size_t smem = (size_t)K * sizeof(uint16_t);
+  const size_t smem = (size_t)K * sizeof(float);
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(lmhead_argmax_noalloc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return noalloc_fail(MPK_ERR_CUDA, cudaGetErrorString(e));

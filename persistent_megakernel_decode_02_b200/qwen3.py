@@ -96,7 +96,8 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   attn_chunks: Optional[int] = None, gemv_tasks: Optional[int] = None, block_dim: int = 0,
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
-                  prefetch_kb: int = 0, fused_attention: Optional[bool] = None) -> Decoder:
+                  prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
+                  debug_stall_op: int = 0) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
@@ -125,8 +126,8 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
         "q": mk.new_tensor((requests, s.q_dim), torch.float32, "q"),
         "k": mk.new_tensor((requests, s.kv_dim), torch.float32, "k"),
         "v": mk.new_tensor((requests, s.kv_dim), torch.float32, "v"),
-        "o": mk.new_tensor((requests, s.q_dim), torch.bfloat16, "o"),
-        "a": mk.new_tensor((requests, s.intermediate), torch.bfloat16, "a"),
+        "o": mk.new_tensor((requests, s.q_dim), torch.float32, "o"),
+        "a": mk.new_tensor((requests, s.intermediate), torch.float32, "a"),
     }
     if attn_chunks is None:
         attn_chunks = default_attn_chunks(s, requests, num_workers, max_seq)
@@ -136,5 +137,6 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                          fused_attention=fused_attention):
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
-    mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb)
+    mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb,
+               debug_stall_op=debug_stall_op)
     return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)

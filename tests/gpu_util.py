@@ -53,7 +53,7 @@ def oracle_teacher_forced(shape, w_cpu, tokens_cpu: torch.Tensor, iters, kc=None
     for _ in range(iters):
         lg = np.full((R, shape.vocab), np.nan)
         hd = np.full((shape.layers + 1, R, shape.hidden), np.nan)
-        ref.iteration(kc, vc, step, toks, None, oracle.ROUND_BF16, lg, hd)
+        ref.iteration(kc, vc, step, toks, None, oracle.ROUND_NONE, lg, hd)
         out.append((lg, hd))
     return out, toks, kc, vc
 

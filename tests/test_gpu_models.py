@@ -1,0 +1,106 @@
+"""GPU parity at the model sizes of the measured workloads (Qwen3-0.6B and
+Qwen3-8B shapes), in the launch configuration the benchmark uses (all SMs but
+four worker SMs' worth of scheduler warps, default task splits and attention
+mode for the sequence length).
+
+The oracle cannot afford hundreds of full-size iterations, so these tests
+sample: the KV cache is pre-filled with seeded N(0,1) bf16 keys/values for
+positions [0, P) (the same input on both sides), and a few teacher-forced
+iterations from step P are compared — logits within rel-L2 2e-2 and every
+layer's residual stream within 1e-2.  P sits at the end of the 39 + 512 token
+workload, and at 32768 for the long-context workload (split-K attention).
+"""
+import numpy as np
+import pytest
+import torch
+
+from synth import qwen3 as sq
+from tests.gpu_util import compare_captures, gpu_teacher_forced, oracle_teacher_forced, to_cuda
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+PROMPT, GENERATED = 39, 512
+
+
+def _u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def _check(shape, w_cpu, w, P, S, iters, **build_kw):
+    from persistent_megakernel_decode_02_b200 import build_decoder
+
+    kc, vc = sq.make_kv_prefill(shape, 1, S, P, seed=11)
+    tokens = sq.make_tokens(shape, 1, S, [S], seed=12, teacher_forced=True)
+    dec = build_decoder(shape, w, requests=1, max_seq=S, k_cache=kc.cuda(), v_cache=vc.cuda(), **build_kw)
+    gpu, gtok, gstep = gpu_teacher_forced(dec, tokens, iters, step0=P)
+    ref, _, rkc, _ = oracle_teacher_forced(shape, w_cpu, tokens, iters, _u16(kc), _u16(vc), step0=P)
+    wl, wh = compare_captures(gpu, ref)
+    print(f"{shape.name} P={P}: worst logits rel-L2 {wl:.2e}, hidden {wh:.2e}")
+    assert int(gstep[0]) == P + iters
+    assert torch.equal(gtok, tokens)
+    # the K cache rows this run wrote are the oracle's up to bf16 rounding flips
+    gk = dec.k_cache[:, :, :, P:P + iters].float().cpu().numpy()
+    rk = (rkc[:, :, :, P:P + iters].astype(np.uint32) << 16).view(np.float32)
+    assert np.linalg.norm(gk - rk) <= 1e-2 * np.linalg.norm(rk)
+    # the pre-filled rows are untouched
+    assert torch.equal(dec.k_cache[:, :, :, :P].cpu().view(torch.int16), kc[:, :, :, :P].view(torch.int16))
+    dec.kernel.close()
+
+
+@pytest.fixture(scope="module")
+def qwen3_0_6b():
+    w_cpu = sq.make_weights(sq.QWEN3_0_6B, seed=0)
+    return w_cpu, to_cuda(w_cpu)
+
+
+@pytest.fixture(scope="module")
+def qwen3_8b():
+    w_cpu = sq.make_weights(sq.QWEN3_8B, seed=0)
+    yield w_cpu, to_cuda(w_cpu)
+    torch.cuda.empty_cache()
+
+
+def test_qwen3_0_6b_from_scratch(qwen3_0_6b):
+    """0.6B shape (tied embeddings): iterations from an empty cache."""
+    w_cpu, w = qwen3_0_6b
+    _check(sq.QWEN3_0_6B, w_cpu, w, 0, PROMPT + GENERATED, 4)
+
+
+def test_qwen3_0_6b_end_of_workload(qwen3_0_6b):
+    w_cpu, w = qwen3_0_6b
+    S = PROMPT + GENERATED
+    _check(sq.QWEN3_0_6B, w_cpu, w, S - 4, S, 3)
+
+
+def test_qwen3_0_6b_op_by_op_bit_identical(qwen3_0_6b):
+    from persistent_megakernel_decode_02_b200 import build_decoder
+
+    _, w = qwen3_0_6b
+    shape, S = sq.QWEN3_0_6B, 16
+    tokens = sq.make_tokens(shape, 1, S, [8], seed=13)
+    outs = []
+    for mode in ("run", "run_op_by_op"):
+        dec = build_decoder(shape, w, requests=1, max_seq=S)
+        tok = tokens.cuda()
+        step = torch.zeros(1, dtype=torch.int32, device="cuda")
+        getattr(dec, mode)(step, tok)
+        torch.cuda.synchronize()
+        dec.kernel.check_status()
+        outs.append((tok.cpu(), dec.pred.cpu(), dec.k_cache.cpu().view(torch.int16)))
+        dec.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_qwen3_8b_end_of_workload(qwen3_8b):
+    """The benchmarked workload: 8B shape, 551 positions, fused attention."""
+    w_cpu, w = qwen3_8b
+    S = PROMPT + GENERATED
+    _check(sq.QWEN3_8B, w_cpu, w, S - 3, S, 2)
+
+
+def test_qwen3_8b_long_context(qwen3_8b):
+    """32768 pre-filled positions: the split-K attention path at full size."""
+    w_cpu, w = qwen3_8b
+    P = 32768
+    _check(sq.QWEN3_8B, w_cpu, w, P, P + 128, 2)

@@ -323,12 +323,14 @@ def test_decoder_gqa_maps_contiguous_groups():
 
 # ---------------------------------------------------------------- independent restatement
 
-def _torch_reference(shape, w, tokens_row, steps):
+def _torch_reference(shape, w, tokens_row, steps, round_mode=oracle.ROUND_BF16):
     """Teacher-forced logits of the decoder written with PyTorch library routines
     (F.rms_norm, F.linear, F.scaled_dot_product_attention with GQA, F.silu) in
-    float64, with the same bf16 rounding points."""
+    float64.  The KV cache is bf16 in both modes; with ROUND_BF16 the inputs of
+    the projections are rounded to bf16 too, with ROUND_NONE they are not."""
     s = shape
-    rb = lambda t: torch.from_numpy(rb_exact(t.numpy()))
+    rkv = lambda t: torch.from_numpy(rb_exact(t.numpy()))
+    rb = rkv if round_mode == oracle.ROUND_BF16 else (lambda t: t)
     W = {k: v.double() for k, v in w.items()}
     d = s.head_dim
     inv = 1.0 / (s.rope_theta ** (torch.arange(0, d // 2, dtype=torch.float64) * 2.0 / d))
@@ -352,8 +354,8 @@ def _torch_reference(shape, w, tokens_row, steps):
             v = F.linear(h, W[p + "v_proj"]).view(s.kv_heads, d)
             q = rot(F.rms_norm(q, (d,), W[p + "q_norm"], eps=s.eps))
             k = rot(F.rms_norm(k, (d,), W[p + "k_norm"], eps=s.eps))
-            Kc[l].append(rb(k))
-            Vc[l].append(rb(v))
+            Kc[l].append(rkv(k))
+            Vc[l].append(rkv(v))
             Ks = torch.stack(Kc[l], dim=1)[None]  # [1, Hkv, T, d]
             Vs = torch.stack(Vc[l], dim=1)[None]
             o = F.scaled_dot_product_attention(q[None, :, None, :], Ks, Vs, enable_gqa=True)
@@ -368,8 +370,9 @@ def _torch_reference(shape, w, tokens_row, steps):
     return np.stack(out)
 
 
+@pytest.mark.parametrize("mode", [oracle.ROUND_NONE, oracle.ROUND_BF16], ids=["round-none", "round-bf16"])
 @pytest.mark.parametrize("shape", [qwen3.TINY, qwen3.Qwen3Shape("pin-t", 2, 64, 4, 2, 16, 96, 200, tied=True)])
-def test_decoder_matches_library_restatement(shape):
+def test_decoder_matches_library_restatement(shape, mode):
     w = qwen3.make_weights(shape, seed=0)
     dec = oracle.Decoder(shape, w)
     S = 10
@@ -379,8 +382,8 @@ def test_decoder_matches_library_restatement(shape):
     got = []
     for _ in range(S - 1):
         lg = np.zeros((1, shape.vocab))
-        dec.iteration(kc, vc, step, toks, None, oracle.ROUND_BF16, lg, None)
+        dec.iteration(kc, vc, step, toks, None, mode, lg, None)
         got.append(lg[0].copy())
-    ref = _torch_reference(shape, w, toks[0], S - 1)
+    ref = _torch_reference(shape, w, toks[0], S - 1, mode)
     err = np.linalg.norm(np.stack(got) - ref) / np.linalg.norm(ref)
     assert err < 1e-9, err
