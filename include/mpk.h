@@ -93,7 +93,12 @@ typedef enum {
      * slice; rope_theta the RoPE base.  grid_dim = (Hkv, chunks, R). */
     MPK_OP_ATTENTION = 3,
     /* x += W a.  inputs[0] = a fp32 [R,K]; weights[0] = W bf16 [N,K];
-     * outputs[0] = x fp32 [R,N] (read and written in place). */
+     * outputs[0] = x fp32 [R,N] (read and written in place).  When K exceeds
+     * MPK_MAX_GEMV_K the reduction is split into the fewest ks equal segments
+     * of at most MPK_MAX_GEMV_K (each a multiple of 256): task t computes
+     * segment t % ks of row block t / ks, and the last segment task of a row
+     * block to finish adds the ks partial sums to x in segment order.  grid_dim
+     * must then give a multiple of ks tasks (MPK_ERR_SHAPE otherwise). */
     MPK_OP_LINEAR_RESIDUAL = 4,
     /* h = rmsnorm(x) * w_norm; a = silu(W_gate h) * (W_up h).
      * inputs[0] = x fp32 [R,K]; weights = w_norm [K], W_gate [I,K], W_up [I,K];
@@ -122,6 +127,8 @@ typedef enum {
 typedef struct { int32_t x, y, z; } mpk_dim3;
 
 #define MPK_MAX_IO 8
+/* Longest reduction (input length K) one GEMV task holds in shared memory. */
+#define MPK_MAX_GEMV_K 4096
 
 /* One fused operation.  Unused name slots are NULL.  grid_dim gives the number
  * of tasks (thread blocks) x*y*z; block_dim the threads per task (a multiple

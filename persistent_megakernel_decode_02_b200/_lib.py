@@ -24,6 +24,7 @@ IO_CUDA, IO_NVSHMEM = 0, 1
 OP_EMBED, OP_RMSNORM_LINEAR, OP_ATTENTION, OP_LINEAR_RESIDUAL = 1, 2, 3, 4
 OP_RMSNORM_LINEAR_SILU_MUL, OP_RMSNORM_LMHEAD_ARGMAX, OP_RMSNORM_QKV_ATTENTION = 5, 6, 7
 MAX_IO = 8
+MAX_GEMV_K = 4096  # MPK_MAX_GEMV_K
 
 
 class Dim3(ctypes.Structure):

@@ -140,7 +140,7 @@ int need(mpk_ctx* c, int li, const char* role, const char* name, mpk_dtype dt, i
 // GEMV geometry: rows per shared-memory stage (each consumer warp owns whole
 // rows, so any K that is a multiple of 256 and fits the input buffer works).
 int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats, bool norm) {
-  const int K = o.K;
+  const int K = o.ksplit > 1 ? o.kseg : o.K;
   if (K % 256 != 0) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d is not a multiple of 256", li, K);
   if (K > MAX_K) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d exceeds %d", li, K, MAX_K);
   if (norm && K > MAX_NORM_K)
@@ -331,7 +331,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   std::vector<OpDesc> ops(n_layers);
   int R = -1, H = -1, V = -1, L = -1, S = -1;
   // attention workspace sizing
-  size_t part_floats = 0, merge_u32 = 0;
+  size_t part_floats = 0, merge_u32 = 0, kpart_floats = 0, blk_u32 = 0;
   std::vector<std::pair<int, size_t>> merge_off(n_layers, {0, 0});
   struct RopeKey { float theta; int d; int S; };
   std::vector<RopeKey> rope_keys;
@@ -404,6 +404,22 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
           op.seg_row0[1] = op.N;
           op.x_out = (float*)out->ptr;
           op.x = (const float*)out->ptr;
+          if (op.K > MAX_K) {
+            // Split the reduction into the fewest segments that fit the input
+            // buffer; task t computes segment t % ksplit of row block t / ksplit.
+            int ks = (op.K + MAX_K - 1) / MAX_K;
+            while (ks <= op.K / 256 && (op.K % ks != 0 || (op.K / ks) % 256 != 0)) ++ks;
+            if (ks > op.K / 256)
+              return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d cannot be split", li, op.K);
+            if (ntasks % ks != 0)
+              return fail(c, MPK_ERR_SHAPE,
+                          "layer %d: reduction length %d is split into %d segments: grid_dim must give a multiple "
+                          "of %d tasks (got %d)", li, op.K, ks, ks, ntasks);
+            op.ksplit = ks;
+            op.kseg = op.K / ks;
+            kpart_floats = std::max(kpart_floats, (size_t)ks * op.N);
+            blk_u32 = std::max(blk_u32, (size_t)(ntasks / ks));
+          }
         } else {
           NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32, 2, &x);
           op.x = (const float*)x->ptr;
@@ -477,7 +493,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
                       li, R);
         int rc = gemv_geometry(c, li, op, silu, !resid);
         if (rc != MPK_OK) return rc;
-        rc = check_grid(c, li, Ly, ntasks, op.N);
+        rc = check_grid(c, li, Ly, ntasks, op.N * (op.ksplit > 1 ? op.ksplit : 1));
         if (rc != MPK_OK) return rc;
         op.signal_per_task = lmh ? 0 : 1;
         op.out_trigger = lmh ? 1 : ntasks;
@@ -667,7 +683,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   }
 
   // ---- workspace
-  // sync block (zeroed before every run): events | q_head | q_tail | ctl | status | keys | arrive | merge counters | timeline_n
+  // sync block (zeroed before every run): events | q_head | q_tail | ctl | status | keys | arrive | merge counters |
+  // timeline_n | split row-block counters
   const size_t line = EVENT_STRIDE * sizeof(uint32_t);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o2 = off; off += (bytes + 127) / 128 * 128; return o2; };
@@ -680,6 +697,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   const size_t o_arrive = take(line);
   const size_t o_merge = take(sizeof(uint32_t) * (merge_u32 ? merge_u32 : 1));
   const size_t o_tln = take(line);
+  const size_t o_blk = take(sizeof(uint32_t) * (blk_u32 ? blk_u32 : 1));
   c->sync_bytes = off;
   uint8_t* sb = nullptr;
   int rc = alloc(c, &sb, off);
@@ -690,6 +708,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (rc != MPK_OK) return rc;
   float* part = nullptr;
   rc = alloc(c, &part, sizeof(float) * (part_floats ? part_floats : 1));
+  if (rc != MPK_OK) return rc;
+  float* kpart = nullptr;
+  rc = alloc(c, &kpart, sizeof(float) * (kpart_floats ? kpart_floats : 1));
   if (rc != MPK_OK) return rc;
   std::vector<float2*> rope_dev(rope_keys.size(), nullptr);
   for (size_t i = 0; i < rope_keys.size(); ++i) {
@@ -719,6 +740,11 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     if (op.kind == TK_QKV_ATTN) {
       op.grp_cnt = reinterpret_cast<uint32_t*>(sb + o_merge) + merge_off[p].second;
       op.rope = rope_dev[rope_of[p]];
+    }
+    if (op.ksplit > 1) {
+      // shared by every split projection: they run one after another
+      op.kpart = kpart;
+      op.blk_cnt = reinterpret_cast<uint32_t*>(sb + o_blk);
     }
     if (op.kind == TK_NORM_GEMV_ARGMAX) {
       op.keys = reinterpret_cast<unsigned long long*>(sb + o_keys);

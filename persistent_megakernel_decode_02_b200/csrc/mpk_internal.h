@@ -2,24 +2,41 @@
 #pragma once
 #include <stdint.h>
 
+#include "mpk.h"
+
 namespace mpk {
 
-// Worker block: one producer warp (weight stream) + CONSUMER_WARPS compute warps.
+// Worker block: a producer warpgroup (its warp 0 streams the weights, the
+// other three only hand their registers over) + CONSUMER_WARPS compute warps
+// in two warpgroups.  The launch gives every thread LAUNCH_REGS registers;
+// setmaxnreg then moves them from the producer warpgroup to the consumers.
 constexpr int CONSUMER_WARPS = 8;
 constexpr int CONSUMER_THREADS = CONSUMER_WARPS * 32;
-constexpr int BLOCK_THREADS = CONSUMER_THREADS + 32;
+constexpr int PRODUCER_WARPS = 4;
+constexpr int BLOCK_THREADS = CONSUMER_THREADS + PRODUCER_WARPS * 32;
+constexpr int LAUNCH_REGS = 168;    // 65536 / 384 threads, rounded down to a multiple of 8
+constexpr int PRODUCER_REGS = 56;
+constexpr int CONSUMER_REGS = 224;
+static_assert(PRODUCER_WARPS * 32 * PRODUCER_REGS + CONSUMER_THREADS * CONSUMER_REGS <= BLOCK_THREADS * LAUNCH_REGS,
+              "register hand-over must stay within the launch's registers");
 #ifndef MPK_STAGE_BYTES
 #define MPK_STAGE_BYTES 32768
 #endif
+#ifndef MPK_GEMV_RB
+#define MPK_GEMV_RB 1   // weight rows per warp sharing each load of the input vector
+#endif
 #ifndef MPK_NSTAGES
-#define MPK_NSTAGES 5
+#define MPK_NSTAGES 6
 #endif
 constexpr int STAGE_BYTES = MPK_STAGE_BYTES;  // one weight stage in shared memory
 constexpr int NSTAGES = MPK_NSTAGES;          // weight ring depth
 constexpr int TASK_FIFO = 4;                // decoded task entries buffered per worker
 constexpr int QUEUE_CAP = 64;               // global task queue entries per worker
 constexpr int MAX_RPS = 64;                 // rows per stage upper bound
-constexpr int MAX_K = 12288;                // longest GEMV input kept in shared memory (fp32)
+constexpr int MAX_K = 4096;                 // longest GEMV input kept in shared memory (fp32);
+                                            // longer residual projections are split (ksplit)
+static_assert(MAX_K % 256 == 0, "the permuted input layout works in blocks of 256");
+static_assert(MAX_K == MPK_MAX_GEMV_K, "the header states the input buffer length");
 constexpr int MAX_NORM_K = 4096;            // longest RMSNorm input (held in registers)
 constexpr int MAX_XS = 1024;                // residual rows of a task preloaded to shared memory
 constexpr int MAX_SEG = 3;
@@ -50,6 +67,10 @@ struct OpDesc {
   int32_t groups;          // row groups (QKV+attention: kv heads; else 1); N = rows per group
   int32_t grp_rows[MAX_SEG];      // rows of segment s per group (matrix row = g * grp_rows + local)
   uint32_t* grp_cnt;       // QKV+attention: finished tasks per (request, group)
+  int32_t ksplit;          // RESID: reduction split into ksplit segments of kseg (1: no split)
+  int32_t kseg;
+  float* kpart;            // RESID split: partial sums [ksplit][N]
+  uint32_t* blk_cnt;       // RESID split: finished segment tasks per row block
   const uint16_t* W[MAX_SEG];   // bf16 weights [rows, K]
   float* y[MAX_SEG];            // fp32 outputs of RMSNORM_LINEAR
   const uint16_t* W_up;         // SILU: up matrix (W[0] = gate)

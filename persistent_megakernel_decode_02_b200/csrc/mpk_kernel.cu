@@ -133,12 +133,33 @@ __device__ bool wait_mbar(const Graph& g, uint64_t* bar, uint32_t parity, int wh
 // ------------------------------------------------------------------ task geometry
 // Rows [row0, row1) of group g that task `task` computes (groups split the
 // tasks evenly; N is the row count of one group).
+// A split residual projection (ksplit > 1) has ntasks / ksplit row blocks;
+// task t computes reduction segment t % ksplit of row block t / ksplit.
 __device__ __forceinline__ void task_rows(const OpDesc& op, int task, int& g, int& row0, int& row1) {
-  const int tpg = op.ntasks / op.groups;
-  g = task / tpg;
-  const int t = task - g * tpg;
+  int tpg = op.ntasks / op.groups, t;
+  if (op.ksplit > 1) {
+    tpg /= op.ksplit;
+    g = 0;
+    t = task / op.ksplit;
+  } else {
+    g = task / tpg;
+    t = task - g * tpg;
+  }
   row0 = (int)(((long long)t * op.N) / tpg);
   row1 = (int)(((long long)(t + 1) * op.N) / tpg);
+}
+
+// First reduction element of the task's segment (0 without a split).
+__device__ __forceinline__ int task_koff(const OpDesc& op, int task) {
+  return op.ksplit > 1 ? (task % op.ksplit) * op.kseg : 0;
+}
+
+// Reduction length of one task (the segment length for a split projection).
+__device__ __forceinline__ int task_k(const OpDesc& op) { return op.ksplit > 1 ? op.kseg : op.K; }
+
+// Weight bytes of one task row in a stage (gate/up: both matrices).
+__device__ __forceinline__ uint32_t stage_row_bytes(const OpDesc& op) {
+  return (uint32_t)task_k(op) * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
 }
 
 __device__ __forceinline__ bool is_gemv(int kind) {
@@ -172,8 +193,16 @@ __device__ __forceinline__ size_t seg_row(const OpDesc& op, int g, int s, int ro
 
 // ------------------------------------------------------------------ producer
 // Issue the bulk copies of one stage: rows [r, r+n) of the op's row space.
-__device__ void issue_stage(const OpDesc& op, int g, int r, int n, uint8_t* dst, uint64_t* bar, uint64_t pol) {
+__device__ void issue_stage(const OpDesc& op, int g, int r, int n, int koff, uint8_t* dst, uint64_t* bar,
+                            uint64_t pol) {
   const uint32_t row_bytes = (uint32_t)op.K * 2u;
+  if (op.ksplit > 1) {
+    // one segment of each row: rows are strided in memory
+    const uint32_t seg_bytes = (uint32_t)op.kseg * 2u;
+    for (int i = 0; i < n; ++i)
+      bulk_g2s(dst + (size_t)i * seg_bytes, op.W[0] + (size_t)(r + i) * op.K + koff, seg_bytes, bar, pol);
+    return;
+  }
   if (op.kind == TK_NORM_GEMV_SILU) {
     bulk_g2s(dst, op.W[0] + (size_t)r * op.K, row_bytes * n, bar, pol);
     bulk_g2s(dst + (size_t)op.rps * row_bytes, op.W_up + (size_t)r * op.K, row_bytes * n, bar, pol);
@@ -191,8 +220,12 @@ __device__ void issue_stage(const OpDesc& op, int g, int r, int n, uint8_t* dst,
 }
 
 // Prefetch rows [r, r+n) of a GEMV operation's weights into L2.
-__device__ void prefetch_rows(const OpDesc& op, int g, int r, int n) {
+__device__ void prefetch_rows(const OpDesc& op, int g, int r, int n, int koff) {
   const uint32_t row_bytes = (uint32_t)op.K * 2u;
+  if (op.ksplit > 1) {
+    for (int i = 0; i < n; ++i) prefetch_l2(op.W[0] + (size_t)(r + i) * op.K + koff, (uint32_t)op.kseg * 2u);
+    return;
+  }
   if (op.kind == TK_NORM_GEMV_SILU) {
     prefetch_l2(op.W[0] + (size_t)r * op.K, row_bytes * n);
     prefetch_l2(op.W_up + (size_t)r * op.K, row_bytes * n);
@@ -263,9 +296,9 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
         pf.have = false;
         continue;
       }
-      const uint32_t rb = (uint32_t)op.K * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
+      const uint32_t rb = stage_row_bytes(op);
       const int n = min(r1 - pf.row, max(1, (int)(65536u / rb)));
-      if (pf.pos + (uint64_t)rb * n > lo) prefetch_rows(op, pg, pf.row, n);
+      if (pf.pos + (uint64_t)rb * n > lo) prefetch_rows(op, pg, pf.row, n, task_koff(op, (int)(pf.e & 0xFFFFu)));
       pf.row += n;
       pf.pos += (uint64_t)rb * n;
     }
@@ -308,7 +341,8 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     if (!is_gemv(op.kind)) continue;
     int grp, row0, row1;
     task_rows(op, task, grp, row0, row1);
-    const uint32_t bytes_row = (uint32_t)op.K * 2u * (op.kind == TK_NORM_GEMV_SILU ? 2u : 1u);
+    const uint32_t bytes_row = stage_row_bytes(op);
+    const int koff = task_koff(op, task);
     for (int r = row0; r < row1; r += op.rps) {
       const int n = min(op.rps, row1 - r);
       const uint32_t slot = pstage % NSTAGES;
@@ -324,7 +358,7 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
       }
       if (g.profiling && r == row0) atomicExch(&sm.fifo_t[f], (unsigned long long)globaltimer());
       mbar_arrive_expect_tx(&sm.full[slot], bytes_row * (uint32_t)n);
-      issue_stage(op, grp, r, n, sm.ring[slot], &sm.full[slot], pol);
+      issue_stage(op, grp, r, n, koff, sm.ring[slot], &sm.full[slot], pol);
       ld_bytes += (uint64_t)bytes_row * n;
       ++pstage;
       if (pf_dist) prefetch_some();
@@ -345,48 +379,66 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
 }
 
 // ------------------------------------------------------------------ consumer helpers
-// Dot product of one bf16 weight row with the fp32 input vector, both in
-// shared memory; lane l covers elements [8l + 256j, 8l + 256j + 8).
-__device__ __forceinline__ float dot_row(const uint16_t* w, const float* h, int K, int lane) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll 4
-  for (int e = lane * 8; e < K; e += 256) {
-    const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
-    const float4 h0 = *reinterpret_cast<const float4*>(h + e);
-    const float4 h1 = *reinterpret_cast<const float4*>(h + e + 4);
-    a0 = fmaf(bf16_lo(wv.x), h0.x, a0);
-    a1 = fmaf(bf16_hi(wv.x), h0.y, a1);
-    a2 = fmaf(bf16_lo(wv.y), h0.z, a2);
-    a3 = fmaf(bf16_hi(wv.y), h0.w, a3);
-    a0 = fmaf(bf16_lo(wv.z), h1.x, a0);
-    a1 = fmaf(bf16_hi(wv.z), h1.y, a1);
-    a2 = fmaf(bf16_lo(wv.w), h1.z, a2);
-    a3 = fmaf(bf16_hi(wv.w), h1.w, a3);
-  }
-  return (a0 + a1) + (a2 + a3);
+// The fp32 input vector h is stored permuted in shared memory so that the
+// GEMV's loads are free of bank conflicts: lane l of a warp multiplies weight
+// elements [8l + 256j, +8) and reads their inputs as two float4 at
+// hperm(8l + 256j) and hperm(8l + 256j + 4), which for one j are 32
+// consecutive float4.  hperm(k) for k a multiple of 4: element block m = k/8,
+// half k/4 mod 2 -> ((m/32)*2 + half)*128 + 4*(m mod 32).
+__device__ __forceinline__ int hperm(int k) {
+  const int q = k >> 2, m = q >> 1;
+  return (((m >> 5) << 1) + (q & 1)) * 128 + ((m & 31) << 2);
 }
 
-// Two rows against the same input: one pass over h serves both.
-__device__ __forceinline__ void dot_row2(const uint16_t* w, const uint16_t* u, const float* h, int K, int lane,
-                                         float& dw, float& du) {
-  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll 2
-  for (int e = lane * 8; e < K; e += 256) {
-    const uint4 wv = *reinterpret_cast<const uint4*>(w + e);
-    const uint4 uv = *reinterpret_cast<const uint4*>(u + e);
-    const float4 hA = *reinterpret_cast<const float4*>(h + e);
-    const float4 hB = *reinterpret_cast<const float4*>(h + e + 4);
-    a0 = fmaf(bf16_lo(wv.x), hA.x, a0); a1 = fmaf(bf16_hi(wv.x), hA.y, a1);
-    a0 = fmaf(bf16_lo(wv.y), hA.z, a0); a1 = fmaf(bf16_hi(wv.y), hA.w, a1);
-    a0 = fmaf(bf16_lo(wv.z), hB.x, a0); a1 = fmaf(bf16_hi(wv.z), hB.y, a1);
-    a0 = fmaf(bf16_lo(wv.w), hB.z, a0); a1 = fmaf(bf16_hi(wv.w), hB.w, a1);
-    b0 = fmaf(bf16_lo(uv.x), hA.x, b0); b1 = fmaf(bf16_hi(uv.x), hA.y, b1);
-    b0 = fmaf(bf16_lo(uv.y), hA.z, b0); b1 = fmaf(bf16_hi(uv.y), hA.w, b1);
-    b0 = fmaf(bf16_lo(uv.z), hB.x, b0); b1 = fmaf(bf16_hi(uv.z), hB.y, b1);
-    b0 = fmaf(bf16_lo(uv.w), hB.z, b0); b1 = fmaf(bf16_hi(uv.w), hB.w, b1);
+// Eight products of one 16-byte chunk of a bf16 row with the matching eight
+// fp32 inputs, into two accumulators.
+__device__ __forceinline__ void fma8(float (&acc)[2], const uint4 w, const float4 h0, const float4 h1) {
+  acc[0] = fmaf(bf16_lo(w.x), h0.x, acc[0]);
+  acc[1] = fmaf(bf16_hi(w.x), h0.y, acc[1]);
+  acc[0] = fmaf(bf16_lo(w.y), h0.z, acc[0]);
+  acc[1] = fmaf(bf16_hi(w.y), h0.w, acc[1]);
+  acc[0] = fmaf(bf16_lo(w.z), h1.x, acc[0]);
+  acc[1] = fmaf(bf16_hi(w.z), h1.y, acc[1]);
+  acc[0] = fmaf(bf16_lo(w.w), h1.z, acc[0]);
+  acc[1] = fmaf(bf16_hi(w.w), h1.w, acc[1]);
+}
+
+// Dot products of NR bf16 weight rows of a stage (and, with PAIR, of the NR
+// partner rows `rps` rows further: gate and up) with the fp32 input vector h,
+// all in shared memory.  One warp; lane l covers elements [8l + 256j, +8), so
+// every 16-byte load of h serves all NR (or 2 NR) rows.  Row indices at or past
+// `n` are clamped to the last row (their results are discarded).  Every lane
+// returns every total.
+template <int NR, bool PAIR>
+__device__ __forceinline__ void dot_group(const uint8_t* stage, int i0, int n, int rps, const float* h, int K,
+                                          int lane, float (&v)[NR], float (&u)[NR]) {
+  const uint16_t* w[NR];
+  const uint16_t* wu[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const int i = min(i0 + r, n - 1);
+    w[r] = reinterpret_cast<const uint16_t*>(stage + (size_t)i * K * 2);
+    wu[r] = reinterpret_cast<const uint16_t*>(stage + (size_t)(rps + i) * K * 2);
   }
-  dw = a0 + a1;
-  du = b0 + b1;
+  float a[NR][2], b[NR][2];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) a[r][0] = a[r][1] = b[r][0] = b[r][1] = 0.f;
+  const float* hp = h + lane * 4;  // hperm(8 lane + 256 j) = 256 j + 4 lane
+#pragma unroll 2
+  for (int e = lane * 8; e < K; e += 256, hp += 256) {
+    const float4 h0 = *reinterpret_cast<const float4*>(hp);
+    const float4 h1 = *reinterpret_cast<const float4*>(hp + 128);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      fma8(a[r], *reinterpret_cast<const uint4*>(w[r] + e), h0, h1);
+      if (PAIR) fma8(b[r], *reinterpret_cast<const uint4*>(wu[r] + e), h0, h1);
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    v[r] = warp_sum(a[r][0] + a[r][1]);
+    u[r] = PAIR ? warp_sum(b[r][0] + b[r][1]) : 0.f;
+  }
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
@@ -404,7 +456,9 @@ template <int KIND>
 __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
                           uint32_t& cstage, int cw, int lane, int worker) {
   const int ctid = cw * 32 + lane;
-  const int K = op.K, rps = op.rps, nw = op.nwarps;
+  const int K = task_k(op), rps = op.rps, nw = op.nwarps;
+  const bool split = KIND == TK_GEMV_RESID && op.ksplit > 1;
+  const int koff = task_koff(op, task);
   int grp, row0, row1;
   task_rows(op, task, grp, row0, row1);
   float* hs = sm.u.g.hs;
@@ -412,11 +466,11 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   // ---- prologue: the input vector, fp32, in shared memory.  Every global
   // load of the prologue is issued before the first use (one L2 round trip).
   const int nrows = row1 - row0;
-  const bool xs_ok = KIND == TK_GEMV_RESID && nrows <= MAX_XS;
+  const bool xs_ok = KIND == TK_GEMV_RESID && !split && nrows <= MAX_XS;
   if (KIND == TK_GEMV_RESID) {
-    // the input goes straight to shared memory (cp.async through L2), the
-    // task's residual rows through registers
-    for (int k = ctid * 4; k < K; k += CONSUMER_THREADS * 4) cp_async16(hs + k, op.a_in + k);
+    // the input (this task's segment of it) goes straight to shared memory
+    // (cp.async through L2), the task's residual rows through registers
+    for (int k = ctid * 4; k < K; k += CONSUMER_THREADS * 4) cp_async16(hs + hperm(k), op.a_in + koff + k);
     float xv[MAX_XS / CONSUMER_THREADS];
 #pragma unroll
     for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
@@ -471,8 +525,8 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
         h0.z = xr[c][2] * rinv * bf16_lo(w.y); h0.w = xr[c][3] * rinv * bf16_hi(w.y);
         h1.x = xr[c][4] * rinv * bf16_lo(w.z); h1.y = xr[c][5] * rinv * bf16_hi(w.z);
         h1.z = xr[c][6] * rinv * bf16_lo(w.w); h1.w = xr[c][7] * rinv * bf16_hi(w.w);
-        *reinterpret_cast<float4*>(hs + k) = h0;
-        *reinterpret_cast<float4*>(hs + k + 4) = h1;
+        *reinterpret_cast<float4*>(hs + hperm(k)) = h0;
+        *reinterpret_cast<float4*>(hs + hperm(k + 4)) = h1;
       }
     }
   }
@@ -490,6 +544,10 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       const int sg = seg_of(op, row);
       op.y[sg][seg_row(op, grp, sg, row)] = v;
     } else if (KIND == TK_GEMV_RESID) {
+      if (split) {
+        op.kpart[(size_t)(task % op.ksplit) * op.N + row] = v;
+        return;
+      }
       const float nx = (xs_ok ? sm.u.g.xs[j] : __ldcg(op.x_out + row)) + v;
       op.x_out[row] = nx;
       if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
@@ -504,9 +562,16 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   };
 
 
-  int jn = cw;  // next task-local row of this warp
+  // Rows of a stage go to warps in groups of RB (RB pairs for gate/up) that
+  // share each load of h; group u of the task goes to warp u % nwarps, and
+  // lane r runs the epilogue of the group's row r.
+  constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
+  constexpr int RB = PAIR ? (MPK_GEMV_RB > 1 ? MPK_GEMV_RB / 2 : 1) : MPK_GEMV_RB;
+  int un = cw;     // next task-local group of this warp
+  int ubase = 0;   // first group of the current stage
   for (int base = 0; base < nrows; base += rps) {
     const int n = min(rps, nrows - base);
+    const int ngroups = (n + RB - 1) / RB;
     const uint32_t slot = cstage % NSTAGES;
     bool ok = true;
     if (lane == 0) ok = wait_mbar(g, &sm.full[slot], (cstage / NSTAGES) & 1u, 3, worker);
@@ -518,29 +583,46 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     if (g.profiling && ctid == 0 && base == 0) sm.t_data = globaltimer();
     const uint8_t* stage = sm.ring[slot];
     if (cw < nw) {
-      int j = jn;
-      for (; j < base + n; j += nw) {
-        const int i = j - base;
-        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(stage + (size_t)i * K * 2);
-        float v, u = 0.f;
-        if (KIND == TK_NORM_GEMV_SILU) {
-          const uint16_t* urow = reinterpret_cast<const uint16_t*>(stage + (size_t)(rps + i) * K * 2);
-          dot_row2(wrow, urow, hs, K, lane, v, u);
-          u = warp_sum(u);
-        } else {
-          v = dot_row(wrow, hs, K, lane);
-        }
-        v = warp_sum(v);
-        if (lane == 0) finish(j, v, u);
+      for (; un < ubase + ngroups; un += nw) {
+        const int i0 = (un - ubase) * RB;
+        float v[RB], u[RB];
+        dot_group<RB, PAIR>(stage, i0, n, rps, hs, K, lane, v, u);
+#pragma unroll
+        for (int r = 0; r < RB; ++r)
+          if (lane == r && i0 + r < n) finish(base + i0 + r, v[r], u[r]);
       }
-      jn = j;
     }
+    ubase += ngroups;
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[slot]);
     ++cstage;
   }
+  if (KIND == TK_NORM_GEMV_ARGMAX) best = warp_max_u64(best);
   if (KIND == TK_NORM_GEMV_ARGMAX && lane == 0) sm.bestk[cw] = best;
   if (consumer_sync_or(fail)) return false;
+
+  if (split) {
+    // The last segment task of this row block to finish adds the partial sums
+    // to the residual, in segment order.
+    if (ctid == 0) {
+      __threadfence();
+      const uint32_t old = atomicAdd(op.blk_cnt + task / op.ksplit, 1u);
+      sm.last = ((old + 1u) % (uint32_t)op.ksplit) == 0u;
+    }
+    consumer_sync();
+    if (sm.last) {
+      __threadfence();
+      for (int j = ctid; j < nrows; j += CONSUMER_THREADS) {
+        const int row = row0 + j;
+        float sum = __ldcg(op.kpart + row);
+        for (int k = 1; k < op.ksplit; ++k) sum += __ldcg(op.kpart + (size_t)k * op.N + row);
+        const float nx = __ldcg(op.x_out + row) + sum;
+        op.x_out[row] = nx;
+        if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
+          g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
+      }
+    }
+  }
 
   if (KIND == TK_QKV_ATTN) {
     // The last projection task of this kv head's group runs its attention.
@@ -1063,11 +1145,13 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_ke
   const int worker = blockIdx.x - g.sched_ctas;
   if (threadIdx.x == 0) init_barriers(sm);
   __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) producer_loop<false>(sm, g, worker, 0, 0);
+  if (warp < PRODUCER_WARPS) {
+    regs_dec<PRODUCER_REGS>();
+    if (warp == 0 && lane == 0) producer_loop<false>(sm, g, worker, 0, 0);
     return;
   }
-  consumer_loop<false>(sm, g, worker, warp - 1, lane);
+  regs_inc<CONSUMER_REGS>();
+  consumer_loop<false>(sm, g, worker, warp - PRODUCER_WARPS, lane);
 }
 
 // One operation of one iteration as an ordinary launch: block b runs task b.
@@ -1077,11 +1161,13 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_kernel(con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) init_barriers(sm);
   __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) producer_loop<true>(sm, g, blockIdx.x, iter, op);
+  if (warp < PRODUCER_WARPS) {
+    regs_dec<PRODUCER_REGS>();
+    if (warp == 0 && lane == 0) producer_loop<true>(sm, g, blockIdx.x, iter, op);
     return;
   }
-  consumer_loop<true>(sm, g, blockIdx.x, warp - 1, lane);
+  regs_inc<CONSUMER_REGS>();
+  consumer_loop<true>(sm, g, blockIdx.x, warp - PRODUCER_WARPS, lane);
 }
 
 // ------------------------------------------------------------------ host-side launch helpers

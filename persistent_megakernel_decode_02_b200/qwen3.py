@@ -14,10 +14,21 @@ from typing import Dict, List, Optional
 
 import torch
 
+from . import _lib
 from .kernel import PersistentKernel
 
 
 FUSED_ATTENTION_MAX_SEQ = 4096
+
+
+def reduction_split(K: int, max_k: int = _lib.MAX_GEMV_K) -> int:
+    """Segments a residual projection of reduction length K is split into (the
+    rule of MPK_OP_LINEAR_RESIDUAL): the fewest equal segments of at most max_k
+    whose length is a multiple of 256."""
+    ks = -(-K // max_k)
+    while ks <= K // 256 and (K % ks or (K // ks) % 256):
+        ks += 1
+    return ks
 
 
 def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
@@ -57,7 +68,8 @@ def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_ta
                          weight_up=p + "up_proj", output="a", grid_dim=min(gt, s.intermediate), block_dim=block_dim,
                          eps=s.eps))
         plan.append(dict(method="linear_residual_layer", input="a", weight=p + "down_proj", residual="x",
-                         grid_dim=min(gt, s.hidden), block_dim=block_dim, capture_slot=l + 1))
+                         grid_dim=min(gt, s.hidden * reduction_split(s.intermediate)), block_dim=block_dim,
+                         capture_slot=l + 1))
     plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
                      weight_lm="embed_tokens" if tied else "lm_head", pred="pred", grid_dim=min(gt, s.vocab),
                      block_dim=block_dim, eps=s.eps))

@@ -77,6 +77,15 @@ def test_layer_plan_fused_attention():
                                                 "rmsnorm_linear_silu_mul_layer", "linear_residual_layer"]
 
 
+def test_reduction_split_rule():
+    from persistent_megakernel_decode_02_b200.qwen3 import reduction_split
+    txt = open(os.path.join(ROOT, "include", "mpk.h")).read()
+    assert int(re.search(r"#define MPK_MAX_GEMV_K (\d+)", txt).group(1)) == _lib.MAX_GEMV_K
+    assert [reduction_split(k) for k in (256, 3072, 4096, 4352, 8192, 12288, 17408)] == [1, 1, 1, 17, 2, 3, 17]
+    plan = layer_plan(sq.QWEN3_8B, requests=1, num_workers=144, attn_chunks=9)
+    assert plan[5]["grid_dim"] == 144 and plan[5]["weight"].endswith("down_proj")
+
+
 def test_default_attention_chunks():
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 551) == 9
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 32897) == 18
