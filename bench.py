@@ -478,7 +478,9 @@ def timeline_summary(tl, shape) -> dict:
     """Per operation kind, means over tasks (us): wait = popped -> dependency met,
     pro = dependency met -> prologue done, data = prologue done -> first weight
     stage ready, lead = first stage issued -> dependency met (how early the
-    producer started on the task's weights), work = dependency met -> done;
+    producer started on the task's weights), work = dependency met -> done,
+    stall = time the consumers waited for weight stages, tail = last stage
+    ready -> done;
     span = first dependency met -> last task done of the operation, gap = last
     task of the previous operation done -> first dependency met here."""
     import collections
@@ -500,7 +502,7 @@ def timeline_summary(tl, shape) -> dict:
         end1 = max(r[4] for r in rows)
         a = acc[k]
         for r in rows:
-            _, _, tp, tr, te, tpro, tdat, tiss = r
+            _, _, tp, tr, te, tpro, tdat, tiss, tstall, tlast, tloop = r
             a["wait"].append((tr - tp) / 1e3)
             a["work"].append((te - tr) / 1e3)
             if tpro:
@@ -509,6 +511,9 @@ def timeline_summary(tl, shape) -> dict:
                 a["data"].append((max(tdat, tpro) - tpro) / 1e3)
             if tiss:
                 a["lead"].append((tr - tiss) / 1e3)
+            if tlast:
+                a["stall"].append(tstall / 1e3)
+                a["tail"].append((te - tlast) / 1e3)
         a["span"].append((end1 - ready0) / 1e3)
         if prev_end is not None and it > first_it:
             a["gap"].append((ready0 - prev_end) / 1e3)
@@ -533,7 +538,11 @@ def write_chrome_trace(tl, dec, path):
         entry, worker, ts, tr, te = rec[:5]
         it, op, task = (entry >> 32) & 0xFFFFFFFF, (entry >> 16) & 0xFFFF, entry & 0xFFFF
         ev.append({"name": f"op{op}", "ph": "X", "pid": 0, "tid": int(worker), "ts": (ts - t0) / 1e3,
-                   "dur": max(te - ts, 0) / 1e3, "args": {"iter": it, "task": task, "wait_us": (tr - ts) / 1e3}})
+                   "dur": max(te - ts, 0) / 1e3,
+                   "args": {"iter": it, "task": task, "wait_us": (tr - ts) / 1e3,
+                            "pro_us": (rec[5] - tr) / 1e3 if rec[5] else 0.0, "stall_us": rec[8] / 1e3,
+                            "tail_us": (te - rec[9]) / 1e3 if rec[9] else 0.0,
+                            "rows_done_us": (rec[10] - tr) / 1e3 if rec[10] else 0.0}})
     with open(path, "w") as f:
         json.dump({"traceEvents": ev}, f)
 

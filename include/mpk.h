@@ -267,10 +267,14 @@ MPK_API int mpk_status(mpk_ctx *ctx);
 MPK_API int mpk_request_abort(mpk_ctx *ctx);
 
 /* Number of timeline records of the last profiled run, and a copy of up to
- * `cap` of them into host memory `out` (8 x uint64 each, %globaltimer ns):
- * packed task id (iter<<32 | op<<16 | task), worker, task popped, dependency
- * met, task done, prologue done (0 if none), first weight stage ready (0 if
- * none), first weight stage issued by the producer (0 if none). */
+ * `cap` of them into host memory `out` (MPK_TIMELINE_FIELDS x uint64 each,
+ * %globaltimer ns): packed task id (iter<<32 | op<<16 | task), worker, task
+ * popped, dependency met, task done, prologue done (0 if none), first weight
+ * stage ready (0 if none), first weight stage issued by the producer (0 if
+ * none), total time the task waited for weight stages (a duration), last
+ * weight stage ready (0 if none), every consumer warp done with its weight
+ * rows (0 if none). */
+#define MPK_TIMELINE_FIELDS 11
 MPK_API int mpk_timeline(mpk_ctx *ctx, uint64_t *out, int cap);
 
 /*

@@ -22,9 +22,6 @@ static_assert(PRODUCER_WARPS * 32 * PRODUCER_REGS + CONSUMER_THREADS * CONSUMER_
 #ifndef MPK_STAGE_BYTES
 #define MPK_STAGE_BYTES 32768
 #endif
-#ifndef MPK_GEMV_RB
-#define MPK_GEMV_RB 1   // weight rows per warp sharing each load of the input vector
-#endif
 #ifndef MPK_NSTAGES
 #define MPK_NSTAGES 6
 #endif
@@ -148,7 +145,10 @@ struct Graph {
   uint32_t* timeline_n;
 };
 
-constexpr int TIMELINE_FIELDS = 8;  // entry, worker, popped, dependency met, end, prologue done, first stage ready, first stage issued
+// entry, worker, popped, dependency met, end, prologue done, first stage ready,
+// first stage issued, time spent waiting for weight stages, last stage ready,
+// rows done
+constexpr int TIMELINE_FIELDS = MPK_TIMELINE_FIELDS;
 constexpr int EVENT_STRIDE = 32;    // uint32 per event / queue counter (128 bytes)
 constexpr unsigned long long QUEUE_TERMINATE = ~0ull;
 

@@ -64,6 +64,8 @@ struct __align__(128) Smem {
   unsigned long long cur_entry;
   unsigned long long fifo_t[TASK_FIFO];          // profiling: first weight stage issued
   unsigned long long t_pro, t_data;              // profiling: prologue done, first stage ready
+  unsigned long long t_stall, t_last;            // profiling: time waited for stages, last stage ready
+  unsigned long long t_loop;                     // profiling: every consumer warp done with its rows
   int32_t last;     // last-arrival flag
 };
 
@@ -562,11 +564,11 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   };
 
 
-  // Rows of a stage go to warps in groups of RB (RB pairs for gate/up) that
-  // share each load of h; group u of the task goes to warp u % nwarps, and
-  // lane r runs the epilogue of the group's row r.
+  // Each warp owns whole rows: task row j goes to warp j % nwarps (rows per
+  // warp group RB = 1; several rows per warp sharing the loads of h measured
+  // slower, the stage's rows then wait on fewer warps).
   constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
-  constexpr int RB = PAIR ? (MPK_GEMV_RB > 1 ? MPK_GEMV_RB / 2 : 1) : MPK_GEMV_RB;
+  constexpr int RB = 1;
   int un = cw;     // next task-local group of this warp
   int ubase = 0;   // first group of the current stage
   for (int base = 0; base < nrows; base += rps) {
@@ -574,13 +576,21 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     const int ngroups = (n + RB - 1) / RB;
     const uint32_t slot = cstage % NSTAGES;
     bool ok = true;
-    if (lane == 0) ok = wait_mbar(g, &sm.full[slot], (cstage / NSTAGES) & 1u, 3, worker);
+    if (lane == 0) {
+      const uint64_t w0 = (g.profiling && ctid == 0) ? globaltimer() : 0ull;
+      ok = wait_mbar(g, &sm.full[slot], (cstage / NSTAGES) & 1u, 3, worker);
+      if (g.profiling && ctid == 0) {
+        const uint64_t w1 = globaltimer();
+        sm.t_stall += w1 - w0;
+        sm.t_last = w1;
+        if (base == 0) sm.t_data = w1;
+      }
+    }
     ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
     if (!ok) {
       fail = true;
       break;
     }
-    if (g.profiling && ctid == 0 && base == 0) sm.t_data = globaltimer();
     const uint8_t* stage = sm.ring[slot];
     if (cw < nw) {
       for (; un < ubase + ngroups; un += nw) {
@@ -600,6 +610,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   if (KIND == TK_NORM_GEMV_ARGMAX) best = warp_max_u64(best);
   if (KIND == TK_NORM_GEMV_ARGMAX && lane == 0) sm.bestk[cw] = best;
   if (consumer_sync_or(fail)) return false;
+  if (g.profiling && ctid == 0) sm.t_loop = globaltimer();
 
   if (split) {
     // The last segment task of this row block to finish adds the partial sums
@@ -996,6 +1007,9 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
       t_start = globaltimer();
       sm.t_pro = 0ull;
       sm.t_data = 0ull;
+      sm.t_stall = 0ull;
+      sm.t_last = 0ull;
+      sm.t_loop = 0ull;
     }
     // dependency: the event of the op this one follows
     if (!kStandalone && ctid == 0) {
@@ -1044,6 +1058,9 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
           rec[5] = sm.t_pro;
           rec[6] = sm.t_data;
           rec[7] = atomicAdd(&sm.fifo_t[(fpos - 1) % TASK_FIFO], 0ull);
+          rec[8] = sm.t_stall;
+          rec[9] = sm.t_last;
+          rec[10] = sm.t_loop;
         }
       }
     }

@@ -250,10 +250,11 @@ class PersistentKernel:
     def request_abort(self) -> None:
         check(self._lib.mpk_request_abort(self._ctx), self._ctx)
 
-    TIMELINE_FIELDS = ("entry", "worker", "popped", "ready", "end", "prologue", "first_data", "first_issue")
+    TIMELINE_FIELDS = ("entry", "worker", "popped", "ready", "end", "prologue", "first_data", "first_issue",
+                       "stage_wait", "last_data", "rows_done")
 
     def timeline(self) -> torch.Tensor:
-        """[n, 8] records (see TIMELINE_FIELDS; times in %globaltimer ns)."""
+        """[n, 11] records (see TIMELINE_FIELDS; times in %globaltimer ns, stage_wait a duration in ns)."""
         n = int(self._lib.mpk_timeline(self._ctx, None, 0))
         out = torch.zeros((max(n, 0), len(self.TIMELINE_FIELDS)), dtype=torch.int64)
         if n > 0:
