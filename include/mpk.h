@@ -60,7 +60,14 @@ typedef enum {
     MPK_ERR_DEVICE = -11      /* device-side consistency check failed            */
 } mpk_error;
 
-typedef enum { MPK_BF16 = 0, MPK_FP32 = 1, MPK_INT32 = 2, MPK_INT64 = 3 } mpk_dtype;
+/* MPK_FP32T, the activations passed between operations: 8 bytes per element,
+ * the fp32 value in the low 32 bits and a version tag in the high 32 bits.  A
+ * writer stores value and tag in one 8-byte store; a reader waits until the
+ * element carries the tag of the write it needs, so no flag or fence is needed
+ * between producing and consuming operations.  Tag of a write by operation p
+ * in iteration n of a run (n counted from 0): n * num_operations + p + 1; the
+ * library zeroes every MPK_FP32T tensor at the start of each run. */
+typedef enum { MPK_BF16 = 0, MPK_FP32 = 1, MPK_INT32 = 2, MPK_INT64 = 3, MPK_FP32T = 4 } mpk_dtype;
 
 /* Memory category of a library-allocated tensor ([EN] "The API"; [ZH]
  * "关键 API 与张量管理"): CUDA memory of this GPU, or NVSHMEM symmetric memory
@@ -156,8 +163,9 @@ typedef struct {
     int32_t prefetch_kb;    /* L2 prefetch distance per worker ahead of the shared-memory
                                weight ring, KiB (<=0: off)                                 */
     int32_t debug_stall_op; /* fault injection for tests: k > 0 makes operation k-1 wait
-                               for one more completion per iteration than its dependency
-                               delivers, so that wait runs out and the run ends with
+                               for an input nothing will produce (a version of the next
+                               iteration, or one completion more than its dependency
+                               delivers), so that wait runs out and the run ends with
                                MPK_ERR_TIMEOUT (0: off)                                    */
 } mpk_options;
 

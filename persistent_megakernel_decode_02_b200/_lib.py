@@ -19,7 +19,7 @@ ERRORS = {
 }
 ERR_CODE = {v: k for k, v in ERRORS.items()}
 
-BF16, FP32, INT32, INT64 = 0, 1, 2, 3
+BF16, FP32, INT32, INT64, FP32T = 0, 1, 2, 3, 4
 IO_CUDA, IO_NVSHMEM = 0, 1
 OP_EMBED, OP_RMSNORM_LINEAR, OP_ATTENTION, OP_LINEAR_RESIDUAL = 1, 2, 3, 4
 OP_RMSNORM_LINEAR_SILU_MUL, OP_RMSNORM_LMHEAD_ARGMAX, OP_RMSNORM_QKV_ATTENTION = 5, 6, 7

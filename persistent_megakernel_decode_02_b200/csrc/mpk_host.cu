@@ -39,6 +39,7 @@ size_t dtype_size(mpk_dtype t) {
     case MPK_FP32: return 4;
     case MPK_INT32: return 4;
     case MPK_INT64: return 8;
+    case MPK_FP32T: return 8;
   }
   return 0;
 }
@@ -49,6 +50,7 @@ const char* dtype_name(mpk_dtype t) {
     case MPK_FP32: return "fp32";
     case MPK_INT32: return "int32";
     case MPK_INT64: return "int64";
+    case MPK_FP32T: return "fp32t";
   }
   return "?";
 }
@@ -73,6 +75,7 @@ struct mpk_ctx {
   int32_t R = 0, S_cache = 0, V = 0, H = 0, L = 0;
   int32_t pred_S = 0;
   std::string err, warnings;
+  std::vector<std::pair<void*, size_t>> zero_each_run;  // tagged activations: versions restart at every run
   int capture_iter = -1;
   float* cap_logits = nullptr;
   float* cap_hidden = nullptr;
@@ -257,7 +260,7 @@ static int register_tensor(mpk_ctx* c, const char* name, void* ptr, mpk_dtype dt
   if (!name || !*name) return fail(c, MPK_ERR_INVALID_ARG, "tensor name is empty");
   if (c->compiled) return fail(c, MPK_ERR_STATE, "tensors cannot be added after compile");
   if (ndim < 1 || ndim > 5 || !dims) return fail(c, MPK_ERR_INVALID_ARG, "'%s': rank must be 1..5", name);
-  if ((int)dtype < 0 || (int)dtype > 3) return fail(c, MPK_ERR_INVALID_ARG, "'%s': unknown dtype %d", name, (int)dtype);
+  if ((int)dtype < 0 || (int)dtype > 4) return fail(c, MPK_ERR_INVALID_ARG, "'%s': unknown dtype %d", name, (int)dtype);
   if (c->tensors.count(name)) return fail(c, MPK_ERR_INVALID_ARG, "tensor '%s' already registered", name);
   Tensor t;
   for (int i = 0; i < ndim; ++i) {
@@ -288,7 +291,7 @@ int mpk_new_tensor(mpk_ctx* c, const char* name, mpk_dtype dtype, int ndim, cons
     return fail(c, MPK_ERR_UNSUPPORTED, "'%s': nvshmem_tensor is for remote GPU access; this build runs on one GPU",
                 name ? name : "");
   if (io != MPK_IO_CUDA) return fail(c, MPK_ERR_INVALID_ARG, "unknown io category %d", (int)io);
-  if ((int)dtype < 0 || (int)dtype > 3) return fail(c, MPK_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if ((int)dtype < 0 || (int)dtype > 4) return fail(c, MPK_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   if (ndim < 1 || ndim > 5 || !dims) return fail(c, MPK_ERR_INVALID_ARG, "rank must be 1..5");
   int64_t n = 1;
   for (int i = 0; i < ndim; ++i) {
@@ -362,7 +365,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       case MPK_OP_EMBED: {
         op.kind = TK_EMBED;
         NEED("weights[0] (embedding)", Ly.weights[0], MPK_BF16, 2, &w0);
-        NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32, 2, &out);
+        NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32T, 2, &out);
         SHAPE_CHECK(out->dims[1] == w0->dims[1], "layer %d: x width %lld != embedding width %lld", li,
                     (long long)out->dims[1], (long long)w0->dims[1]);
         SHAPE_CHECK(out->dims[1] % 8 == 0, "layer %d: hidden size must be a multiple of 8", li);
@@ -370,7 +373,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         SHAPE_CHECK(out->dims[0] == R, "layer %d: request count mismatch", li);
         SHAPE_CHECK(ntasks == R, "layer %d: EMBED needs grid_dim = number of requests (%d)", li, R);
         op.table = (const uint16_t*)w0->ptr;
-        op.x_out = (float*)out->ptr;
+        op.x_out = (uint64_t*)out->ptr;
         op.N = (int)out->dims[1];
         if (V < 0) V = (int)w0->dims[0];
         if (H < 0) H = op.N;
@@ -387,11 +390,11 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         const bool lmh = Ly.op == MPK_OP_RMSNORM_LMHEAD_ARGMAX;
         op.kind = resid ? TK_GEMV_RESID : silu ? TK_NORM_GEMV_SILU : lmh ? TK_NORM_GEMV_ARGMAX : TK_NORM_GEMV;
         if (resid) {
-          NEED("inputs[0] (a)", Ly.inputs[0], MPK_FP32, 2, &x);
-          op.a_in = (const float*)x->ptr;
+          NEED("inputs[0] (a)", Ly.inputs[0], MPK_FP32T, 2, &x);
+          op.a_in = (const uint64_t*)x->ptr;
           op.K = (int)x->dims[1];
           NEED("weights[0] (W)", Ly.weights[0], MPK_BF16, 2, &w0);
-          NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32, 2, &out);
+          NEED("outputs[0] (x)", Ly.outputs[0], MPK_FP32T, 2, &out);
           SHAPE_CHECK(w0->dims[1] == op.K, "layer %d: W is %s but input has %d features", li,
                       dims_str(w0->dims).c_str(), op.K);
           SHAPE_CHECK(out->dims[1] == w0->dims[0] && out->dims[0] == x->dims[0],
@@ -402,8 +405,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
           op.nseg = 1;
           op.seg_row0[0] = 0;
           op.seg_row0[1] = op.N;
-          op.x_out = (float*)out->ptr;
-          op.x = (const float*)out->ptr;
+          op.x_out = (uint64_t*)out->ptr;
+          op.x = (const uint64_t*)out->ptr;
           if (op.K > MAX_K) {
             // Split the reduction into the fewest segments that fit the input
             // buffer; task t computes segment t % ksplit of row block t / ksplit.
@@ -421,8 +424,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
             blk_u32 = std::max(blk_u32, (size_t)(ntasks / ks));
           }
         } else {
-          NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32, 2, &x);
-          op.x = (const float*)x->ptr;
+          NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32T, 2, &x);
+          op.x = (const uint64_t*)x->ptr;
           op.K = (int)x->dims[1];
           NEED("weights[0] (norm)", Ly.weights[0], MPK_BF16, 1, &w0);
           SHAPE_CHECK(w0->dims[0] == op.K, "layer %d: norm weight %s, input width %d", li, dims_str(w0->dims).c_str(),
@@ -431,7 +434,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
           if (silu) {
             NEED("weights[1] (gate)", Ly.weights[1], MPK_BF16, 2, &w1);
             NEED("weights[2] (up)", Ly.weights[2], MPK_BF16, 2, &w2);
-            NEED("outputs[0] (a)", Ly.outputs[0], MPK_FP32, 2, &out);
+            NEED("outputs[0] (a)", Ly.outputs[0], MPK_FP32T, 2, &out);
             SHAPE_CHECK(w1->dims == w2->dims && w1->dims[1] == op.K, "layer %d: gate %s / up %s vs K=%d", li,
                         dims_str(w1->dims).c_str(), dims_str(w2->dims).c_str(), op.K);
             SHAPE_CHECK(out->dims[1] == w1->dims[0] && out->dims[0] == x->dims[0], "layer %d: output %s", li,
@@ -442,7 +445,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
             op.nseg = 1;
             op.seg_row0[0] = 0;
             op.seg_row0[1] = op.N;
-            op.a_out = (float*)out->ptr;
+            op.a_out = (uint64_t*)out->ptr;
           } else if (lmh) {
             NEED("weights[1] (lm head)", Ly.weights[1], MPK_BF16, 2, &w1);
             SHAPE_CHECK(w1->dims[1] == op.K, "layer %d: LM head %s vs K=%d", li, dims_str(w1->dims).c_str(), op.K);
@@ -469,12 +472,12 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
               const Tensor *ws, *ys;
               NEED("weights[1+i] (linear)", Ly.weights[1 + s], MPK_BF16, 2, &ws);
               if (!Ly.outputs[s]) return fail(c, MPK_ERR_INVALID_ARG, "layer %d: outputs[%d] missing", li, s);
-              NEED("outputs[i]", Ly.outputs[s], MPK_FP32, 2, &ys);
+              NEED("outputs[i]", Ly.outputs[s], MPK_FP32T, 2, &ys);
               SHAPE_CHECK(ws->dims[1] == op.K && ys->dims[1] == ws->dims[0] && ys->dims[0] == x->dims[0],
                           "layer %d: linear %d W %s, y %s, K=%d", li, s, dims_str(ws->dims).c_str(),
                           dims_str(ys->dims).c_str(), op.K);
               op.W[s] = (const uint16_t*)ws->ptr;
-              op.y[s] = (float*)ys->ptr;
+              op.y[s] = (uint64_t*)ys->ptr;
               op.seg_row0[s] = rows;
               rows += (int)ws->dims[0];
               op.nseg = s + 1;
@@ -503,14 +506,14 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       case MPK_OP_ATTENTION: {
         op.kind = TK_ATTN;
         const Tensor *q, *k, *v, *qn, *kn, *kc, *vc, *o;
-        NEED("inputs[0] (q)", Ly.inputs[0], MPK_FP32, 2, &q);
-        NEED("inputs[1] (k)", Ly.inputs[1], MPK_FP32, 2, &k);
-        NEED("inputs[2] (v)", Ly.inputs[2], MPK_FP32, 2, &v);
+        NEED("inputs[0] (q)", Ly.inputs[0], MPK_FP32T, 2, &q);
+        NEED("inputs[1] (k)", Ly.inputs[1], MPK_FP32T, 2, &k);
+        NEED("inputs[2] (v)", Ly.inputs[2], MPK_FP32T, 2, &v);
         NEED("weights[0] (q_norm)", Ly.weights[0], MPK_BF16, 1, &qn);
         NEED("weights[1] (k_norm)", Ly.weights[1], MPK_BF16, 1, &kn);
         NEED("weights[2] (k_cache)", Ly.weights[2], MPK_BF16, 5, &kc);
         NEED("weights[3] (v_cache)", Ly.weights[3], MPK_BF16, 5, &vc);
-        NEED("outputs[0] (o)", Ly.outputs[0], MPK_FP32, 2, &o);
+        NEED("outputs[0] (o)", Ly.outputs[0], MPK_FP32T, 2, &o);
         SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
         const int d = (int)kc->dims[4], Hkv = (int)kc->dims[2];
         SHAPE_CHECK(qn->dims[0] == d && kn->dims[0] == d, "layer %d: norm weights must have head_dim %d", li, d);
@@ -537,10 +540,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.L = (int)kc->dims[0];
         op.S = (int)kc->dims[3];
         op.layer = Ly.layer;
-        op.q = (const float*)q->ptr; op.k = (const float*)k->ptr; op.v = (const float*)v->ptr;
+        op.q = (const uint64_t*)q->ptr; op.k = (const uint64_t*)k->ptr; op.v = (const uint64_t*)v->ptr;
         op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
         op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
-        op.a_out = (float*)o->ptr;
+        op.a_out = (uint64_t*)o->ptr;
         op.N = Hq * d;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
         part_floats = std::max(part_floats, (size_t)R * Hq * gy * (d + 2));
@@ -562,7 +565,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       case MPK_OP_RMSNORM_QKV_ATTENTION: {
         op.kind = TK_QKV_ATTN;
         const Tensor *x, *wn, *wq, *wk, *wv, *qn, *kn, *kc, *vc, *q, *k, *v, *o;
-        NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32, 2, &x);
+        NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32T, 2, &x);
         NEED("weights[0] (norm)", Ly.weights[0], MPK_BF16, 1, &wn);
         NEED("weights[1] (Wq)", Ly.weights[1], MPK_BF16, 2, &wq);
         NEED("weights[2] (Wk)", Ly.weights[2], MPK_BF16, 2, &wk);
@@ -571,10 +574,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         NEED("weights[5] (k_norm)", Ly.weights[5], MPK_BF16, 1, &kn);
         NEED("weights[6] (k_cache)", Ly.weights[6], MPK_BF16, 5, &kc);
         NEED("weights[7] (v_cache)", Ly.weights[7], MPK_BF16, 5, &vc);
-        NEED("outputs[0] (q)", Ly.outputs[0], MPK_FP32, 2, &q);
-        NEED("outputs[1] (k)", Ly.outputs[1], MPK_FP32, 2, &k);
-        NEED("outputs[2] (v)", Ly.outputs[2], MPK_FP32, 2, &v);
-        NEED("outputs[3] (o)", Ly.outputs[3], MPK_FP32, 2, &o);
+        NEED("outputs[0] (q)", Ly.outputs[0], MPK_FP32T, 2, &q);
+        NEED("outputs[1] (k)", Ly.outputs[1], MPK_FP32T, 2, &k);
+        NEED("outputs[2] (v)", Ly.outputs[2], MPK_FP32T, 2, &v);
+        NEED("outputs[3] (o)", Ly.outputs[3], MPK_FP32T, 2, &o);
         op.K = (int)x->dims[1];
         SHAPE_CHECK(wn->dims[0] == op.K, "layer %d: norm weight %s, input width %d", li, dims_str(wn->dims).c_str(), op.K);
         SHAPE_CHECK(kc->dims == vc->dims, "layer %d: k/v caches differ", li);
@@ -622,10 +625,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.W[0] = (const uint16_t*)wq->ptr;
         op.W[1] = (const uint16_t*)wk->ptr;
         op.W[2] = (const uint16_t*)wv->ptr;
-        op.y[0] = (float*)q->ptr;
-        op.y[1] = (float*)k->ptr;
-        op.y[2] = (float*)v->ptr;
-        op.x = (const float*)x->ptr;
+        op.y[0] = (uint64_t*)q->ptr;
+        op.y[1] = (uint64_t*)k->ptr;
+        op.y[2] = (uint64_t*)v->ptr;
+        op.x = (const uint64_t*)x->ptr;
         op.norm_w = (const uint16_t*)wn->ptr;
         op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = 1;
         op.L = (int)kc->dims[0];
@@ -634,7 +637,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.q = op.y[0]; op.k = op.y[1]; op.v = op.y[2];
         op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
         op.kc = (uint16_t*)kc->ptr; op.vc = (uint16_t*)vc->ptr;
-        op.a_out = (float*)o->ptr;
+        op.a_out = (uint64_t*)o->ptr;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
         merge_off[li] = {1, merge_u32};
         merge_u32 += (size_t)R * Hkv;
@@ -666,6 +669,73 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   // events: op p signals event p; op p waits on event p-1 (op 0 on the last op,
   // one iteration behind).
   const int P = n_layers;
+
+  // versions: for every tagged input, the operation that last wrote it earlier
+  // in the iteration (a reader waits for that writer's tag)
+  {
+    std::map<const void*, int> writer;
+    auto wr = [&](const void* b) {
+      auto it = writer.find(b);
+      return it == writer.end() ? -1 : it->second;
+    };
+    for (int p = 0; p < P; ++p) {
+      OpDesc& op = ops[p];
+      op.self = p;
+      op.x_writer = -1;
+      op.a_writer = -1;
+      op.tagged = op.kind == TK_EMBED ? 0 : 1;
+      switch (op.kind) {
+        case TK_NORM_GEMV:
+        case TK_NORM_GEMV_SILU:
+        case TK_NORM_GEMV_ARGMAX:
+        case TK_QKV_ATTN:
+          op.x_writer = wr(op.x);
+          if (op.kind == TK_QKV_ATTN) op.a_writer = p;
+          break;
+        case TK_GEMV_RESID:
+          op.x_writer = wr(op.x_out);
+          op.a_writer = wr(op.a_in);
+          if (op.a_writer < 0)
+            return fail(c, MPK_ERR_INVALID_ARG, "layer %d: its input is not written by an earlier operation", p);
+          break;
+        case TK_ATTN:
+          op.a_writer = wr(op.q);
+          if (op.a_writer < 0 || wr(op.k) != op.a_writer || wr(op.v) != op.a_writer)
+            return fail(c, MPK_ERR_INVALID_ARG, "layer %d: q, k and v must come from one earlier operation", p);
+          break;
+        default:
+          break;
+      }
+      if (op.kind != TK_EMBED && op.kind != TK_ATTN && op.x_writer < 0)
+        return fail(c, MPK_ERR_INVALID_ARG, "layer %d: its x is not written by an earlier operation", p);
+      switch (op.kind) {
+        case TK_EMBED:
+        case TK_GEMV_RESID:
+          writer[op.x_out] = p;
+          break;
+        case TK_NORM_GEMV:
+          for (int sg = 0; sg < op.nseg; ++sg) writer[op.y[sg]] = p;
+          break;
+        case TK_QKV_ATTN:
+          for (int sg = 0; sg < 3; ++sg) writer[op.y[sg]] = p;
+          writer[op.a_out] = p;
+          break;
+        case TK_NORM_GEMV_SILU:
+        case TK_ATTN:
+          writer[op.a_out] = p;
+          break;
+        default:
+          break;
+      }
+    }
+  }
+  c->zero_each_run.clear();
+  for (auto& kv : c->tensors)
+    if (kv.second.dtype == MPK_FP32T) {
+      size_t n = 1;
+      for (int64_t d : kv.second.dims) n *= (size_t)d;
+      c->zero_each_run.push_back({kv.second.ptr, n * 8});
+    }
   for (int p = 0; p < P; ++p) {
     ops[p].out_event = p;
     const int dp = (p + P - 1) % P;
@@ -677,9 +747,15 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     const int p = o.debug_stall_op - 1;
     if (p >= P)
       return fail(c, MPK_ERR_INVALID_ARG, "debug_stall_op %d beyond the %d operations", o.debug_stall_op, P);
-    // one more completion per iteration than the dependency ever delivers
-    ops[p].dep_trigger += 1;
-    ops[p].dep_iter_offset = 1;
+    if (ops[p].tagged) {
+      // wait for the versions of the next iteration, which only this op's own
+      // completion could lead to
+      ops[p].tag_skew = (uint32_t)P;
+    } else {
+      // one more completion per iteration than the dependency ever delivers
+      ops[p].dep_trigger += 1;
+      ops[p].dep_iter_offset = 1;
+    }
   }
 
   // ---- workspace
@@ -709,9 +785,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   float* part = nullptr;
   rc = alloc(c, &part, sizeof(float) * (part_floats ? part_floats : 1));
   if (rc != MPK_OK) return rc;
-  float* kpart = nullptr;
-  rc = alloc(c, &kpart, sizeof(float) * (kpart_floats ? kpart_floats : 1));
+  uint64_t* kpart = nullptr;
+  rc = alloc(c, &kpart, sizeof(uint64_t) * (kpart_floats ? kpart_floats : 1));
   if (rc != MPK_OK) return rc;
+  c->zero_each_run.push_back({kpart, sizeof(uint64_t) * (kpart_floats ? kpart_floats : 1)});
   std::vector<float2*> rope_dev(rope_keys.size(), nullptr);
   for (size_t i = 0; i < rope_keys.size(); ++i) {
     const RopeKey& k = rope_keys[i];
@@ -813,6 +890,7 @@ static int prepare_run(mpk_ctx* c, int32_t* step, int64_t* tokens, const int32_t
   g.cap_logits = c->cap_logits;
   g.cap_hidden = c->cap_hidden;
   CUDA_OR_FAIL(c, cudaMemsetAsync(c->sync_block, 0, c->sync_bytes, s));
+  for (const auto& z : c->zero_each_run) CUDA_OR_FAIL(c, cudaMemsetAsync(z.first, 0, z.second, s));
   return MPK_OK;
 }
 
@@ -869,8 +947,9 @@ int mpk_status(mpk_ctx* c) {
   if (st.code == 0) return MPK_OK;
   static const char* where[] = {"?", "worker dependency wait", "producer queue wait", "weight ring wait",
                                 "task fifo wait", "scheduler gate wait", "scheduler queue space wait", "start",
-                                "embedding token check", "task dispatch", "iteration boundary"};
-  const char* w = (st.where >= 0 && st.where < 11) ? where[st.where] : "?";
+                                "embedding token check", "task dispatch", "iteration boundary",
+                                "tagged input wait"};
+  const char* w = (st.where >= 0 && st.where < 12) ? where[st.where] : "?";
   fail(c, st.code, "device status %d at %s: op %d task %d worker %d iter %d observed %u expected %u", st.code, w, st.op,
        st.task, st.worker, st.iter, st.observed, st.expected);
   return st.code;

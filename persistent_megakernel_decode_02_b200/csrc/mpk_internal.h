@@ -66,23 +66,23 @@ struct OpDesc {
   uint32_t* grp_cnt;       // QKV+attention: finished tasks per (request, group)
   int32_t ksplit;          // RESID: reduction split into ksplit segments of kseg (1: no split)
   int32_t kseg;
-  float* kpart;            // RESID split: partial sums [ksplit][N]
+  uint64_t* kpart;         // RESID split: tagged partial sums [ksplit][N]
   uint32_t* blk_cnt;       // RESID split: finished segment tasks per row block
   const uint16_t* W[MAX_SEG];   // bf16 weights [rows, K]
-  float* y[MAX_SEG];            // fp32 outputs of RMSNORM_LINEAR
+  uint64_t* y[MAX_SEG];         // tagged outputs of RMSNORM_LINEAR
   const uint16_t* W_up;         // SILU: up matrix (W[0] = gate)
-  const float* x;               // fp32 input (norm ops) / residual (RESID)
-  const float* a_in;            // fp32 input of RESID
+  const uint64_t* x;            // tagged input (norm ops) / residual (RESID)
+  const uint64_t* a_in;         // tagged input of RESID
   const uint16_t* norm_w;       // bf16 [K]
-  float* x_out;                 // RESID: residual updated in place; EMBED: x
-  float* a_out;                 // SILU / ATTN output (fp32)
+  uint64_t* x_out;              // RESID: residual updated in place; EMBED: x (tagged)
+  uint64_t* a_out;              // SILU / ATTN output (tagged)
   float eps;
   int32_t capture_slot;
   // attention
   int32_t layer, L, Hq, Hkv, d, G, C, S;
-  const float* q;
-  const float* k;
-  const float* v;
+  const uint64_t* q;            // tagged
+  const uint64_t* k;
+  const uint64_t* v;
   const uint16_t* qn_w;
   const uint16_t* kn_w;
   uint16_t* kc;
@@ -95,6 +95,12 @@ struct OpDesc {
   unsigned long long* keys;     // ARGMAX: per-request packed (value, index) maxima
   uint32_t* arrive;             // ARGMAX: arrival counter
   int64_t* pred;                // ARGMAX: optional [R][S]
+  // versions: the tag of a value written by op w in iteration n is n * nops + w + 1
+  int32_t self;                 // this op's index (the writer of its outputs)
+  int32_t x_writer;             // op that last wrote the x this op reads (-1: none)
+  int32_t a_writer;             // op that wrote a_in (RESID) or q/k/v (attention)
+  int32_t tagged;               // 1: inputs are waited for through their tags; 0: through dep_event
+  uint32_t tag_skew;            // added to every expected input tag (0; fault injection for tests)
   // events
   int32_t dep_event;            // event this op waits on
   int32_t dep_trigger;          // increments of dep_event per iteration

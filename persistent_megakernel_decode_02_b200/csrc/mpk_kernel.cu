@@ -132,6 +132,50 @@ __device__ bool wait_mbar(const Graph& g, uint64_t* bar, uint32_t parity, int wh
   }
 }
 
+// Version tag of the values op `writer` writes in iteration `iter`.
+__device__ __forceinline__ uint32_t vtag(const Graph& g, uint32_t iter, int writer) {
+  return iter * (uint32_t)g.nops + (uint32_t)writer + 1u;
+}
+
+// Value of a tagged element once it carries `tag` (the word already loaded is
+// tried first).  False on abort or timeout (the value is then meaningless).
+__device__ __noinline__ bool poll_tagged(const Graph& g, const uint64_t* p, uint64_t w, uint32_t tag, float& v,
+                                         int op, int worker, int iter) {
+  if (word_tag(w) == tag) {
+    v = word_value(w);
+    return true;
+  }
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    w = ld_tagged(p);
+    if (word_tag(w) == tag) {
+      v = word_value(w);
+      return true;
+    }
+    if (check_stop(g, t0, it, 11, op, -1, worker, iter, word_tag(w), tag)) {
+      v = 0.f;
+      return false;
+    }
+  }
+}
+
+// n consecutive tagged elements into fp32: all loads issued first, stragglers
+// polled.  Returns false on abort or timeout.
+template <int N>
+__device__ __forceinline__ bool load_tagged(const Graph& g, const uint64_t* p, uint32_t tag, float* out, int op,
+                                            int worker, int iter) {
+  uint64_t w[N];
+#pragma unroll
+  for (int e = 0; e < N; ++e) w[e] = ld_tagged(p + e);
+  bool ok = true;
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    if (word_tag(w[e]) == tag) out[e] = word_value(w[e]);
+    else ok &= poll_tagged(g, p + e, w[e], tag, out[e], op, worker, iter);
+  }
+  return ok;
+}
+
 // ------------------------------------------------------------------ task geometry
 // Rows [row0, row1) of group g that task `task` computes (groups split the
 // tasks evenly; N is the row count of one group).
@@ -446,7 +490,7 @@ __device__ __forceinline__ void dot_group(const uint8_t* stage, int i0, int n, i
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
 __device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
-                              int cw, int lane);
+                              int cw, int lane, uint32_t iter, int worker);
 
 // ------------------------------------------------------------------ GEMV tasks
 // Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector h
@@ -469,22 +513,29 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   // load of the prologue is issued before the first use (one L2 round trip).
   const int nrows = row1 - row0;
   const bool xs_ok = KIND == TK_GEMV_RESID && !split && nrows <= MAX_XS;
+  // versions of the inputs (and of what this task writes)
+  const uint32_t xtag = vtag(g, iter, op.x_writer) + op.tag_skew;
+  const uint32_t atag = vtag(g, iter, op.a_writer) + op.tag_skew;
+  const uint32_t mytag = vtag(g, iter, op.self);
+  bool pfail = false;
   if (KIND == TK_GEMV_RESID) {
-    // the input (this task's segment of it) goes straight to shared memory
-    // (cp.async through L2), the task's residual rows through registers
-    for (int k = ctid * 4; k < K; k += CONSUMER_THREADS * 4) cp_async16(hs + hperm(k), op.a_in + koff + k);
-    float xv[MAX_XS / CONSUMER_THREADS];
+    // the input (this task's segment of it) into shared memory once every
+    // element carries its writer's tag, the task's residual rows likewise
 #pragma unroll
-    for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
-      const int j = c * CONSUMER_THREADS + ctid;
-      if (xs_ok && j < nrows) xv[c] = __ldcg(op.x_out + row0 + j);
+    for (int c = 0; c < MAX_K / (CONSUMER_THREADS * 4); ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 4;
+      if (k < K) {
+        float v[4];
+        pfail |= !load_tagged<4>(g, op.a_in + koff + k, atag, v, op.self, worker, (int)iter);
+        *reinterpret_cast<float4*>(hs + hperm(k)) = make_float4(v[0], v[1], v[2], v[3]);
+      }
     }
-#pragma unroll
-    for (int c = 0; c < MAX_XS / CONSUMER_THREADS; ++c) {
-      const int j = c * CONSUMER_THREADS + ctid;
-      if (xs_ok && j < nrows) sm.u.g.xs[j] = xv[c];
+    for (int j = ctid; xs_ok && j < nrows; j += CONSUMER_THREADS) {
+      float xv;
+      pfail |= !poll_tagged(g, op.x_out + row0 + j, ld_tagged(op.x_out + row0 + j), xtag, xv, op.self, worker,
+                            (int)iter);
+      sm.u.g.xs[j] = xv;
     }
-    cp_async_wait_all();
   } else {
     // RMSNorm: x and the norm weight are read once into registers, the
     // statistics are reduced in a fixed order.
@@ -494,12 +545,12 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int k = (c * CONSUMER_THREADS + ctid) * 8;
-      if (k < K) {
-        const float4 x0 = ldcg_f4(op.x + k), x1 = ldcg_f4(op.x + k + 4);
-        wr[c] = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
-        xr[c][0] = x0.x; xr[c][1] = x0.y; xr[c][2] = x0.z; xr[c][3] = x0.w;
-        xr[c][4] = x1.x; xr[c][5] = x1.y; xr[c][6] = x1.z; xr[c][7] = x1.w;
-      }
+      if (k < K) wr[c] = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
+    }
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 8;
+      if (k < K) pfail |= !load_tagged<8>(g, op.x + k, xtag, xr[c], op.self, worker, (int)iter);
     }
     float ss = 0.f;
 #pragma unroll
@@ -532,7 +583,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       }
     }
   }
-  consumer_sync();
+  if (consumer_sync_or(pfail)) return false;
   if (g.profiling && ctid == 0) sm.t_pro = globaltimer();
 
   const bool capture = (g.capture_iter == (int)iter);
@@ -544,18 +595,21 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     const int row = row0 + j;
     if (KIND == TK_NORM_GEMV || KIND == TK_QKV_ATTN) {
       const int sg = seg_of(op, row);
-      op.y[sg][seg_row(op, grp, sg, row)] = v;
+      st_tagged(op.y[sg] + seg_row(op, grp, sg, row), v, mytag);
     } else if (KIND == TK_GEMV_RESID) {
       if (split) {
-        op.kpart[(size_t)(task % op.ksplit) * op.N + row] = v;
+        st_tagged(op.kpart + (size_t)(task % op.ksplit) * op.N + row, v, mytag);
         return;
       }
-      const float nx = (xs_ok ? sm.u.g.xs[j] : __ldcg(op.x_out + row)) + v;
-      op.x_out[row] = nx;
+      float xo;
+      if (xs_ok) xo = sm.u.g.xs[j];
+      else poll_tagged(g, op.x_out + row, ld_tagged(op.x_out + row), xtag, xo, op.self, worker, (int)iter);
+      const float nx = xo + v;
+      st_tagged(op.x_out + row, nx, mytag);
       if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
         g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
     } else if (KIND == TK_NORM_GEMV_SILU) {
-      op.a_out[row] = silu_f(v) * u;
+      st_tagged(op.a_out + row, silu_f(v) * u, mytag);
     } else {  // LM head
       const unsigned long long key = argmax_key(v, (uint32_t)row);
       best = key > best ? key : best;
@@ -615,37 +669,43 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   if (split) {
     // The last segment task of this row block to finish adds the partial sums
     // to the residual, in segment order.
+    // (no fence: the finisher waits for the partials' tags)
     if (ctid == 0) {
-      __threadfence();
       const uint32_t old = atomicAdd(op.blk_cnt + task / op.ksplit, 1u);
       sm.last = ((old + 1u) % (uint32_t)op.ksplit) == 0u;
     }
     consumer_sync();
     if (sm.last) {
-      __threadfence();
+      bool ffail = false;
       for (int j = ctid; j < nrows; j += CONSUMER_THREADS) {
         const int row = row0 + j;
-        float sum = __ldcg(op.kpart + row);
-        for (int k = 1; k < op.ksplit; ++k) sum += __ldcg(op.kpart + (size_t)k * op.N + row);
-        const float nx = __ldcg(op.x_out + row) + sum;
-        op.x_out[row] = nx;
+        float sum = 0.f, xo = 0.f;
+        for (int k = 0; k < op.ksplit; ++k) {
+          const uint64_t* pk = op.kpart + (size_t)k * op.N + row;
+          float pv;
+          ffail |= !poll_tagged(g, pk, ld_tagged(pk), mytag, pv, op.self, worker, (int)iter);
+          sum = k == 0 ? pv : sum + pv;
+        }
+        ffail |= !poll_tagged(g, op.x_out + row, ld_tagged(op.x_out + row), xtag, xo, op.self, worker, (int)iter);
+        const float nx = xo + sum;
+        st_tagged(op.x_out + row, nx, mytag);
         if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
           g.cap_hidden[(size_t)op.capture_slot * g.R * g.H + row] = nx;
       }
+      if (consumer_sync_or(ffail)) return false;
     }
   }
 
   if (KIND == TK_QKV_ATTN) {
     // The last projection task of this kv head's group runs its attention.
+    // (no fence: the attention waits for q, k and v through their tags)
     if (ctid == 0) {
-      __threadfence();
       const uint32_t old = atomicAdd(op.grp_cnt + grp, 1u);
       sm.last = ((old + 1u) % (uint32_t)(op.ntasks / op.groups)) == 0u;
     }
     consumer_sync();
     if (sm.last) {
-      __threadfence();
-      if (!attn_dispatch(sm, g, op, grp, 0, 1, 0, true, cw, lane)) return false;
+      if (!attn_dispatch(sm, g, op, grp, 0, 1, 0, true, cw, lane, iter, worker)) return false;
       consumer_sync();
       if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
     }
@@ -698,7 +758,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // chunk order and signals the operation's event.
 template <int G, int D>
 __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
-                          int cw, int lane) {
+                          int cw, int lane, uint32_t iter, int worker) {
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
   constexpr int NSTEP = 4;           // warp steps whose loads are in flight together
@@ -713,16 +773,34 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
   // are issued before it is read.
   constexpr int EL = D / 32;  // elements per lane
   const int prow = cw;
+  const uint32_t intag = vtag(g, iter, op.a_writer) + op.tag_skew;
+  const uint32_t mytag = vtag(g, iter, op.self);
   float x[EL];
+  uint64_t xw[EL];
+  const uint64_t* src = prow < G ? op.q + (size_t)r * op.Hq * D + (size_t)(j * G + prow) * D
+                      : prow == G ? op.k + (size_t)r * Hkv * D + (size_t)j * D
+                                  : op.v + (size_t)r * Hkv * D + (size_t)j * D;
   if (prow < G + 2) {
-    const float* src = prow < G ? op.q + (size_t)r * op.Hq * D + (size_t)(j * G + prow) * D
-                     : prow == G ? op.k + (size_t)r * Hkv * D + (size_t)j * D
-                                 : op.v + (size_t)r * Hkv * D + (size_t)j * D;
 #pragma unroll
-    for (int e = 0; e < EL; ++e) x[e] = __ldcg(src + lane + 32 * e);
+    for (int e = 0; e < EL; ++e) xw[e] = ld_tagged(src + lane + 32 * e);
   }
   int s;
   const bool active = request_active(g, r, s);
+  bool afail = false;
+  if (active && prow < G + 2) {
+    // q, k, v of this iteration (their tags), then the cache: positions below
+    // s were appended by this operation's attention tasks of earlier
+    // iterations, which released its event after appending
+#pragma unroll
+    for (int e = 0; e < EL; ++e) {
+      if (word_tag(xw[e]) == intag) x[e] = word_value(xw[e]);
+      else afail |= !poll_tagged(g, src + lane + 32 * e, xw[e], intag, x[e], op.self, worker, (int)iter);
+    }
+  }
+  if (active && ctid == 0 && iter > 0 &&
+      !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 1, op.self,
+                    -1, worker, (int)iter))
+    afail = true;
 
   if (active) {
     const int npos = s + 1;
@@ -762,7 +840,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         else A.vs[i] = f32_to_bf16_rn(x[e]);
       }
     }
-    consumer_sync();
+    if (consumer_sync_or(afail)) return false;
     if (hi == npos && ctid < D / 4) {
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
@@ -879,7 +957,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         }
       }
       if (direct) {
-        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = Os / Ls;
+        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
       } else {
         float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
         p[2 + i] = Os;
@@ -922,7 +1000,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
           Ls = fmaf(lc, f, Ls);
           Os = fmaf(oc, f, Os);
         }
-        op.a_out[(size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i] = Os / Ls;
+        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
       }
     }
     consumer_sync();
@@ -942,14 +1020,17 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
       return true;
     }
     const uint16_t* row = op.table + (size_t)tok * op.N;
-    float* x = op.x_out + (size_t)r * op.N;
+    uint64_t* x = op.x_out + (size_t)r * op.N;
+    const uint32_t mytag = vtag(g, iter, op.self);
     const bool capture = (g.capture_iter == (int)iter) && g.cap_hidden != nullptr && op.capture_slot >= 0;
     for (int i = ctid * 8; i < op.N; i += CONSUMER_THREADS * 8) {
       const uint4 w = __ldg(reinterpret_cast<const uint4*>(row + i));
       const float4 a = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
       const float4 b = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
-      *reinterpret_cast<float4*>(x + i) = a;
-      *reinterpret_cast<float4*>(x + i + 4) = b;
+      st_tagged(x + i + 0, a.x, mytag); st_tagged(x + i + 1, a.y, mytag);
+      st_tagged(x + i + 2, a.z, mytag); st_tagged(x + i + 3, a.w, mytag);
+      st_tagged(x + i + 4, b.x, mytag); st_tagged(x + i + 5, b.y, mytag);
+      st_tagged(x + i + 6, b.z, mytag); st_tagged(x + i + 7, b.w, mytag);
       if (capture) {
         float* hc = g.cap_hidden + ((size_t)op.capture_slot * g.R + r) * g.H + i;
         *reinterpret_cast<float4*>(hc) = a;
@@ -964,15 +1045,15 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 // Not inlined: attention gets its own register allocation, so its per-head
 // arrays never push the GEMV loops into spills.
 __device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
-                                           bool direct, int cw, int lane) {
+                                           bool direct, int cw, int lane, uint32_t iter, int worker) {
   const int key = op.G * 1000 + op.d;
   switch (key) {
-    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
-    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
-    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, direct, cw, lane);
-    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
-    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
-    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, direct, cw, lane);
+    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
     default: return false;
   }
 }
@@ -1012,7 +1093,7 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
       sm.t_loop = 0ull;
     }
     // dependency: the event of the op this one follows
-    if (!kStandalone && ctid == 0) {
+    if (!kStandalone && ctid == 0 && !op.tagged) {
       const uint32_t target = (iter + (uint32_t)op.dep_iter_offset) * (uint32_t)op.dep_trigger;
       if (target != 0 &&
           !wait_counter(g, g.events + (size_t)op.dep_event * EVENT_STRIDE, target, 1, opi, task, worker, (int)iter))
@@ -1034,7 +1115,7 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
         break;
       case TK_ATTN:
         ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C), false, cw,
-                           lane);
+                           lane, iter, worker);
         break;
       case TK_QKV_ATTN: ok = gemv_task<TK_QKV_ATTN>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       default: ok = false;
@@ -1045,7 +1126,9 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     }
     consumer_sync();
     if (ctid == 0) {
-      if (op.signal_per_task) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+      // progress count for the scheduler's dispatch window (data readiness
+      // travels with the tagged values, so no release is needed here)
+      if (op.signal_per_task) red_relaxed_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
       if (g.profiling) {
         const uint32_t k = atomicAdd(g.timeline_n, 1u);
         if (k < (uint32_t)g.max_timeline) {

@@ -25,15 +25,24 @@ from ._lib import MpkError, check
 _DTYPES = {torch.bfloat16: _lib.BF16, torch.float32: _lib.FP32, torch.int32: _lib.INT32,
            torch.int64: _lib.INT64}
 _TORCH = {v: k for k, v in _DTYPES.items()}
+# Activations passed between operations (MPK_FP32T): 8 bytes per element, the
+# fp32 value in the low half, a version tag in the high half.  Seen from torch
+# as int64; `untag` gives the values.
+FP32_TAGGED = "fp32_tagged"
 _IO = {"cuda_tensor": _lib.IO_CUDA, "nvshmem_tensor": _lib.IO_NVSHMEM}
 
 Name = Union[str, torch.Tensor]
 
 
+def untag(t: torch.Tensor) -> torch.Tensor:
+    """fp32 values of a tagged activation tensor (int64 view of MPK_FP32T)."""
+    return t.contiguous().view(torch.float32)[..., 0::2]
+
+
 class _DeviceArray:
     """__cuda_array_interface__ view of library-owned memory (for torch.as_tensor)."""
 
-    _TYPESTR = {_lib.BF16: "<f2", _lib.FP32: "<f4", _lib.INT32: "<i4", _lib.INT64: "<i8"}
+    _TYPESTR = {_lib.BF16: "<f2", _lib.FP32: "<f4", _lib.INT32: "<i4", _lib.INT64: "<i8", _lib.FP32T: "<i8"}
 
     def __init__(self, ptr: int, dims: Sequence[int], dtype: int):
         self.__cuda_array_interface__ = {
@@ -88,13 +97,13 @@ class PersistentKernel:
                    io_category: str = "cuda_tensor") -> torch.Tensor:
         if io_category not in _IO:
             raise MpkError(_lib.ERR_CODE["INVALID_ARG"], f"io_category {io_category!r}")
-        if dtype not in _DTYPES:
+        if dtype != FP32_TAGGED and dtype not in _DTYPES:
             raise MpkError(_lib.ERR_CODE["DTYPE"], f"dtype {dtype} not supported")
+        code = _lib.FP32T if dtype == FP32_TAGGED else _DTYPES[dtype]
         cd = (ctypes.c_int64 * len(dims))(*dims)
         ptr = ctypes.c_void_p()
-        check(self._lib.mpk_new_tensor(self._ctx, name.encode(), _DTYPES[dtype], len(dims), cd, _IO[io_category],
+        check(self._lib.mpk_new_tensor(self._ctx, name.encode(), code, len(dims), cd, _IO[io_category],
                                        ctypes.byref(ptr)), self._ctx)
-        code = _DTYPES[dtype]
         if dtype == torch.bfloat16:
             view = torch.as_tensor(_DeviceArray(ptr.value, dims, code), device="cuda").view(torch.bfloat16)
         else:

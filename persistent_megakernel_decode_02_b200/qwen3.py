@@ -15,7 +15,7 @@ from typing import Dict, List, Optional
 import torch
 
 from . import _lib
-from .kernel import PersistentKernel
+from .kernel import FP32_TAGGED, PersistentKernel
 
 
 FUSED_ATTENTION_MAX_SEQ = 4096
@@ -134,12 +134,12 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     pred = torch.full((requests, max_seq), -1, dtype=torch.int64, device=dev)
     mk.attach_input(pred, "pred")
     bufs = {
-        "x": mk.new_tensor((requests, s.hidden), torch.float32, "x"),
-        "q": mk.new_tensor((requests, s.q_dim), torch.float32, "q"),
-        "k": mk.new_tensor((requests, s.kv_dim), torch.float32, "k"),
-        "v": mk.new_tensor((requests, s.kv_dim), torch.float32, "v"),
-        "o": mk.new_tensor((requests, s.q_dim), torch.float32, "o"),
-        "a": mk.new_tensor((requests, s.intermediate), torch.float32, "a"),
+        "x": mk.new_tensor((requests, s.hidden), FP32_TAGGED, "x"),
+        "q": mk.new_tensor((requests, s.q_dim), FP32_TAGGED, "q"),
+        "k": mk.new_tensor((requests, s.kv_dim), FP32_TAGGED, "k"),
+        "v": mk.new_tensor((requests, s.kv_dim), FP32_TAGGED, "v"),
+        "o": mk.new_tensor((requests, s.q_dim), FP32_TAGGED, "o"),
+        "a": mk.new_tensor((requests, s.intermediate), FP32_TAGGED, "a"),
     }
     if attn_chunks is None:
         attn_chunks = default_attn_chunks(s, requests, num_workers, max_seq)
