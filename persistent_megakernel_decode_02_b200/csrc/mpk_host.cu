@@ -660,6 +660,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         return fail(c, MPK_ERR_INVALID_ARG, "layer %d: unknown op %d", li, Ly.op);
     }
   }
+  if (R > MAX_REQUESTS)
+    return fail(c, MPK_ERR_UNSUPPORTED, "%d requests (at most %d)", R, MAX_REQUESTS);
   if (n_argmax != 1 || ops[n_layers - 1].kind != TK_NORM_GEMV_ARGMAX)
     return fail(c, MPK_ERR_INVALID_ARG, "the graph must end with one RMSNORM_LMHEAD_ARGMAX operation");
   if (ops[0].kind != TK_EMBED)
@@ -902,6 +904,7 @@ int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_
   int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
   if (rc != MPK_OK) return rc;
   *(volatile int32_t*)c->abort_host = 0;
+  c->graph.op_by_op = 0;
   CUDA_OR_FAIL(c, launch_persistent(c->graph, c->sms, s));
   return MPK_OK;
 }
@@ -924,9 +927,11 @@ int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_request
     const int64_t end = std::min<int64_t>(se[r], seq_len - 1);
     if (st[r] >= 0 && st[r] < end) n_iter = std::max<int64_t>(n_iter, end - st[r]);
   }
+  c->graph.op_by_op = 1;
   for (int64_t it = 0; it < n_iter; ++it)
     for (int p = 0; p < (int)c->ops.size(); ++p)
       CUDA_OR_FAIL(c, launch_op(c->graph, p, c->ops[p].ntasks, (uint32_t)it, s));
+  c->graph.op_by_op = 0;
   return MPK_OK;
 }
 

@@ -117,15 +117,23 @@ struct Status {
   uint32_t observed, expected;
 };
 
+constexpr int MAX_REQUESTS = 64;
 struct Control {
   uint32_t ready;
   uint32_t n_iter;
   uint32_t pad[30];
+  // per request, read at the start of a run: step[r] and the last position it
+  // may reach, min(step_end[r], S - 1).  While a request is active its step
+  // advances by exactly one per iteration, so in iteration n it is
+  // step0[r] + n.
+  int32_t step0[MAX_REQUESTS];
+  int32_t stop[MAX_REQUESTS];
 };
 
 struct Graph {
   const OpDesc* ops;
   int32_t nops;
+  int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
   int32_t R, S, V, H, L;
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;

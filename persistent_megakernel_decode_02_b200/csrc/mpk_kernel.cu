@@ -67,6 +67,8 @@ struct __align__(128) Smem {
   unsigned long long t_stall, t_last;            // profiling: time waited for stages, last stage ready
   unsigned long long t_loop;                     // profiling: every consumer warp done with its rows
   int32_t last;     // last-arrival flag
+  int32_t attn_s;   // fused QKV + attention: position of the request (-1: inactive), read in the prologue
+  float2 rope_row[MAX_D / 2];                    // its RoPE (cos, sin) row
 };
 
 // ------------------------------------------------------------------ status / waits
@@ -213,6 +215,15 @@ __device__ __forceinline__ bool is_gemv(int kind) {
          kind == TK_NORM_GEMV_ARGMAX || kind == TK_QKV_ATTN;
 }
 
+// Position of request r in iteration `iter` of a persistent run (from the
+// run-start state, so nothing written during the run is read), and whether it
+// is active.
+__device__ __forceinline__ bool request_at(const Graph& g, int r, uint32_t iter, int& s) {
+  const int s0 = __ldcg(&g.ctl->step0[r]);
+  s = s0 + (int)iter;
+  return s0 >= 0 && s < __ldcg(&g.ctl->stop[r]);
+}
+
 __device__ __forceinline__ bool request_active(const Graph& g, int r, int& s) {
   s = __ldcg(g.step + r);
   int end = g.S - 1;
@@ -221,6 +232,13 @@ __device__ __forceinline__ bool request_active(const Graph& g, int r, int& s) {
     end = e < end ? e : end;
   }
   return s >= 0 && s < end;
+}
+
+// Position and activity of request r in iteration `iter`: from the run-start
+// state in a persistent run, from `step` itself when every operation is its
+// own launch (the launches order the updates).
+__device__ __forceinline__ bool request_state(const Graph& g, int r, uint32_t iter, int& s) {
+  return g.op_by_op ? request_active(g, r, s) : request_at(g, r, iter, s);
 }
 
 // Locate global row `row` of a stacked multi-matrix operation.
@@ -518,6 +536,37 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   const uint32_t atag = vtag(g, iter, op.a_writer) + op.tag_skew;
   const uint32_t mytag = vtag(g, iter, op.self);
   bool pfail = false;
+  if (KIND == TK_QKV_ATTN) {
+    // What this operation's attention needs besides q, k and v, fetched while
+    // the input is awaited: the request's position, its RoPE row, and the
+    // ordering of the cache (this operation's attention releases its event
+    // after appending; positions below s were appended in earlier iterations).
+    if (ctid < op.d / 2) {
+      int sp;
+      const bool act = request_state(g, 0, iter, sp);
+      if (act) sm.rope_row[ctid] = __ldg(op.rope + (size_t)sp * (op.d / 2) + ctid);
+      if (ctid == 0) {
+        sm.attn_s = act ? sp : -1;
+        if (act && sp > 0) {
+          // this task's share of the head's cached positions into L2, so the
+          // group's attention (run by whichever task finishes last) reads
+          // them at L2 latency
+          const int tpg = op.ntasks / op.groups, t = task - grp * tpg;
+          const int p0 = (int)(((long long)t * sp) / tpg), p1 = (int)(((long long)(t + 1) * sp) / tpg);
+          if (p1 > p0) {
+            const size_t base = (((size_t)op.layer * g.R) * op.Hkv + grp) * (size_t)op.S * op.d;
+            const uint32_t bytes = (uint32_t)(p1 - p0) * (uint32_t)op.d * 2u;
+            prefetch_l2(op.kc + base + (size_t)p0 * op.d, bytes);
+            prefetch_l2(op.vc + base + (size_t)p0 * op.d, bytes);
+          }
+        }
+      }
+    }
+    if (ctid == 0 && iter > 0 &&
+        !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 1, op.self,
+                      task, worker, (int)iter))
+      pfail = true;
+  }
   if (KIND == TK_GEMV_RESID) {
     // the input (this task's segment of it) into shared memory once every
     // element carries its writer's tag, the task's residual rows likewise
@@ -728,7 +777,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       if (ctid < g.R) {
         const int rq = ctid;
         int s;
-        if (request_active(g, rq, s)) {
+        if (request_state(g, rq, iter, s)) {
           const unsigned long long key = atomicAdd(op.keys + rq, 0ull);
           const int64_t nxt = (int64_t)argmax_key_index(key);
           int64_t* trow = g.tokens + (size_t)rq * g.S;
@@ -785,7 +834,14 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
     for (int e = 0; e < EL; ++e) xw[e] = ld_tagged(src + lane + 32 * e);
   }
   int s;
-  const bool active = request_active(g, r, s);
+  bool active;
+  if (direct) {
+    // fused with the projections: state fetched in that task's prologue
+    s = sm.attn_s;
+    active = s >= 0;
+  } else {
+    active = request_state(g, r, iter, s);
+  }
   bool afail = false;
   if (active && prow < G + 2) {
     // q, k, v of this iteration (their tags), then the cache: positions below
@@ -797,7 +853,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       else afail |= !poll_tagged(g, src + lane + 32 * e, xw[e], intag, x[e], op.self, worker, (int)iter);
     }
   }
-  if (active && ctid == 0 && iter > 0 &&
+  if (!direct && active && ctid == 0 && iter > 0 &&
       !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 1, op.self,
                     -1, worker, (int)iter))
     afail = true;
@@ -811,7 +867,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         float2 rc[EL / 2];
         const float2* cs = op.rope + (size_t)s * (D / 2);
 #pragma unroll
-        for (int e = 0; e < EL / 2; ++e) rc[e] = __ldg(cs + lane + 32 * e);
+        for (int e = 0; e < EL / 2; ++e) rc[e] = direct ? sm.rope_row[lane + 32 * e] : __ldg(cs + lane + 32 * e);
         const uint16_t* wn = prow < G ? op.qn_w : op.kn_w;
         uint16_t wb[EL];
 #pragma unroll
@@ -1013,7 +1069,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
 __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t iter, int ctid) {
   const int r = task;
   int s;
-  if (r < g.R && request_active(g, r, s)) {
+  if (r < g.R && request_state(g, r, iter, s)) {
     const int64_t tok = __ldcg(g.tokens + (size_t)r * g.S + s);
     if (tok < 0 || tok >= g.V) {
       if (ctid == 0) record_error(g, -11 /*DEVICE*/, 8, -1, task, -1, (int)iter, (uint32_t)tok, (uint32_t)g.V);
@@ -1226,11 +1282,12 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_ke
       uint32_t n_iter = 0;
       for (int r = 0; r < g.R; ++r) {
         int s;
-        if (request_active(g, r, s)) {
-          int end = g.S - 1;
-          if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + r));
-          n_iter = max(n_iter, (uint32_t)(end - s));
-        }
+        const bool act = request_active(g, r, s);
+        int end = g.S - 1;
+        if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + r));
+        if (act) n_iter = max(n_iter, (uint32_t)(end - s));
+        g.ctl->step0[r] = act ? s : -1;
+        g.ctl->stop[r] = end;
       }
       g.ctl->n_iter = n_iter;
       st_release(&g.ctl->ready, 1u);
