@@ -19,7 +19,7 @@ size_t kernel_smem_bytes();
 cudaError_t prepare_kernels();
 cudaError_t max_blocks_per_sm(int* n);
 cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream);
-cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, cudaStream_t stream);
+cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, bool cooperative, cudaStream_t stream);
 }  // namespace mpk
 
 using namespace mpk;
@@ -334,7 +334,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   std::vector<OpDesc> ops(n_layers);
   int R = -1, H = -1, V = -1, L = -1, S = -1;
   // attention workspace sizing
-  size_t part_floats = 0, merge_u32 = 0, kpart_floats = 0, blk_u32 = 0;
+  size_t part_floats = 0, merge_u32 = 0, kpart_floats = 0, blk_u32 = 0, gpart_words = 0;
   std::vector<std::pair<int, size_t>> merge_off(n_layers, {0, 0});
   struct RopeKey { float theta; int d; int S; };
   std::vector<RopeKey> rope_keys;
@@ -630,7 +630,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.y[2] = (uint64_t*)v->ptr;
         op.x = (const uint64_t*)x->ptr;
         op.norm_w = (const uint16_t*)wn->ptr;
-        op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = 1;
+        op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G;
         op.L = (int)kc->dims[0];
         op.S = (int)kc->dims[3];
         op.layer = Ly.layer;
@@ -641,6 +641,12 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
         merge_off[li] = {1, merge_u32};
         merge_u32 += (size_t)R * Hkv;
+        // group mode needs every task of the operation on its own worker
+        op.group_sync = ntasks <= c->num_workers ? 1 : 0;
+        // attention chunks per kv head (run by the group's first tasks); chunk
+        // partials [Hkv][C][G][d + 2], written in both modes
+        op.C = std::min(gx, MAX_GCHUNK);
+        gpart_words = std::max(gpart_words, (size_t)Hkv * op.C * G * (d + 2));
         const float theta = Ly.rope_theta > 0 ? Ly.rope_theta : 1.0e6f;
         int ri = -1;
         for (size_t i = 0; i < rope_keys.size(); ++i)
@@ -791,6 +797,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   rc = alloc(c, &kpart, sizeof(uint64_t) * (kpart_floats ? kpart_floats : 1));
   if (rc != MPK_OK) return rc;
   c->zero_each_run.push_back({kpart, sizeof(uint64_t) * (kpart_floats ? kpart_floats : 1)});
+  uint64_t* gpart = nullptr;
+  rc = alloc(c, &gpart, sizeof(uint64_t) * (gpart_words ? gpart_words : 1));
+  if (rc != MPK_OK) return rc;
+  c->zero_each_run.push_back({gpart, sizeof(uint64_t) * (gpart_words ? gpart_words : 1)});
   std::vector<float2*> rope_dev(rope_keys.size(), nullptr);
   for (size_t i = 0; i < rope_keys.size(); ++i) {
     const RopeKey& k = rope_keys[i];
@@ -817,6 +827,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       op.rope = rope_dev[rope_of[p]];
     }
     if (op.kind == TK_QKV_ATTN) {
+      op.gpart = gpart;  // one group-mode operation at a time uses it
       op.grp_cnt = reinterpret_cast<uint32_t*>(sb + o_merge) + merge_off[p].second;
       op.rope = rope_dev[rope_of[p]];
     }
@@ -930,7 +941,7 @@ int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_request
   c->graph.op_by_op = 1;
   for (int64_t it = 0; it < n_iter; ++it)
     for (int p = 0; p < (int)c->ops.size(); ++p)
-      CUDA_OR_FAIL(c, launch_op(c->graph, p, c->ops[p].ntasks, (uint32_t)it, s));
+      CUDA_OR_FAIL(c, launch_op(c->graph, p, c->ops[p].ntasks, (uint32_t)it, c->ops[p].group_sync != 0, s));
   c->graph.op_by_op = 0;
   return MPK_OK;
 }

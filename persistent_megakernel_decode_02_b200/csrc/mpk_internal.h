@@ -39,6 +39,7 @@ constexpr int MAX_XS = 1024;                // residual rows of a task preloaded
 constexpr int MAX_SEG = 3;
 constexpr int MAX_G = 8;                    // query heads per kv head
 constexpr int MAX_D = 128;                  // head dim
+constexpr int MAX_GCHUNK = 8;               // fused op: attention chunks per kv head (tasks 0.. of the group)
 constexpr int SCHED_WARPS_PER_SM = 4;
 
 enum TaskKind : int32_t {
@@ -88,6 +89,8 @@ struct OpDesc {
   uint16_t* kc;
   uint16_t* vc;
   float* part;                  // [R][Hq][C][d + 2]
+  uint64_t* gpart;              // group mode: tagged chunk partials [Hkv][C][G][d + 2]
+  int32_t group_sync;           // fused op: every task of a group attends to a chunk (tasks <= workers)
   uint32_t* merge_cnt;          // [R][Hkv]
   const float2* rope;           // [S][d/2] (cos, sin)
   // embed / LM head

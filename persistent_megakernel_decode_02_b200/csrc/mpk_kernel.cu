@@ -44,6 +44,8 @@ struct AttnScratch {
   float wacc[CONSUMER_WARPS][MAX_G * MAX_D / 2]; // per-warp unnormalised outputs
 };
 static_assert(MAX_G * MAX_D / 2 >= 512, "attention scratch");
+static_assert(sizeof(AttnScratch) >= sizeof(float) * MAX_GCHUNK * (MAX_G / 2) * (MAX_D + 2),
+              "the group merge gathers every chunk partial of a kv head into the attention scratch");
 
 struct __align__(128) Smem {
   uint8_t ring[NSTAGES][STAGE_BYTES];
@@ -507,7 +509,13 @@ __device__ __forceinline__ void dot_group(const uint8_t* stage, int i0, int n, i
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 
-__device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
+// Attention task modes: a chunk of the split-K ATTENTION operation (partials,
+// merged by the last chunk to arrive), or a chunk of a fused
+// projections+attention operation's kv-head group (tagged partials, merged by
+// chunk 0).
+constexpr int ATTN_SPLIT_OP = 0, ATTN_GROUP = 1;
+
+__device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
                               int cw, int lane, uint32_t iter, int worker);
 
 // ------------------------------------------------------------------ GEMV tasks
@@ -745,16 +753,31 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     }
   }
 
-  if (KIND == TK_QKV_ATTN) {
-    // The last projection task of this kv head's group runs its attention.
-    // (no fence: the attention waits for q, k and v through their tags)
+  if (KIND == TK_QKV_ATTN && op.group_sync) {
+    // The group's first op.C tasks each attend to a chunk of the positions
+    // (once the group's q, k, v carry their tags) and chunk 0 merges; each
+    // task of the operation runs on its own worker, so the waits on the
+    // group's other tasks always end.
+    const int tpg = op.ntasks / op.groups, t = task - grp * tpg;
+    if (t < op.C && !attn_dispatch(sm, g, op, grp, t, op.C, 0, ATTN_GROUP, cw, lane, iter, worker)) return false;
+    if (t == 0) {
+      consumer_sync();
+      if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+    }
+  } else if (KIND == TK_QKV_ATTN) {
+    // More tasks than workers: the last projection task of this kv head's
+    // group to finish runs the group's attention.  (No fence: the attention
+    // waits for q, k and v through their tags.)
     if (ctid == 0) {
       const uint32_t old = atomicAdd(op.grp_cnt + grp, 1u);
       sm.last = ((old + 1u) % (uint32_t)(op.ntasks / op.groups)) == 0u;
     }
     consumer_sync();
     if (sm.last) {
-      if (!attn_dispatch(sm, g, op, grp, 0, 1, 0, true, cw, lane, iter, worker)) return false;
+      // the same chunks as in group mode, one after another, chunk 0 (the
+      // merge) last: results are identical whichever mode runs
+      for (int cc = op.C - 1; cc >= 0; --cc)
+        if (!attn_dispatch(sm, g, op, grp, cc, op.C, 0, ATTN_GROUP, cw, lane, iter, worker)) return false;
       consumer_sync();
       if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
     }
@@ -795,19 +818,21 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 }
 
 // ------------------------------------------------------------------ attention task
-// Attention of kv head j for request r at position s = step[r], over the
-// positions of chunk c of C (split-K) or over all of 0..s (direct).
-// Prologue: RMSNorm over the head dim and rotate-half RoPE of the G query
-// heads of the group and of k; the chunk holding s appends bf16 k, v at
-// position s.  Main loop: LP = D/8 lanes per position (8 dims per lane),
-// 32/LP positions per warp step, NSTEP steps' K/V loads issued before any is
-// used, online softmax in base 2 per query head.  Direct: o = bf16(output)
-// is written here.  Split-K: (max, sum, unnormalised output) partials go to
-// global memory and the last chunk task of (r, j) to arrive merges them in
-// chunk order and signals the operation's event.
+// Attention of kv head j for request r at position s, over the positions
+// [c (s+1) / C, (c+1) (s+1) / C) of chunk c of C.  Prologue: RMSNorm over the
+// head dim and rotate-half RoPE of the G query heads of the group and of k;
+// the cache append of k, v at s (by the chunk holding s, or in group mode by
+// chunk 0).  Main loop: LP = D/8 lanes per position (8 dims per lane), 32/LP
+// positions per warp step, NSTEP steps' K/V loads issued before any is used,
+// online softmax in base 2 per query head.  The chunk's (max, sum,
+// unnormalised output) partial goes to global memory; the split operation's
+// last chunk task of (r, j) to arrive merges the partials in chunk order and
+// signals the operation's event, in group mode chunk 0 merges once every
+// partial carries this iteration's tag and writes o.
 template <int G, int D>
-__device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, bool direct,
+__device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
                           int cw, int lane, uint32_t iter, int worker) {
+  const bool fused = mode == ATTN_GROUP;  // state fetched in the projections' prologue
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
   constexpr int NSTEP = 4;           // warp steps whose loads are in flight together
@@ -835,7 +860,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
   }
   int s;
   bool active;
-  if (direct) {
+  if (fused) {
     // fused with the projections: state fetched in that task's prologue
     s = sm.attn_s;
     active = s >= 0;
@@ -853,7 +878,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       else afail |= !poll_tagged(g, src + lane + 32 * e, xw[e], intag, x[e], op.self, worker, (int)iter);
     }
   }
-  if (!direct && active && ctid == 0 && iter > 0 &&
+  if (!fused && active && ctid == 0 && iter > 0 &&
       !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 1, op.self,
                     -1, worker, (int)iter))
     afail = true;
@@ -867,7 +892,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         float2 rc[EL / 2];
         const float2* cs = op.rope + (size_t)s * (D / 2);
 #pragma unroll
-        for (int e = 0; e < EL / 2; ++e) rc[e] = direct ? sm.rope_row[lane + 32 * e] : __ldg(cs + lane + 32 * e);
+        for (int e = 0; e < EL / 2; ++e) rc[e] = fused ? sm.rope_row[lane + 32 * e] : __ldg(cs + lane + 32 * e);
         const uint16_t* wn = prow < G ? op.qn_w : op.kn_w;
         uint16_t wb[EL];
 #pragma unroll
@@ -897,7 +922,9 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       }
     }
     if (consumer_sync_or(afail)) return false;
-    if (hi == npos && ctid < D / 4) {
+    // the cache append at s: by the chunk holding s, or in group mode by the
+    // merging task (chunk 0), whose release after the merge covers it
+    if ((mode == ATTN_GROUP ? c == 0 : hi == npos) && ctid < D / 4) {
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
@@ -999,7 +1026,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       }
     }
     consumer_sync();
-    // merge the warps in fixed order -> the output (direct) or this chunk's partial
+    // merge the warps in fixed order -> this chunk's partial
     for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
       const int hh = idx / D, i = idx % D;
       float M = -INFINITY;
@@ -1012,8 +1039,13 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
           Os = fmaf(A.wacc[w][hh * D + i], f, Os);
         }
       }
-      if (direct) {
-        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
+      if (fused) {
+        uint64_t* p = op.gpart + (((size_t)j * C + c) * G + hh) * (D + 2);
+        st_tagged(p + 2 + i, Os, mytag);
+        if (i == 0) {
+          st_tagged(p, M, mytag);
+          st_tagged(p + 1, Ls, mytag);
+        }
       } else {
         float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
         p[2 + i] = Os;
@@ -1024,7 +1056,57 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       }
     }
   }
-  if (direct) return true;
+  if (fused) {
+    if (c != 0 || !active) return true;
+    // chunk 0 merges the group's chunks in chunk order once each partial
+    // carries this iteration's tag (online rescaling, as for the split op):
+    // all partial words are first gathered into shared memory, eight loads in
+    // flight per thread, then merged from there
+    float* pv = reinterpret_cast<float*>(&A);
+    const int nwords = C * G * (D + 2);
+    const uint64_t* pg = op.gpart + (size_t)j * nwords;
+    bool mfail = false;
+    consumer_sync();  // the chunk's own use of the scratch is over
+    for (int base = 0; base < nwords; base += 8 * CONSUMER_THREADS) {
+      uint64_t w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = base + u * CONSUMER_THREADS + ctid;
+        w[u] = q < nwords ? ld_tagged(pg + q) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int q = base + u * CONSUMER_THREADS + ctid;
+        if (q < nwords) {
+          float v;
+          if (word_tag(w[u]) == mytag) v = word_value(w[u]);
+          else mfail |= !poll_tagged(g, pg + q, w[u], mytag, v, op.self, worker, (int)iter);
+          pv[q] = v;
+        }
+      }
+    }
+    if (consumer_sync_or(mfail)) return false;
+    for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
+      const int hh = idx / D, i = idx % D;
+      float M = -INFINITY, Ls = 0.f, Os = 0.f;
+      for (int cc = 0; cc < C; ++cc) {
+        const float* p = pv + ((size_t)cc * G + hh) * (D + 2);
+        const float mc = p[0], lc = p[1], oc = p[2 + i];
+        if (mc == -INFINITY) continue;
+        if (mc > M) {
+          const float sc = exp2f(M - mc);  // M = -inf -> 0
+          Ls *= sc;
+          Os *= sc;
+          M = mc;
+        }
+        const float f = exp2f(mc - M);
+        Ls = fmaf(lc, f, Ls);
+        Os = fmaf(oc, f, Os);
+      }
+      st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
+    }
+    return !consumer_sync_or(mfail);
+  }
   consumer_sync();
   if (ctid == 0) {
     __threadfence();
@@ -1101,15 +1183,15 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 // Not inlined: attention gets its own register allocation, so its per-head
 // arrays never push the GEMV loops into spills.
 __device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
-                                           bool direct, int cw, int lane, uint32_t iter, int worker) {
+                                           int mode, int cw, int lane, uint32_t iter, int worker) {
   const int key = op.G * 1000 + op.d;
   switch (key) {
-    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
-    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
-    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
-    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
-    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
-    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, direct, cw, lane, iter, worker);
+    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
+    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
+    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
+    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
+    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
+    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
     default: return false;
   }
 }
@@ -1170,8 +1252,8 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
         ok = gemv_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
       case TK_ATTN:
-        ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C), false, cw,
-                           lane, iter, worker);
+        ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C),
+                           ATTN_SPLIT_OP, cw, lane, iter, worker);
         break;
       case TK_QKV_ATTN: ok = gemv_task<TK_QKV_ATTN>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       default: ok = false;
@@ -1347,7 +1429,14 @@ cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream) {
                                      sizeof(Smem), stream);
 }
 
-cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, cudaStream_t stream) {
+// An operation whose tasks wait on one another (group mode) is launched
+// cooperatively, so all of its blocks are resident together.
+cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, bool cooperative, cudaStream_t stream) {
+  if (cooperative) {
+    void* args[] = {const_cast<Graph*>(&g), &op, &iter};
+    return cudaLaunchCooperativeKernel((const void*)mpk_op_kernel, dim3(ntasks), dim3(BLOCK_THREADS), args,
+                                       sizeof(Smem), stream);
+  }
   mpk_op_kernel<<<ntasks, BLOCK_THREADS, sizeof(Smem), stream>>>(g, op, iter);
   return cudaGetLastError();
 }
