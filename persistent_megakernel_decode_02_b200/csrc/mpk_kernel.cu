@@ -675,11 +675,13 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   };
 
 
-  // Each warp owns whole rows: task row j goes to warp j % nwarps (rows per
-  // warp group RB = 1; several rows per warp sharing the loads of h measured
-  // slower, the stage's rows then wait on fewer warps).
+  // Each warp owns groups of RB whole rows that share every load of h from
+  // shared memory (gate/up: one gate row and one up row); group u of the task
+  // goes to warp u % nwarps.  RB = 2 measured best for single matrices: it
+  // halves the shared-memory reads of h, more rows per warp leave too few
+  // warps working on each stage.
   constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
-  constexpr int RB = 1;
+  constexpr int RB = PAIR ? 1 : 2;
   int un = cw;     // next task-local group of this warp
   int ubase = 0;   // first group of the current stage
   for (int base = 0; base < nrows; base += rps) {
