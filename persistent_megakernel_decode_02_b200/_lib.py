@@ -53,6 +53,7 @@ class Options(ctypes.Structure):
         ("timeout_s", ctypes.c_double),
         ("max_timeline", ctypes.c_int32),
         ("prefetch_kb", ctypes.c_int32),
+        ("dynamic_tasks", ctypes.c_int32),
         ("debug_stall_op", ctypes.c_int32),
     ]
 

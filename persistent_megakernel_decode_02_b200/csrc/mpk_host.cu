@@ -737,6 +737,18 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       }
     }
   }
+  // Plain GEMV operations are claimed dynamically (tasks of an op are shared
+  // out by a counter, so workers that finish the previous op early take more);
+  // the fused projections+attention op keeps its fixed task-to-worker mapping
+  // (its group tasks wait on one another).
+  for (int p = 0; p < P; ++p) {
+    OpDesc& op = ops[p];
+    op.dynamic = (o.dynamic_tasks >= 0) &&
+                 (op.kind == TK_NORM_GEMV || op.kind == TK_GEMV_RESID || op.kind == TK_NORM_GEMV_SILU ||
+                  op.kind == TK_NORM_GEMV_ARGMAX) ? 1 : 0;
+    if (op.dynamic && op.ntasks >= (int)TASK_CLAIM)
+      return fail(c, MPK_ERR_INVALID_ARG, "layer %d: at most %u tasks", p, TASK_CLAIM - 1);
+  }
   c->zero_each_run.clear();
   for (auto& kv : c->tensors)
     if (kv.second.dtype == MPK_FP32T) {
@@ -773,6 +785,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o2 = off; off += (bytes + 127) / 128 * 128; return o2; };
   const size_t o_events = take(line * P);
+  const size_t o_claims = take(line * P * CLAIM_SLOTS);
   const size_t o_qhead = take(line * c->num_workers);
   const size_t o_qtail = take(line * c->num_workers);
   const size_t o_ctl = take(sizeof(Control));
@@ -859,6 +872,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   g.lookahead = o.sched_lookahead;
   g.prefetch_bytes = o.prefetch_kb > 0 ? (uint32_t)o.prefetch_kb * 1024u : 0u;
   g.events = reinterpret_cast<uint32_t*>(sb + o_events);
+  g.claims = reinterpret_cast<uint32_t*>(sb + o_claims);
   g.queue = queue;
   g.q_head = reinterpret_cast<uint32_t*>(sb + o_qhead);
   g.q_tail = reinterpret_cast<uint32_t*>(sb + o_qtail);

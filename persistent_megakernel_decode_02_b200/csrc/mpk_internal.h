@@ -103,6 +103,7 @@ struct OpDesc {
   int32_t x_writer;             // op that last wrote the x this op reads (-1: none)
   int32_t a_writer;             // op that wrote a_in (RESID) or q/k/v (attention)
   int32_t tagged;               // 1: inputs are waited for through their tags; 0: through dep_event
+  int32_t dynamic;              // 1: workers claim this op's tasks from a shared counter
   uint32_t tag_skew;            // added to every expected input tag (0; fault injection for tests)
   // events
   int32_t dep_event;            // event this op waits on
@@ -143,6 +144,7 @@ struct Graph {
   int32_t lookahead;
   uint32_t prefetch_bytes;          // L2 prefetch distance per worker (0 = off)
   uint32_t* events;                 // [nops] (one 128-byte line each)
+  uint32_t* claims;                 // [CLAIM_SLOTS][nops] task-claim counters (one line each)
   unsigned long long* queue;        // [num_workers][QUEUE_CAP]
   uint32_t* q_head;                 // [num_workers] (one line each)
   uint32_t* q_tail;
@@ -168,6 +170,10 @@ struct Graph {
 constexpr int TIMELINE_FIELDS = MPK_TIMELINE_FIELDS;
 constexpr int EVENT_STRIDE = 32;    // uint32 per event / queue counter (128 bytes)
 constexpr unsigned long long QUEUE_TERMINATE = ~0ull;
+// Task field of a queue entry that stands for "claim tasks of this dynamic
+// operation until none is left" (one such entry per worker).
+constexpr uint32_t TASK_CLAIM = 0xFFFFu;
+constexpr int CLAIM_SLOTS = 4;  // claim counters per op, used by iteration n % CLAIM_SLOTS
 
 __host__ __device__ inline unsigned long long pack_entry(uint32_t iter, uint32_t op, uint32_t task) {
   return ((unsigned long long)iter << 32) | ((unsigned long long)op << 16) | (unsigned long long)task;

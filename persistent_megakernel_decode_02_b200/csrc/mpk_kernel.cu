@@ -70,6 +70,7 @@ struct __align__(128) Smem {
   unsigned long long t_loop;                     // profiling: every consumer warp done with its rows
   int32_t last;     // last-arrival flag
   int32_t attn_s;   // fused QKV + attention: position of the request (-1: inactive), read in the prologue
+  unsigned long long h_key;  // (iteration, op, segment) whose input vector hs holds (~0: none)
   float2 rope_row[MAX_D / 2];                    // its RoPE (cos, sin) row
 };
 
@@ -183,14 +184,16 @@ __device__ __forceinline__ bool load_tagged(const Graph& g, const uint64_t* p, u
 // ------------------------------------------------------------------ task geometry
 // Rows [row0, row1) of group g that task `task` computes (groups split the
 // tasks evenly; N is the row count of one group).
-// A split residual projection (ksplit > 1) has ntasks / ksplit row blocks;
-// task t computes reduction segment t % ksplit of row block t / ksplit.
+// A split residual projection (ksplit > 1) has nb = ntasks / ksplit row
+// blocks; task t computes reduction segment t / nb of row block t % nb
+// (consecutive tasks share a segment, so a worker claiming several keeps its
+// input segment).
 __device__ __forceinline__ void task_rows(const OpDesc& op, int task, int& g, int& row0, int& row1) {
   int tpg = op.ntasks / op.groups, t;
   if (op.ksplit > 1) {
     tpg /= op.ksplit;
     g = 0;
-    t = task / op.ksplit;
+    t = task % tpg;
   } else {
     g = task / tpg;
     t = task - g * tpg;
@@ -200,9 +203,10 @@ __device__ __forceinline__ void task_rows(const OpDesc& op, int task, int& g, in
 }
 
 // First reduction element of the task's segment (0 without a split).
-__device__ __forceinline__ int task_koff(const OpDesc& op, int task) {
-  return op.ksplit > 1 ? (task % op.ksplit) * op.kseg : 0;
+__device__ __forceinline__ int task_seg(const OpDesc& op, int task) {
+  return op.ksplit > 1 ? task / (op.ntasks / op.ksplit) : 0;
 }
+__device__ __forceinline__ int task_koff(const OpDesc& op, int task) { return task_seg(op, task) * op.kseg; }
 
 // Reduction length of one task (the segment length for a split projection).
 __device__ __forceinline__ int task_k(const OpDesc& op) { return op.ksplit > 1 ? op.kseg : op.K; }
@@ -352,6 +356,12 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
         pf.done = true;
         return;
       }
+      if ((pf.e & 0xFFFFu) == TASK_CLAIM) {  // tasks claimed later: nothing to prefetch for yet
+        ++pf.q;
+        pf.row = -1;
+        pf.have = false;
+        continue;
+      }
       const OpDesc& op = g.ops[(int)((pf.e >> 16) & 0xFFFFu)];
       int r0 = 0, r1 = 0, pg = 0;
       if (is_gemv(op.kind)) task_rows(op, (int)(pf.e & 0xFFFFu), pg, r0, r1);
@@ -370,13 +380,36 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     }
   };
 
+  int claim_op = -1;       // dynamic op whose tasks this worker is claiming (-1: none)
+  uint32_t claim_iter = 0;
   while (true) {
     unsigned long long entry;
     if (kStandalone) {
       entry = (fpos == 0) ? pack_entry(sa_iter, (uint32_t)sa_op, blockIdx.x) : QUEUE_TERMINATE;
+    } else if (claim_op >= 0) {
+      // Claim the next task of the dynamic op, now that the ring has taken
+      // the previous one.  Every worker claims until the counter passes the
+      // task count; the last of those ntasks + W claims resets the counter,
+      // whose slot serves iteration claim_iter + CLAIM_SLOTS next.
+      const OpDesc& co = g.ops[claim_op];
+      uint32_t* ctr = g.claims + ((size_t)(claim_iter % CLAIM_SLOTS) * g.nops + claim_op) * EVENT_STRIDE;
+      const uint32_t c = atomicAdd(ctr, 1u);
+      if (c >= (uint32_t)co.ntasks) {
+        if (c == (uint32_t)(co.ntasks + g.num_workers - 1)) atomicExch(ctr, 0u);
+        claim_op = -1;
+        continue;
+      }
+      entry = pack_entry(claim_iter, (uint32_t)claim_op, c);
     } else {
       if (!wait_counter(g, qtail, qpos + 1, 2, -1, -1, worker, -1)) { ok = false; break; }
       entry = __ldcg(queue + (qpos % QUEUE_CAP));
+      if (entry != QUEUE_TERMINATE && (entry & 0xFFFFu) == TASK_CLAIM) {
+        ++qpos;
+        st_release(qhead, qpos);
+        claim_op = (int)((entry >> 16) & 0xFFFFu);
+        claim_iter = (uint32_t)(entry >> 32);
+        continue;
+      }
       // a prefetch cursor that has not passed this task restarts at its first row
       if (pf.q < qpos || (pf.q == qpos && !pf.have)) {
         // the cursor is behind: restart it at this task (the stream offset of
@@ -544,6 +577,11 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   const uint32_t atag = vtag(g, iter, op.a_writer) + op.tag_skew;
   const uint32_t mytag = vtag(g, iter, op.self);
   bool pfail = false;
+  // consecutive claimed tasks of one dynamic op (same segment) share the
+  // input vector already in shared memory
+  const unsigned long long hkey =
+      ((unsigned long long)iter << 32) | ((unsigned long long)op.self << 16) | (unsigned long long)task_seg(op, task);
+  const bool reuse = op.dynamic && sm.h_key == hkey;
   if (KIND == TK_QKV_ATTN) {
     // What this operation's attention needs besides q, k and v, fetched while
     // the input is awaited: the request's position, its RoPE row, and the
@@ -581,7 +619,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 #pragma unroll
     for (int c = 0; c < MAX_K / (CONSUMER_THREADS * 4); ++c) {
       const int k = (c * CONSUMER_THREADS + ctid) * 4;
-      if (k < K) {
+      if (k < K && !reuse) {
         float v[4];
         pfail |= !load_tagged<4>(g, op.a_in + koff + k, atag, v, op.self, worker, (int)iter);
         *reinterpret_cast<float4*>(hs + hperm(k)) = make_float4(v[0], v[1], v[2], v[3]);
@@ -593,7 +631,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
                             (int)iter);
       sm.u.g.xs[j] = xv;
     }
-  } else {
+  } else if (!reuse) {
     // RMSNorm: x and the norm weight are read once into registers, the
     // statistics are reduced in a fixed order.
     constexpr int NCH = MAX_NORM_K / (CONSUMER_THREADS * 8);
@@ -641,6 +679,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     }
   }
   if (consumer_sync_or(pfail)) return false;
+  if (ctid == 0) sm.h_key = hkey;  // every thread read the previous key before the barrier
   if (g.profiling && ctid == 0) sm.t_pro = globaltimer();
 
   const bool capture = (g.capture_iter == (int)iter);
@@ -655,7 +694,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       st_tagged(op.y[sg] + seg_row(op, grp, sg, row), v, mytag);
     } else if (KIND == TK_GEMV_RESID) {
       if (split) {
-        st_tagged(op.kpart + (size_t)(task % op.ksplit) * op.N + row, v, mytag);
+        st_tagged(op.kpart + (size_t)task_seg(op, task) * op.N + row, v, mytag);
         return;
       }
       float xo;
@@ -730,7 +769,7 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
     // to the residual, in segment order.
     // (no fence: the finisher waits for the partials' tags)
     if (ctid == 0) {
-      const uint32_t old = atomicAdd(op.blk_cnt + task / op.ksplit, 1u);
+      const uint32_t old = atomicAdd(op.blk_cnt + task % (op.ntasks / op.ksplit), 1u);
       sm.last = ((old + 1u) % (uint32_t)op.ksplit) == 0u;
     }
     consumer_sync();
@@ -835,6 +874,7 @@ template <int G, int D>
 __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
                           int cw, int lane, uint32_t iter, int worker) {
   const bool fused = mode == ATTN_GROUP;  // state fetched in the projections' prologue
+  if (cw == 0 && lane == 0) sm.h_key = ~0ull;  // the attention scratch overlays the GEMV input vector
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
   constexpr int NSTEP = 4;           // warp steps whose loads are in flight together
@@ -1332,6 +1372,11 @@ __device__ void scheduler_lane(const Graph& g, int si, int lane) {
                           pp, -1, wk, (int)nn))
           return;
       }
+      if (g.ops[p].dynamic) {
+        // every worker claims this op's tasks itself
+        if (!push(pack_entry(n, (uint32_t)p, TASK_CLAIM))) return;
+        continue;
+      }
       const int nt = g.ops[p].ntasks;
       int t0 = ((wk - (int)off) % W + W) % W;
       for (int t = t0; t < nt; t += W)
@@ -1344,6 +1389,7 @@ __device__ void scheduler_lane(const Graph& g, int si, int lane) {
 
 // ------------------------------------------------------------------ kernels
 __device__ __forceinline__ void init_barriers(Smem& sm) {
+  sm.h_key = ~0ull;
   for (int i = 0; i < NSTAGES; ++i) {
     mbar_init(&sm.full[i], 1);
     mbar_init(&sm.empty[i], CONSUMER_WARPS);

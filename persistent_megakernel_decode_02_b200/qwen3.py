@@ -32,14 +32,16 @@ def reduction_split(K: int, max_k: int = _lib.MAX_GEMV_K) -> int:
 
 
 def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
-               block_dim: int = 0, tied: Optional[bool] = None, fused_attention: bool = False) -> List[dict]:
+               block_dim: int = 0, tied: Optional[bool] = None, fused_attention: bool = False,
+               tasks_per_worker: int = 2) -> List[dict]:
     """The fused-layer list (pure host logic, no GPU): one dict per operation with
     the method name and its keyword arguments.  With ``fused_attention`` the q/k/v
     projections and the attention are one operation (tasks grouped per kv head,
     the last task of a group runs its attention); otherwise attention is its own
     split-K operation with ``attn_chunks`` chunks."""
     s = shape
-    gt = gemv_tasks or num_workers
+    gt = gemv_tasks or num_workers                       # fused projections+attention: one task per worker
+    dt = gemv_tasks or num_workers * tasks_per_worker    # claimed GEMV ops: more, smaller tasks
     tied = s.tied if tied is None else tied
     plan: List[dict] = [dict(method="embed_layer", embedding="embed_tokens", output="x", grid_dim=requests,
                              block_dim=block_dim, capture_slot=0)]
@@ -56,22 +58,22 @@ def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_ta
         else:
             plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
                              weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
-                             grid_dim=min(gt, s.q_dim + 2 * s.kv_dim), block_dim=block_dim, eps=s.eps))
+                             grid_dim=min(dt, s.q_dim + 2 * s.kv_dim), block_dim=block_dim, eps=s.eps))
             plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm",
                              k_norm=p + "k_norm", k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
                              grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
                              rope_theta=s.rope_theta))
         plan.append(dict(method="linear_residual_layer", input="o", weight=p + "o_proj", residual="x",
-                         grid_dim=min(gt, s.hidden), block_dim=block_dim))
+                         grid_dim=min(dt, s.hidden), block_dim=block_dim))
         plan.append(dict(method="rmsnorm_linear_silu_mul_layer", input="x",
                          weight_norm=p + "post_attention_layernorm", weight_gate=p + "gate_proj",
-                         weight_up=p + "up_proj", output="a", grid_dim=min(gt, s.intermediate), block_dim=block_dim,
+                         weight_up=p + "up_proj", output="a", grid_dim=min(dt, s.intermediate), block_dim=block_dim,
                          eps=s.eps))
         plan.append(dict(method="linear_residual_layer", input="a", weight=p + "down_proj", residual="x",
-                         grid_dim=min(gt, s.hidden * reduction_split(s.intermediate)), block_dim=block_dim,
+                         grid_dim=min(dt, s.hidden * reduction_split(s.intermediate)), block_dim=block_dim,
                          capture_slot=l + 1))
     plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
-                     weight_lm="embed_tokens" if tied else "lm_head", pred="pred", grid_dim=min(gt, s.vocab),
+                     weight_lm="embed_tokens" if tied else "lm_head", pred="pred", grid_dim=min(dt, s.vocab),
                      block_dim=block_dim, eps=s.eps))
     return plan
 
@@ -109,7 +111,7 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
-                  debug_stall_op: int = 0) -> Decoder:
+                  debug_stall_op: int = 0, dynamic_tasks: bool = True, tasks_per_worker: int = 2) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
@@ -146,9 +148,9 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     if fused_attention is None:
         fused_attention = requests == 1 and max_seq <= FUSED_ATTENTION_MAX_SEQ
     for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim,
-                         fused_attention=fused_attention):
+                         fused_attention=fused_attention, tasks_per_worker=tasks_per_worker if dynamic_tasks else 1):
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
     mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb,
-               debug_stall_op=debug_stall_op)
+               debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks)
     return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)

@@ -58,7 +58,10 @@ def test_layer_plan_structure():
     assert kinds == ["rmsnorm_linear_layer", "attention_layer", "linear_residual_layer",
                      "rmsnorm_linear_silu_mul_layer", "linear_residual_layer"]
     assert plan[2]["grid_dim"] == (8, 9, 1)
-    assert all(p["grid_dim"] == 144 for p in plan[1:-1] if p["method"] != "attention_layer")
+    # claimed GEMV ops get two tasks per worker
+    assert all(p["grid_dim"] == 288 for p in plan[1:-1] if p["method"] != "attention_layer")
+    assert all(p["grid_dim"] == 144 for p in layer_plan(s, 1, 144, 9, tasks_per_worker=1)[1:-1]
+               if p["method"] != "attention_layer")
     assert plan[-1]["weight_lm"] == "lm_head"
     assert layer_plan(sq.QWEN3_0_6B, 1, 144, 4)[-1]["weight_lm"] == "embed_tokens"
     # the down projection of layer l captures residual slot l+1
@@ -83,7 +86,7 @@ def test_reduction_split_rule():
     assert int(re.search(r"#define MPK_MAX_GEMV_K (\d+)", txt).group(1)) == _lib.MAX_GEMV_K
     assert [reduction_split(k) for k in (256, 3072, 4096, 4352, 8192, 12288, 17408)] == [1, 1, 1, 17, 2, 3, 17]
     plan = layer_plan(sq.QWEN3_8B, requests=1, num_workers=144, attn_chunks=9)
-    assert plan[5]["grid_dim"] == 144 and plan[5]["weight"].endswith("down_proj")
+    assert plan[5]["grid_dim"] == 288 and plan[5]["weight"].endswith("down_proj")
 
 
 def test_default_attention_chunks():

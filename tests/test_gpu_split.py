@@ -62,3 +62,24 @@ def test_split_needs_task_multiple(weights):
     _, w = weights
     with pytest.raises(MpkError, match="multiple of 3 tasks"):
         build_decoder(WIDE, w, requests=1, max_seq=S, gemv_tasks=100)
+
+
+def test_split_claimed_tasks_bit_identical_to_fixed_mapping(weights):
+    from persistent_megakernel_decode_02_b200 import build_decoder
+
+    _, w = weights
+    tokens = sq.make_tokens(WIDE, 1, S, [PROMPT], seed=23)
+    outs = []
+    for dynamic in (False, True):
+        dec = build_decoder(WIDE, w, requests=1, max_seq=S, gemv_tasks=96, dynamic_tasks=dynamic)
+        hd = torch.zeros((WIDE.layers + 1, 1, WIDE.hidden), device="cuda")
+        dec.kernel.set_capture(S - 3, None, hd)
+        tok = tokens.cuda()
+        step = torch.zeros(1, dtype=torch.int32, device="cuda")
+        dec.run(step, tok)
+        torch.cuda.synchronize()
+        dec.kernel.check_status()
+        outs.append((tok.cpu(), dec.pred.cpu(), hd.cpu()))
+        dec.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)

@@ -207,3 +207,23 @@ def test_no_active_request_is_a_no_op(weights):
     dec.kernel.check_status()
     assert int(step.item()) == 3
     dec.kernel.close()
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-attention", "split-attention"])
+def test_claimed_tasks_bit_identical_to_fixed_mapping(weights, fused):
+    """Claiming GEMV tasks from a shared counter (whichever worker is free takes
+    the next) gives exactly the results of the fixed task-to-worker mapping with
+    the same task split."""
+    _, w = weights
+    tokens = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=10)
+    outs = []
+    for dynamic in (False, True):
+        dec = _build(w, gemv_tasks=40, fused_attention=fused, dynamic_tasks=dynamic)
+        lg = torch.zeros((1, SHAPE.vocab), device="cuda")
+        hd = torch.zeros((SHAPE.layers + 1, 1, SHAPE.hidden), device="cuda")
+        dec.kernel.set_capture(S - 3, lg, hd)
+        got, _ = _greedy(dec, tokens)
+        outs.append((got, dec.pred.cpu(), lg.cpu(), hd.cpu(), dec.k_cache.cpu().view(torch.int16)))
+        dec.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
