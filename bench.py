@@ -58,6 +58,9 @@ def parse():
     p.add_argument("--timeline-out", default="")
     p.add_argument("--cpu-budget-s", type=float, default=20.0)
     p.add_argument("--prefetch-kb", type=int, default=0, help="L2 prefetch distance per worker (<=0 off)")
+    p.add_argument("--tasks-per-worker", type=int, default=2, help="tasks per worker of the claimed GEMV ops")
+    p.add_argument("--claim-tasks", action="store_true",
+                   help="GEMV ops hand tasks out through a shared counter instead of the fixed mapping")
     p.add_argument("--attention", choices=["auto", "fused", "split"], default="auto")
     p.add_argument("--layers", type=int, default=0, help="override the layer count (profiling cases)")
     p.add_argument("--vocab", type=int, default=0, help="override the vocabulary (profiling cases)")
@@ -339,7 +342,8 @@ def main():
     dec = build_decoder(shape, w, requests=1, max_seq=S, num_workers=W, num_local_schedulers=ls,
                         attn_chunks=args.attn_chunks or None, sched_lookahead=args.lookahead,
                         profiling=args.profiling, prefetch_kb=args.prefetch_kb,
-                        fused_attention={"auto": None, "fused": True, "split": False}[args.attention])
+                        fused_attention={"auto": None, "fused": True, "split": False}[args.attention],
+                        dynamic_tasks=args.claim_tasks, tasks_per_worker=args.tasks_per_worker)
     stream = torch.cuda.current_stream(dev)
     tok = tokens_cpu.to(dev)
     step = torch.zeros(1, dtype=torch.int32, device=dev)

@@ -162,12 +162,12 @@ typedef struct {
     int32_t max_timeline;   /* timeline entries kept when profiling (<=0: 1<<20)         */
     int32_t prefetch_kb;    /* L2 prefetch distance per worker ahead of the shared-memory
                                weight ring, KiB (<=0: off)                                 */
-    int32_t dynamic_tasks;  /* >= 0: the GEMV operations (all but the fused projections +
+    int32_t dynamic_tasks;  /* > 0: the GEMV operations (all but the fused projections +
                                attention) hand their tasks out through a shared counter:
                                each worker claims the next task when its weight ring has
                                room, so the work follows the workers that are ahead;
-                               < 0: fixed mapping, task t on worker (t + offset) % W.
-                               Results are identical either way.                        */
+                               <= 0 (default): fixed mapping, task t on worker
+                               (t + offset) % W.  Results are identical either way.     */
     int32_t debug_stall_op; /* fault injection for tests: k > 0 makes operation k-1 wait
                                for an input nothing will produce (a version of the next
                                iteration, or one completion more than its dependency

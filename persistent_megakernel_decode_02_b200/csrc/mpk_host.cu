@@ -743,7 +743,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   // (its group tasks wait on one another).
   for (int p = 0; p < P; ++p) {
     OpDesc& op = ops[p];
-    op.dynamic = (o.dynamic_tasks >= 0) &&
+    op.dynamic = (o.dynamic_tasks > 0) &&
                  (op.kind == TK_NORM_GEMV || op.kind == TK_GEMV_RESID || op.kind == TK_NORM_GEMV_SILU ||
                   op.kind == TK_NORM_GEMV_ARGMAX) ? 1 : 0;
     if (op.dynamic && op.ntasks >= (int)TASK_CLAIM)

@@ -111,7 +111,7 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
-                  debug_stall_op: int = 0, dynamic_tasks: bool = True, tasks_per_worker: int = 2) -> Decoder:
+                  debug_stall_op: int = 0, dynamic_tasks: bool = False, tasks_per_worker: int = 2) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
