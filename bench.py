@@ -16,6 +16,13 @@ the value counts the tokens of all ranks.
 
 --impl reference times the CPU oracle (the reference arm of this build) on
 the host cores with the same metric.
+
+--workload batch8 measures the batched configuration instead: 8 concurrent
+requests in tokens[8, 1024], prompt lengths uniform in [32, 512], 256 greedy
+tokens each.  The prompts are ingested first (untimed, one decode iteration
+per prompt token), then 256 lock-step iterations (every request one token per
+iteration, each at its own position) run in ONE timed launch; a step is one
+such iteration, reported in ms/step.  The projections run on the tensor cores.
 """
 from __future__ import annotations
 
@@ -39,11 +46,17 @@ METRIC = "decode ms/token (Qwen3-8B-shape, batch 1) and HBM GB/s vs ~8 TB/s peak
 UNIT = "ms/token"
 A100_MPK_MS = 12.5  # the pages' MPK figure on one A100 40GB for this workload (context)
 
+BATCH, BATCH_SEQ, BATCH_PROMPT, BATCH_GENERATED = 8, 1024, (32, 512), 256
+METRIC_BATCH = "decode ms/step (Qwen3-8B-shape, 8 requests) and HBM GB/s vs ~8 TB/s peak"
+UNIT_BATCH = "ms/step"
+
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=512)
+    p.add_argument("--workload", choices=["batch1", "batch8"], default="batch1",
+                   help="batch1: one request, 39-token prompt + 512 tokens (default); batch8: 8 requests")
+    p.add_argument("--steps", type=int, default=0, help="timed steps (default: 512 for batch1, 256 for batch8)")
     p.add_argument("--warmup", type=int, default=8)
     p.add_argument("--impl", choices=["mpk", "reference"], default="mpk")
     p.add_argument("--shape", default="qwen3-8b", help="qwen3-8b (default), qwen3-0.6b or tiny")
@@ -64,7 +77,10 @@ def parse():
     p.add_argument("--attention", choices=["auto", "fused", "split"], default="auto")
     p.add_argument("--layers", type=int, default=0, help="override the layer count (profiling cases)")
     p.add_argument("--vocab", type=int, default=0, help="override the vocabulary (profiling cases)")
-    return p.parse_args()
+    args = p.parse_args()
+    if not args.steps:
+        args.steps = GENERATED if args.workload == "batch1" else BATCH_GENERATED
+    return args
 
 
 def measured_peaks():
@@ -313,10 +329,164 @@ def workload_config(shape, args, dec):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def batch_algorithmic_bytes(shape, first_pos, iters: int) -> int:
+    """Bytes one lock-step iteration of several requests must move, summed over
+    iterations: every streamed weight byte once (shared by the batch), and per
+    request the K/V of positions 0..s read and position s written."""
+    per_pos = shape.kv_bytes_per_position()
+    total = 0
+    for i in range(iters):
+        total += shape.streamed_weight_bytes()
+        for p in first_pos:
+            total += (int(p) + i + 1) * per_pos + per_pos
+    return total
+
+
+def main_batch(args):
+    """The batched configuration: 8 requests, prompts U[32, 512], 256 lock-step
+    decode iterations timed in one launch."""
+    import torch
+    world, rank, local, pg = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from synth import qwen3 as sq
+    from persistent_megakernel_decode_02_b200 import build_decoder, load
+
+    shape = sq.SHAPES[args.shape]
+    R, S, G = BATCH, BATCH_SEQ, BATCH_GENERATED
+    steps = args.steps
+    if not (1 <= steps <= G and 0 <= args.warmup <= G):
+        raise SystemExit(f"--steps must be in 1..{G} and --warmup in 0..{G}")
+    t0 = time.time()
+    w_cpu = sq.make_weights(shape, seed=0)
+    w = {k: v.to(dev) for k, v in w_cpu.items()}
+    t_gen = time.time() - t0
+    lens = sq.make_prompt_lengths(R, BATCH_PROMPT[0], BATCH_PROMPT[1], seed=0)
+    tokens_cpu = sq.make_tokens(shape, R, S, lens, seed=0)
+    ls = args.local_schedulers
+    W = args.workers or (load().mpk_device_sm_count() - ls // 4)
+    dec = build_decoder(shape, w, requests=R, max_seq=S, num_workers=W, num_local_schedulers=ls,
+                        attn_chunks=args.attn_chunks or None, sched_lookahead=args.lookahead,
+                        profiling=args.profiling)
+    stream = torch.cuda.current_stream(dev)
+    tok = tokens_cpu.to(dev)
+    p_end = (lens - 1).to(torch.int32).to(dev)          # each request has consumed its prompt
+    step = torch.zeros(R, dtype=torch.int32, device=dev)
+    dec.run(step, tok, p_end)                            # phase A: prompts (prefill-as-decode)
+    dec.run(step, tok, p_end + args.warmup)              # warm-up iterations
+    torch.cuda.synchronize(dev)
+    dec.kernel.check_status()
+    tok.copy_(tokens_cpu.to(dev))                        # rewind to the end of the prompts
+    step.copy_(p_end)
+    stop = p_end + steps
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(local)
+    clk.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    dec.run(step, tok, stop, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    barrier(pg, dev)
+    dec.kernel.check_status()
+    ms_launch = e0.elapsed_time(e1)
+    assert torch.equal(step, stop), "not every request ran its timed steps"
+    gen = [tok[r, int(lens[r]):int(lens[r]) + steps].cpu() for r in range(R)]
+    assert all(bool((g >= 0).all()) for g in gen), "some timed tokens were not generated"
+    ms_max = max_over_ranks(pg, ms_launch, dev)
+    ms_per_step = ms_max / steps
+    tokens_per_s = 1e3 * R * steps * world / ms_max
+    p_host = (lens - 1).tolist()
+    bytes_launch = batch_algorithmic_bytes(shape, p_host, steps)
+    gbs = bytes_launch / (ms_launch * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    timeline_stats = None
+    if args.profiling:
+        tl = dec.kernel.timeline()
+        if args.timeline_out:
+            write_chrome_trace(tl, dec, args.timeline_out)
+        op_kind.per_layer = (dec.kernel.num_ops() - 2) // shape.layers
+        timeline_stats = timeline_summary(tl, shape)
+
+    # end to end through the public API with host buffers: tokens in from pinned
+    # memory, prompts + the timed steps in one launch, tokens back to the host
+    e2e = None
+    if not args.no_e2e:
+        host_tok = tokens_cpu.clone().pin_memory()
+        host_step = torch.zeros(R, dtype=torch.int32).pin_memory()
+        host_end = ((lens - 1) + steps).to(torch.int32).pin_memory()
+        out_tok = torch.empty_like(host_tok).pin_memory()
+        barrier(pg, dev)
+        torch.cuda.synchronize(dev)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        tok.copy_(host_tok, non_blocking=True)
+        step.copy_(host_step, non_blocking=True)
+        stop.copy_(host_end, non_blocking=True)
+        dec.run(step, tok, stop, stream)
+        out_tok.copy_(tok, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), dev)
+        for r in range(R):
+            assert torch.equal(out_tok[r, int(lens[r]):int(lens[r]) + steps], gen[r]), "e2e tokens differ"
+        e2e = {"value": e2e_ms / steps, "unit": UNIT_BATCH,
+               "h2d_bytes_per_step": (host_tok.numel() * 8 + 8 * R) / steps,
+               "d2h_bytes_per_step": out_tok.numel() * 8 / steps,
+               "includes": "H2D of tokens/step/step_end, every request's prompt iterations + the timed "
+                           "iterations in one launch, D2H of tokens"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms_cpu, n, cores, desc = time_oracle(shape, w_cpu, tokens_cpu, args.cpu_budget_s, layer_sample=2)
+        cpu = {"value": ms_cpu, "unit": UNIT_BATCH, "cores": cores, "kind": "oracle",
+               "sample": desc.replace("of the same request", f"of all {R} requests")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC_BATCH, "value": ms_per_step, "unit": UNIT_BATCH, "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": f"{shape.name}-shape greedy decode, {R} requests, tokens[{R},{S}], prompt lengths "
+                            f"U[{BATCH_PROMPT[0]},{BATCH_PROMPT[1]}] (seed 0), {steps} lock-step tokens each",
+                "requests": R, "prompt_tokens": [int(x) for x in lens], "seq_len": S, "timed_steps": steps,
+                "weights": "seeded synthetic bf16 N(0,0.02), norms 1.0",
+                "projections": "tcgen05 MMA over the batch (bf16 inputs, fp32 accumulate)",
+                "l2": "no flush: every step streams all weights (15.1 GB), larger than the 126 MB L2",
+                "num_workers": dec.kernel.num_workers, "num_local_schedulers": dec.kernel.num_local_schedulers,
+                "parallelism": "replicas"},
+            "tokens_per_s": tokens_per_s,
+            "hbm_gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_launch,
+                         "kernel": "mpk_persistent_batch_kernel"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 1,
+            "clocks": clocks,
+            "timeline": timeline_stats,
+            "setup_s": {"weights": round(t_gen, 1)},
+        }
+        print(json.dumps(line), flush=True)
+    dec.kernel.close()
+    if pg is not None:
+        pg.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "batch8":
+        return main_batch(args)
     import torch
     world, rank, local, pg = dist_setup(args)
     torch.cuda.set_device(local)

@@ -1,0 +1,423 @@
+// Projections of a batch of requests on the tensor cores (tcgen05, sm_100a).
+//
+// With R = 2..MAX_BATCH requests in the graph, every projection of a decoding
+// iteration is a dense contraction Y[R, N] = X[R, K] W^T ("Mirage Persistent
+// Kernel: Fusing Multi-GPU LLM Inference into One Kernel Launch", section "How
+// MPK Works": the same fused layers, now with several requests per step).
+// Tasks form a grid of (row-block runs) x (reduction segments):
+//
+//  * producer: the weight tiles (BM rows x BK elements, 16 KB) come in by 2-D
+//    tiled TMA copies with 128-byte swizzle, two tiles per ring stage, into
+//    NSTB stages of the ring;
+//  * consumers, prologue: the batch's input rows for the task's reduction
+//    segment (after RMSNorm for the norm operations) are split into bf16
+//    hi/lo pairs and written into the ring's remaining stages in the same
+//    swizzled K-major layout: K block b at b * B_KBLOCK_BYTES, the hi rows as
+//    one 8-row atom, the lo rows as the next; request r at 128 r inside an
+//    atom, its 16-byte chunk c at 16 (c ^ r);
+//  * one consumer thread issues the MMAs (M = BM weight rows, N = BN columns,
+//    K = 16 per instruction) into a tensor-memory accumulator and commits each
+//    stage back to the producer;
+//  * the first consumer warpgroup reads the accumulator (lane = weight row,
+//    column = hi/lo input row), adds each request's hi and lo columns and runs
+//    the operation's epilogue, or writes partial sums when the reduction is
+//    split; the last segment task of a row block to arrive adds the partials
+//    in segment order and runs the epilogue.
+//
+// Included by mpk_kernel.cu inside namespace mpk.
+
+// Row blocks [rb0, rb1) and K blocks [kb0, kb1) of a task; seg is its
+// reduction segment.  Task t computes segment t / ntb (of bsplit) for the run
+// of row blocks [u nb / ntb, (u+1) nb / ntb), u = t mod ntb.
+__device__ __forceinline__ void btask(const OpDesc& op, int task, int& rb0, int& rb1, int& kb0, int& kb1, int& seg) {
+  seg = task / op.ntb;
+  const int u = task - seg * op.ntb;
+  rb0 = (int)(((long long)u * op.nb) / op.ntb);
+  rb1 = (int)(((long long)(u + 1) * op.nb) / op.ntb);
+  kb0 = (int)(((long long)seg * op.nkb) / op.bsplit);
+  kb1 = (int)(((long long)(seg + 1) * op.nkb) / op.bsplit);
+}
+
+// Ring stages of one row block: gate/up take one K block of both matrices per
+// stage, the other operations two K blocks of one matrix.
+__device__ __forceinline__ int bstages(const OpDesc& op, int nkbs) {
+  return op.kind == TK_NORM_GEMV_SILU ? nkbs : (nkbs + 1) / 2;
+}
+
+// Producer side of a batched task: its weight tiles, stage by stage.  False on
+// abort or timeout.  t_issue (profiling) receives the first stage's issue time.
+__device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
+                         uint64_t pol, unsigned long long* t_issue) {
+  int rb0, rb1, kb0, kb1, seg;
+  btask(op, task, rb0, rb1, kb0, kb1, seg);
+  const bool pair = op.kind == TK_NORM_GEMV_SILU;
+  for (int rb = rb0; rb < rb1; ++rb) {
+    const int row = rb * BM;
+    const int s = pair ? 0 : seg_of(op, row);
+    const int mrow = row - op.seg_row0[s];  // row within matrix s (rows past its end read as zeros)
+    const void* tm = op.tmap[s];
+    for (int kb = kb0; kb < kb1; kb += pair ? 1 : 2) {
+      const uint32_t slot = pstage % NSTB;
+      const uint32_t par = ((pstage / NSTB) & 1u) ^ 1u;
+      if (!wait_mbar(g, &sm.empty[slot], par, 3, worker)) return false;
+      if (t_issue != nullptr && rb == rb0 && kb == kb0) atomicExch(t_issue, (unsigned long long)globaltimer());
+      const int nbox = pair ? 2 : min(2, kb1 - kb);
+      mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)(nbox * BOX_BYTES));
+      tma_load_2d(sm.ring[slot], tm, kb * BK, mrow, &sm.full[slot], pol);
+      if (pair) tma_load_2d(sm.ring[slot] + BOX_BYTES, op.tmap_up, kb * BK, mrow, &sm.full[slot], pol);
+      else if (nbox == 2) tma_load_2d(sm.ring[slot] + BOX_BYTES, tm, (kb + 1) * BK, mrow, &sm.full[slot], pol);
+      ++pstage;
+    }
+  }
+  return true;
+}
+
+// Epilogue of output row `row` for every request: v[r] is the row's dot
+// product with request r's input (gate/up: v gate, u up).  RESID leaves the
+// new residual values in nx (0 for rows past the end), for the block's sums
+// of squares.
+template <int KIND>
+__device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int row, const float* v, const float* u,
+                                          uint32_t iter, uint32_t xtag, uint32_t mytag, bool capture,
+                                          unsigned long long (&best)[MAX_BATCH], float (&nx)[MAX_BATCH],
+                                          bool& fail, int worker) {
+  const int R = g.R;
+  if (KIND == TK_NORM_GEMV) {
+    const int s = seg_of(op, row);
+    const int local = row - op.seg_row0[s], ns = op.grp_rows[s];
+#pragma unroll
+    for (int r = 0; r < MAX_BATCH; ++r)
+      if (r < R) st_tagged(op.y[s] + (size_t)r * ns + local, v[r], mytag);
+  } else if (KIND == TK_GEMV_RESID) {
+    uint64_t w[MAX_BATCH];
+#pragma unroll
+    for (int r = 0; r < MAX_BATCH; ++r) w[r] = r < R ? ld_tagged(op.x_out + (size_t)r * op.N + row) : 0ull;
+#pragma unroll
+    for (int r = 0; r < MAX_BATCH; ++r) {
+      if (r < R) {
+        uint64_t* p = op.x_out + (size_t)r * op.N + row;
+        if (word_tag(w[r]) != xtag) {
+          w[r] = poll_word(g, p, xtag, op.self, worker, (int)iter);
+          fail |= word_tag(w[r]) != xtag;
+        }
+        nx[r] = word_value(w[r]) + v[r];
+        st_tagged(p, nx[r], mytag);
+        if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
+          g.cap_hidden[((size_t)op.capture_slot * R + r) * g.H + row] = nx[r];
+      }
+    }
+  } else if (KIND == TK_NORM_GEMV_SILU) {
+#pragma unroll
+    for (int r = 0; r < MAX_BATCH; ++r)
+      if (r < R) st_tagged(op.a_out + (size_t)r * op.N + row, silu_f(v[r]) * u[r], mytag);
+  } else {  // LM head
+#pragma unroll
+    for (int r = 0; r < MAX_BATCH; ++r) {
+      if (r < R) {
+        const unsigned long long key = argmax_key(v[r], (uint32_t)row);
+        best[r] = key > best[r] ? key : best[r];
+        if (capture && g.cap_logits != nullptr) g.cap_logits[(size_t)r * g.V + row] = v[r];
+      }
+    }
+  }
+}
+
+// Two bf16 (bits) in one word, element k in the low half.
+__device__ __forceinline__ uint32_t pack2(uint16_t a, uint16_t b) { return (uint32_t)a | ((uint32_t)b << 16); }
+
+// hi = bf16(v) and lo = bf16(v - hi) of eight values (v - hi is exact in fp32).
+__device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo) {
+  uint16_t h[8], l[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    h[e] = f32_to_bf16_rn(v[e]);
+    l[e] = f32_to_bf16_rn(v[e] - __uint_as_float((uint32_t)h[e] << 16));
+  }
+  hi = make_uint4(pack2(h[0], h[1]), pack2(h[2], h[3]), pack2(h[4], h[5]), pack2(h[6], h[7]));
+  lo = make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
+}
+
+// Consumer side of a batched task (all CONSUMER_THREADS threads).  cstage
+// counts ring stages, accn accumulator uses; both advance identically in every
+// consumer thread.  Roles inside the task: consumer warp MMA_WARP's lane 0
+// issues every row block's MMAs, alternating between two tensor-memory
+// accumulators; warps 0..3 (tensor-memory lanes 0..127, one weight row per
+// thread) read each accumulator as soon as it is complete and run the
+// epilogue, so the next block's MMAs overlap it.
+template <int KIND>
+__device__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter, uint32_t& cstage,
+                           uint32_t& accn, int cw, int lane, int worker) {
+  constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
+  constexpr bool NORM = KIND != TK_GEMV_RESID;
+  constexpr int MMA_WARP = 4;
+  const int ctid = cw * 32 + lane;
+  const int R = g.R;
+  int rb0, rb1, kb0, kb1, seg;
+  btask(op, task, rb0, rb1, kb0, kb1, seg);
+  const int nkbs = kb1 - kb0;
+  const int nst = bstages(op, nkbs);
+  const int nblk = rb1 - rb0;
+  const bool split = op.bsplit > 1;
+  uint8_t* bsm = sm.ring[NSTB];
+  const uint32_t xtag = vtag(g, iter, op.x_writer) + op.tag_skew;
+  const uint32_t atag = vtag(g, iter, op.a_writer) + op.tag_skew;
+  const uint32_t mytag = vtag(g, iter, op.self);
+  const uint64_t* src = NORM ? op.x : op.a_in;
+  const uint32_t stag = NORM ? xtag : atag;
+  bool pfail = false;
+
+  // ---- prologue.  RMSNorm factor of every request from the per-block sums of
+  // squares its writer published (warp r: request r, blocks in a fixed order).
+  if (NORM) {
+    if (cw < R) {
+      float ss = 0.f;
+      for (int b = lane; b < op.xss_blocks; b += 32) {
+        const uint64_t* p = op.xss_in + (size_t)b * R + cw;
+        uint64_t w = ld_tagged(p);
+        if (word_tag(w) != stag) {
+          w = poll_word(g, p, stag, op.self, worker, (int)iter);
+          pfail |= word_tag(w) != stag;
+        }
+        ss += word_value(w);
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) sm.brinv[cw] = 1.0f / sqrtf(ss / (float)op.K + op.eps);
+    }
+    consumer_sync();
+  }
+  // The input rows of the segment as bf16 hi/lo pairs into the swizzled
+  // layout; FL chunks of 8 elements per thread in flight.
+  {
+    const int nch = nkbs * 8;  // 16-byte chunks per request row
+    const int total = MAX_BATCH * nch;
+    constexpr int FL = 2;
+    for (int q0 = ctid; q0 < total; q0 += FL * CONSUMER_THREADS) {
+      uint64_t w[FL][8];
+#pragma unroll
+      for (int u = 0; u < FL; ++u) {
+        const int q = q0 + u * CONSUMER_THREADS;
+        const int r = q / nch;
+        if (q < total && r < R) {
+          const uint64_t* p = src + (size_t)r * op.K + (size_t)kb0 * BK + (size_t)(q - r * nch) * 8;
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) ld_tagged2(p + e, w[u][e], w[u][e + 1]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < FL; ++u) {
+        const int q = q0 + u * CONSUMER_THREADS;
+        if (q < total) {
+          const int r = q / nch, cc = q - r * nch;
+          const int kbl = cc >> 3, ch = cc & 7;
+          uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+          if (r < R) {
+            const int k = kb0 * BK + cc * 8;
+            const uint64_t* p = src + (size_t)r * op.K + k;
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if (word_tag(w[u][e]) != stag) {
+                w[u][e] = poll_word(g, p + e, stag, op.self, worker, (int)iter);
+                pfail |= word_tag(w[u][e]) != stag;
+              }
+              v[e] = word_value(w[u][e]);
+            }
+            if (NORM) {
+              const uint4 nw = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
+              const float ri = sm.brinv[r];
+              v[0] = v[0] * ri * bf16_lo(nw.x); v[1] = v[1] * ri * bf16_hi(nw.x);
+              v[2] = v[2] * ri * bf16_lo(nw.y); v[3] = v[3] * ri * bf16_hi(nw.y);
+              v[4] = v[4] * ri * bf16_lo(nw.z); v[5] = v[5] * ri * bf16_hi(nw.z);
+              v[6] = v[6] * ri * bf16_lo(nw.w); v[7] = v[7] * ri * bf16_hi(nw.w);
+            }
+            split8(v, hi, lo);
+          }
+          uint8_t* dst = bsm + kbl * B_KBLOCK_BYTES + r * (BK * 2) + ((ch ^ r) << 4);
+          *reinterpret_cast<uint4*>(dst) = hi;
+          *reinterpret_cast<uint4*>(dst + B_KBLOCK_BYTES / 2) = lo;
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();  // the tensor cores read these bytes next
+  if (consumer_sync_or(pfail)) return false;
+  if (g.profiling && ctid == 0) sm.t_pro = globaltimer();
+
+  // ---- row blocks
+  const uint32_t tmem = sm.tmem_base;
+  const int nrows = op.N;
+  const size_t NP = (size_t)(PAIR ? 2 : 1) * (size_t)nrows;  // partial-sum row length
+  bool fail = false;
+  unsigned long long best[MAX_BATCH];
+#pragma unroll
+  for (int r = 0; r < MAX_BATCH; ++r) best[r] = 0ull;
+  if (cw == MMA_WARP) {
+    if (lane == 0) {
+      const uint32_t idesc = mma_idesc_bf16(BM, BN);
+      bool ok = true;
+      for (int i = 0; i < nblk; ++i) {
+        const uint32_t a = accn + (uint32_t)i, buf = a & 1u, use = a >> 1;
+        // the epilogue has read this accumulator's previous block
+        if (ok) ok = wait_mbar(g, &sm.acc_empty[buf], (use & 1u) ^ 1u, 3, worker);
+        tc_fence_after_sync();
+        const uint32_t dacc = tmem + buf * (uint32_t)(2 * BN);
+        for (int st = 0; ok && st < nst; ++st) {
+          const uint32_t cs = cstage + (uint32_t)(i * nst + st);
+          const uint32_t slot = cs % NSTB;
+          const uint64_t w0 = g.profiling ? globaltimer() : 0ull;
+          ok = wait_mbar(g, &sm.full[slot], (cs / NSTB) & 1u, 3, worker);
+          if (g.profiling) {
+            const uint64_t w1 = globaltimer();
+            sm.t_stall += w1 - w0;
+            sm.t_last = w1;
+            if (i == 0 && st == 0) sm.t_data = w1;
+          }
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t a0 = smem_u32(sm.ring[slot]);
+          if (PAIR) {
+            const uint32_t b0 = smem_u32(bsm) + (uint32_t)st * B_KBLOCK_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t bd = sw128_desc(b0 + kk * 32);
+              const uint32_t acc = (st | kk) != 0;
+              mma_bf16_ss(dacc, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+              mma_bf16_ss(dacc + BN, sw128_desc(a0 + BOX_BYTES + kk * 32), bd, idesc, acc);
+            }
+          } else {
+            const int nbox = min(2, nkbs - 2 * st);
+            for (int b = 0; b < nbox; ++b) {
+              const uint32_t b0 = smem_u32(bsm) + (uint32_t)(2 * st + b) * B_KBLOCK_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                mma_bf16_ss(dacc, sw128_desc(a0 + b * BOX_BYTES + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                            (st | b | kk) != 0);
+            }
+          }
+          mma_commit(&sm.empty[slot]);  // the stage returns to the producer once these MMAs have read it
+        }
+        mma_commit(&sm.acc_full[buf]);  // also after a failure: it ends the epilogue's wait
+      }
+      fail = !ok;
+    }
+    __syncwarp();
+  } else if (cw < 4) {
+    const bool capture = (g.capture_iter == (int)iter);
+    const uint32_t lanes = (uint32_t)(cw * 32) << 16;
+    for (int i = 0; i < nblk; ++i) {
+      const int rb = rb0 + i;
+      const uint32_t a = accn + (uint32_t)i, buf = a & 1u, use = a >> 1;
+      bool ok = true;
+      if (lane == 0) ok = wait_mbar(g, &sm.acc_full[buf], use & 1u, 3, worker);
+      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+      tc_fence_after_sync();
+      float d[16], du[16];
+      const uint32_t dacc = tmem + buf * (uint32_t)(2 * BN) + lanes;
+      tmem_ld16(dacc, d);
+      if (PAIR) tmem_ld16(dacc + BN, du);
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+      fail |= !ok;
+      // W hi + W lo per request
+      float v[MAX_BATCH], u[MAX_BATCH], nx[MAX_BATCH];
+#pragma unroll
+      for (int r = 0; r < MAX_BATCH; ++r) {
+        v[r] = d[r] + d[MAX_BATCH + r];
+        u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
+        nx[r] = 0.f;
+      }
+      const int row = rb * BM + cw * 32 + lane;
+      bool finish = !split;  // this task runs the block's epilogue
+      if (split) {
+        if (ok && row < nrows) {
+          float* pp = op.bpart + (size_t)seg * R * NP;
+#pragma unroll
+          for (int r = 0; r < MAX_BATCH; ++r) {
+            if (r < R) {
+              pp[(size_t)r * NP + row] = v[r];
+              if (PAIR) pp[(size_t)r * NP + nrows + row] = u[r];
+            }
+          }
+        }
+        // The last segment task of this row block to arrive adds the partial
+        // sums in segment order and runs the epilogue.
+        epi_sync();
+        if (ctid == 0) {
+          __threadfence();
+          const uint32_t old = atomicAdd(op.blk_cnt + rb, 1u);
+          sm.blast = ((old + 1u) % (uint32_t)op.bsplit) == 0u;
+        }
+        epi_sync();
+        finish = sm.blast != 0;
+        if (finish) {
+          __threadfence();
+          if (row < nrows) {
+            for (int sg = 0; sg < op.bsplit; ++sg) {
+              const float* pp = op.bpart + (size_t)sg * R * NP;
+#pragma unroll
+              for (int r = 0; r < MAX_BATCH; ++r) {
+                if (r < R) {
+                  const float pa = __ldcg(pp + (size_t)r * NP + row);
+                  v[r] = sg == 0 ? pa : v[r] + pa;
+                  if (PAIR) {
+                    const float pb = __ldcg(pp + (size_t)r * NP + nrows + row);
+                    u[r] = sg == 0 ? pb : u[r] + pb;
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+      if (finish) {
+        if (ok && row < nrows) bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
+        if (KIND == TK_GEMV_RESID && op.xss_out != nullptr) {
+          // the block's sums of squares of the new x, per request: lanes, then
+          // warps 0..3 in order
+#pragma unroll
+          for (int r = 0; r < MAX_BATCH; ++r) {
+            const float ssr = warp_sum(nx[r] * nx[r]);
+            if (lane == 0) sm.bss[i & 1][cw][r] = ssr;
+          }
+          epi_sync();
+          if (ctid < R) {
+            const float t = sm.bss[i & 1][0][ctid] + sm.bss[i & 1][1][ctid] + sm.bss[i & 1][2][ctid] +
+                            sm.bss[i & 1][3][ctid];
+            st_tagged(op.xss_out + (size_t)rb * R + ctid, t, mytag);
+          }
+        }
+      }
+    }
+  }
+  accn += (uint32_t)nblk;
+  cstage += (uint32_t)(nblk * nst);
+  if (consumer_sync_or(fail)) return false;
+  if (g.profiling && ctid == 0) sm.t_loop = globaltimer();
+
+  if (KIND == TK_NORM_GEMV_ARGMAX) {
+    // per-request maxima of the task -> one 64-bit atomicMax each; the last
+    // task of the operation to arrive writes the tokens
+    if (cw < 4) {
+#pragma unroll
+      for (int r = 0; r < MAX_BATCH; ++r) {
+        const unsigned long long b = warp_max_u64(best[r]);
+        if (lane == 0) sm.bbest[cw][r] = b;
+      }
+    }
+    consumer_sync();
+    if (ctid == 0) {
+      for (int r = 0; r < R; ++r) {
+        unsigned long long b = 0ull;
+        for (int w = 0; w < 4; ++w) b = sm.bbest[w][r] > b ? sm.bbest[w][r] : b;
+        if (b != 0ull) atomicMax(op.keys + r, b);
+      }
+      __threadfence();
+      const uint32_t old = atomicAdd(op.arrive, 1u);
+      sm.last = ((old + 1u) % (uint32_t)op.ntasks) == 0u;
+    }
+    consumer_sync();
+    argmax_tokens(sm, g, op, iter, ctid);
+  }
+  return true;
+}

@@ -1,6 +1,8 @@
 // Host side of the C ABI declared in include/mpk.h: tensor registry, graph
 // compiler (validation, task split, event assignment, workspace layout) and
 // the launch of the persistent kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -153,6 +155,72 @@ int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats, bool norm) {
   if (rps < 1) return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: one weight row (%d bytes) exceeds a stage", li, row_bytes);
   if (rps > MAX_RPS) rps = MAX_RPS;
   o.rps = rps;
+  return MPK_OK;
+}
+
+// Tensor-core geometry of a projection over R >= 2 requests: row blocks of BM,
+// K blocks of BK; grid_dim = (tasks per reduction segment, reduction segments,
+// 1).  Task t computes segment t / gx for the run of row blocks
+// [u nb / gx, (u+1) nb / gx), u = t mod gx, so gx <= nb; each segment must fit
+// the input buffer (B_MAX_KBLOCKS blocks).
+int batched_geometry(mpk_ctx* c, int li, OpDesc& o, int R, const mpk_layer& Ly) {
+  if (R > MAX_BATCH)
+    return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: %d requests (the batched projections take at most %d)", li, R,
+                MAX_BATCH);
+  if (o.K % BK != 0)
+    return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d is not a multiple of %d", li, o.K, BK);
+  for (int s = 1; s < o.nseg; ++s)
+    if (o.seg_row0[s] % BM != 0)
+      return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: stacked matrix %d starts at row %d, not a multiple of %d", li, s,
+                  o.seg_row0[s], BM);
+  const int gx = Ly.grid_dim.x, gy = Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1,
+            gz = Ly.grid_dim.z > 0 ? Ly.grid_dim.z : 1;
+  o.batched = 1;
+  o.nb = (o.N + BM - 1) / BM;
+  o.nkb = o.K / BK;
+  o.ntb = gx;
+  o.bsplit = gy;
+  if (gz != 1)
+    return fail(c, MPK_ERR_SHAPE, "layer %d: a batched projection takes grid_dim = (row-block tasks, reduction "
+                "segments, 1)", li);
+  if (gx > o.nb)
+    return fail(c, MPK_ERR_SHAPE, "layer %d: %d rows are %d blocks of %d: grid_dim.x = %d tasks per segment is more",
+                li, o.N, o.nb, BM, gx);
+  if (gy > o.nkb)
+    return fail(c, MPK_ERR_SHAPE, "layer %d: grid_dim.y = %d segments for a reduction of %d blocks of %d", li, gy,
+                o.nkb, BK);
+  const int longest = (o.nkb + gy - 1) / gy;
+  if (longest > B_MAX_KBLOCKS)
+    return fail(c, MPK_ERR_SHAPE,
+                "layer %d: reduction length %d in %d segment(s) leaves %d elements per task (at most %d): "
+                "grid_dim.y must be at least %d", li, o.K, gy, longest * BK, B_MAX_KBLOCKS * BK,
+                (o.nkb + B_MAX_KBLOCKS - 1) / B_MAX_KBLOCKS);
+  o.dynamic = 0;
+  return MPK_OK;
+}
+
+// Tensor map of a bf16 [rows, K] row-major matrix for BM x BK tiles with
+// 128-byte swizzle (the layout the MMA's shared-memory descriptors describe).
+int make_weight_map(mpk_ctx* c, int li, CUtensorMap* m, const void* ptr, int64_t rows, int64_t K) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return fail(c, MPK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(c, MPK_ERR_CUDA, "layer %d: tensor map of a [%lld, %lld] weight failed (CUresult %d)", li,
+                (long long)rows, (long long)K, (int)r);
   return MPK_OK;
 }
 
@@ -407,9 +475,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
           op.seg_row0[1] = op.N;
           op.x_out = (uint64_t*)out->ptr;
           op.x = (const uint64_t*)out->ptr;
-          if (op.K > MAX_K) {
-            // Split the reduction into the fewest segments that fit the input
-            // buffer; task t computes segment t % ksplit of row block t / ksplit.
+          if (op.K > MAX_K && x->dims[0] < 2) {
+            // One request: split the reduction into the fewest segments that
+            // fit the input buffer (several requests split it on their own
+            // terms, see batched_geometry).
             int ks = (op.K + MAX_K - 1) / MAX_K;
             while (ks <= op.K / 256 && (op.K % ks != 0 || (op.K / ks) % 256 != 0)) ++ks;
             if (ks > op.K / 256)
@@ -491,13 +560,20 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         }
         if (R < 0) R = (int)x->dims[0];
         SHAPE_CHECK(x->dims[0] == R, "layer %d: %lld requests, graph has %d", li, (long long)x->dims[0], R);
-        if (R != 1)
-          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: projections with %d requests are not built yet (1 supported)",
-                      li, R);
-        int rc = gemv_geometry(c, li, op, silu, !resid);
-        if (rc != MPK_OK) return rc;
-        rc = check_grid(c, li, Ly, ntasks, op.N * (op.ksplit > 1 ? op.ksplit : 1));
-        if (rc != MPK_OK) return rc;
+        if (R >= 2) {
+          // several requests: the projection is a dense contraction on the tensor cores
+          op.ksplit = 0;
+          op.kseg = 0;
+          int rc = batched_geometry(c, li, op, R, Ly);
+          if (rc != MPK_OK) return rc;
+          rc = check_grid(c, li, Ly, ntasks, 0);
+          if (rc != MPK_OK) return rc;
+        } else {
+          int rc = gemv_geometry(c, li, op, silu, !resid);
+          if (rc != MPK_OK) return rc;
+          rc = check_grid(c, li, Ly, ntasks, op.N * (op.ksplit > 1 ? op.ksplit : 1));
+          if (rc != MPK_OK) return rc;
+        }
         op.signal_per_task = lmh ? 0 : 1;
         op.out_trigger = lmh ? 1 : ntasks;
         if (resid && H < 0) H = op.N;
@@ -601,8 +677,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
                     dims_str(v->dims).c_str(), dims_str(o->dims).c_str());
         SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range", li, Ly.layer);
         if (R != 1)
-          return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: projections with %d requests are not built yet (1 supported)",
-                      li, R);
+          return fail(c, MPK_ERR_UNSUPPORTED,
+                      "layer %d: the fused projections + attention operation serves one request (got %d); several "
+                      "requests take RMSNORM_LINEAR + ATTENTION", li, R);
         const int G = Hq / Hkv;
         if (!((d == 64 || d == 128) && (G == 1 || G == 2 || G == 4)))
           return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: head_dim %d with %d query heads per kv head", li, d, G);
@@ -743,7 +820,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   // (its group tasks wait on one another).
   for (int p = 0; p < P; ++p) {
     OpDesc& op = ops[p];
-    op.dynamic = (o.dynamic_tasks > 0) &&
+    op.dynamic = (o.dynamic_tasks > 0) && !op.batched &&
                  (op.kind == TK_NORM_GEMV || op.kind == TK_GEMV_RESID || op.kind == TK_NORM_GEMV_SILU ||
                   op.kind == TK_NORM_GEMV_ARGMAX) ? 1 : 0;
     if (op.dynamic && op.ntasks >= (int)TASK_CLAIM)
@@ -795,6 +872,19 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   const size_t o_merge = take(sizeof(uint32_t) * (merge_u32 ? merge_u32 : 1));
   const size_t o_tln = take(line);
   const size_t o_blk = take(sizeof(uint32_t) * (blk_u32 ? blk_u32 : 1));
+  // batched projections with a split reduction: their own row-block counters
+  // and partial sums per operation (consecutive projections can overlap)
+  std::vector<size_t> bblk_off(P, 0), bpart_off(P, 0);
+  size_t bblk_u32 = 0, bpart_floats = 0;
+  for (int p = 0; p < P; ++p) {
+    const OpDesc& op = ops[p];
+    if (!op.batched || op.bsplit <= 1) continue;
+    bblk_off[p] = bblk_u32;
+    bblk_u32 += (size_t)op.nb;
+    bpart_off[p] = bpart_floats;
+    bpart_floats += (size_t)op.bsplit * R * op.N * (op.kind == TK_NORM_GEMV_SILU ? 2 : 1);
+  }
+  const size_t o_bblk = take(sizeof(uint32_t) * (bblk_u32 ? bblk_u32 : 1));
   c->sync_bytes = off;
   uint8_t* sb = nullptr;
   int rc = alloc(c, &sb, off);
@@ -826,6 +916,75 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     rc = alloc(c, &rope_dev[i], tab.size() * sizeof(float2));
     if (rc != MPK_OK) return rc;
     CUDA_OR_FAIL(c, cudaMemcpy(rope_dev[i], tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice));
+  }
+  float* bpart = nullptr;
+  if (bpart_floats) {
+    rc = alloc(c, &bpart, sizeof(float) * bpart_floats);
+    if (rc != MPK_OK) return rc;
+  }
+  // tensor maps of the batched projections' weights (64-byte aligned device copies)
+  std::vector<CUtensorMap> tmaps;
+  std::vector<std::pair<int, int>> tmap_of;  // (op, slot): slot MAX_SEG = the up matrix
+  for (int p = 0; p < P; ++p) {
+    const OpDesc& op = ops[p];
+    if (!op.batched) continue;
+    for (int sg = 0; sg <= MAX_SEG; ++sg) {
+      const void* w = sg < MAX_SEG ? (sg < op.nseg ? op.W[sg] : nullptr)
+                                   : (op.kind == TK_NORM_GEMV_SILU ? op.W_up : nullptr);
+      if (!w) continue;
+      const int64_t rows = (sg < MAX_SEG && op.nseg > 1) ? op.grp_rows[sg] : op.N;
+      CUtensorMap m;
+      rc = make_weight_map(c, p, &m, w, rows, op.K);
+      if (rc != MPK_OK) return rc;
+      tmaps.push_back(m);
+      tmap_of.push_back({p, sg});
+    }
+  }
+  if (!tmaps.empty()) {
+    CUtensorMap* tm_dev = nullptr;
+    rc = alloc(c, &tm_dev, sizeof(CUtensorMap) * tmaps.size());
+    if (rc != MPK_OK) return rc;
+    CUDA_OR_FAIL(c, cudaMemcpy(tm_dev, tmaps.data(), sizeof(CUtensorMap) * tmaps.size(), cudaMemcpyHostToDevice));
+    for (size_t i = 0; i < tmap_of.size(); ++i) {
+      OpDesc& op = ops[tmap_of[i].first];
+      if (tmap_of[i].second < MAX_SEG) op.tmap[tmap_of[i].second] = tm_dev + i;
+      else op.tmap_up = tm_dev + i;
+    }
+  }
+  for (int p = 0; p < P; ++p) {
+    OpDesc& op = ops[p];
+    if (op.batched && op.bsplit > 1) {
+      op.bpart = bpart + bpart_off[p];
+      op.blk_cnt = reinterpret_cast<uint32_t*>(sb + o_bblk) + bblk_off[p];
+    }
+  }
+  if (R >= 2) {
+    // per-block sums of squares of every residual stream (tagged, versioned
+    // like the stream itself): one buffer per x tensor, published by its
+    // writers, read by the RMSNorm operations
+    std::map<const void*, uint64_t*> xss;
+    for (int p = 0; p < P; ++p) {
+      OpDesc& op = ops[p];
+      if (op.kind != TK_EMBED && op.kind != TK_GEMV_RESID) continue;
+      uint64_t*& buf = xss[op.x_out];
+      const size_t words = (size_t)((op.N + BM - 1) / BM) * R;
+      if (!buf) {
+        rc = alloc(c, &buf, words * sizeof(uint64_t));
+        if (rc != MPK_OK) return rc;
+        c->zero_each_run.push_back({buf, words * sizeof(uint64_t)});
+      }
+      op.xss_out = buf;
+      op.xss_blocks = (op.N + BM - 1) / BM;
+    }
+    for (int p = 0; p < P; ++p) {
+      OpDesc& op = ops[p];
+      if (op.kind != TK_NORM_GEMV && op.kind != TK_NORM_GEMV_SILU && op.kind != TK_NORM_GEMV_ARGMAX) continue;
+      auto it = xss.find(op.x);
+      if (it == xss.end())
+        return fail(c, MPK_ERR_INVALID_ARG, "layer %d: its input is written by no embedding or residual operation", p);
+      op.xss_in = it->second;
+      op.xss_blocks = (op.K + BM - 1) / BM;
+    }
   }
   unsigned long long* timeline = nullptr;
   if (o.profiling) {
@@ -862,6 +1021,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   memset(&g, 0, sizeof(g));
   g.ops = c->ops_dev;
   g.nops = P;
+  g.batched = R >= 2 ? 1 : 0;
   g.R = R;
   g.V = V;
   g.H = H;

@@ -42,6 +42,26 @@ constexpr int MAX_D = 128;                  // head dim
 constexpr int MAX_GCHUNK = 8;               // fused op: attention chunks per kv head (tasks 0.. of the group)
 constexpr int SCHED_WARPS_PER_SM = 4;
 
+// Tensor-core path (an operation over 2..MAX_BATCH requests): every
+// projection is a dense contraction [R, K] x W^T computed by tcgen05 MMAs of
+// M = BM weight rows x N = BN columns, K in blocks of BK elements.  The fp32
+// input of request r is split into two bf16 rows, hi = bf16(h) in column r and
+// lo = bf16(h - hi) in column MAX_BATCH + r, so one MMA yields W hi + W lo: the
+// contraction sees the input to about 16 significant bits, with the weights
+// exact.  Weights arrive as BM x BK tiles (TMA, 128-byte swizzle); the input
+// rows are held in the ring's last stages in the same layout; accumulators
+// live in tensor memory.
+constexpr int MAX_BATCH = 8;
+constexpr int BM = 128;                     // weight rows per MMA (tensor-memory lanes)
+constexpr int BN = 2 * MAX_BATCH;           // MMA N: hi columns, then lo columns (a valid shape for M = 128)
+constexpr int BK = 64;                      // K elements per tile row (128 bytes)
+constexpr int BOX_BYTES = BM * BK * 2;      // one weight tile: 16 KB
+constexpr int NSTB = 5;                     // weight stages of the ring in this mode
+constexpr int B_MAX_KBLOCKS = 24;           // longest reduction segment held for the inputs: 1536
+constexpr int B_KBLOCK_BYTES = BN * BK * 2; // the hi and lo rows of one K block: two 1 KB swizzle atoms
+static_assert(STAGE_BYTES == 2 * BOX_BYTES, "a weight stage holds two tiles");
+static_assert(MAX_BATCH == 8, "one 8-row swizzle atom per half of the input columns");
+
 enum TaskKind : int32_t {
   TK_EMBED = 1,
   TK_NORM_GEMV = 2,
@@ -112,6 +132,21 @@ struct OpDesc {
   int32_t out_event;            // event this op signals
   int32_t out_trigger;          // increments of out_event per iteration
   int32_t signal_per_task;      // 1: every task signals; 0: merges / finisher signal
+  // tensor-core path (batched)
+  int32_t batched;              // 1: the projection runs as tcgen05 MMAs over the batch
+  int32_t nb;                   // row blocks of BM rows (gate/up: of one matrix)
+  int32_t nkb;                  // K blocks of BK elements
+  int32_t bsplit;               // reduction segments (grid_dim.y)
+  int32_t ntb;                  // tasks per segment (grid_dim.x), each owning a run of row blocks
+  const void* tmap[MAX_SEG];    // tensor maps of W[s] (device memory, 64-byte aligned)
+  const void* tmap_up;          // SILU: tensor map of the up matrix
+  float* bpart;                 // bsplit > 1: partial sums [bsplit][R][rows] (gate/up: rows = 2N)
+  // per-block sums of squares of x (batched graphs): EMBED and RESID publish
+  // them for every BM-row block of the x they write, tagged [blocks][R]; the
+  // RMSNorm operations read them instead of the whole of x
+  uint64_t* xss_out;
+  const uint64_t* xss_in;
+  int32_t xss_blocks;
 };
 
 struct Status {
@@ -138,6 +173,7 @@ struct Graph {
   const OpDesc* ops;
   int32_t nops;
   int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
+  int32_t batched;                  // 1: projections run on the tensor-core path (R >= 2)
   int32_t R, S, V, H, L;
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;

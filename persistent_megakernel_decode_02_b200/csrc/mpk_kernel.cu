@@ -72,7 +72,18 @@ struct __align__(128) Smem {
   int32_t attn_s;   // fused QKV + attention: position of the request (-1: inactive), read in the prologue
   unsigned long long h_key;  // (iteration, op, segment) whose input vector hs holds (~0: none)
   float2 rope_row[MAX_D / 2];                    // its RoPE (cos, sin) row
+  // tensor-core path
+  uint64_t acc_full[2];                          // accumulator b holds a finished row block
+  uint64_t acc_empty[2];                         // accumulator b has been read (one arrival per epilogue warp)
+  uint64_t fin_bar;                              // drain of outstanding MMAs before exit
+  uint32_t tmem_base;                            // tensor-memory address of the accumulators
+  int32_t blast;                                 // this task finishes the current row block
+  float brinv[MAX_BATCH];                        // per-request RMSNorm factor of the task's input
+  float bss[2][4][MAX_BATCH];                    // per block parity, epilogue warp, request: sums of squares
+  unsigned long long bbest[4][MAX_BATCH];        // LM head: per epilogue warp and request (value, index) maxima
 };
+static_assert((NSTAGES - NSTB) * STAGE_BYTES + sizeof(((Smem*)nullptr)->u) >= B_MAX_KBLOCKS * B_KBLOCK_BYTES,
+              "the batch input rows fit in the stages the ring leaves free and the scratch after them");
 
 // ------------------------------------------------------------------ status / waits
 __device__ __forceinline__ bool aborted(const Graph& g) {
@@ -161,6 +172,19 @@ __device__ __noinline__ bool poll_tagged(const Graph& g, const uint64_t* p, uint
       v = 0.f;
       return false;
     }
+  }
+}
+
+// The word at p once it carries `tag`; on abort or timeout the last word read
+// (its tag differs, which the caller checks).  Takes no address of the
+// caller's variables, so their arrays stay in registers.
+__device__ __noinline__ uint64_t poll_word(const Graph& g, const uint64_t* p, uint32_t tag, int op, int worker,
+                                           int iter) {
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    const uint64_t w = ld_tagged(p);
+    if (word_tag(w) == tag) return w;
+    if (check_stop(g, t0, it, 11, op, -1, worker, iter, word_tag(w), tag)) return w;
   }
 }
 
@@ -326,8 +350,13 @@ struct PrefetchCursor {
   uint64_t pos;            // stream byte offset of (q, row)
 };
 
-template <bool kStandalone>
+// Producer side of a tensor-core (batched) task; defined with the batched path.
+__device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
+                         uint64_t pol, unsigned long long* t_issue);
+
+template <bool kStandalone, bool kBatch>
 __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
+  constexpr int NR = kBatch ? NSTB : NSTAGES;  // weight stages of the ring
   const uint64_t pol = policy_evict_first();
   uint32_t qpos = 0, fpos = 0, pstage = 0;
   bool ok = true;
@@ -337,8 +366,8 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
   uint32_t tail_seen = 0;
   uint64_t ld_bytes = 0;
   PrefetchCursor pf{0u, -1, false, false, 0ull, 0ull};
-  const uint64_t pf_dist = kStandalone ? 0ull : (uint64_t)g.prefetch_bytes;
-  constexpr uint64_t RING = (uint64_t)NSTAGES * STAGE_BYTES;
+  const uint64_t pf_dist = (kStandalone || kBatch) ? 0ull : (uint64_t)g.prefetch_bytes;
+  constexpr uint64_t RING = (uint64_t)NR * STAGE_BYTES;
 
   auto prefetch_some = [&]() {
     const uint64_t lo = ld_bytes + RING, hi = lo + pf_dist;
@@ -438,6 +467,13 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     const int task = (int)(entry & 0xFFFFu);
     const OpDesc& op = g.ops[opi];
     if (!is_gemv(op.kind)) continue;
+    if constexpr (kBatch) {
+      if (!bproduce(sm, g, op, task, pstage, worker, pol, g.profiling ? &sm.fifo_t[f] : nullptr)) {
+        ok = false;
+        break;
+      }
+      continue;
+    }
     int grp, row0, row1;
     task_rows(op, task, grp, row0, row1);
     const uint32_t bytes_row = stage_row_bytes(op);
@@ -467,10 +503,10 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
   if (!ok || aborted(g)) {
     // Never leave the block with bulk copies in flight: wait (bounded) for the
     // most recent stages to land before returning.
-    const uint32_t first = pstage > (uint32_t)NSTAGES ? pstage - NSTAGES : 0u;
+    const uint32_t first = pstage > (uint32_t)NR ? pstage - NR : 0u;
     for (uint32_t s = first; s < pstage; ++s) {
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(&sm.full[s % NSTAGES], (s / NSTAGES) & 1u)) {
+      while (!mbar_try_wait(&sm.full[s % NR], (s / NR) & 1u)) {
         if (globaltimer() - t0 > 200000000ull) break;
       }
     }
@@ -550,6 +586,29 @@ constexpr int ATTN_SPLIT_OP = 0, ATTN_GROUP = 1;
 
 __device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
                               int cw, int lane, uint32_t iter, int worker);
+
+// The LM head's last task to arrive (sm.last) turns every active request's
+// maximum key into its next token: written to tokens[r, s+1] if that slot
+// holds -1, always to pred; step[r] advances; the keys are reset.
+__device__ __forceinline__ void argmax_tokens(Smem& sm, const Graph& g, const OpDesc& op, uint32_t iter, int ctid) {
+  if (!sm.last) return;
+  __threadfence();
+  if (ctid < g.R) {
+    const int rq = ctid;
+    int s;
+    if (request_state(g, rq, iter, s)) {
+      const unsigned long long key = atomicAdd(op.keys + rq, 0ull);
+      const int64_t nxt = (int64_t)argmax_key_index(key);
+      int64_t* trow = g.tokens + (size_t)rq * g.S;
+      if (__ldcg(trow + s + 1) == -1) trow[s + 1] = nxt;
+      if (op.pred != nullptr) op.pred[(size_t)rq * g.S + s + 1] = nxt;
+      g.step[rq] = s + 1;
+    }
+    op.keys[rq] = 0ull;
+  }
+  consumer_sync();
+  if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+}
 
 // ------------------------------------------------------------------ GEMV tasks
 // Rows [row0,row1) of W (bf16, [rows, K] row-major) against one input vector h
@@ -836,27 +895,13 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       sm.last = ((old + 1u) % (uint32_t)op.ntasks) == 0u;
     }
     consumer_sync();
-    if (sm.last) {
-      __threadfence();
-      if (ctid < g.R) {
-        const int rq = ctid;
-        int s;
-        if (request_state(g, rq, iter, s)) {
-          const unsigned long long key = atomicAdd(op.keys + rq, 0ull);
-          const int64_t nxt = (int64_t)argmax_key_index(key);
-          int64_t* trow = g.tokens + (size_t)rq * g.S;
-          if (__ldcg(trow + s + 1) == -1) trow[s + 1] = nxt;
-          if (op.pred != nullptr) op.pred[(size_t)rq * g.S + s + 1] = nxt;
-          g.step[rq] = s + 1;
-        }
-        op.keys[rq] = 0ull;
-      }
-      consumer_sync();
-      if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
-    }
+    argmax_tokens(sm, g, op, iter, ctid);
   }
   return true;
 }
+
+// ------------------------------------------------------------------ batched projections (tensor cores)
+#include "mpk_batch.cuh"
 
 // ------------------------------------------------------------------ attention task
 // Attention of kv head j for request r at position s, over the positions
@@ -1182,6 +1227,11 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
         }
         st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
       }
+    } else {
+      // an inactive request still publishes this iteration's version of its
+      // output (zeros), which the next projection waits for
+      for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS)
+        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)j * G * D + idx, 0.f, mytag);
     }
     consumer_sync();
     if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
@@ -1193,7 +1243,17 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
 __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t iter, int ctid) {
   const int r = task;
   int s;
-  if (r < g.R && request_state(g, r, iter, s)) {
+  if (r < g.R && !request_state(g, r, iter, s)) {
+    // inactive request (several requests, this one done): x carries this
+    // iteration's version with zeros, so every reader's wait ends; nothing
+    // of it reaches the request's tokens or cache
+    const uint32_t mytag = vtag(g, iter, op.self);
+    for (int i = ctid; i < op.N; i += CONSUMER_THREADS) st_tagged(op.x_out + (size_t)r * op.N + i, 0.f, mytag);
+    if (op.xss_out != nullptr)
+      for (int b = ctid; b < op.xss_blocks; b += CONSUMER_THREADS) st_tagged(op.xss_out + (size_t)b * g.R + r, 0.f, mytag);
+    return true;
+  }
+  if (r < g.R) {
     const int64_t tok = __ldcg(g.tokens + (size_t)r * g.S + s);
     if (tok < 0 || tok >= g.V) {
       if (ctid == 0) record_error(g, -11 /*DEVICE*/, 8, -1, task, -1, (int)iter, (uint32_t)tok, (uint32_t)g.V);
@@ -1217,6 +1277,22 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
         *reinterpret_cast<float4*>(hc + 4) = b;
       }
     }
+    if (op.xss_out != nullptr) {
+      // per-block sums of squares of the row (batched graphs): warp w takes
+      // blocks w, w + 8, ..., lane l elements 4l..4l+3 of the block
+      const int cw = ctid >> 5, lane = ctid & 31;
+      for (int b = cw; b < op.xss_blocks; b += CONSUMER_WARPS) {
+        float ss = 0.f;
+        const int i = b * BM + lane * 4;
+        if (i < op.N) {
+          const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + i));
+          const float e0 = bf16_lo(w.x), e1 = bf16_hi(w.x), e2 = bf16_lo(w.y), e3 = bf16_hi(w.y);
+          ss = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) st_tagged(op.xss_out + (size_t)b * g.R + r, ss, mytag);
+      }
+    }
   }
   return true;
 }
@@ -1238,10 +1314,10 @@ __device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDes
   }
 }
 
-template <bool kStandalone>
+template <bool kStandalone, bool kBatch>
 __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int lane) {
   const int ctid = cw * 32 + lane;
-  uint32_t fpos = 0, cstage = 0;
+  uint32_t fpos = 0, cstage = 0, accn = 0;
   while (true) {
     // fetch the next task entry (elected wait, shared decision)
     bool fail = false;
@@ -1283,7 +1359,26 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     if (consumer_sync_or(fail)) return;
 
     bool ok = true;
-    switch (op.kind) {
+    if constexpr (kBatch) {
+      switch (op.kind) {
+        case TK_EMBED: ok = embed_task(g, op, task, iter, ctid); break;
+        case TK_NORM_GEMV: ok = bgemm_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, accn, cw, lane, worker); break;
+        case TK_GEMV_RESID:
+          ok = bgemm_task<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          break;
+        case TK_NORM_GEMV_SILU:
+          ok = bgemm_task<TK_NORM_GEMV_SILU>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          break;
+        case TK_NORM_GEMV_ARGMAX:
+          ok = bgemm_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          break;
+        case TK_ATTN:
+          ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C),
+                             ATTN_SPLIT_OP, cw, lane, iter, worker);
+          break;
+        default: ok = false;  // the fused projections + attention operation takes one request
+      }
+    } else switch (op.kind) {
       case TK_EMBED: ok = embed_task(g, op, task, iter, ctid); break;
       case TK_NORM_GEMV: ok = gemv_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       case TK_GEMV_RESID: ok = gemv_task<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
@@ -1388,12 +1483,20 @@ __device__ void scheduler_lane(const Graph& g, int si, int lane) {
 }
 
 // ------------------------------------------------------------------ kernels
+// The ring's stages are released by every consumer warp (GEMV path) or by
+// one MMA completion (tensor-core path).
+template <bool kBatch>
 __device__ __forceinline__ void init_barriers(Smem& sm) {
   sm.h_key = ~0ull;
   for (int i = 0; i < NSTAGES; ++i) {
     mbar_init(&sm.full[i], 1);
-    mbar_init(&sm.empty[i], CONSUMER_WARPS);
+    mbar_init(&sm.empty[i], kBatch ? 1 : CONSUMER_WARPS);
   }
+  for (int i = 0; i < 2; ++i) {
+    mbar_init(&sm.acc_full[i], 1);
+    mbar_init(&sm.acc_empty[i], 4);
+  }
+  mbar_init(&sm.fin_bar, 1);
   for (int i = 0; i < TASK_FIFO; ++i) {
     mbar_init(&sm.fifo_full[i], 1);
     mbar_init(&sm.fifo_empty[i], 1);
@@ -1401,9 +1504,53 @@ __device__ __forceinline__ void init_barriers(Smem& sm) {
   fence_mbar_init();
 }
 
-extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_kernel(const Graph g) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+// Dynamic shared memory: the layout plus slack to start it on a 1024-byte
+// boundary (the swizzled tensor-core operands need that alignment).
+extern __shared__ __align__(1024) uint8_t smem_raw[];
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;
+static_assert(SMEM_BYTES <= 232448, "one worker block per SM: at most 227 KB of shared memory");
+
+__device__ __forceinline__ Smem& smem_layout(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return *reinterpret_cast<Smem*>(raw + ((1024u - (a & 1023u)) & 1023u));
+}
+
+// A worker block: barriers (and, on the tensor-core path, the accumulator's
+// tensor memory, allocated by consumer warp 0 and released by it after the
+// last task, once no MMA is in flight), then the producer and consumer roles.
+template <bool kStandalone, bool kBatch>
+__device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) init_barriers<kBatch>(sm);
+  if (kBatch && warp == PRODUCER_WARPS) tmem_alloc(&sm.tmem_base);
+  if (kBatch) tc_fence_before_sync();
+  __syncthreads();
+  if (kBatch) tc_fence_after_sync();
+  if (warp < PRODUCER_WARPS) {
+    regs_dec<PRODUCER_REGS>();
+    if (warp == 0 && lane == 0) producer_loop<kStandalone, kBatch>(sm, g, worker, sa_iter, sa_op);
+    return;
+  }
+  regs_inc<CONSUMER_REGS>();
+  consumer_loop<kStandalone, kBatch>(sm, g, worker, warp - PRODUCER_WARPS, lane);
+  if (kBatch) {
+    // the MMA-issuing thread waits (bounded) until none of its MMAs is outstanding
+    if (warp == PRODUCER_WARPS + 4 && lane == 0) {
+      mma_commit(&sm.fin_bar);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&sm.fin_bar, 0u) && globaltimer() - t0 < 200000000ull) {
+      }
+    }
+    __syncwarp();
+    tc_fence_before_sync();
+    consumer_sync();
+    tc_fence_after_sync();
+    if (warp == PRODUCER_WARPS) tmem_dealloc(sm.tmem_base);
+  }
+}
+
+template <bool kBatch>
+__device__ __forceinline__ void persistent_body(const Graph& g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if ((int)blockIdx.x < g.sched_ctas) {
@@ -1428,65 +1575,61 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_ke
     }
     return;
   }
+  worker_block<false, kBatch>(smem_layout(smem_raw), g, blockIdx.x - g.sched_ctas, 0, 0);
+}
 
-  const int worker = blockIdx.x - g.sched_ctas;
-  if (threadIdx.x == 0) init_barriers(sm);
-  __syncthreads();
-  if (warp < PRODUCER_WARPS) {
-    regs_dec<PRODUCER_REGS>();
-    if (warp == 0 && lane == 0) producer_loop<false>(sm, g, worker, 0, 0);
-    return;
-  }
-  regs_inc<CONSUMER_REGS>();
-  consumer_loop<false>(sm, g, worker, warp - PRODUCER_WARPS, lane);
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_kernel(const Graph g) {
+  persistent_body<false>(g);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_batch_kernel(const Graph g) {
+  persistent_body<true>(g);
 }
 
 // One operation of one iteration as an ordinary launch: block b runs task b.
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_kernel(const Graph g, int op, uint32_t iter) {
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) init_barriers(sm);
-  __syncthreads();
-  if (warp < PRODUCER_WARPS) {
-    regs_dec<PRODUCER_REGS>();
-    if (warp == 0 && lane == 0) producer_loop<true>(sm, g, blockIdx.x, iter, op);
-    return;
-  }
-  regs_inc<CONSUMER_REGS>();
-  consumer_loop<true>(sm, g, blockIdx.x, warp - PRODUCER_WARPS, lane);
+  worker_block<true, false>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_batch_kernel(const Graph g, int op,
+                                                                                  uint32_t iter) {
+  worker_block<true, true>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
 }
 
 // ------------------------------------------------------------------ host-side launch helpers
-size_t kernel_smem_bytes() { return sizeof(Smem); }
+size_t kernel_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t prepare_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(mpk_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sizeof(Smem));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(mpk_op_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+  const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_batch_kernel,
+                      (const void*)mpk_op_kernel, (const void*)mpk_op_batch_kernel};
+  for (const void* k : ks) {
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t max_blocks_per_sm(int* n) {
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(n, mpk_persistent_kernel, BLOCK_THREADS, sizeof(Smem));
+  int a = 0, b = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, mpk_persistent_kernel, BLOCK_THREADS, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mpk_persistent_batch_kernel, BLOCK_THREADS, SMEM_BYTES);
+  *n = a < b ? a : b;
+  return e;
 }
 
 cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream) {
   void* args[] = {const_cast<Graph*>(&g)};
-  return cudaLaunchCooperativeKernel((const void*)mpk_persistent_kernel, dim3(grid), dim3(BLOCK_THREADS), args,
-                                     sizeof(Smem), stream);
+  const void* k = g.batched ? (const void*)mpk_persistent_batch_kernel : (const void*)mpk_persistent_kernel;
+  return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
 }
 
 // An operation whose tasks wait on one another (group mode) is launched
 // cooperatively, so all of its blocks are resident together.
 cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, bool cooperative, cudaStream_t stream) {
-  if (cooperative) {
-    void* args[] = {const_cast<Graph*>(&g), &op, &iter};
-    return cudaLaunchCooperativeKernel((const void*)mpk_op_kernel, dim3(ntasks), dim3(BLOCK_THREADS), args,
-                                       sizeof(Smem), stream);
-  }
-  mpk_op_kernel<<<ntasks, BLOCK_THREADS, sizeof(Smem), stream>>>(g, op, iter);
-  return cudaGetLastError();
+  const void* k = g.batched ? (const void*)mpk_op_batch_kernel : (const void*)mpk_op_kernel;
+  void* args[] = {const_cast<Graph*>(&g), &op, &iter};
+  if (cooperative)
+    return cudaLaunchCooperativeKernel(k, dim3(ntasks), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
+  return cudaLaunchKernel(k, dim3(ntasks), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
 }
 
 }  // namespace mpk

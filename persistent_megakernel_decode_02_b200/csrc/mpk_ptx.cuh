@@ -1,6 +1,7 @@
 // Thin wrappers over the sm_100a PTX the runtime uses: mbarriers, 1-D bulk
-// (TMA) copies global -> shared, scoped acquire/release accesses and the
-// global nanosecond timer.  No cluster multicast anywhere.
+// and 2-D tiled (TMA) copies global -> shared, tensor-memory allocation,
+// tcgen05 MMAs and loads, scoped acquire/release accesses and the global
+// nanosecond timer.  No cluster multicast anywhere.
 #pragma once
 #include <stdint.h>
 
@@ -78,6 +79,95 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// 2-D tiled tensor (TMA) copy global -> this CTA's shared memory: the box at
+// coordinates (x, y) of the tensor map (x innermost, in elements), completing
+// the box's bytes on `bar`.  The map lives in global memory; x * element size
+// must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// ---------------------------------------------------------------- tensor memory and tcgen05 MMA
+// Columns of tensor memory one worker block allocates (a power of two >= 32):
+// two accumulators of 2 x 16 columns.
+constexpr uint32_t TMEM_COLS = 64;
+
+// Allocation by one whole warp; the tensor-memory address lands in *dst.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(TMEM_COLS)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(TMEM_COLS) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// Orders this thread's ordinary shared-memory stores before later reads of
+// the same bytes by the tensor cores (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Shared-memory matrix descriptor of a K-major bf16 operand in the 128-byte
+// swizzled layout: rows of 128 bytes (64 elements of K), 8-row atoms of 1024
+// bytes stacked along M/N; the atom base must be 1024-byte aligned.  Bits:
+// start address >> 4 [0,14), leading offset >> 4 [16,30) (unused for this
+// layout: 1), stride offset >> 4 [32,46) = 1024 >> 4, descriptor version 1 at
+// [46,48), layout 2 (128-byte swizzle) at [61,64).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+// Instruction descriptor of a dense kind::f16 MMA: fp32 accumulator (bits
+// [4,6) = 1), bf16 A and B ([7,10) = 1, [10,13) = 1), both K-major (bits 15,
+// 16 = 0), N >> 3 at [17,23), M >> 4 at [24,29).
+__host__ __device__ constexpr uint32_t mma_idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// D (tensor memory) = A * B^T (+ D when `accumulate`), A and B from shared
+// memory descriptors.  Issued by one thread.
+__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane (warp w
+// of a warpgroup reads lanes 32 (w mod 4) ..; taddr carries the lane in its
+// upper half), waited for before returning.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // ---------------------------------------------------------------- scoped accesses
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;
@@ -118,8 +208,16 @@ __device__ __forceinline__ uint64_t ld_tagged(const uint64_t* p) {
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
   return w;
 }
+// Two consecutive tagged words (16-byte aligned) in one access.
+__device__ __forceinline__ void ld_tagged2(const uint64_t* p, uint64_t& a, uint64_t& b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p) : "memory");
+}
 __device__ __forceinline__ float word_value(uint64_t w) { return __uint_as_float((uint32_t)w); }
 __device__ __forceinline__ uint32_t word_tag(uint64_t w) { return (uint32_t)(w >> 32); }
+
+// Named barrier 2 over the first consumer warpgroup (the accumulator readers
+// of the tensor-core path).
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, %0;" ::"r"(128) : "memory"); }
 
 // Named barrier 1 over the 256 consumer threads (the producer warp never joins).
 __device__ __forceinline__ void consumer_sync() {

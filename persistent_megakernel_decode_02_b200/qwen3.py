@@ -10,7 +10,7 @@ RMSNorm + LM head + greedy argmax, which advances `step` and writes `tokens`.
 from __future__ import annotations
 
 from dataclasses import dataclass
-from typing import Dict, List, Optional
+from typing import Dict, List, Optional, Tuple
 
 import torch
 
@@ -31,6 +31,74 @@ def reduction_split(K: int, max_k: int = _lib.MAX_GEMV_K) -> int:
     return ks
 
 
+# Tensor-core projections over several requests (the rule of the batched path
+# in mpk.h): row blocks of BATCH_BM rows, K blocks of BATCH_BK elements, at most
+# BATCH_MAX_KBLOCKS K blocks per reduction segment; grid_dim = (tasks per
+# segment, segments).
+BATCH_BM, BATCH_BK, BATCH_MAX_KBLOCKS = 128, 64, 24
+# Task-size model used to choose the grid: a worker streams weights at about
+# its share of HBM bandwidth and pays a fixed cost per task.
+_WORKER_BYTES_PER_S = 43e9
+_TASK_OVERHEAD_S = 3e-6
+
+
+def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[int, int]:
+    """grid_dim (tasks per reduction segment, segments) of a projection over
+    several requests: among segment counts s (enough that each fits the input
+    buffer) and, per number of rounds k of the workers, the largest run split
+    gx <= row blocks with gx * s <= k * workers, the one with the least
+    rounds x (largest task's weight bytes / bandwidth + task cost); fewer
+    segments on ties."""
+    nb = -(-rows // BATCH_BM)
+    nkb = K // BATCH_BK
+    smin = -(-nkb // BATCH_MAX_KBLOCKS)
+    block_bytes = BATCH_BM * K * 2 * (2 if pair else 1)
+    best = None
+    for s in range(smin, min(nkb, max(smin, 16)) + 1):
+        for k in range(1, 5):
+            gx = max(1, min(nb, (k * workers) // s))
+            rounds = -(-(gx * s) // workers)
+            t = rounds * ((-(-nb // gx)) * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S)
+            if best is None or t < best[0] * (1 - 1e-2):
+                best = (t, gx, s)
+    return best[1], best[2]
+
+
+def batched_layer_plan(shape, requests: int, plan_workers: int, attn_chunks: int, block_dim: int = 0,
+                       tied: Optional[bool] = None) -> List[dict]:
+    """The fused-layer list for several requests: projections on the tensor
+    cores (grids from batched_grid for plan_workers workers), attention as its
+    own split-K operation."""
+    s = shape
+    W = plan_workers
+    tied = s.tied if tied is None else tied
+    plan: List[dict] = [dict(method="embed_layer", embedding="embed_tokens", output="x", grid_dim=requests,
+                             block_dim=block_dim, capture_slot=0)]
+    for l in range(s.layers):
+        p = f"layers.{l}."
+        plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
+                         weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
+                         grid_dim=batched_grid(s.q_dim + 2 * s.kv_dim, s.hidden, W), block_dim=block_dim, eps=s.eps))
+        plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm",
+                         k_norm=p + "k_norm", k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
+                         grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
+                         rope_theta=s.rope_theta))
+        plan.append(dict(method="linear_residual_layer", input="o", weight=p + "o_proj", residual="x",
+                         grid_dim=batched_grid(s.hidden, s.q_dim, W), block_dim=block_dim))
+        plan.append(dict(method="rmsnorm_linear_silu_mul_layer", input="x",
+                         weight_norm=p + "post_attention_layernorm", weight_gate=p + "gate_proj",
+                         weight_up=p + "up_proj", output="a",
+                         grid_dim=batched_grid(s.intermediate, s.hidden, W, pair=True), block_dim=block_dim,
+                         eps=s.eps))
+        plan.append(dict(method="linear_residual_layer", input="a", weight=p + "down_proj", residual="x",
+                         grid_dim=batched_grid(s.hidden, s.intermediate, W), block_dim=block_dim,
+                         capture_slot=l + 1))
+    plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
+                     weight_lm="embed_tokens" if tied else "lm_head", pred="pred",
+                     grid_dim=batched_grid(s.vocab, s.hidden, W), block_dim=block_dim, eps=s.eps))
+    return plan
+
+
 def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_tasks: Optional[int] = None,
                block_dim: int = 0, tied: Optional[bool] = None, fused_attention: bool = False,
                tasks_per_worker: int = 2) -> List[dict]:
@@ -38,7 +106,10 @@ def layer_plan(shape, requests: int, num_workers: int, attn_chunks: int, gemv_ta
     the method name and its keyword arguments.  With ``fused_attention`` the q/k/v
     projections and the attention are one operation (tasks grouped per kv head,
     the last task of a group runs its attention); otherwise attention is its own
-    split-K operation with ``attn_chunks`` chunks."""
+    split-K operation with ``attn_chunks`` chunks.  Several requests take
+    batched_layer_plan."""
+    if requests >= 2:
+        return batched_layer_plan(shape, requests, gemv_tasks or num_workers, attn_chunks, block_dim, tied)
     s = shape
     gt = gemv_tasks or num_workers                       # fused projections+attention: one task per worker
     dt = gemv_tasks or num_workers * tasks_per_worker    # claimed GEMV ops: more, smaller tasks

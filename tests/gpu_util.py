@@ -21,13 +21,20 @@ def to_cuda(weights):
     return {k: v.cuda() for k, v in weights.items()}
 
 
-def gpu_teacher_forced(dec, tokens_cpu: torch.Tensor, iters, step0: int = 0):
+def _steps(step0, R):
+    """step0 as one position for every request or one per request."""
+    a = np.asarray(step0, dtype=np.int32)
+    return np.full(R, int(a), np.int32) if a.ndim == 0 else a.astype(np.int32).copy()
+
+
+def gpu_teacher_forced(dec, tokens_cpu: torch.Tensor, iters, step0=0):
     """Run one persistent launch per iteration with capture on; returns the
-    per-iteration (logits [R,V], hidden [L+1,R,H]) as float64 numpy arrays."""
+    per-iteration (logits [R,V], hidden [L+1,R,H]) as float64 numpy arrays.
+    step0: the first position, shared or per request."""
     s = dec.shape
     R = tokens_cpu.shape[0]
     tok = tokens_cpu.cuda()
-    step = torch.full((R,), step0, dtype=torch.int32, device="cuda")
+    step = torch.from_numpy(_steps(step0, R)).cuda()
     out = []
     for it in range(iters):
         lg = torch.full((R, s.vocab), float("nan"), device="cuda")
@@ -42,18 +49,19 @@ def gpu_teacher_forced(dec, tokens_cpu: torch.Tensor, iters, step0: int = 0):
     return out, tok.cpu(), step.cpu()
 
 
-def oracle_teacher_forced(shape, w_cpu, tokens_cpu: torch.Tensor, iters, kc=None, vc=None, step0: int = 0):
+def oracle_teacher_forced(shape, w_cpu, tokens_cpu: torch.Tensor, iters, kc=None, vc=None, step0=0,
+                          round_mode=oracle.ROUND_NONE):
     ref = oracle.Decoder(shape, w_cpu)
     toks = tokens_cpu.numpy().copy()
     R, S = toks.shape
     if kc is None:
         kc, vc = ref.new_cache(R, S)
-    step = np.full(R, step0, np.int32)
+    step = _steps(step0, R)
     out = []
     for _ in range(iters):
         lg = np.full((R, shape.vocab), np.nan)
         hd = np.full((shape.layers + 1, R, shape.hidden), np.nan)
-        ref.iteration(kc, vc, step, toks, None, oracle.ROUND_NONE, lg, hd)
+        ref.iteration(kc, vc, step, toks, None, round_mode, lg, hd)
         out.append((lg, hd))
     return out, toks, kc, vc
 

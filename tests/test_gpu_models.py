@@ -104,3 +104,31 @@ def test_qwen3_8b_long_context(qwen3_8b):
     w_cpu, w = qwen3_8b
     P = 32768
     _check(sq.QWEN3_8B, w_cpu, w, P, P + 128, 2)
+
+
+def test_qwen3_8b_batch8(qwen3_8b):
+    """The batched workload's shape: 8 requests (prompt lengths U[32,512]) half
+    way through their 256 generated tokens, each at its own position: tensor-core
+    projections over the batch, split-K attention per request.  Compared with
+    the plain (unrounded) reading of the oracle."""
+    from persistent_megakernel_decode_02_b200 import build_decoder
+
+    w_cpu, w = qwen3_8b
+    shape, R, S = sq.QWEN3_8B, 8, 1024
+    lens = sq.make_prompt_lengths(R, 32, 512, seed=0)
+    p0 = (lens - 1 + 128).numpy().astype(np.int32)
+    kc, vc = sq.make_kv_prefill(shape, R, S, int(p0.max()), seed=21)
+    tokens = sq.make_tokens(shape, R, S, [S] * R, seed=22, teacher_forced=True)
+    dec = build_decoder(shape, w, requests=R, max_seq=S, k_cache=kc.cuda(), v_cache=vc.cuda())
+    gpu, gtok, gstep = gpu_teacher_forced(dec, tokens, 2, step0=p0)
+    ref, _, rkc, _ = oracle_teacher_forced(shape, w_cpu, tokens, 2, _u16(kc), _u16(vc), step0=p0)
+    wl, wh = compare_captures(gpu, ref)
+    print(f"{shape.name} x{R}: worst logits rel-L2 {wl:.2e}, hidden {wh:.2e}")
+    assert np.array_equal(gstep.numpy(), p0 + 2)
+    assert torch.equal(gtok, tokens)
+    for r in range(R):
+        a = int(p0[r])
+        gk = dec.k_cache[:, r, :, a:a + 2].float().cpu().numpy()
+        rk = (rkc[:, r, :, a:a + 2].astype(np.uint32) << 16).view(np.float32)
+        assert np.linalg.norm(gk - rk) <= 1e-2 * np.linalg.norm(rk)
+    dec.kernel.close()
