@@ -38,6 +38,15 @@ __device__ __forceinline__ void btask(const OpDesc& op, int task, int& rb0, int&
   kb1 = (int)(((long long)(seg + 1) * op.nkb) / op.bsplit);
 }
 
+// A task's K blocks are processed in passes of at most B_MAX_KBLOCKS (the
+// input rows held in shared memory): passes of the task's row blocks
+// accumulate into one tensor-memory slot per block.
+__device__ __forceinline__ int bpasses(int nkbs) { return (nkbs + B_MAX_KBLOCKS - 1) / B_MAX_KBLOCKS; }
+__device__ __forceinline__ void bpass(int kb0, int kb1, int npass, int ps, int& kp0, int& kp1) {
+  kp0 = kb0 + (int)(((long long)ps * (kb1 - kb0)) / npass);
+  kp1 = kb0 + (int)(((long long)(ps + 1) * (kb1 - kb0)) / npass);
+}
+
 // Ring stages of one row block: gate/up take one K block of both matrices per
 // stage, the other operations two K blocks of one matrix.
 __device__ __forceinline__ int bstages(const OpDesc& op, int nkbs) {
@@ -51,22 +60,28 @@ __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, u
   int rb0, rb1, kb0, kb1, seg;
   btask(op, task, rb0, rb1, kb0, kb1, seg);
   const bool pair = op.kind == TK_NORM_GEMV_SILU;
-  for (int rb = rb0; rb < rb1; ++rb) {
-    const int row = rb * BM;
-    const int s = pair ? 0 : seg_of(op, row);
-    const int mrow = row - op.seg_row0[s];  // row within matrix s (rows past its end read as zeros)
-    const void* tm = op.tmap[s];
-    for (int kb = kb0; kb < kb1; kb += pair ? 1 : 2) {
-      const uint32_t slot = pstage % NSTB;
-      const uint32_t par = ((pstage / NSTB) & 1u) ^ 1u;
-      if (!wait_mbar(g, &sm.empty[slot], par, 3, worker)) return false;
-      if (t_issue != nullptr && rb == rb0 && kb == kb0) atomicExch(t_issue, (unsigned long long)globaltimer());
-      const int nbox = pair ? 2 : min(2, kb1 - kb);
-      mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)(nbox * BOX_BYTES));
-      tma_load_2d(sm.ring[slot], tm, kb * BK, mrow, &sm.full[slot], pol);
-      if (pair) tma_load_2d(sm.ring[slot] + BOX_BYTES, op.tmap_up, kb * BK, mrow, &sm.full[slot], pol);
-      else if (nbox == 2) tma_load_2d(sm.ring[slot] + BOX_BYTES, tm, (kb + 1) * BK, mrow, &sm.full[slot], pol);
-      ++pstage;
+  const int npass = bpasses(kb1 - kb0);
+  for (int ps = 0; ps < npass; ++ps) {
+    int kp0, kp1;
+    bpass(kb0, kb1, npass, ps, kp0, kp1);
+    for (int rb = rb0; rb < rb1; ++rb) {
+      const int row = rb * BM;
+      const int s = pair ? 0 : seg_of(op, row);
+      const int mrow = row - op.seg_row0[s];  // row within matrix s (rows past its end read as zeros)
+      const void* tm = op.tmap[s];
+      for (int kb = kp0; kb < kp1; kb += pair ? 1 : 2) {
+        const uint32_t slot = pstage % NSTB;
+        const uint32_t par = ((pstage / NSTB) & 1u) ^ 1u;
+        if (!wait_mbar(g, &sm.empty[slot], par, 3, worker)) return false;
+        if (t_issue != nullptr && ps == 0 && rb == rb0 && kb == kp0)
+          atomicExch(t_issue, (unsigned long long)globaltimer());
+        const int nbox = pair ? 2 : min(2, kp1 - kb);
+        mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)(nbox * BOX_BYTES));
+        tma_load_2d(sm.ring[slot], tm, kb * BK, mrow, &sm.full[slot], pol);
+        if (pair) tma_load_2d(sm.ring[slot] + BOX_BYTES, op.tmap_up, kb * BK, mrow, &sm.full[slot], pol);
+        else if (nbox == 2) tma_load_2d(sm.ring[slot] + BOX_BYTES, tm, (kb + 1) * BK, mrow, &sm.full[slot], pol);
+        ++pstage;
+      }
     }
   }
   return true;
@@ -144,9 +159,12 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo
 // accumulators; warps 0..3 (tensor-memory lanes 0..127, one weight row per
 // thread) read each accumulator as soon as it is complete and run the
 // epilogue, so the next block's MMAs overlap it.
+//
+// Not inlined: the task gets its own register allocation, so neither its
+// arrays nor the attention's are spilled around the other.
 template <int KIND>
-__device__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter, uint32_t& cstage,
-                           uint32_t& accn, int cw, int lane, int worker) {
+__device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
+                                        uint32_t& cstage, uint32_t& accn, int cw, int lane, int worker) {
   constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
   constexpr bool NORM = KIND != TK_GEMV_RESID;
   constexpr int MMA_WARP = 4;
@@ -154,9 +172,8 @@ __device__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task,
   const int R = g.R;
   int rb0, rb1, kb0, kb1, seg;
   btask(op, task, rb0, rb1, kb0, kb1, seg);
-  const int nkbs = kb1 - kb0;
-  const int nst = bstages(op, nkbs);
   const int nblk = rb1 - rb0;
+  const int npass = bpasses(kb1 - kb0);
   const bool split = op.bsplit > 1;
   uint8_t* bsm = sm.ring[NSTB];
   const uint32_t xtag = vtag(g, iter, op.x_writer) + op.tag_skew;
@@ -164,11 +181,21 @@ __device__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task,
   const uint32_t mytag = vtag(g, iter, op.self);
   const uint64_t* src = NORM ? op.x : op.a_in;
   const uint32_t stag = NORM ? xtag : atag;
-  bool pfail = false;
+  const uint32_t tmem = sm.tmem_base;
+  const int nrows = op.N;
+  // partial sums: [segment][row][PW] floats, PW = the requests' values (gate/up:
+  // then the up values), so a thread moves its row with 16-byte accesses
+  constexpr int PW = PAIR ? 2 * MAX_BATCH : MAX_BATCH;
+  const size_t SEGW = (size_t)nrows * PW;
+  bool fail = false;
+  unsigned long long best[MAX_BATCH];
+#pragma unroll
+  for (int r = 0; r < MAX_BATCH; ++r) best[r] = 0ull;
 
-  // ---- prologue.  RMSNorm factor of every request from the per-block sums of
-  // squares its writer published (warp r: request r, blocks in a fixed order).
+  // ---- RMSNorm factor of every request from the per-block sums of squares
+  // its writer published (warp r: request r, blocks in a fixed order)
   if (NORM) {
+    bool pfail = false;
     if (cw < R) {
       float ss = 0.f;
       for (int b = lane; b < op.xss_blocks; b += 32) {
@@ -183,215 +210,236 @@ __device__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task,
       ss = warp_sum(ss);
       if (lane == 0) sm.brinv[cw] = 1.0f / sqrtf(ss / (float)op.K + op.eps);
     }
-    consumer_sync();
+    if (consumer_sync_or(pfail)) return false;
   }
-  // The input rows of the segment as bf16 hi/lo pairs into the swizzled
-  // layout; FL chunks of 8 elements per thread in flight.
-  {
-    const int nch = nkbs * 8;  // 16-byte chunks per request row
-    const int total = MAX_BATCH * nch;
-    constexpr int FL = 2;
-    for (int q0 = ctid; q0 < total; q0 += FL * CONSUMER_THREADS) {
-      uint64_t w[FL][8];
-#pragma unroll
-      for (int u = 0; u < FL; ++u) {
-        const int q = q0 + u * CONSUMER_THREADS;
-        const int r = q / nch;
-        if (q < total && r < R) {
-          const uint64_t* p = src + (size_t)r * op.K + (size_t)kb0 * BK + (size_t)(q - r * nch) * 8;
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) ld_tagged2(p + e, w[u][e], w[u][e + 1]);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < FL; ++u) {
-        const int q = q0 + u * CONSUMER_THREADS;
-        if (q < total) {
-          const int r = q / nch, cc = q - r * nch;
-          const int kbl = cc >> 3, ch = cc & 7;
-          uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
-          if (r < R) {
-            const int k = kb0 * BK + cc * 8;
-            const uint64_t* p = src + (size_t)r * op.K + k;
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              if (word_tag(w[u][e]) != stag) {
-                w[u][e] = poll_word(g, p + e, stag, op.self, worker, (int)iter);
-                pfail |= word_tag(w[u][e]) != stag;
-              }
-              v[e] = word_value(w[u][e]);
-            }
-            if (NORM) {
-              const uint4 nw = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
-              const float ri = sm.brinv[r];
-              v[0] = v[0] * ri * bf16_lo(nw.x); v[1] = v[1] * ri * bf16_hi(nw.x);
-              v[2] = v[2] * ri * bf16_lo(nw.y); v[3] = v[3] * ri * bf16_hi(nw.y);
-              v[4] = v[4] * ri * bf16_lo(nw.z); v[5] = v[5] * ri * bf16_hi(nw.z);
-              v[6] = v[6] * ri * bf16_lo(nw.w); v[7] = v[7] * ri * bf16_hi(nw.w);
-            }
-            split8(v, hi, lo);
-          }
-          uint8_t* dst = bsm + kbl * B_KBLOCK_BYTES + r * (BK * 2) + ((ch ^ r) << 4);
-          *reinterpret_cast<uint4*>(dst) = hi;
-          *reinterpret_cast<uint4*>(dst + B_KBLOCK_BYTES / 2) = lo;
-        }
-      }
-    }
-  }
-  fence_proxy_async_smem();  // the tensor cores read these bytes next
-  if (consumer_sync_or(pfail)) return false;
-  if (g.profiling && ctid == 0) sm.t_pro = globaltimer();
 
-  // ---- row blocks
-  const uint32_t tmem = sm.tmem_base;
-  const int nrows = op.N;
-  const size_t NP = (size_t)(PAIR ? 2 : 1) * (size_t)nrows;  // partial-sum row length
-  bool fail = false;
-  unsigned long long best[MAX_BATCH];
-#pragma unroll
-  for (int r = 0; r < MAX_BATCH; ++r) best[r] = 0ull;
-  if (cw == MMA_WARP) {
-    if (lane == 0) {
-      const uint32_t idesc = mma_idesc_bf16(BM, BN);
+  for (int ps = 0; ps < npass; ++ps) {
+    int kp0, kp1;
+    bpass(kb0, kb1, npass, ps, kp0, kp1);
+    const int nkbs = kp1 - kp0;
+    const int nst = bstages(op, nkbs);
+    const bool last = ps == npass - 1;
+    if (ps > 0) {
+      // the previous pass's MMAs are done reading the input rows
       bool ok = true;
-      for (int i = 0; i < nblk; ++i) {
-        const uint32_t a = accn + (uint32_t)i, buf = a & 1u, use = a >> 1;
-        // the epilogue has read this accumulator's previous block
-        if (ok) ok = wait_mbar(g, &sm.acc_empty[buf], (use & 1u) ^ 1u, 3, worker);
-        tc_fence_after_sync();
-        const uint32_t dacc = tmem + buf * (uint32_t)(2 * BN);
-        for (int st = 0; ok && st < nst; ++st) {
-          const uint32_t cs = cstage + (uint32_t)(i * nst + st);
-          const uint32_t slot = cs % NSTB;
-          const uint64_t w0 = g.profiling ? globaltimer() : 0ull;
-          ok = wait_mbar(g, &sm.full[slot], (cs / NSTB) & 1u, 3, worker);
-          if (g.profiling) {
-            const uint64_t w1 = globaltimer();
-            sm.t_stall += w1 - w0;
-            sm.t_last = w1;
-            if (i == 0 && st == 0) sm.t_data = w1;
-          }
-          if (!ok) break;
-          tc_fence_after_sync();
-          const uint32_t a0 = smem_u32(sm.ring[slot]);
-          if (PAIR) {
-            const uint32_t b0 = smem_u32(bsm) + (uint32_t)st * B_KBLOCK_BYTES;
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk) {
-              const uint64_t bd = sw128_desc(b0 + kk * 32);
-              const uint32_t acc = (st | kk) != 0;
-              mma_bf16_ss(dacc, sw128_desc(a0 + kk * 32), bd, idesc, acc);
-              mma_bf16_ss(dacc + BN, sw128_desc(a0 + BOX_BYTES + kk * 32), bd, idesc, acc);
-            }
-          } else {
-            const int nbox = min(2, nkbs - 2 * st);
-            for (int b = 0; b < nbox; ++b) {
-              const uint32_t b0 = smem_u32(bsm) + (uint32_t)(2 * st + b) * B_KBLOCK_BYTES;
-#pragma unroll
-              for (int kk = 0; kk < BK / 16; ++kk)
-                mma_bf16_ss(dacc, sw128_desc(a0 + b * BOX_BYTES + kk * 32), sw128_desc(b0 + kk * 32), idesc,
-                            (st | b | kk) != 0);
-            }
-          }
-          mma_commit(&sm.empty[slot]);  // the stage returns to the producer once these MMAs have read it
-        }
-        mma_commit(&sm.acc_full[buf]);  // also after a failure: it ends the epilogue's wait
+      if (ctid == 0) {
+        ok = wait_mbar(g, &sm.bfree, sm.bfn & 1u, 3, worker);
+        ++sm.bfn;
       }
-      fail = !ok;
+      if (consumer_sync_or(fail || !ok)) return false;
     }
-    __syncwarp();
-  } else if (cw < 4) {
-    const bool capture = (g.capture_iter == (int)iter);
-    const uint32_t lanes = (uint32_t)(cw * 32) << 16;
-    for (int i = 0; i < nblk; ++i) {
-      const int rb = rb0 + i;
-      const uint32_t a = accn + (uint32_t)i, buf = a & 1u, use = a >> 1;
-      bool ok = true;
-      if (lane == 0) ok = wait_mbar(g, &sm.acc_full[buf], use & 1u, 3, worker);
-      ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
-      tc_fence_after_sync();
-      float d[16], du[16];
-      const uint32_t dacc = tmem + buf * (uint32_t)(2 * BN) + lanes;
-      tmem_ld16(dacc, d);
-      if (PAIR) tmem_ld16(dacc + BN, du);
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
-      fail |= !ok;
-      // W hi + W lo per request
-      float v[MAX_BATCH], u[MAX_BATCH], nx[MAX_BATCH];
+    // ---- the input rows of this pass's K blocks as bf16 hi/lo pairs into
+    // the swizzled layout; FL chunks of 8 elements per thread in flight
+    {
+      bool pfail = false;
+      const int nch = nkbs * 8;  // 16-byte chunks per request row
+      const int total = MAX_BATCH * nch;
+      constexpr int FL = 2;
+      for (int q0 = ctid; q0 < total; q0 += FL * CONSUMER_THREADS) {
+        uint64_t w[FL][8];
 #pragma unroll
-      for (int r = 0; r < MAX_BATCH; ++r) {
-        v[r] = d[r] + d[MAX_BATCH + r];
-        u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
-        nx[r] = 0.f;
-      }
-      const int row = rb * BM + cw * 32 + lane;
-      bool finish = !split;  // this task runs the block's epilogue
-      if (split) {
-        if (ok && row < nrows) {
-          float* pp = op.bpart + (size_t)seg * R * NP;
+        for (int u = 0; u < FL; ++u) {
+          const int q = q0 + u * CONSUMER_THREADS;
+          const int r = q / nch;
+          if (q < total && r < R) {
+            const uint64_t* p = src + (size_t)r * op.K + (size_t)kp0 * BK + (size_t)(q - r * nch) * 8;
 #pragma unroll
-          for (int r = 0; r < MAX_BATCH; ++r) {
-            if (r < R) {
-              pp[(size_t)r * NP + row] = v[r];
-              if (PAIR) pp[(size_t)r * NP + nrows + row] = u[r];
-            }
+            for (int e = 0; e < 8; e += 2) ld_tagged2(p + e, w[u][e], w[u][e + 1]);
           }
         }
-        // The last segment task of this row block to arrive adds the partial
-        // sums in segment order and runs the epilogue.
-        epi_sync();
-        if (ctid == 0) {
-          __threadfence();
-          const uint32_t old = atomicAdd(op.blk_cnt + rb, 1u);
-          sm.blast = ((old + 1u) % (uint32_t)op.bsplit) == 0u;
-        }
-        epi_sync();
-        finish = sm.blast != 0;
-        if (finish) {
-          __threadfence();
-          if (row < nrows) {
-            for (int sg = 0; sg < op.bsplit; ++sg) {
-              const float* pp = op.bpart + (size_t)sg * R * NP;
 #pragma unroll
-              for (int r = 0; r < MAX_BATCH; ++r) {
-                if (r < R) {
-                  const float pa = __ldcg(pp + (size_t)r * NP + row);
-                  v[r] = sg == 0 ? pa : v[r] + pa;
-                  if (PAIR) {
-                    const float pb = __ldcg(pp + (size_t)r * NP + nrows + row);
-                    u[r] = sg == 0 ? pb : u[r] + pb;
+        for (int u = 0; u < FL; ++u) {
+          const int q = q0 + u * CONSUMER_THREADS;
+          if (q < total) {
+            const int r = q / nch, cc = q - r * nch;
+            const int kbl = cc >> 3, ch = cc & 7;
+            uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = hi;
+            if (r < R) {
+              const int k = kp0 * BK + cc * 8;
+              const uint64_t* p = src + (size_t)r * op.K + k;
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (word_tag(w[u][e]) != stag) {
+                  w[u][e] = poll_word(g, p + e, stag, op.self, worker, (int)iter);
+                  pfail |= word_tag(w[u][e]) != stag;
+                }
+                v[e] = word_value(w[u][e]);
+              }
+              if (NORM) {
+                const uint4 nw = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
+                const float ri = sm.brinv[r];
+                v[0] = v[0] * ri * bf16_lo(nw.x); v[1] = v[1] * ri * bf16_hi(nw.x);
+                v[2] = v[2] * ri * bf16_lo(nw.y); v[3] = v[3] * ri * bf16_hi(nw.y);
+                v[4] = v[4] * ri * bf16_lo(nw.z); v[5] = v[5] * ri * bf16_hi(nw.z);
+                v[6] = v[6] * ri * bf16_lo(nw.w); v[7] = v[7] * ri * bf16_hi(nw.w);
+              }
+              split8(v, hi, lo);
+            }
+            uint8_t* dst = bsm + kbl * B_KBLOCK_BYTES + r * (BK * 2) + ((ch ^ r) << 4);
+            *reinterpret_cast<uint4*>(dst) = hi;
+            *reinterpret_cast<uint4*>(dst + B_KBLOCK_BYTES / 2) = lo;
+          }
+        }
+      }
+      fence_proxy_async_smem();  // the tensor cores read these bytes next
+      if (consumer_sync_or(pfail)) return false;
+    }
+    if (ps == 0 && g.profiling && ctid == 0) sm.t_pro = globaltimer();
+
+    if (cw == MMA_WARP) {
+      // ---- MMAs of this pass for every row block: block i accumulates in
+      // slot (accn + i) mod NSLOT, handed to the epilogue after the last pass
+      if (lane == 0) {
+        const uint32_t idesc = mma_idesc_bf16(BM, BN);
+        bool ok = true;
+        for (int i = 0; i < nblk; ++i) {
+          const uint32_t a = accn + (uint32_t)i, slot = a % NSLOT, use = a / NSLOT;
+          // the epilogue has read this slot's previous block
+          if (ps == 0 && ok) ok = wait_mbar(g, &sm.acc_empty[slot], (use & 1u) ^ 1u, 3, worker);
+          tc_fence_after_sync();
+          const uint32_t dacc = tmem + slot * (uint32_t)(2 * BN);
+          for (int st = 0; ok && st < nst; ++st) {
+            const uint32_t cs = cstage + (uint32_t)(i * nst + st);
+            const uint32_t rs = cs % NSTB;
+            const uint64_t w0 = g.profiling ? globaltimer() : 0ull;
+            ok = wait_mbar(g, &sm.full[rs], (cs / NSTB) & 1u, 3, worker);
+            if (g.profiling) {
+              const uint64_t w1 = globaltimer();
+              sm.t_stall += w1 - w0;
+              sm.t_last = w1;
+              if (ps == 0 && i == 0 && st == 0) sm.t_data = w1;
+            }
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint32_t a0 = smem_u32(sm.ring[rs]);
+            if (PAIR) {
+              const uint32_t b0 = smem_u32(bsm) + (uint32_t)st * B_KBLOCK_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk) {
+                const uint64_t bd = sw128_desc(b0 + kk * 32);
+                const uint32_t acc = (ps | st | kk) != 0;
+                mma_bf16_ss(dacc, sw128_desc(a0 + kk * 32), bd, idesc, acc);
+                mma_bf16_ss(dacc + BN, sw128_desc(a0 + BOX_BYTES + kk * 32), bd, idesc, acc);
+              }
+            } else {
+              const int nbox = min(2, nkbs - 2 * st);
+              for (int b = 0; b < nbox; ++b) {
+                const uint32_t b0 = smem_u32(bsm) + (uint32_t)(2 * st + b) * B_KBLOCK_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                  mma_bf16_ss(dacc, sw128_desc(a0 + b * BOX_BYTES + kk * 32), sw128_desc(b0 + kk * 32), idesc,
+                              (ps | st | b | kk) != 0);
+              }
+            }
+            mma_commit(&sm.empty[rs]);  // the stage returns to the producer once these MMAs have read it
+          }
+          if (last) mma_commit(&sm.acc_full[slot]);  // also after a failure: it ends the epilogue's wait
+        }
+        if (!last) mma_commit(&sm.bfree);  // also after a failure: it ends the next pass's wait
+        fail |= !ok;
+      }
+      __syncwarp();
+    } else if (cw < 4 && last) {
+      // ---- epilogue of every row block, in order, as soon as its slot is complete
+      const bool capture = (g.capture_iter == (int)iter);
+      const uint32_t lanes = (uint32_t)(cw * 32) << 16;
+      for (int i = 0; i < nblk; ++i) {
+        const int rb = rb0 + i;
+        const uint32_t a = accn + (uint32_t)i, slot = a % NSLOT, use = a / NSLOT;
+        bool ok = true;
+        if (lane == 0) ok = wait_mbar(g, &sm.acc_full[slot], use & 1u, 3, worker);
+        ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
+        tc_fence_after_sync();
+        float d[16], du[16];
+        const uint32_t dacc = tmem + slot * (uint32_t)(2 * BN) + lanes;
+        tmem_ld16(dacc, d);
+        if (PAIR) tmem_ld16(dacc + BN, du);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
+        fail |= !ok;
+        // W hi + W lo per request
+        float v[MAX_BATCH], u[MAX_BATCH], nx[MAX_BATCH];
+#pragma unroll
+        for (int r = 0; r < MAX_BATCH; ++r) {
+          v[r] = d[r] + d[MAX_BATCH + r];
+          u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
+          nx[r] = 0.f;
+        }
+        const int row = rb * BM + cw * 32 + lane;
+        bool finish = !split;  // this task runs the block's epilogue
+        if (split) {
+          if (ok && row < nrows) {
+            float4* pp = reinterpret_cast<float4*>(op.bpart + (size_t)seg * SEGW + (size_t)row * PW);
+            pp[0] = make_float4(v[0], v[1], v[2], v[3]);
+            pp[1] = make_float4(v[4], v[5], v[6], v[7]);
+            if (PAIR) {
+              pp[2] = make_float4(u[0], u[1], u[2], u[3]);
+              pp[3] = make_float4(u[4], u[5], u[6], u[7]);
+            }
+          }
+          // The last segment task of this row block to arrive adds the
+          // partial sums in segment order and runs the epilogue.  (Thread 0's
+          // acquire-release arrival, then the barrier, order the other tasks'
+          // partials before every thread's reads.)
+          epi_sync();
+          if (ctid == 0) {
+            const uint32_t old = atom_add_acq_rel(op.blk_cnt + rb, 1u);
+            sm.blast = ((old + 1u) % (uint32_t)op.bsplit) == 0u;
+          }
+          epi_sync();
+          finish = sm.blast != 0;
+          if (finish && row < nrows) {
+            constexpr int V4 = PW / 4;  // float4 per partial row
+            const float4* base = reinterpret_cast<const float4*>(op.bpart + (size_t)row * PW);
+            const size_t seg4 = SEGW / 4;
+            // segments in pairs, both segments' loads issued first
+            for (int s0 = 0; s0 < op.bsplit; s0 += 2) {
+              float4 q[2][V4];
+#pragma unroll
+              for (int j = 0; j < 2; ++j)
+                if (s0 + j < op.bsplit)
+#pragma unroll
+                  for (int c4 = 0; c4 < V4; ++c4) q[j][c4] = __ldcg(base + (size_t)(s0 + j) * seg4 + c4);
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                if (s0 + j < op.bsplit) {
+                  const float* f = reinterpret_cast<const float*>(q[j]);
+#pragma unroll
+                  for (int r = 0; r < MAX_BATCH; ++r) {
+                    v[r] = (s0 + j) == 0 ? f[r] : v[r] + f[r];
+                    if (PAIR) u[r] = (s0 + j) == 0 ? f[MAX_BATCH + r] : u[r] + f[MAX_BATCH + r];
                   }
                 }
               }
             }
           }
         }
-      }
-      if (finish) {
-        if (ok && row < nrows) bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
-        if (KIND == TK_GEMV_RESID && op.xss_out != nullptr) {
-          // the block's sums of squares of the new x, per request: lanes, then
-          // warps 0..3 in order
+        if (finish) {
+          if (ok && row < nrows)
+            bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
+          if (KIND == TK_GEMV_RESID && op.xss_out != nullptr) {
+            // the block's sums of squares of the new x, per request: lanes,
+            // then warps 0..3 in order
 #pragma unroll
-          for (int r = 0; r < MAX_BATCH; ++r) {
-            const float ssr = warp_sum(nx[r] * nx[r]);
-            if (lane == 0) sm.bss[i & 1][cw][r] = ssr;
-          }
-          epi_sync();
-          if (ctid < R) {
-            const float t = sm.bss[i & 1][0][ctid] + sm.bss[i & 1][1][ctid] + sm.bss[i & 1][2][ctid] +
-                            sm.bss[i & 1][3][ctid];
-            st_tagged(op.xss_out + (size_t)rb * R + ctid, t, mytag);
+            for (int r = 0; r < MAX_BATCH; ++r) {
+              const float ssr = warp_sum(nx[r] * nx[r]);
+              if (lane == 0) sm.bss[i & 1][cw][r] = ssr;
+            }
+            epi_sync();
+            if (ctid < R) {
+              const float t = sm.bss[i & 1][0][ctid] + sm.bss[i & 1][1][ctid] + sm.bss[i & 1][2][ctid] +
+                              sm.bss[i & 1][3][ctid];
+              st_tagged(op.xss_out + (size_t)rb * R + ctid, t, mytag);
+            }
           }
         }
       }
     }
+    cstage += (uint32_t)(nblk * nst);
   }
   accn += (uint32_t)nblk;
-  cstage += (uint32_t)(nblk * nst);
   if (consumer_sync_or(fail)) return false;
   if (g.profiling && ctid == 0) sm.t_loop = globaltimer();
 

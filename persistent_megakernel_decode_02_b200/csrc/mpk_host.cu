@@ -161,8 +161,7 @@ int gemv_geometry(mpk_ctx* c, int li, OpDesc& o, bool two_mats, bool norm) {
 // Tensor-core geometry of a projection over R >= 2 requests: row blocks of BM,
 // K blocks of BK; grid_dim = (tasks per reduction segment, reduction segments,
 // 1).  Task t computes segment t / gx for the run of row blocks
-// [u nb / gx, (u+1) nb / gx), u = t mod gx, so gx <= nb; each segment must fit
-// the input buffer (B_MAX_KBLOCKS blocks).
+// [u nb / gx, (u+1) nb / gx), u = t mod gx, so gx <= nb.
 int batched_geometry(mpk_ctx* c, int li, OpDesc& o, int R, const mpk_layer& Ly) {
   if (R > MAX_BATCH)
     return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: %d requests (the batched projections take at most %d)", li, R,
@@ -189,12 +188,15 @@ int batched_geometry(mpk_ctx* c, int li, OpDesc& o, int R, const mpk_layer& Ly) 
   if (gy > o.nkb)
     return fail(c, MPK_ERR_SHAPE, "layer %d: grid_dim.y = %d segments for a reduction of %d blocks of %d", li, gy,
                 o.nkb, BK);
+  // a segment longer than the input buffer runs in passes, which keep every
+  // row block of the task in its own tensor-memory accumulator slot
   const int longest = (o.nkb + gy - 1) / gy;
-  if (longest > B_MAX_KBLOCKS)
+  const int most_blocks = (o.nb + gx - 1) / gx;
+  if (longest > B_MAX_KBLOCKS && most_blocks > NSLOT)
     return fail(c, MPK_ERR_SHAPE,
-                "layer %d: reduction length %d in %d segment(s) leaves %d elements per task (at most %d): "
-                "grid_dim.y must be at least %d", li, o.K, gy, longest * BK, B_MAX_KBLOCKS * BK,
-                (o.nkb + B_MAX_KBLOCKS - 1) / B_MAX_KBLOCKS);
+                "layer %d: tasks of %d row blocks over %d elements of the reduction: a task longer than %d elements "
+                "takes at most %d row blocks (more tasks per segment, grid_dim.x, or more segments, grid_dim.y)",
+                li, most_blocks, longest * BK, B_MAX_KBLOCKS * BK, NSLOT);
   o.dynamic = 0;
   return MPK_OK;
 }
@@ -622,7 +624,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.a_out = (uint64_t*)o->ptr;
         op.N = Hq * d;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
-        part_floats = std::max(part_floats, (size_t)R * Hq * gy * (d + 2));
+        part_floats = std::max(part_floats, (size_t)R * Hq * gy * R * (d + 2));
         merge_off[li] = {1, merge_u32};
         merge_u32 += (size_t)R * Hkv;
         const float theta = Ly.rope_theta > 0 ? Ly.rope_theta : 1.0e6f;
@@ -882,7 +884,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     bblk_off[p] = bblk_u32;
     bblk_u32 += (size_t)op.nb;
     bpart_off[p] = bpart_floats;
-    bpart_floats += (size_t)op.bsplit * R * op.N * (op.kind == TK_NORM_GEMV_SILU ? 2 : 1);
+    bpart_floats += (size_t)op.bsplit * op.N * MAX_BATCH * (op.kind == TK_NORM_GEMV_SILU ? 2 : 1);
   }
   const size_t o_bblk = take(sizeof(uint32_t) * (bblk_u32 ? bblk_u32 : 1));
   c->sync_bytes = off;

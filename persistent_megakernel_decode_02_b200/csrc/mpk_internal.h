@@ -60,6 +60,7 @@ constexpr int NSTB = 5;                     // weight stages of the ring in this
 constexpr int B_MAX_KBLOCKS = 24;           // longest reduction segment held for the inputs: 1536
 constexpr int B_KBLOCK_BYTES = BN * BK * 2; // the hi and lo rows of one K block: two 1 KB swizzle atoms
 static_assert(STAGE_BYTES == 2 * BOX_BYTES, "a weight stage holds two tiles");
+constexpr int NSLOT = 16;                   // accumulator slots of 2 BN tensor-memory columns (512 columns)
 static_assert(MAX_BATCH == 8, "one 8-row swizzle atom per half of the input columns");
 
 enum TaskKind : int32_t {
@@ -140,7 +141,7 @@ struct OpDesc {
   int32_t ntb;                  // tasks per segment (grid_dim.x), each owning a run of row blocks
   const void* tmap[MAX_SEG];    // tensor maps of W[s] (device memory, 64-byte aligned)
   const void* tmap_up;          // SILU: tensor map of the up matrix
-  float* bpart;                 // bsplit > 1: partial sums [bsplit][R][rows] (gate/up: rows = 2N)
+  float* bpart;                 // bsplit > 1: partial sums [bsplit][N][MAX_BATCH] (gate/up: [..][2 MAX_BATCH])
   // per-block sums of squares of x (batched graphs): EMBED and RESID publish
   // them for every BM-row block of the x they write, tagged [blocks][R]; the
   // RMSNorm operations read them instead of the whole of x

@@ -73,8 +73,10 @@ struct __align__(128) Smem {
   unsigned long long h_key;  // (iteration, op, segment) whose input vector hs holds (~0: none)
   float2 rope_row[MAX_D / 2];                    // its RoPE (cos, sin) row
   // tensor-core path
-  uint64_t acc_full[2];                          // accumulator b holds a finished row block
-  uint64_t acc_empty[2];                         // accumulator b has been read (one arrival per epilogue warp)
+  uint64_t acc_full[NSLOT];                      // accumulator slot b holds a finished row block
+  uint64_t acc_empty[NSLOT];                     // slot b has been read (one arrival per epilogue warp)
+  uint64_t bfree;                                // the MMAs of a pass are done with the input rows
+  uint32_t bfn;                                  // completed phases of bfree (read and advanced by consumer thread 0)
   uint64_t fin_bar;                              // drain of outstanding MMAs before exit
   uint32_t tmem_base;                            // tensor-memory address of the accumulators
   int32_t blast;                                 // this task finishes the current row block
@@ -584,8 +586,49 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z));
 // chunk 0).
 constexpr int ATTN_SPLIT_OP = 0, ATTN_GROUP = 1;
 
-__device__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
-                              int cw, int lane, uint32_t iter, int worker);
+__device__ __forceinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                              int mode, int cw, int lane, uint32_t iter, int worker);
+
+// Chunk slots of the split-K attention operation: each kv head has NQ = C x R
+// slots (C = grid_dim.y).  Request r takes C_r = 1 + floor(w_r (NQ - R) /
+// sum w) of them, w_r = s_r + 1 positions (an inactive request takes one,
+// which publishes zeros); the slots left over go one at a time to the request
+// with the most positions per chunk (lowest index on ties).  Slots are laid
+// out in request order, so chunks cover about the same number of positions
+// whatever the requests' lengths; slots past the last request's are unused.
+// Slot q of iteration iter -> (request r, chunk c of Cr); false when unused.
+__device__ bool attn_slot(const Graph& g, const OpDesc& op, int q, uint32_t iter, int& r, int& c, int& Cr) {
+  const int R = g.R, NQ = op.C * R;
+  int w[MAX_REQUESTS], cr[MAX_REQUESTS];
+  long long tot = 0;
+  for (int i = 0; i < R; ++i) {
+    int s;
+    w[i] = request_state(g, i, iter, s) ? s + 1 : 0;
+    tot += w[i];
+  }
+  int used = 0;
+  for (int i = 0; i < R; ++i) {
+    cr[i] = (w[i] > 0 && tot > 0) ? 1 + (int)(((long long)w[i] * (NQ - R)) / tot) : 1;
+    used += cr[i];
+  }
+  for (; used < NQ && tot > 0; ++used) {
+    int best = 0;
+    for (int i = 1; i < R; ++i)  // w[i] / cr[i] > w[best] / cr[best]
+      if ((long long)w[i] * cr[best] > (long long)w[best] * cr[i]) best = i;
+    ++cr[best];
+  }
+  int acc = 0;
+  for (int i = 0; i < R; ++i) {
+    if (q < acc + cr[i]) {
+      r = i;
+      c = q - acc;
+      Cr = cr[i];
+      return true;
+    }
+    acc += cr[i];
+  }
+  return false;
+}
 
 // The LM head's last task to arrive (sm.last) turns every active request's
 // maximum key into its next token: written to tokens[r, s+1] if that slot
@@ -915,8 +958,11 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // last chunk task of (r, j) to arrive merges the partials in chunk order and
 // signals the operation's event, in group mode chunk 0 merges once every
 // partial carries this iteration's tag and writes o.
+//
+// Not inlined, one function per (G, D): each gets its own register
+// allocation, independent of the projection code it shares a kernel with.
 template <int G, int D>
-__device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
+__device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
                           int cw, int lane, uint32_t iter, int worker) {
   const bool fused = mode == ATTN_GROUP;  // state fetched in the projections' prologue
   if (cw == 0 && lane == 0) sm.h_key = ~0ull;  // the attention scratch overlays the GEMV input vector
@@ -928,7 +974,8 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
   const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
   const size_t kvbase = ((((size_t)op.layer * g.R + r) * Hkv + j) * (size_t)op.S) * D;
-  const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * C) * (D + 2);
+  const int CS = op.C * g.R;  // split op: chunk partials per (request, query head)
+  const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * CS) * (D + 2);
   // Prologue rows: warp cw < G takes query head cw of the group, warp G the
   // key, warp G+1 the value.  Their loads do not depend on the step, so they
   // are issued before it is read.
@@ -1134,7 +1181,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
           st_tagged(p + 1, Ls, mytag);
         }
       } else {
-        float* p = const_cast<float*>(pbase) + ((size_t)hh * C + c) * (D + 2);
+        float* p = const_cast<float*>(pbase) + ((size_t)hh * CS + c) * (D + 2);
         p[2 + i] = Os;
         if (i == 0) {
           p[0] = M;
@@ -1198,7 +1245,10 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
   if (ctid == 0) {
     __threadfence();
     const uint32_t old = atomicAdd(op.merge_cnt + (size_t)r * Hkv + j, 1u);
-    sm.last = ((old + 1u) % (uint32_t)C) == 0u;
+    sm.last = (old + 1u) == (uint32_t)C;
+    // the merging task restarts the count for the next iteration (whose
+    // tasks depend on this merge's output)
+    if (sm.last) atomicExch(op.merge_cnt + (size_t)r * Hkv + j, 0u);
   }
   consumer_sync();
   if (sm.last) {
@@ -1207,7 +1257,7 @@ __device__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int
       // one pass over the chunk partials, in chunk order (online rescaling)
       for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
         const int hh = idx / D, i = idx % D;
-        const float* p = pbase + (size_t)hh * C * (D + 2);
+        const float* p = pbase + (size_t)hh * CS * (D + 2);
         float M = -INFINITY, Ls = 0.f, Os = 0.f;
 #pragma unroll 4
         for (int cc = 0; cc < C; ++cc) {
@@ -1298,10 +1348,8 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 }
 
 // ------------------------------------------------------------------ dispatch
-// Not inlined: attention gets its own register allocation, so its per-head
-// arrays never push the GEMV loops into spills.
-__device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
-                                           int mode, int cw, int lane, uint32_t iter, int worker) {
+__device__ __forceinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                              int mode, int cw, int lane, uint32_t iter, int worker) {
   const int key = op.G * 1000 + op.d;
   switch (key) {
     case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
@@ -1372,10 +1420,12 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
         case TK_NORM_GEMV_ARGMAX:
           ok = bgemm_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
           break;
-        case TK_ATTN:
-          ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C),
-                             ATTN_SPLIT_OP, cw, lane, iter, worker);
+        case TK_ATTN: {
+          int r, c, Cr;
+          if (attn_slot(g, op, task / op.Hkv, iter, r, c, Cr))
+            ok = attn_dispatch(sm, g, op, task % op.Hkv, c, Cr, r, ATTN_SPLIT_OP, cw, lane, iter, worker);
           break;
+        }
         default: ok = false;  // the fused projections + attention operation takes one request
       }
     } else switch (op.kind) {
@@ -1388,10 +1438,12 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
       case TK_NORM_GEMV_ARGMAX:
         ok = gemv_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
-      case TK_ATTN:
-        ok = attn_dispatch(sm, g, op, task % op.Hkv, (task / op.Hkv) % op.C, op.C, task / (op.Hkv * op.C),
-                           ATTN_SPLIT_OP, cw, lane, iter, worker);
+      case TK_ATTN: {
+        int r, c, Cr;
+        if (attn_slot(g, op, task / op.Hkv, iter, r, c, Cr))
+          ok = attn_dispatch(sm, g, op, task % op.Hkv, c, Cr, r, ATTN_SPLIT_OP, cw, lane, iter, worker);
         break;
+      }
       case TK_QKV_ATTN: ok = gemv_task<TK_QKV_ATTN>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
       default: ok = false;
     }
@@ -1492,10 +1544,12 @@ __device__ __forceinline__ void init_barriers(Smem& sm) {
     mbar_init(&sm.full[i], 1);
     mbar_init(&sm.empty[i], kBatch ? 1 : CONSUMER_WARPS);
   }
-  for (int i = 0; i < 2; ++i) {
+  for (int i = 0; i < NSLOT; ++i) {
     mbar_init(&sm.acc_full[i], 1);
     mbar_init(&sm.acc_empty[i], 4);
   }
+  mbar_init(&sm.bfree, 1);
+  sm.bfn = 0;
   mbar_init(&sm.fin_bar, 1);
   for (int i = 0; i < TASK_FIFO; ++i) {
     mbar_init(&sm.fifo_full[i], 1);

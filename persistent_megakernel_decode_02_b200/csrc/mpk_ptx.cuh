@@ -94,8 +94,8 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
 
 // ---------------------------------------------------------------- tensor memory and tcgen05 MMA
 // Columns of tensor memory one worker block allocates (a power of two >= 32):
-// two accumulators of 2 x 16 columns.
-constexpr uint32_t TMEM_COLS = 64;
+// all of it (one worker block per SM), as accumulator slots of 2 x 16 columns.
+constexpr uint32_t TMEM_COLS = 512;
 
 // Allocation by one whole warp; the tensor-memory address lands in *dst.
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst) {
@@ -187,6 +187,15 @@ __device__ __forceinline__ void st_release(uint32_t* p, uint32_t v) {
 
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {
   asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Fetch-and-add with acquire-release semantics at GPU scope: the caller's
+// earlier writes (and those its CTA barrier ordered before) are visible before
+// the increment, and writes released by earlier increments are visible after.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void red_relaxed_add(uint32_t* p, uint32_t v) {

@@ -37,28 +37,37 @@ def reduction_split(K: int, max_k: int = _lib.MAX_GEMV_K) -> int:
 # segment, segments).
 BATCH_BM, BATCH_BK, BATCH_MAX_KBLOCKS = 128, 64, 24
 # Task-size model used to choose the grid: a worker streams weights at about
-# its share of HBM bandwidth and pays a fixed cost per task.
+# its share of HBM bandwidth and pays a fixed cost per task, per extra pass
+# over the input rows, and (split reductions) for the finishing task's
+# partial-sum reduction.
 _WORKER_BYTES_PER_S = 43e9
 _TASK_OVERHEAD_S = 3e-6
+_PASS_OVERHEAD_S = 4e-6
+_SPLIT_OVERHEAD_S = 6e-6
+BATCH_SLOTS = 16  # accumulator slots: row blocks a task may hold across passes
 
 
 def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[int, int]:
     """grid_dim (tasks per reduction segment, segments) of a projection over
-    several requests: among segment counts s (enough that each fits the input
-    buffer) and, per number of rounds k of the workers, the largest run split
-    gx <= row blocks with gx * s <= k * workers, the one with the least
-    rounds x (largest task's weight bytes / bandwidth + task cost); fewer
-    segments on ties."""
+    several requests: among segment counts s and, per number of rounds k of
+    the workers, the largest run split gx <= row blocks with gx * s <= k *
+    workers, the one with the least rounds x (largest task's weight bytes /
+    bandwidth + task, pass and split costs); fewer segments on ties.  A task
+    longer than the input rows (passes) holds at most BATCH_SLOTS row blocks."""
     nb = -(-rows // BATCH_BM)
     nkb = K // BATCH_BK
-    smin = -(-nkb // BATCH_MAX_KBLOCKS)
     block_bytes = BATCH_BM * K * 2 * (2 if pair else 1)
     best = None
-    for s in range(smin, min(nkb, max(smin, 16)) + 1):
+    for s in range(1, min(nkb, 16) + 1):
+        npass = -(-(-(-nkb // s)) // BATCH_MAX_KBLOCKS)
         for k in range(1, 5):
             gx = max(1, min(nb, (k * workers) // s))
+            most = -(-nb // gx)
+            if npass > 1 and most > BATCH_SLOTS:
+                continue
             rounds = -(-(gx * s) // workers)
-            t = rounds * ((-(-nb // gx)) * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S)
+            t = rounds * (most * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S +
+                          (npass - 1) * _PASS_OVERHEAD_S) + (_SPLIT_OVERHEAD_S if s > 1 else 0.0)
             if best is None or t < best[0] * (1 - 1e-2):
                 best = (t, gx, s)
     return best[1], best[2]

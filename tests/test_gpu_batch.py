@@ -215,3 +215,61 @@ def test_request_permutation_is_exact(weights):
         assert np.array_equal(l0[perm], l1)
         assert np.array_equal(h0[:, perm], h1)
     assert torch.equal(k0[:, perm], k1)
+
+
+WIDE = sq.Qwen3Shape("tiny-wide", 2, 256, 4, 2, 64, 4096, 1024, tied=False)
+
+
+@pytest.fixture(scope="module")
+def wide_weights():
+    w_cpu = sq.make_weights(WIDE, seed=4)
+    return w_cpu, to_cuda(w_cpu)
+
+
+@pytest.mark.parametrize("down_grid,gu_grid,lm_grid", [
+    ((1, 1), (1, 1), (1, 1)),    # one task per op: the 4096-long down reduction in 3 passes, 16 gate/up blocks
+    ((2, 2), (4, 1), (8, 1)),    # split in two segments of 2048, each in 2 passes
+    ((2, 3), (32, 1), (8, 4)),   # three segments of 1365 (single pass), one block per gate/up task
+    ((1, 64), (2, 4), (4, 2)),   # every K block its own task (64-way split)
+])
+def test_reduction_passes_and_splits(wide_weights, monkeypatch, down_grid, gu_grid, lm_grid):
+    """Reductions longer than the shared-memory input rows run in passes that
+    keep each row block in its own tensor-memory accumulator, alone or combined
+    with cross-task splits: all within tight tolerance of the oracle."""
+    import persistent_megakernel_decode_02_b200.qwen3 as q3
+    from persistent_megakernel_decode_02_b200 import build_decoder
+
+    grids = {(WIDE.hidden, WIDE.intermediate, False): down_grid, (WIDE.intermediate, WIDE.hidden, True): gu_grid,
+             (WIDE.vocab, WIDE.hidden, False): lm_grid}
+    orig = q3.batched_grid
+    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, w, pair=False: grids.get((rows, K, pair)) or
+                        orig(rows, K, w, pair))
+    w_cpu, w = wide_weights
+    R = 4
+    p0 = _positions(R, seed=19)
+    kc, vc = sq.make_kv_prefill(WIDE, R, S, int(p0.max()), seed=20)
+    tokens = sq.make_tokens(WIDE, R, S, [S] * R, seed=21, teacher_forced=True)
+    dec = build_decoder(WIDE, w, requests=R, max_seq=S, k_cache=kc.cuda(), v_cache=vc.cuda())
+    gpu, _, gstep = gpu_teacher_forced(dec, tokens, 2, step0=p0)
+    ref, _, _, _ = oracle_teacher_forced(WIDE, w_cpu, tokens, 2, _u16(kc), _u16(vc), step0=p0)
+    wl, wh = compare_captures(gpu, ref)
+    print(f"down {down_grid} gate/up {gu_grid} lm {lm_grid}: worst logits rel-L2 {wl:.2e}, hidden {wh:.2e}")
+    assert wl <= 1e-3 and wh <= 1e-3
+    assert np.array_equal(gstep.numpy(), p0 + 2)
+    dec.kernel.close()
+
+
+def test_too_many_blocks_for_passes_is_rejected(wide_weights, monkeypatch):
+    """A task that needs passes must fit its row blocks in the accumulator
+    slots: 32 gate/up blocks of one task over a reduction longer than the
+    input rows are refused at compile time."""
+    import persistent_megakernel_decode_02_b200.qwen3 as q3
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    from persistent_megakernel_decode_02_b200._lib import MpkError
+
+    shape = sq.Qwen3Shape("tiny-long", 1, 2048, 4, 2, 64, 4096, 1024, tied=False)
+    w = to_cuda(sq.make_weights(shape, seed=5))
+    orig = q3.batched_grid
+    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, wk, pair=False: (1, 1) if pair else orig(rows, K, wk, pair))
+    with pytest.raises(MpkError, match="at most 16 row blocks"):
+        build_decoder(shape, w, requests=2, max_seq=16)
