@@ -23,6 +23,9 @@ tokens each.  The prompts are ingested first (untimed, one decode iteration
 per prompt token), then 256 lock-step iterations (every request one token per
 iteration, each at its own position) run in ONE timed launch; a step is one
 such iteration, reported in ms/step.  The projections run on the tensor cores.
+
+--workload long measures one request over a KV cache pre-filled with 32768
+positions (seeded N(0,1) bf16): 128 greedy iterations in one timed launch.
 """
 from __future__ import annotations
 
@@ -50,12 +53,16 @@ BATCH, BATCH_SEQ, BATCH_PROMPT, BATCH_GENERATED = 8, 1024, (32, 512), 256
 METRIC_BATCH = "decode ms/step (Qwen3-8B-shape, 8 requests) and HBM GB/s vs ~8 TB/s peak"
 UNIT_BATCH = "ms/step"
 
+LONG_CONTEXT, LONG_GENERATED = 32768, 128
+METRIC_LONG = "decode ms/token (Qwen3-8B-shape, batch 1, 32768 cached positions) and HBM GB/s vs ~8 TB/s peak"
+
 
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--workload", choices=["batch1", "batch8"], default="batch1",
-                   help="batch1: one request, 39-token prompt + 512 tokens (default); batch8: 8 requests")
+    p.add_argument("--workload", choices=["batch1", "batch8", "long"], default="batch1",
+                   help="batch1: one request, 39-token prompt + 512 tokens (default); batch8: 8 requests; "
+                        "long: one request over 32768 pre-filled positions")
     p.add_argument("--steps", type=int, default=0, help="timed steps (default: 512 for batch1, 256 for batch8)")
     p.add_argument("--warmup", type=int, default=8)
     p.add_argument("--impl", choices=["mpk", "reference"], default="mpk")
@@ -79,7 +86,7 @@ def parse():
     p.add_argument("--vocab", type=int, default=0, help="override the vocabulary (profiling cases)")
     args = p.parse_args()
     if not args.steps:
-        args.steps = GENERATED if args.workload == "batch1" else BATCH_GENERATED
+        args.steps = {"batch1": GENERATED, "batch8": BATCH_GENERATED, "long": LONG_GENERATED}[args.workload]
     return args
 
 
@@ -145,16 +152,16 @@ def kernel_source_digest() -> str:
     import hashlib
     csrc = os.path.join(ROOT, "persistent_megakernel_decode_02_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("mpk_kernel.cu", "mpk_internal.h", "mpk_ptx.cuh"):
+    for f in ("mpk_kernel.cu", "mpk_internal.h", "mpk_ptx.cuh", "mpk_batch.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def traffic_ratio():
-    """DRAM bytes per algorithmic byte from the committed ncu summary, when it was
-    taken on the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "mpk_persistent_kernel_dram_traffic.txt")
+def traffic_ratio(kernel: str = "mpk_persistent_kernel"):
+    """DRAM bytes per algorithmic byte of `kernel` from the committed ncu summary,
+    when it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_dram_traffic.txt")
     if not os.path.exists(path):
         return None
     kv = {}
@@ -329,6 +336,16 @@ def workload_config(shape, args, dec):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def sized_shape(sq, args):
+    """The --shape, with --layers / --vocab overrides (smaller profiling cases)."""
+    shape = sq.SHAPES[args.shape]
+    if args.layers or args.vocab:
+        import dataclasses
+        shape = dataclasses.replace(shape, name=f"{shape.name}-L{args.layers or shape.layers}-V{args.vocab or shape.vocab}",
+                                    layers=args.layers or shape.layers, vocab=args.vocab or shape.vocab)
+    return shape
+
+
 def batch_algorithmic_bytes(shape, first_pos, iters: int) -> int:
     """Bytes one lock-step iteration of several requests must move, summed over
     iterations: every streamed weight byte once (shared by the batch), and per
@@ -352,7 +369,7 @@ def main_batch(args):
     from synth import qwen3 as sq
     from persistent_megakernel_decode_02_b200 import build_decoder, load
 
-    shape = sq.SHAPES[args.shape]
+    shape = sized_shape(sq, args)
     R, S, G = BATCH, BATCH_SEQ, BATCH_GENERATED
     steps = args.steps
     if not (1 <= steps <= G and 0 <= args.warmup <= G):
@@ -465,7 +482,10 @@ def main_batch(args):
             "tokens_per_s": tokens_per_s,
             "hbm_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "peak_kind": peak_kind,
+                         "traffic": (None if traffic_ratio("mpk_persistent_batch_kernel") is None
+                                     else traffic_ratio("mpk_persistent_batch_kernel") * bytes_launch),
+                         "traffic_source": "ncu dram bytes of a 4-layer case scaled by algorithmic bytes",
+                         "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_launch,
                          "kernel": "mpk_persistent_batch_kernel"},
             "cpu_baseline": cpu,
@@ -481,12 +501,9 @@ def main_batch(args):
         pg.destroy_process_group()
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
-    if args.workload == "batch8":
-        return main_batch(args)
+def main_long(args):
+    """Long-context decode: one request whose KV cache holds 32768 pre-filled
+    positions (seeded N(0,1) bf16), 128 greedy iterations timed in one launch."""
     import torch
     world, rank, local, pg = dist_setup(args)
     torch.cuda.set_device(local)
@@ -495,10 +512,93 @@ def main():
     from persistent_megakernel_decode_02_b200 import build_decoder, load
 
     shape = sq.SHAPES[args.shape]
-    if args.layers or args.vocab:
-        import dataclasses
-        shape = dataclasses.replace(shape, name=f"{shape.name}-L{args.layers or shape.layers}-V{args.vocab or shape.vocab}",
-                                    layers=args.layers or shape.layers, vocab=args.vocab or shape.vocab)
+    P, steps = LONG_CONTEXT, args.steps
+    if not (1 <= steps <= LONG_GENERATED and 0 <= args.warmup <= LONG_GENERATED):
+        raise SystemExit(f"--steps must be in 1..{LONG_GENERATED} and --warmup in 0..{LONG_GENERATED}")
+    S = P + LONG_GENERATED + 1
+    t0 = time.time()
+    w = {k: v.to(dev) for k, v in sq.make_weights(shape, seed=0).items()}
+    kc, vc = sq.make_kv_prefill(shape, 1, S, P, seed=11)
+    kc, vc = kc.to(dev), vc.to(dev)
+    t_gen = time.time() - t0
+    tokens_cpu = sq.make_tokens(shape, 1, S, [P + 1], seed=12)
+    ls = args.local_schedulers
+    W = args.workers or (load().mpk_device_sm_count() - ls // 4)
+    dec = build_decoder(shape, w, requests=1, max_seq=S, num_workers=W, num_local_schedulers=ls,
+                        attn_chunks=args.attn_chunks or None, k_cache=kc, v_cache=vc, profiling=args.profiling)
+    stream = torch.cuda.current_stream(dev)
+    tok = tokens_cpu.to(dev)
+    step = torch.full((1,), P, dtype=torch.int32, device=dev)
+    end = lambda n: torch.full((1,), n, dtype=torch.int32, device=dev)
+    dec.run(step, tok, end(P + args.warmup))             # warm-up iterations
+    torch.cuda.synchronize(dev)
+    dec.kernel.check_status()
+    tok.copy_(tokens_cpu.to(dev))                        # rewind (positions >= P are rewritten)
+    step.fill_(P)
+    stop = end(P + steps)
+    barrier(pg, dev)
+    torch.cuda.synchronize(dev)
+    clk = ClockSampler(local)
+    clk.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    dec.run(step, tok, stop, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = clk.stop()
+    barrier(pg, dev)
+    dec.kernel.check_status()
+    ms_launch = e0.elapsed_time(e1)
+    assert int(step.item()) == P + steps
+    gen = tok[0, P + 1:P + 1 + steps].cpu()
+    assert bool((gen >= 0).all()), "some timed tokens were not generated"
+    ms_max = max_over_ranks(pg, ms_launch, dev)
+    value, tokens_per_s = whole_job(ms_max, steps, world)
+    bytes_launch = algorithmic_bytes(shape, P, steps)
+    gbs = bytes_launch / (ms_launch * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    if rank == 0:
+        line = {
+            "metric": METRIC_LONG, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / steps, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{shape.name}-shape greedy decode, batch 1, KV cache pre-filled with {P} "
+                                   f"positions of seeded N(0,1) bf16, {steps} greedy tokens",
+                       "requests": 1, "cached_positions": P, "seq_len": S, "timed_tokens": steps,
+                       "weights": "seeded synthetic bf16 N(0,0.02), norms 1.0",
+                       "attention": "split-K operation", "num_workers": dec.kernel.num_workers,
+                       "l2": "no flush: every step streams all weights (15.1 GB) and 4.8 GB of KV",
+                       "parallelism": "replicas"},
+            "tokens_per_s": tokens_per_s, "hbm_gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
+                         "launch_ms": ms_launch, "kernel": "mpk_persistent_kernel"},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": 1, "clocks": clocks,
+            "setup_s": {"weights_and_kv": round(t_gen, 1)},
+        }
+        print(json.dumps(line), flush=True)
+    dec.kernel.close()
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.workload == "batch8":
+        return main_batch(args)
+    if args.workload == "long":
+        return main_long(args)
+    import torch
+    world, rank, local, pg = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from synth import qwen3 as sq
+    from persistent_megakernel_decode_02_b200 import build_decoder, load
+
+    shape = sized_shape(sq, args)
     S = PROMPT + GENERATED
     if not (1 <= args.steps <= GENERATED and 0 <= args.warmup <= GENERATED):
         raise SystemExit(f"--steps must be in 1..{GENERATED} and --warmup in 0..{GENERATED}")

@@ -97,7 +97,10 @@ typedef enum {
      * inputs = q fp32 [R,Hq*d], k fp32 [R,Hkv*d], v fp32 [R,Hkv*d];
      * weights = q_norm bf16 [d], k_norm bf16 [d], k_cache, v_cache bf16
      * [L,R,Hkv,S,d]; outputs[0] = o fp32 [R,Hq*d].  layer selects the cache
-     * slice; rope_theta the RoPE base.  grid_dim = (Hkv, chunks, R). */
+     * slice; rope_theta the RoPE base.  grid_dim = (Hkv, C, R): task
+     * (j, c, r) attends to chunk c of C of request r's positions (a split
+     * that never depends on the other requests); a request that is not active
+     * publishes zeros as its output. */
     MPK_OP_ATTENTION = 3,
     /* x += W a.  inputs[0] = a fp32 [R,K]; weights[0] = W bf16 [N,K];
      * outputs[0] = x fp32 [R,N] (read and written in place).  When K exceeds
@@ -141,7 +144,27 @@ typedef struct { int32_t x, y, z; } mpk_dim3;
  * of tasks (thread blocks) x*y*z; block_dim the threads per task (a multiple
  * of 32, at most mpk_worker_threads()).  [EN] "The API": both are specified per
  * fused layer, and the total number of thread blocks should be a multiple of
- * the number of workers (a warning, not an error, when it is not). */
+ * the number of workers (a warning, not an error, when it is not).
+ *
+ * Several requests (R = 2..MPK_MAX_BATCH): the projection operations
+ * (RMSNORM_LINEAR, LINEAR_RESIDUAL, RMSNORM_LINEAR_SILU_MUL,
+ * RMSNORM_LMHEAD_ARGMAX) run on the tensor cores as [R,K] x W^T contractions
+ * (tcgen05: weight tiles of MPK_BATCH_BM rows x 64 by TMA, every fp32 input
+ * split into bf16 hi + lo parts so the products see it to ~16 bits, fp32
+ * accumulation in tensor memory).  Their grid_dim is then (gx, gy, 1): the N
+ * rows form nb = ceil(N / MPK_BATCH_BM) row blocks (gate/up: of one matrix)
+ * and the reduction gy segments (gy <= K / 64); task t computes segment
+ * t / gx for the row blocks [u*nb/gx, (u+1)*nb/gx), u = t % gx (gx <= nb).
+ * With gy > 1 the last segment task of a row block to finish adds the partial
+ * sums in segment order.  A task whose segment is longer than
+ * MPK_BATCH_MAX_PASS_K runs it in passes and then holds at most
+ * MPK_BATCH_SLOTS row blocks.  K must be a multiple of 64 and stacked
+ * matrices start at multiples of MPK_BATCH_BM rows (MPK_ERR_UNSUPPORTED
+ * otherwise); RMSNORM_QKV_ATTENTION takes one request. */
+#define MPK_MAX_BATCH 8
+#define MPK_BATCH_BM 128
+#define MPK_BATCH_MAX_PASS_K 1536
+#define MPK_BATCH_SLOTS 16
 typedef struct {
     int32_t op;                         /* mpk_op */
     const char *inputs[MPK_MAX_IO];

@@ -624,7 +624,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         op.a_out = (uint64_t*)o->ptr;
         op.N = Hq * d;
         if (c->S_cache == 0 || op.S < c->S_cache) c->S_cache = op.S;
-        part_floats = std::max(part_floats, (size_t)R * Hq * gy * R * (d + 2));
+        part_floats = std::max(part_floats, (size_t)R * Hq * gy * (d + 2));
         merge_off[li] = {1, merge_u32};
         merge_u32 += (size_t)R * Hkv;
         const float theta = Ly.rope_theta > 0 ? Ly.rope_theta : 1.0e6f;

@@ -62,6 +62,9 @@ constexpr int B_KBLOCK_BYTES = BN * BK * 2; // the hi and lo rows of one K block
 static_assert(STAGE_BYTES == 2 * BOX_BYTES, "a weight stage holds two tiles");
 constexpr int NSLOT = 16;                   // accumulator slots of 2 BN tensor-memory columns (512 columns)
 static_assert(MAX_BATCH == 8, "one 8-row swizzle atom per half of the input columns");
+static_assert(MAX_BATCH == MPK_MAX_BATCH && BM == MPK_BATCH_BM && B_MAX_KBLOCKS * BK == MPK_BATCH_MAX_PASS_K &&
+                  NSLOT == MPK_BATCH_SLOTS,
+              "the header states the batched geometry");
 
 enum TaskKind : int32_t {
   TK_EMBED = 1,

@@ -589,45 +589,17 @@ constexpr int ATTN_SPLIT_OP = 0, ATTN_GROUP = 1;
 __device__ __forceinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
                                               int mode, int cw, int lane, uint32_t iter, int worker);
 
-// Chunk slots of the split-K attention operation: each kv head has NQ = C x R
-// slots (C = grid_dim.y).  Request r takes C_r = 1 + floor(w_r (NQ - R) /
-// sum w) of them, w_r = s_r + 1 positions (an inactive request takes one,
-// which publishes zeros); the slots left over go one at a time to the request
-// with the most positions per chunk (lowest index on ties).  Slots are laid
-// out in request order, so chunks cover about the same number of positions
-// whatever the requests' lengths; slots past the last request's are unused.
-// Slot q of iteration iter -> (request r, chunk c of Cr); false when unused.
-__device__ bool attn_slot(const Graph& g, const OpDesc& op, int q, uint32_t iter, int& r, int& c, int& Cr) {
-  const int R = g.R, NQ = op.C * R;
-  int w[MAX_REQUESTS], cr[MAX_REQUESTS];
-  long long tot = 0;
-  for (int i = 0; i < R; ++i) {
-    int s;
-    w[i] = request_state(g, i, iter, s) ? s + 1 : 0;
-    tot += w[i];
-  }
-  int used = 0;
-  for (int i = 0; i < R; ++i) {
-    cr[i] = (w[i] > 0 && tot > 0) ? 1 + (int)(((long long)w[i] * (NQ - R)) / tot) : 1;
-    used += cr[i];
-  }
-  for (; used < NQ && tot > 0; ++used) {
-    int best = 0;
-    for (int i = 1; i < R; ++i)  // w[i] / cr[i] > w[best] / cr[best]
-      if ((long long)w[i] * cr[best] > (long long)w[best] * cr[i]) best = i;
-    ++cr[best];
-  }
-  int acc = 0;
-  for (int i = 0; i < R; ++i) {
-    if (q < acc + cr[i]) {
-      r = i;
-      c = q - acc;
-      Cr = cr[i];
-      return true;
-    }
-    acc += cr[i];
-  }
-  return false;
+// Chunk slots of the split-K attention operation: grid_dim = (Hkv, C, R),
+// task (j, c, r) attends to chunk c of C of request r's positions.  The split
+// of a request never depends on the other requests, so its results do not
+// depend on the batch it shares an iteration with.
+__device__ __forceinline__ bool attn_slot(const Graph& g, const OpDesc& op, int q, uint32_t iter, int& r, int& c,
+                                          int& Cr) {
+  (void)iter;
+  r = q / op.C;
+  c = q - r * op.C;
+  Cr = op.C;
+  return r < g.R;
 }
 
 // The LM head's last task to arrive (sm.last) turns every active request's
@@ -974,7 +946,7 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
   const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
   const size_t kvbase = ((((size_t)op.layer * g.R + r) * Hkv + j) * (size_t)op.S) * D;
-  const int CS = op.C * g.R;  // split op: chunk partials per (request, query head)
+  const int CS = op.C;  // split op: chunk partials per (request, query head)
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * CS) * (D + 2);
   // Prologue rows: warp cw < G takes query head cw of the group, warp G the
   // key, warp G+1 the value.  Their loads do not depend on the step, so they

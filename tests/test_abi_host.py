@@ -93,3 +93,53 @@ def test_default_attention_chunks():
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 551) == 9
     assert default_attn_chunks(sq.QWEN3_8B, 1, 144, 32897) == 18
     assert default_attn_chunks(sq.TINY, 1, 144, 24) == 1
+
+
+def _header_define(name):
+    import re
+    txt = open(os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "mpk.h")).read()
+    m = re.search(rf"#define {name} (\d+)", txt)
+    return int(m.group(1))
+
+
+def test_batched_grid_rule():
+    """The batched projections' grid (tasks per segment, segments) obeys the
+    header's geometry for every model shape and worker count: at most one task
+    per row block and segment, at most one segment per K block, and a task
+    whose segment needs passes holds at most the accumulator slots."""
+    from persistent_megakernel_decode_02_b200.qwen3 import BATCH_BM, BATCH_MAX_KBLOCKS, BATCH_SLOTS, batched_grid
+    assert BATCH_BM == _header_define("MPK_BATCH_BM")
+    assert BATCH_MAX_KBLOCKS * 64 == _header_define("MPK_BATCH_MAX_PASS_K")
+    assert BATCH_SLOTS == _header_define("MPK_BATCH_SLOTS")
+    for shape in (sq.TINY, sq.QWEN3_0_6B, sq.QWEN3_8B):
+        cases = [(shape.q_dim + 2 * shape.kv_dim, shape.hidden, False), (shape.hidden, shape.q_dim, False),
+                 (shape.intermediate, shape.hidden, True), (shape.hidden, shape.intermediate, False),
+                 (shape.vocab, shape.hidden, False)]
+        for rows, K, pair in cases:
+            for W in (1, 7, 100, 144, 300):
+                gx, gy = batched_grid(rows, K, W, pair)
+                nb, nkb = -(-rows // BATCH_BM), K // 64
+                assert 1 <= gx <= nb and 1 <= gy <= nkb
+                if -(-nkb // gy) > BATCH_MAX_KBLOCKS:
+                    assert -(-nb // gx) <= BATCH_SLOTS
+    # the 8B plan for 144 workers: one round of tasks for the projections, the
+    # reductions split three or nine ways
+    assert batched_grid(6144, 4096, 144) == (48, 3)
+    assert batched_grid(12288, 4096, 144, True) == (48, 3)
+    assert batched_grid(4096, 12288, 144) == (16, 9)
+
+
+def test_batched_layer_plan():
+    """Several requests: split-K attention (no fused projections+attention op)
+    and two-dimensional grids for every projection."""
+    s = sq.QWEN3_8B
+    plan = layer_plan(s, requests=8, num_workers=144, attn_chunks=2)
+    methods = [p["method"] for p in plan]
+    assert "rmsnorm_qkv_attention_layer" not in methods
+    assert methods.count("attention_layer") == s.layers
+    assert plan[0]["grid_dim"] == 8
+    for p in plan[1:]:
+        if p["method"] == "attention_layer":
+            assert p["grid_dim"] == (s.kv_heads, 2, 8)
+        else:
+            assert isinstance(p["grid_dim"], tuple) and len(p["grid_dim"]) == 2

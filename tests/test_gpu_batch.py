@@ -273,3 +273,24 @@ def test_too_many_blocks_for_passes_is_rejected(wide_weights, monkeypatch):
     monkeypatch.setattr(q3, "batched_grid", lambda rows, K, wk, pair=False: (1, 1) if pair else orig(rows, K, wk, pair))
     with pytest.raises(MpkError, match="at most 16 row blocks"):
         build_decoder(shape, w, requests=2, max_seq=16)
+
+
+def test_results_do_not_depend_on_the_batch(weights):
+    """A request decodes to the same tokens, predictions and cache whether it
+    shares its iterations with one other request or with seven of different
+    lengths (every step of the path treats a request on its own)."""
+    _, w = weights
+    lens = [9, 3, 11, 5, 2, 7, 10, 4]
+    tokens = sq.make_tokens(SHAPE, 8, S, lens, seed=23)
+    outs = []
+    for R in (2, 8):
+        dec = _build(w, R)
+        tok = tokens[:R].cuda()
+        step = torch.zeros(R, dtype=torch.int32, device="cuda")
+        dec.run(step, tok, torch.full((R,), 30, dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        dec.kernel.check_status()
+        outs.append((tok[0].cpu(), dec.pred[0].cpu(), dec.k_cache[:, 0].cpu().view(torch.int16)))
+        dec.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
