@@ -558,6 +558,13 @@ def main_long(args):
     bytes_launch = algorithmic_bytes(shape, P, steps)
     gbs = bytes_launch / (ms_launch * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
+    timeline_stats = None
+    if args.profiling:
+        tl = dec.kernel.timeline()
+        if args.timeline_out:
+            write_chrome_trace(tl, dec, args.timeline_out)
+        op_kind.per_layer = (dec.kernel.num_ops() - 2) // shape.layers
+        timeline_stats = timeline_summary(tl, shape)
     if rank == 0:
         line = {
             "metric": METRIC_LONG, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -575,6 +582,7 @@ def main_long(args):
                          "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
                          "launch_ms": ms_launch, "kernel": "mpk_persistent_kernel"},
             "cpu_baseline": None, "e2e": None, "gpu_launches": 1, "clocks": clocks,
+            "timeline": timeline_stats,
             "setup_s": {"weights_and_kv": round(t_gen, 1)},
         }
         print(json.dumps(line), flush=True)

@@ -53,6 +53,21 @@ __device__ __forceinline__ int bstages(const OpDesc& op, int nkbs) {
   return op.kind == TK_NORM_GEMV_SILU ? nkbs : (nkbs + 1) / 2;
 }
 
+// Ring stages and accumulator slots a batched task takes.
+__device__ __forceinline__ void bgemm_counts(const OpDesc& op, int task, uint32_t& stages, uint32_t& blocks) {
+  int rb0, rb1, kb0, kb1, seg;
+  btask(op, task, rb0, rb1, kb0, kb1, seg);
+  const int npass = bpasses(kb1 - kb0);
+  uint32_t st = 0;
+  for (int ps = 0; ps < npass; ++ps) {
+    int kp0, kp1;
+    bpass(kb0, kb1, npass, ps, kp0, kp1);
+    st += (uint32_t)bstages(op, kp1 - kp0);
+  }
+  stages = st * (uint32_t)(rb1 - rb0);
+  blocks = (uint32_t)(rb1 - rb0);
+}
+
 // Producer side of a batched task: its weight tiles, stage by stage.  False on
 // abort or timeout.  t_issue (profiling) receives the first stage's issue time.
 __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
@@ -152,9 +167,9 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo
   lo = make_uint4(pack2(l[0], l[1]), pack2(l[2], l[3]), pack2(l[4], l[5]), pack2(l[6], l[7]));
 }
 
-// Consumer side of a batched task (all CONSUMER_THREADS threads).  cstage
-// counts ring stages, accn accumulator uses; both advance identically in every
-// consumer thread.  Roles inside the task: consumer warp MMA_WARP's lane 0
+// Consumer side of a batched task (all CONSUMER_THREADS threads).  cstage and
+// accn are the ring stage and accumulator use the task starts at (the caller
+// advances them by bgemm_counts).  Roles inside the task: consumer warp MMA_WARP's lane 0
 // issues every row block's MMAs, alternating between two tensor-memory
 // accumulators; warps 0..3 (tensor-memory lanes 0..127, one weight row per
 // thread) read each accumulator as soon as it is complete and run the
@@ -164,7 +179,7 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo
 // arrays nor the attention's are spilled around the other.
 template <int KIND>
 __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
-                                        uint32_t& cstage, uint32_t& accn, int cw, int lane, int worker) {
+                                        uint32_t cstage, uint32_t accn, int cw, int lane, int worker) {
   constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
   constexpr bool NORM = KIND != TK_GEMV_RESID;
   constexpr int MMA_WARP = 4;
@@ -439,7 +454,6 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
     }
     cstage += (uint32_t)(nblk * nst);
   }
-  accn += (uint32_t)nblk;
   if (consumer_sync_or(fail)) return false;
   if (g.profiling && ctid == 0) sm.t_loop = globaltimer();
 

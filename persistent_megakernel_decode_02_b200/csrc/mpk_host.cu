@@ -1024,6 +1024,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   g.ops = c->ops_dev;
   g.nops = P;
   g.batched = R >= 2 ? 1 : 0;
+  g.split_attn = 0;
+  for (int p = 0; p < P; ++p)
+    if (ops[p].kind == TK_ATTN) g.split_attn = 1;
   g.R = R;
   g.V = V;
   g.H = H;

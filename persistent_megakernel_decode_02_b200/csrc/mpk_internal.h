@@ -178,6 +178,7 @@ struct Graph {
   int32_t nops;
   int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
   int32_t batched;                  // 1: projections run on the tensor-core path (R >= 2)
+  int32_t split_attn;               // 1: the graph has split-K attention operations
   int32_t R, S, V, H, L;
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;

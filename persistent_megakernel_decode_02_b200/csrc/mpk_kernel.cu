@@ -352,11 +352,76 @@ struct PrefetchCursor {
   uint64_t pos;            // stream byte offset of (q, row)
 };
 
+// Chunk slots of the split-K attention operation: grid_dim = (Hkv, C, R),
+// task (j, c, r) attends to chunk c of C of request r's positions.  The split
+// of a request never depends on the other requests, so its results do not
+// depend on the batch it shares an iteration with.
+__device__ __forceinline__ bool attn_slot(const Graph& g, const OpDesc& op, int q, uint32_t iter, int& r, int& c,
+                                          int& Cr) {
+  (void)iter;
+  r = q / op.C;
+  c = q - r * op.C;
+  Cr = op.C;
+  return r < g.R;
+}
+
+// Producer side of a split-K attention task: the cached positions of its
+// chunk, [lo, min(hi, s)), into the ring, PB positions of K then PB of V per
+// stage (1-D bulk copies), once the previous iteration's attention has
+// released the operation (so those positions are in the cache).  The consumer
+// takes exactly these stages.  False on abort or timeout.
+// Ring stages a split-K attention task takes (the producer issues them, the
+// consumer reads them): its chunk's cached positions in blocks of
+// STAGE_BYTES / (4 d).
+__device__ __forceinline__ uint32_t attn_stages(const Graph& g, const OpDesc& op, int task, uint32_t iter) {
+  int r, c, Cr, s;
+  if (!attn_slot(g, op, task / op.Hkv, iter, r, c, Cr) || !request_state(g, r, iter, s)) return 0u;
+  const int npos = s + 1;
+  const int lo = (int)(((long long)c * npos) / Cr);
+  int hi = (int)(((long long)(c + 1) * npos) / Cr);
+  hi = hi < s ? hi : s;
+  const int PB = STAGE_BYTES / (4 * op.d);
+  return hi > lo ? (uint32_t)((hi - lo + PB - 1) / PB) : 0u;
+}
+
+// Not inlined, so it adds nothing to the producer loop's registers.
+__device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
+                                          uint32_t& pstage, int worker, uint64_t pol, int nr) {
+  int r, c, Cr;
+  if (!attn_slot(g, op, task / op.Hkv, iter, r, c, Cr)) return true;
+  const int j = task % op.Hkv;
+  int s;
+  if (!request_state(g, r, iter, s)) return true;
+  const int npos = s + 1;
+  const int lo = (int)(((long long)c * npos) / Cr);
+  int hi = (int)(((long long)(c + 1) * npos) / Cr);
+  hi = hi < s ? hi : s;
+  if (hi <= lo) return true;
+  if (iter > 0 && !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 2,
+                                op.self, task, worker, (int)iter))
+    return false;
+  const int D = op.d, PB = STAGE_BYTES / (4 * D);
+  const size_t kvbase = ((((size_t)op.layer * g.R + r) * op.Hkv + j) * (size_t)op.S) * D;
+  for (int p = lo; p < hi; p += PB) {
+    const int n = min(PB, hi - p);
+    const uint32_t slot = pstage % (uint32_t)nr;
+    if (!wait_mbar(g, &sm.empty[slot], ((pstage / (uint32_t)nr) & 1u) ^ 1u, 3, worker)) return false;
+    const uint32_t bytes = (uint32_t)n * (uint32_t)D * 2u;
+    mbar_arrive_expect_tx(&sm.full[slot], 2u * bytes);
+    bulk_g2s(sm.ring[slot], op.kc + kvbase + (size_t)p * D, bytes, &sm.full[slot], pol);
+    bulk_g2s(sm.ring[slot] + (size_t)PB * D * 2, op.vc + kvbase + (size_t)p * D, bytes, &sm.full[slot], pol);
+    ++pstage;
+  }
+  return true;
+}
+
 // Producer side of a tensor-core (batched) task; defined with the batched path.
 __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
                          uint64_t pol, unsigned long long* t_issue);
 
-template <bool kStandalone, bool kBatch>
+// kSplit: the graph has split-K attention operations, whose K/V the producer
+// streams (kernels without them leave the code out entirely).
+template <bool kStandalone, bool kBatch, bool kSplit>
 __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
   constexpr int NR = kBatch ? NSTB : NSTAGES;  // weight stages of the ring
   const uint64_t pol = policy_evict_first();
@@ -468,6 +533,15 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     const int opi = (int)((entry >> 16) & 0xFFFFu);
     const int task = (int)(entry & 0xFFFFu);
     const OpDesc& op = g.ops[opi];
+    if constexpr (kSplit) {
+      if (op.kind == TK_ATTN) {
+        if (!attn_produce(sm, g, op, task, (uint32_t)(entry >> 32), pstage, worker, pol, NR)) {
+          ok = false;
+          break;
+        }
+        continue;
+      }
+    }
     if (!is_gemv(op.kind)) continue;
     if constexpr (kBatch) {
       if (!bproduce(sm, g, op, task, pstage, worker, pol, g.profiling ? &sm.fifo_t[f] : nullptr)) {
@@ -586,21 +660,9 @@ __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z));
 // chunk 0).
 constexpr int ATTN_SPLIT_OP = 0, ATTN_GROUP = 1;
 
-__device__ __forceinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
-                                              int mode, int cw, int lane, uint32_t iter, int worker);
+__device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                           int mode, int cw, int lane, uint32_t iter, int worker);
 
-// Chunk slots of the split-K attention operation: grid_dim = (Hkv, C, R),
-// task (j, c, r) attends to chunk c of C of request r's positions.  The split
-// of a request never depends on the other requests, so its results do not
-// depend on the batch it shares an iteration with.
-__device__ __forceinline__ bool attn_slot(const Graph& g, const OpDesc& op, int q, uint32_t iter, int& r, int& c,
-                                          int& Cr) {
-  (void)iter;
-  r = q / op.C;
-  c = q - r * op.C;
-  Cr = op.C;
-  return r < g.R;
-}
 
 // The LM head's last task to arrive (sm.last) turns every active request's
 // maximum key into its next token: written to tokens[r, s+1] if that slot
@@ -918,6 +980,13 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // ------------------------------------------------------------------ batched projections (tensor cores)
 #include "mpk_batch.cuh"
 
+__device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32_t& cstage, uint32_t& accn) {
+  uint32_t st, bl;
+  bgemm_counts(op, task, st, bl);
+  cstage += st;
+  accn += bl;
+}
+
 // ------------------------------------------------------------------ attention task
 // Attention of kv head j for request r at position s, over the positions
 // [c (s+1) / C, (c+1) (s+1) / C) of chunk c of C.  Prologue: RMSNorm over the
@@ -930,12 +999,9 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // last chunk task of (r, j) to arrive merges the partials in chunk order and
 // signals the operation's event, in group mode chunk 0 merges once every
 // partial carries this iteration's tag and writes o.
-//
-// Not inlined, one function per (G, D): each gets its own register
-// allocation, independent of the projection code it shares a kernel with.
-template <int G, int D>
-__device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r, int mode,
-                          int cw, int lane, uint32_t iter, int worker) {
+template <int G, int D, bool STREAMED>
+__device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                          int mode, int cw, int lane, uint32_t iter, int worker, uint32_t cstage) {
   const bool fused = mode == ATTN_GROUP;  // state fetched in the projections' prologue
   if (cw == 0 && lane == 0) sm.h_key = ~0ull;  // the attention scratch overlays the GEMV input vector
   constexpr int LP = D / 8;          // lanes per position
@@ -1049,56 +1115,111 @@ __device__ __noinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& o
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
     }
-    const uint16_t* kg = op.kc + kvbase + sub * 8;
-    const uint16_t* vg = op.vc + kvbase + sub * 8;
-    for (int base = lo + cw * PPW; base < hi; base += NSTEP * CONSUMER_WARPS * PPW) {
-      uint4 kv[NSTEP], vv[NSTEP];
+    // one position's K/V (8 dims per lane) into the warp's online softmax
+    auto consume = [&](const uint4 kvu, const uint4 vvu, bool valid) {
+      const float kf[8] = {bf16_lo(kvu.x), bf16_hi(kvu.x), bf16_lo(kvu.y), bf16_hi(kvu.y),
+                           bf16_lo(kvu.z), bf16_hi(kvu.z), bf16_lo(kvu.w), bf16_hi(kvu.w)};
+      float sc[G];
 #pragma unroll
-      for (int u = 0; u < NSTEP; ++u) {
-        const int t = base + u * CONSUMER_WARPS * PPW + grp;
-        kv[u] = make_uint4(0, 0, 0, 0);
-        vv[u] = make_uint4(0, 0, 0, 0);
-        if (t < hi) {
-          if (t == s) {
-            kv[u] = *reinterpret_cast<const uint4*>(A.ks + sub * 8);
-            vv[u] = *reinterpret_cast<const uint4*>(A.vs + sub * 8);
-          } else {
-            kv[u] = ldcg_u4(kg + (size_t)t * D);
-            vv[u] = ldcg_u4(vg + (size_t)t * D);
-          }
-        }
+      for (int hh = 0; hh < G; ++hh) {
+        const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
+        const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
+        float a = q0.x * kf[0];
+        a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+        a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
+#pragma unroll
+        for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+        sc[hh] = a;
       }
-#pragma unroll
-      for (int u = 0; u < NSTEP; ++u) {
-        const bool valid = base + u * CONSUMER_WARPS * PPW + grp < hi;
-        const float kf[8] = {bf16_lo(kv[u].x), bf16_hi(kv[u].x), bf16_lo(kv[u].y), bf16_hi(kv[u].y),
-                             bf16_lo(kv[u].z), bf16_hi(kv[u].z), bf16_lo(kv[u].w), bf16_hi(kv[u].w)};
-        float sc[G];
+      if (valid) {
+        const float vf[8] = {bf16_lo(vvu.x), bf16_hi(vvu.x), bf16_lo(vvu.y), bf16_hi(vvu.y),
+                             bf16_lo(vvu.z), bf16_hi(vvu.z), bf16_lo(vvu.w), bf16_hi(vvu.w)};
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
-          const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
-          float a = q0.x * kf[0];
-          a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
-          a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
+          const float mn = fmaxf(m[hh], sc[hh]);
+          const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
+          const float p = exp2f(sc[hh] - mn);
+          l[hh] = l[hh] * al + p;
 #pragma unroll
-          for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-          sc[hh] = a;
+          for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
+          m[hh] = mn;
         }
-        if (valid) {
-          const float vf[8] = {bf16_lo(vv[u].x), bf16_hi(vv[u].x), bf16_lo(vv[u].y), bf16_hi(vv[u].y),
-                               bf16_lo(vv[u].z), bf16_hi(vv[u].z), bf16_lo(vv[u].w), bf16_hi(vv[u].w)};
+      }
+    };
+    if constexpr (STREAMED) {
+      // Split-K operation: the chunk's cached positions [lo, min(hi, s))
+      // arrive through the weight ring (the producer streams them with bulk
+      // copies, PB positions of K then of V per stage); position s, if in
+      // this chunk, comes from shared memory.
+      constexpr int PB = STAGE_BYTES / (4 * D);
+      const int nr = g.batched ? NSTB : NSTAGES;
+      const int chi = hi < s ? hi : s;
+      bool sfail = false;
+      for (int p0 = lo; p0 < chi; p0 += PB) {
+        const int n = min(PB, chi - p0);
+        const uint32_t cs = cstage;
+        const uint32_t slot = cs % (uint32_t)nr;
+        bool okk = true;
+        if (ctid == 0) okk = wait_mbar(g, &sm.full[slot], (cs / (uint32_t)nr) & 1u, 3, worker);
+        if (consumer_sync_or(!okk)) {
+          sfail = true;
+          break;
+        }
+        const uint16_t* Ks = reinterpret_cast<const uint16_t*>(sm.ring[slot]) + sub * 8;
+        const uint16_t* Vs = Ks + PB * D;
+        for (int b = cw * PPW; b < n; b += NSTEP * CONSUMER_WARPS * PPW) {
+          uint4 kv[NSTEP], vv[NSTEP];
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            const float mn = fmaxf(m[hh], sc[hh]);
-            const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
-            const float p = exp2f(sc[hh] - mn);
-            l[hh] = l[hh] * al + p;
+          for (int u = 0; u < NSTEP; ++u) {
+            const int t = b + u * CONSUMER_WARPS * PPW + grp;
+            kv[u] = make_uint4(0, 0, 0, 0);
+            vv[u] = make_uint4(0, 0, 0, 0);
+            if (t < n) {
+              kv[u] = *reinterpret_cast<const uint4*>(Ks + (size_t)t * D);
+              vv[u] = *reinterpret_cast<const uint4*>(Vs + (size_t)t * D);
+            }
+          }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
-            m[hh] = mn;
+          for (int u = 0; u < NSTEP; ++u) consume(kv[u], vv[u], b + u * CONSUMER_WARPS * PPW + grp < n);
+        }
+        // every warp is done with the stage: release it (the ring's empty
+        // barrier expects one arrival per consumer warp on the GEMV path, one
+        // on the tensor-core path)
+        consumer_sync();
+        if (ctid == 0) {
+          const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
+          for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[slot]);
+        }
+        cstage = cs + 1u;
+      }
+      if (sfail) return false;
+      if (hi == npos && cw == 0) {
+        const uint4 kvs = grp == 0 ? *reinterpret_cast<const uint4*>(A.ks + sub * 8) : make_uint4(0, 0, 0, 0);
+        const uint4 vvs = grp == 0 ? *reinterpret_cast<const uint4*>(A.vs + sub * 8) : make_uint4(0, 0, 0, 0);
+        consume(kvs, vvs, grp == 0);
+      }
+    } else {
+      const uint16_t* kg = op.kc + kvbase + sub * 8;
+      const uint16_t* vg = op.vc + kvbase + sub * 8;
+      for (int base = lo + cw * PPW; base < hi; base += NSTEP * CONSUMER_WARPS * PPW) {
+        uint4 kv[NSTEP], vv[NSTEP];
+#pragma unroll
+        for (int u = 0; u < NSTEP; ++u) {
+          const int t = base + u * CONSUMER_WARPS * PPW + grp;
+          kv[u] = make_uint4(0, 0, 0, 0);
+          vv[u] = make_uint4(0, 0, 0, 0);
+          if (t < hi) {
+            if (t == s) {
+              kv[u] = *reinterpret_cast<const uint4*>(A.ks + sub * 8);
+              vv[u] = *reinterpret_cast<const uint4*>(A.vs + sub * 8);
+            } else {
+              kv[u] = ldcg_u4(kg + (size_t)t * D);
+              vv[u] = ldcg_u4(vg + (size_t)t * D);
+            }
           }
         }
+#pragma unroll
+        for (int u = 0; u < NSTEP; ++u) consume(kv[u], vv[u], base + u * CONSUMER_WARPS * PPW + grp < hi);
       }
     }
     // merge the position groups of the warp
@@ -1320,21 +1441,55 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
 }
 
 // ------------------------------------------------------------------ dispatch
-__device__ __forceinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
-                                              int mode, int cw, int lane, uint32_t iter, int worker) {
-  const int key = op.G * 1000 + op.d;
-  switch (key) {
-    case 1000 + 64: return attn_task<1, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    case 2000 + 64: return attn_task<2, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    case 4000 + 64: return attn_task<4, 64>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    case 1000 + 128: return attn_task<1, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    case 2000 + 128: return attn_task<2, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    case 4000 + 128: return attn_task<4, 128>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker);
-    default: return false;
-  }
+// Attention dispatch by (G, D).  The fused projections + attention operation
+// calls one non-inlined dispatch with every body inlined into it (the GEMV
+// tasks' consumer loop then keeps its registers); the split-K operation calls
+// a non-inlined function per (G, D), each with its own register allocation.
+template <int G, int D, bool STREAMED>
+__device__ __noinline__ bool attn_task_call(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                            int mode, int cw, int lane, uint32_t iter, int worker, uint32_t cstage) {
+  return attn_task<G, D, STREAMED>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker, cstage);
 }
 
-template <bool kStandalone, bool kBatch>
+__device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
+                                           int mode, int cw, int lane, uint32_t iter, int worker) {
+#define MPK_ATTN_CASE(GG, DD) \
+  case GG * 1000 + DD: return attn_task<GG, DD, false>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker, 0u);
+  switch (op.G * 1000 + op.d) {
+    MPK_ATTN_CASE(1, 64) MPK_ATTN_CASE(2, 64) MPK_ATTN_CASE(4, 64)
+    MPK_ATTN_CASE(1, 128) MPK_ATTN_CASE(2, 128) MPK_ATTN_CASE(4, 128)
+    default: return false;
+  }
+#undef MPK_ATTN_CASE
+}
+
+__device__ __forceinline__ bool attn_dispatch_split(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C,
+                                                    int r, int mode, int cw, int lane, uint32_t iter, int worker,
+                                                    uint32_t cstage) {
+#define MPK_ATTN_CASE(GG, DD)                                                                                 \
+  case GG * 1000 + DD:                                                                                        \
+    return attn_task_call<GG, DD, true>(sm, g, op, j, c, C, r, mode, cw, lane, iter, worker, cstage);
+  switch (op.G * 1000 + op.d) {
+    MPK_ATTN_CASE(1, 64) MPK_ATTN_CASE(2, 64) MPK_ATTN_CASE(4, 64)
+    MPK_ATTN_CASE(1, 128) MPK_ATTN_CASE(2, 128) MPK_ATTN_CASE(4, 128)
+    default: return false;
+  }
+#undef MPK_ATTN_CASE
+}
+
+// A task of the split-K attention operation, its K/V streamed through the ring
+// from stage cstage on.  Returns the stages it took, -1 on failure.  Not
+// inlined, so the consumer loop keeps its registers.
+__device__ __noinline__ int attn_split_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
+                                            int cw, int lane, int worker, uint32_t cstage) {
+  int r, c, Cr;
+  bool ok = true;
+  if (attn_slot(g, op, task / op.Hkv, iter, r, c, Cr))
+    ok = attn_dispatch_split(sm, g, op, task % op.Hkv, c, Cr, r, ATTN_SPLIT_OP, cw, lane, iter, worker, cstage);
+  return ok ? (int)attn_stages(g, op, task, iter) : -1;
+}
+
+template <bool kStandalone, bool kBatch, bool kSplit>
 __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int lane) {
   const int ctid = cw * 32 + lane;
   uint32_t fpos = 0, cstage = 0, accn = 0;
@@ -1382,20 +1537,24 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     if constexpr (kBatch) {
       switch (op.kind) {
         case TK_EMBED: ok = embed_task(g, op, task, iter, ctid); break;
-        case TK_NORM_GEMV: ok = bgemm_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, accn, cw, lane, worker); break;
+        case TK_NORM_GEMV: ok = bgemm_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance(op, task, cstage, accn); break;
         case TK_GEMV_RESID:
           ok = bgemm_task<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance(op, task, cstage, accn);
           break;
         case TK_NORM_GEMV_SILU:
           ok = bgemm_task<TK_NORM_GEMV_SILU>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance(op, task, cstage, accn);
           break;
         case TK_NORM_GEMV_ARGMAX:
           ok = bgemm_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance(op, task, cstage, accn);
           break;
         case TK_ATTN: {
-          int r, c, Cr;
-          if (attn_slot(g, op, task / op.Hkv, iter, r, c, Cr))
-            ok = attn_dispatch(sm, g, op, task % op.Hkv, c, Cr, r, ATTN_SPLIT_OP, cw, lane, iter, worker);
+          const int n = attn_split_task(sm, g, op, task, iter, cw, lane, worker, cstage);
+          ok = n >= 0;
+          cstage += ok ? (uint32_t)n : 0u;
           break;
         }
         default: ok = false;  // the fused projections + attention operation takes one request
@@ -1411,9 +1570,13 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
         ok = gemv_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, cw, lane, worker);
         break;
       case TK_ATTN: {
-        int r, c, Cr;
-        if (attn_slot(g, op, task / op.Hkv, iter, r, c, Cr))
-          ok = attn_dispatch(sm, g, op, task % op.Hkv, c, Cr, r, ATTN_SPLIT_OP, cw, lane, iter, worker);
+        if constexpr (kSplit) {
+          const int n = attn_split_task(sm, g, op, task, iter, cw, lane, worker, cstage);
+          ok = n >= 0;
+          cstage += ok ? (uint32_t)n : 0u;
+        } else {
+          ok = false;  // the host runs graphs with split-K attention on the kSplit kernels
+        }
         break;
       }
       case TK_QKV_ATTN: ok = gemv_task<TK_QKV_ATTN>(sm, g, op, task, iter, cstage, cw, lane, worker); break;
@@ -1544,7 +1707,7 @@ __device__ __forceinline__ Smem& smem_layout(uint8_t* raw) {
 // A worker block: barriers (and, on the tensor-core path, the accumulator's
 // tensor memory, allocated by consumer warp 0 and released by it after the
 // last task, once no MMA is in flight), then the producer and consumer roles.
-template <bool kStandalone, bool kBatch>
+template <bool kStandalone, bool kBatch, bool kSplit>
 __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) init_barriers<kBatch>(sm);
@@ -1554,11 +1717,11 @@ __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worke
   if (kBatch) tc_fence_after_sync();
   if (warp < PRODUCER_WARPS) {
     regs_dec<PRODUCER_REGS>();
-    if (warp == 0 && lane == 0) producer_loop<kStandalone, kBatch>(sm, g, worker, sa_iter, sa_op);
+    if (warp == 0 && lane == 0) producer_loop<kStandalone, kBatch, kSplit>(sm, g, worker, sa_iter, sa_op);
     return;
   }
   regs_inc<CONSUMER_REGS>();
-  consumer_loop<kStandalone, kBatch>(sm, g, worker, warp - PRODUCER_WARPS, lane);
+  consumer_loop<kStandalone, kBatch, kSplit>(sm, g, worker, warp - PRODUCER_WARPS, lane);
   if (kBatch) {
     // the MMA-issuing thread waits (bounded) until none of its MMAs is outstanding
     if (warp == PRODUCER_WARPS + 4 && lane == 0) {
@@ -1575,7 +1738,7 @@ __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worke
   }
 }
 
-template <bool kBatch>
+template <bool kBatch, bool kSplit>
 __device__ __forceinline__ void persistent_body(const Graph& g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1601,31 +1764,42 @@ __device__ __forceinline__ void persistent_body(const Graph& g) {
     }
     return;
   }
-  worker_block<false, kBatch>(smem_layout(smem_raw), g, blockIdx.x - g.sched_ctas, 0, 0);
+  worker_block<false, kBatch, kSplit>(smem_layout(smem_raw), g, blockIdx.x - g.sched_ctas, 0, 0);
 }
 
+// Kernels: one request without split-K attention (the fused projections +
+// attention operation), one request with it (long contexts), several requests
+// (tensor-core projections, split-K attention).
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_kernel(const Graph g) {
-  persistent_body<false>(g);
+  persistent_body<false, false>(g);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_split_kernel(const Graph g) {
+  persistent_body<false, true>(g);
 }
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_batch_kernel(const Graph g) {
-  persistent_body<true>(g);
+  persistent_body<true, true>(g);
 }
 
 // One operation of one iteration as an ordinary launch: block b runs task b.
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_kernel(const Graph g, int op, uint32_t iter) {
-  worker_block<true, false>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+  worker_block<true, false, false>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_split_kernel(const Graph g, int op,
+                                                                                  uint32_t iter) {
+  worker_block<true, false, true>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
 }
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_batch_kernel(const Graph g, int op,
                                                                                   uint32_t iter) {
-  worker_block<true, true>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+  worker_block<true, true, true>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
 }
 
 // ------------------------------------------------------------------ host-side launch helpers
 size_t kernel_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t prepare_kernels() {
-  const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_batch_kernel,
-                      (const void*)mpk_op_kernel, (const void*)mpk_op_batch_kernel};
+  const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_split_kernel,
+                      (const void*)mpk_persistent_batch_kernel, (const void*)mpk_op_kernel,
+                      (const void*)mpk_op_split_kernel, (const void*)mpk_op_batch_kernel};
   for (const void* k : ks) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -1634,24 +1808,31 @@ cudaError_t prepare_kernels() {
 }
 
 cudaError_t max_blocks_per_sm(int* n) {
-  int a = 0, b = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, mpk_persistent_kernel, BLOCK_THREADS, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, mpk_persistent_batch_kernel, BLOCK_THREADS, SMEM_BYTES);
-  *n = a < b ? a : b;
-  return e;
+  const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_split_kernel,
+                      (const void*)mpk_persistent_batch_kernel};
+  int m = 1 << 30;
+  for (const void* k : ks) {
+    int a = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, k, BLOCK_THREADS, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    m = a < m ? a : m;
+  }
+  *n = m;
+  return cudaSuccess;
 }
 
 cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream) {
   void* args[] = {const_cast<Graph*>(&g)};
-  const void* k = g.batched ? (const void*)mpk_persistent_batch_kernel : (const void*)mpk_persistent_kernel;
+  const void* k = g.batched ? (const void*)mpk_persistent_batch_kernel
+                  : g.split_attn ? (const void*)mpk_persistent_split_kernel : (const void*)mpk_persistent_kernel;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
 }
 
 // An operation whose tasks wait on one another (group mode) is launched
 // cooperatively, so all of its blocks are resident together.
 cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, bool cooperative, cudaStream_t stream) {
-  const void* k = g.batched ? (const void*)mpk_op_batch_kernel : (const void*)mpk_op_kernel;
+  const void* k = g.batched ? (const void*)mpk_op_batch_kernel
+                  : g.split_attn ? (const void*)mpk_op_split_kernel : (const void*)mpk_op_kernel;
   void* args[] = {const_cast<Graph*>(&g), &op, &iter};
   if (cooperative)
     return cudaLaunchCooperativeKernel(k, dim3(ntasks), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
