@@ -511,7 +511,7 @@ def main_long(args):
     from synth import qwen3 as sq
     from persistent_megakernel_decode_02_b200 import build_decoder, load
 
-    shape = sq.SHAPES[args.shape]
+    shape = sized_shape(sq, args)
     P, steps = LONG_CONTEXT, args.steps
     if not (1 <= steps <= LONG_GENERATED and 0 <= args.warmup <= LONG_GENERATED):
         raise SystemExit(f"--steps must be in 1..{LONG_GENERATED} and --warmup in 0..{LONG_GENERATED}")
@@ -579,8 +579,11 @@ def main_long(args):
                        "parallelism": "replicas"},
             "tokens_per_s": tokens_per_s, "hbm_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": None, "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
-                         "launch_ms": ms_launch, "kernel": "mpk_persistent_kernel"},
+                         "traffic": (None if traffic_ratio("mpk_persistent_split_kernel") is None
+                                     else traffic_ratio("mpk_persistent_split_kernel") * bytes_launch),
+                         "traffic_source": "ncu dram bytes of a 2-iteration run scaled by algorithmic bytes",
+                         "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
+                         "launch_ms": ms_launch, "kernel": "mpk_persistent_split_kernel"},
             "cpu_baseline": None, "e2e": None, "gpu_launches": 1, "clocks": clocks,
             "timeline": timeline_stats,
             "setup_s": {"weights_and_kv": round(t_gen, 1)},
