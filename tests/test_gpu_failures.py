@@ -100,3 +100,38 @@ def test_host_abort_then_resume(weights):
     print(f"aborted at step {s_abort} of {S - 1}")
     dec.kernel.close()
     ref.kernel.close()
+
+
+@pytest.mark.parametrize("stall_op", [2, 3, 4, 6, 12])
+def test_batched_unsatisfiable_dependency_times_out(weights, stall_op):
+    """The batched kernel (tensor-core projections, streamed split-K attention)
+    under a stalled operation: RMSNorm + QKV (op 2), attention (3), o projection
+    (4), down projection (6), LM head (12).  The run ends with MPK_ERR_TIMEOUT
+    within the wait limit, after the accumulators' tensor memory is drained and
+    released, and a fresh batched decoder then runs normally."""
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    from persistent_megakernel_decode_02_b200._lib import ERR_CODE
+
+    S, R = 24, 4
+    tok = sq.make_tokens(SHAPE, R, S, [8, 5, 7, 3], seed=1).cuda()
+    step = torch.zeros(R, dtype=torch.int32, device="cuda")
+    dec = build_decoder(SHAPE, weights, requests=R, max_seq=S, timeout_s=0.2, debug_stall_op=stall_op)
+    before = tok.cpu()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    dec.run(step, tok)
+    torch.cuda.synchronize()
+    took = time.time() - t0
+    assert dec.kernel.status() == ERR_CODE["TIMEOUT"], dec.kernel.last_error()
+    assert took < 5.0, took
+    assert not step.any()
+    assert torch.equal(tok.cpu(), before)
+    dec.kernel.close()
+    ok = build_decoder(SHAPE, weights, requests=R, max_seq=S)
+    tok = sq.make_tokens(SHAPE, R, S, [8, 5, 7, 3], seed=1).cuda()
+    step = torch.zeros(R, dtype=torch.int32, device="cuda")
+    ok.run(step, tok)
+    torch.cuda.synchronize()
+    ok.kernel.check_status()
+    assert (step == S - 1).all()
+    ok.kernel.close()
