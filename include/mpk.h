@@ -78,7 +78,10 @@ typedef enum { MPK_IO_CUDA = 0, MPK_IO_NVSHMEM = 1 } mpk_io;
  * to build the graph; rmsnorm_linear_layer is the one the pages name).
  * Number format: weights and the KV cache are bf16; every activation (the
  * residual stream x, normed inputs h, q/k/v, the attention output o, the MLP
- * product a, logits) is fp32; dot products accumulate in fp32. */
+ * product a, logits) is fp32; dot products accumulate in fp32.  The
+ * activation tensors passed between operations (x, q, k, v, o, a below,
+ * written "fp32") are registered as MPK_FP32T: fp32 values carrying version
+ * tags; MPK_ERR_DTYPE otherwise. */
 typedef enum {
     /* x[r,:] = fp32(E[tokens[r, step[r]], :]).
      * weights[0] = E bf16 [V,H]; outputs[0] = x fp32 [R,H].  grid_dim = R tasks. */

@@ -4,7 +4,8 @@ projection a tensor-core (tcgen05) contraction over the batch.
 Expected values come from the CPU oracle only (its plain ROUND_NONE reading).
 The batched projections feed each fp32 input to the MMA as a bf16 hi/lo pair,
 so they see it to about 16 significant bits; the results stay within the
-spec tolerances with a wide margin, and greedy tokens match exactly.
+decode tolerances (logits 2e-2, hidden 1e-2 rel-L2) with a wide margin, and
+greedy tokens match exactly.
 """
 import numpy as np
 import pytest
@@ -44,7 +45,7 @@ def _positions(R, seed):
 @pytest.mark.parametrize("R", [2, 3, 8])
 def test_teacher_forced_batch(weights, R):
     """R requests at different positions (KV pre-filled below the largest):
-    logits and every layer's residual stream within the benchmark spec's tolerances,
+    logits (rel-L2 2e-2) and every layer's residual stream (1e-2) within tolerance,
     and the cache rows each request appends."""
     w_cpu, w = weights
     p0 = _positions(R, seed=R)
