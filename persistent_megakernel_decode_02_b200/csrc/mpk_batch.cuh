@@ -152,6 +152,19 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
   }
 }
 
+// Element k of request r's row of x into the next RMSNorm operation's
+// published input rows: bf16 hi/lo of x * w_next[k] at row r (hi) and 8 + r
+// (lo) of K block k / 64, 16-byte chunk (k mod 64) / 8 swizzled by r.
+__device__ __forceinline__ void publish_xb(const OpDesc& op, int k, int r, float x) {
+  const float h = x * __uint_as_float((uint32_t)op.xb_w[k] << 16);
+  const uint16_t hi = f32_to_bf16_rn(h);
+  const uint16_t lo = f32_to_bf16_rn(h - __uint_as_float((uint32_t)hi << 16));
+  uint16_t* blk = op.xb_out + (size_t)(k >> 6) * (B_KBLOCK_BYTES / 2);
+  const int off = r * BK + ((((k & 63) >> 3) ^ r) << 3) + (k & 7);
+  blk[off] = hi;
+  blk[MAX_BATCH * BK + off] = lo;
+}
+
 // Two bf16 (bits) in one word, element k in the low half.
 __device__ __forceinline__ uint32_t pack2(uint16_t a, uint16_t b) { return (uint32_t)a | ((uint32_t)b << 16); }
 
@@ -224,6 +237,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       }
       ss = warp_sum(ss);
       if (lane == 0) sm.brinv[cw] = 1.0f / sqrtf(ss / (float)op.K + op.eps);
+      if (op.xb_in != nullptr) __threadfence();  // acquire: the rows published before these sums
     }
     if (consumer_sync_or(pfail)) return false;
   }
@@ -243,6 +257,20 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       }
       if (consumer_sync_or(fail || !ok)) return false;
     }
+    const bool published = NORM && op.xb_in != nullptr;
+    if (published) {
+      // the writers' published rows (their per-block sums of squares, all
+      // checked above, were released after them): one bulk copy of this
+      // pass's K blocks, waited for by the MMA-issuing thread
+      if (ctid == 0) {
+        fence_acq_rel_gpu();
+        fence_proxy_async_global();
+        const uint32_t bytes = (uint32_t)nkbs * (uint32_t)B_KBLOCK_BYTES;
+        mbar_arrive_expect_tx(&sm.bload, bytes);
+        bulk_g2s(bsm, op.xb_in + (size_t)kp0 * (B_KBLOCK_BYTES / 2), bytes, &sm.bload, policy_evict_first());
+      }
+      consumer_sync();
+    } else {
     // ---- the input rows of this pass's K blocks as bf16 hi/lo pairs into
     // the swizzled layout; FL chunks of 8 elements per thread in flight
     {
@@ -300,6 +328,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       fence_proxy_async_smem();  // the tensor cores read these bytes next
       if (consumer_sync_or(pfail)) return false;
     }
+    }
     if (ps == 0 && g.profiling && ctid == 0) sm.t_pro = globaltimer();
 
     if (cw == MMA_WARP) {
@@ -308,6 +337,15 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       if (lane == 0) {
         const uint32_t idesc = mma_idesc_bf16(BM, BN);
         bool ok = true;
+        if (published) {
+          ok = wait_mbar(g, &sm.bload, sm.bload_n & 1u, 3, worker);
+          if (!ok) {  // never leave the block with the copy in flight
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&sm.bload, sm.bload_n & 1u) && globaltimer() - t0 < 200000000ull) {
+            }
+          }
+          ++sm.bload_n;
+        }
         for (int i = 0; i < nblk; ++i) {
           const uint32_t a = accn + (uint32_t)i, slot = a % NSLOT, use = a / NSLOT;
           // the epilogue has read this slot's previous block
@@ -374,12 +412,16 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
         fail |= !ok;
-        // W hi + W lo per request
+        // W hi + W lo per request (published rows: times the request's RMS factor)
         float v[MAX_BATCH], u[MAX_BATCH], nx[MAX_BATCH];
 #pragma unroll
         for (int r = 0; r < MAX_BATCH; ++r) {
           v[r] = d[r] + d[MAX_BATCH + r];
           u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
+          if (published) {
+            v[r] *= sm.brinv[r];
+            u[r] *= sm.brinv[r];
+          }
           nx[r] = 0.f;
         }
         const int row = rb * BM + cw * 32 + lane;
@@ -434,6 +476,11 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         if (finish) {
           if (ok && row < nrows)
             bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
+          if (KIND == TK_GEMV_RESID && op.xb_out != nullptr && row < nrows) {
+#pragma unroll
+            for (int r = 0; r < MAX_BATCH; ++r)
+              if (r < R) publish_xb(op, row, r, nx[r]);
+          }
           if (KIND == TK_GEMV_RESID && op.xss_out != nullptr) {
             // the block's sums of squares of the new x, per request: lanes,
             // then warps 0..3 in order
@@ -446,6 +493,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
             if (ctid < R) {
               const float t = sm.bss[i & 1][0][ctid] + sm.bss[i & 1][1][ctid] + sm.bss[i & 1][2][ctid] +
                               sm.bss[i & 1][3][ctid];
+              if (op.xb_out != nullptr) __threadfence();  // the block's published rows first
               st_tagged(op.xss_out + (size_t)rb * R + ctid, t, mytag);
             }
           }

@@ -987,6 +987,33 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       op.xss_in = it->second;
       op.xss_blocks = (op.K + BM - 1) / BM;
     }
+    // published input rows: every writer of x also writes, for the next
+    // RMSNorm operation that reads this version of x, its rows as the
+    // tensor-core input (bf16 hi/lo of x * that operation's norm weight, in
+    // the swizzled shared-memory layout); one buffer per x tensor, zero in
+    // the unused request rows and past the end of x
+    std::map<const void*, uint16_t*> xb;
+    for (int p = 0; p < P; ++p) {
+      OpDesc& op = ops[p];
+      if (op.kind != TK_EMBED && op.kind != TK_GEMV_RESID) continue;
+      int q = -1;
+      for (int t = p + 1; t < P && q < 0; ++t) {
+        if ((ops[t].kind == TK_EMBED || ops[t].kind == TK_GEMV_RESID) && ops[t].x_out == op.x_out) break;
+        const bool norm = ops[t].kind == TK_NORM_GEMV || ops[t].kind == TK_NORM_GEMV_SILU ||
+                          ops[t].kind == TK_NORM_GEMV_ARGMAX;
+        if (norm && ops[t].x == op.x_out && ops[t].x_writer == p && ops[t].xb_in == nullptr) q = t;
+      }
+      if (q < 0) continue;
+      uint16_t*& buf = xb[op.x_out];
+      if (!buf) {
+        const size_t bytes = (size_t)((op.N + BK - 1) / BK) * B_KBLOCK_BYTES;
+        rc = alloc(c, &buf, bytes);
+        if (rc != MPK_OK) return rc;
+      }
+      op.xb_out = buf;
+      op.xb_w = ops[q].norm_w;
+      ops[q].xb_in = buf;
+    }
   }
   unsigned long long* timeline = nullptr;
   if (o.profiling) {

@@ -151,6 +151,16 @@ struct OpDesc {
   uint64_t* xss_out;
   const uint64_t* xss_in;
   int32_t xss_blocks;
+  // the next RMSNorm operation's input rows (batched graphs): writers of x
+  // (EMBED, RESID) also store bf16 hi/lo of x * w_norm of the next operation
+  // that normalises this x, in the swizzled layout of the shared-memory input
+  // buffer ([K/64 blocks][2 x 8 rows][64], 2 KB per block; rows past R zero),
+  // before publishing the block's sums of squares with release; the reader
+  // copies its K blocks with one bulk copy and applies the RMS factor to the
+  // products
+  uint16_t* xb_out;
+  const uint16_t* xb_w;
+  const uint16_t* xb_in;
 };
 
 struct Status {

@@ -77,6 +77,8 @@ struct __align__(128) Smem {
   uint64_t acc_empty[NSLOT];                     // slot b has been read (one arrival per epilogue warp)
   uint64_t bfree;                                // the MMAs of a pass are done with the input rows
   uint32_t bfn;                                  // completed phases of bfree (read and advanced by consumer thread 0)
+  uint64_t bload;                                // the published input rows of a pass have landed
+  uint32_t bload_n;                              // completed phases of bload (the MMA-issuing thread's)
   uint64_t fin_bar;                              // drain of outstanding MMAs before exit
   uint32_t tmem_base;                            // tensor-memory address of the accumulators
   int32_t blast;                                 // this task finishes the current row block
@@ -1392,8 +1394,17 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
     // of it reaches the request's tokens or cache
     const uint32_t mytag = vtag(g, iter, op.self);
     for (int i = ctid; i < op.N; i += CONSUMER_THREADS) st_tagged(op.x_out + (size_t)r * op.N + i, 0.f, mytag);
-    if (op.xss_out != nullptr)
-      for (int b = ctid; b < op.xss_blocks; b += CONSUMER_THREADS) st_tagged(op.xss_out + (size_t)b * g.R + r, 0.f, mytag);
+    if (op.xss_out != nullptr) {
+      const int cw = ctid >> 5, lane = ctid & 31;
+      for (int b = cw; b < op.xss_blocks; b += CONSUMER_WARPS) {
+        if (op.xb_out != nullptr) {
+          for (int i = b * BM + lane; i < min(op.N, (b + 1) * BM); i += 32) publish_xb(op, i, r, 0.f);
+          __threadfence();
+        }
+        __syncwarp();
+        if (lane == 0) st_tagged(op.xss_out + (size_t)b * g.R + r, 0.f, mytag);
+      }
+    }
     return true;
   }
   if (r < g.R) {
@@ -1431,7 +1442,13 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
           const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + i));
           const float e0 = bf16_lo(w.x), e1 = bf16_hi(w.x), e2 = bf16_lo(w.y), e3 = bf16_hi(w.y);
           ss = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
+          if (op.xb_out != nullptr) {
+            // the rows the next RMSNorm operation reads, before the sums
+            publish_xb(op, i, r, e0); publish_xb(op, i + 1, r, e1);
+            publish_xb(op, i + 2, r, e2); publish_xb(op, i + 3, r, e3);
+          }
         }
+        if (op.xb_out != nullptr) __threadfence();
         ss = warp_sum(ss);
         if (lane == 0) st_tagged(op.xss_out + (size_t)b * g.R + r, ss, mytag);
       }
@@ -1685,6 +1702,8 @@ __device__ __forceinline__ void init_barriers(Smem& sm) {
   }
   mbar_init(&sm.bfree, 1);
   sm.bfn = 0;
+  mbar_init(&sm.bload, 1);
+  sm.bload_n = 0;
   mbar_init(&sm.fin_bar, 1);
   for (int i = 0; i < TASK_FIFO; ++i) {
     mbar_init(&sm.fifo_full[i], 1);
