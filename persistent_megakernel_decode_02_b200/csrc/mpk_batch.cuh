@@ -138,8 +138,12 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
     }
   } else if (KIND == TK_NORM_GEMV_SILU) {
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r)
-      if (r < R) st_tagged(op.a_out + (size_t)r * op.N + row, silu_f(v[r]) * u[r], mytag);
+    for (int r = 0; r < MAX_BATCH; ++r) {
+      if (r < R) {
+        nx[r] = silu_f(v[r]) * u[r];
+        st_tagged(op.a_out + (size_t)r * op.N + row, nx[r], mytag);
+      }
+    }
   } else {  // LM head
 #pragma unroll
     for (int r = 0; r < MAX_BATCH; ++r) {
@@ -152,11 +156,12 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
   }
 }
 
-// Element k of request r's row of x into the next RMSNorm operation's
-// published input rows: bf16 hi/lo of x * w_next[k] at row r (hi) and 8 + r
-// (lo) of K block k / 64, 16-byte chunk (k mod 64) / 8 swizzled by r.
+// Element k of request r's input row into the next projection's published
+// input rows: bf16 hi/lo of x (times w_next[k] when the next operation is an
+// RMSNorm) at row r (hi) and 8 + r (lo) of K block k / 64, 16-byte chunk
+// (k mod 64) / 8 swizzled by r.
 __device__ __forceinline__ void publish_xb(const OpDesc& op, int k, int r, float x) {
-  const float h = x * __uint_as_float((uint32_t)op.xb_w[k] << 16);
+  const float h = op.xb_w != nullptr ? x * __uint_as_float((uint32_t)op.xb_w[k] << 16) : x;
   const uint16_t hi = f32_to_bf16_rn(h);
   const uint16_t lo = f32_to_bf16_rn(h - __uint_as_float((uint32_t)hi << 16));
   uint16_t* blk = op.xb_out + (size_t)(k >> 6) * (B_KBLOCK_BYTES / 2);
@@ -242,6 +247,24 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
     if (consumer_sync_or(pfail)) return false;
   }
 
+  // ---- published plain inputs: the tagged flags covering this task's K range
+  // (each thread acquires what it observed; the barrier hands it on)
+  if (!NORM && op.xb_in != nullptr) {
+    bool pfail = false;
+    const int g0 = kb0 * BK / op.xf_grp, g1 = min(kb1 * BK - 1, op.K - 1) / op.xf_grp;
+    const int ng = g1 - g0 + 1, nq = ng * (op.xf_rstride != 0 ? R : 1);
+    for (int q = ctid; q < nq; q += CONSUMER_THREADS) {
+      const uint64_t* p = op.xf_in + (size_t)(q / ng) * op.xf_rstride + g0 + q % ng;
+      uint64_t w = ld_tagged(p);
+      if (word_tag(w) != stag) {
+        w = poll_word(g, p, stag, op.self, worker, (int)iter);
+        pfail |= word_tag(w) != stag;
+      }
+      __threadfence();
+    }
+    if (consumer_sync_or(pfail)) return false;
+  }
+
   for (int ps = 0; ps < npass; ++ps) {
     int kp0, kp1;
     bpass(kb0, kb1, npass, ps, kp0, kp1);
@@ -257,11 +280,11 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       }
       if (consumer_sync_or(fail || !ok)) return false;
     }
-    const bool published = NORM && op.xb_in != nullptr;
+    const bool published = op.xb_in != nullptr;
     if (published) {
-      // the writers' published rows (their per-block sums of squares, all
-      // checked above, were released after them): one bulk copy of this
-      // pass's K blocks, waited for by the MMA-issuing thread
+      // the writers' published rows (released before the sums of squares or
+      // flags acquired above): one bulk copy of this pass's K blocks, waited
+      // for by the MMA-issuing thread
       if (ctid == 0) {
         fence_acq_rel_gpu();
         fence_proxy_async_global();
@@ -418,7 +441,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         for (int r = 0; r < MAX_BATCH; ++r) {
           v[r] = d[r] + d[MAX_BATCH + r];
           u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
-          if (published) {
+          if (NORM && published) {
             v[r] *= sm.brinv[r];
             u[r] *= sm.brinv[r];
           }
@@ -476,10 +499,18 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         if (finish) {
           if (ok && row < nrows)
             bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
-          if (KIND == TK_GEMV_RESID && op.xb_out != nullptr && row < nrows) {
+          if ((KIND == TK_GEMV_RESID || KIND == TK_NORM_GEMV_SILU) && op.xb_out != nullptr && row < nrows) {
 #pragma unroll
             for (int r = 0; r < MAX_BATCH; ++r)
               if (r < R) publish_xb(op, row, r, nx[r]);
+          }
+          if (KIND == TK_NORM_GEMV_SILU && op.xb_out != nullptr) {
+            // the row block's flag, after all its rows
+            epi_sync();
+            if (ctid == 0) {
+              __threadfence();
+              st_tagged(op.xf_out + rb, 0.f, mytag);
+            }
           }
           if (KIND == TK_GEMV_RESID && op.xss_out != nullptr) {
             // the block's sums of squares of the new x, per request: lanes,

@@ -1014,6 +1014,44 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       op.xb_w = ops[q].norm_w;
       ops[q].xb_in = buf;
     }
+    // published plain inputs of the o and down projections: the attention's
+    // merge (flag per request and kv head) and the gate/up epilogue (flag per
+    // row block) publish the rows; flags are tagged, so zeroed every run
+    std::map<std::pair<const void*, int>, std::pair<uint16_t*, uint64_t*>> ab;
+    for (int q = 0; q < P; ++q) {
+      OpDesc& rd = ops[q];
+      if (rd.kind != TK_GEMV_RESID || !rd.batched || rd.a_writer < 0) continue;
+      OpDesc& wr = ops[rd.a_writer];
+      int grp, rstride;
+      size_t nflags;
+      if (wr.kind == TK_ATTN) {
+        grp = wr.G * wr.d;
+        rstride = wr.Hkv;
+        nflags = (size_t)R * wr.Hkv;
+      } else if (wr.kind == TK_NORM_GEMV_SILU && wr.batched) {
+        grp = BM;
+        rstride = 0;
+        nflags = (size_t)((wr.N + BM - 1) / BM);
+      } else {
+        continue;
+      }
+      if (wr.xb_out != nullptr || rd.K % BK != 0 || grp % BK != 0) continue;
+      auto& e = ab[{rd.a_in, wr.kind}];
+      if (!e.first) {
+        rc = alloc(c, &e.first, (size_t)(rd.K / BK) * B_KBLOCK_BYTES);
+        if (rc != MPK_OK) return rc;
+        rc = alloc(c, &e.second, nflags * sizeof(uint64_t));
+        if (rc != MPK_OK) return rc;
+        c->zero_each_run.push_back({e.second, nflags * sizeof(uint64_t)});
+      }
+      wr.xb_out = e.first;
+      wr.xb_w = nullptr;
+      wr.xf_out = e.second;
+      rd.xb_in = e.first;
+      rd.xf_in = e.second;
+      rd.xf_grp = grp;
+      rd.xf_rstride = rstride;
+    }
   }
   unsigned long long* timeline = nullptr;
   if (o.profiling) {

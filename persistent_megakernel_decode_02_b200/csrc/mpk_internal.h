@@ -151,16 +151,22 @@ struct OpDesc {
   uint64_t* xss_out;
   const uint64_t* xss_in;
   int32_t xss_blocks;
-  // the next RMSNorm operation's input rows (batched graphs): writers of x
-  // (EMBED, RESID) also store bf16 hi/lo of x * w_norm of the next operation
-  // that normalises this x, in the swizzled layout of the shared-memory input
-  // buffer ([K/64 blocks][2 x 8 rows][64], 2 KB per block; rows past R zero),
-  // before publishing the block's sums of squares with release; the reader
-  // copies its K blocks with one bulk copy and applies the RMS factor to the
-  // products
+  // published input rows (batched graphs): the writer of a projection's input
+  // also stores it as bf16 hi/lo in the swizzled layout of the shared-memory
+  // input buffer ([K/64 blocks][2 x 8 rows][64], 2 KB per block; rows past R
+  // zero) and the reader copies its K blocks with one bulk copy.  Writers of x
+  // (EMBED, RESID) store x * w_norm of the next RMSNorm operation (xb_w) and
+  // release the rows with the block's sums of squares; the reader applies the
+  // RMS factor to the products.  Writers of a projection's plain input (the
+  // attention's merge, the gate/up epilogue; xb_w null) release them with tagged
+  // flags: flag r * xf_rstride + k / xf_grp covers element k of request r.
   uint16_t* xb_out;
   const uint16_t* xb_w;
   const uint16_t* xb_in;
+  uint64_t* xf_out;
+  const uint64_t* xf_in;
+  int32_t xf_grp;
+  int32_t xf_rstride;
 };
 
 struct Status {

@@ -1371,15 +1371,25 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
           Os = fmaf(oc, f, Os);
         }
         st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
+        if (op.xb_out != nullptr) publish_xb(op, (j * G + hh) * D + i, r, Os / Ls);
       }
     } else {
       // an inactive request still publishes this iteration's version of its
       // output (zeros), which the next projection waits for
-      for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS)
+      for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
         st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)j * G * D + idx, 0.f, mytag);
+        if (op.xb_out != nullptr) publish_xb(op, j * G * D + idx, r, 0.f);
+      }
     }
     consumer_sync();
-    if (ctid == 0) red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+    if (ctid == 0) {
+      if (op.xb_out != nullptr) {
+        // the group's published rows, then their flag
+        __threadfence();
+        st_tagged(op.xf_out + (size_t)r * Hkv + j, 0.f, mytag);
+      }
+      red_release_add(g.events + (size_t)op.out_event * EVENT_STRIDE, 1u);
+    }
   }
   return true;
 }
