@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-#define MPK_ABI_VERSION 1
+#define MPK_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MPK_API __attribute__((visibility("default")))
@@ -199,6 +199,13 @@ typedef struct {
                                iteration, or one completion more than its dependency
                                delivers), so that wait runs out and the run ends with
                                MPK_ERR_TIMEOUT (0: off)                                    */
+    int32_t poll_inputs;    /* several requests: > 0 makes every tensor-core projection
+                               read its input element by element (poll each tagged word,
+                               apply the RMSNorm, split into bf16 hi/lo) instead of the
+                               rows its writer publishes in the shared-memory layout;
+                               <= 0 (default): published rows wherever the graph allows.
+                               The RMSNorm factor then scales the input instead of the
+                               products, so results agree to rounding, not bit for bit. */
 } mpk_options;
 
 /* Library build facts. */

@@ -55,6 +55,7 @@ class Options(ctypes.Structure):
         ("prefetch_kb", ctypes.c_int32),
         ("dynamic_tasks", ctypes.c_int32),
         ("debug_stall_op", ctypes.c_int32),
+        ("poll_inputs", ctypes.c_int32),
     ]
 
 

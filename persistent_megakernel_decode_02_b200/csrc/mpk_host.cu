@@ -993,7 +993,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     // the swizzled shared-memory layout); one buffer per x tensor, zero in
     // the unused request rows and past the end of x
     std::map<const void*, uint16_t*> xb;
-    for (int p = 0; p < P; ++p) {
+    for (int p = 0; p < P && o.poll_inputs <= 0; ++p) {
       OpDesc& op = ops[p];
       if (op.kind != TK_EMBED && op.kind != TK_GEMV_RESID) continue;
       int q = -1;
@@ -1018,7 +1018,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     // merge (flag per request and kv head) and the gate/up epilogue (flag per
     // row block) publish the rows; flags are tagged, so zeroed every run
     std::map<std::pair<const void*, int>, std::pair<uint16_t*, uint64_t*>> ab;
-    for (int q = 0; q < P; ++q) {
+    for (int q = 0; q < P && o.poll_inputs <= 0; ++q) {
       OpDesc& rd = ops[q];
       if (rd.kind != TK_GEMV_RESID || !rd.batched || rd.a_writer < 0) continue;
       OpDesc& wr = ops[rd.a_writer];

@@ -191,7 +191,8 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   k_cache: Optional[torch.Tensor] = None, v_cache: Optional[torch.Tensor] = None,
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
-                  debug_stall_op: int = 0, dynamic_tasks: bool = False, tasks_per_worker: int = 2) -> Decoder:
+                  debug_stall_op: int = 0, dynamic_tasks: bool = False, tasks_per_worker: int = 2,
+                  poll_inputs: bool = False) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
@@ -232,5 +233,5 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
     mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb,
-               debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks)
+               debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks, poll_inputs=poll_inputs)
     return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)

@@ -25,8 +25,31 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(lib, n), n
         assert n in _lib.SIGNATURES, f"binding lacks {n}"
-    assert lib.mpk_abi_version() == 1
+    txt = open(os.path.join(ROOT, "include", "mpk.h")).read()
+    assert lib.mpk_abi_version() == int(re.search(r"#define MPK_ABI_VERSION (\d+)", txt).group(1))
     assert lib.mpk_worker_threads() == 256
+
+
+def _header_struct_fields(name):
+    """Member names, in order, of `typedef struct { ... } name;` in the header."""
+    txt = open(os.path.join(ROOT, "include", "mpk.h")).read()
+    body = re.search(r"typedef struct \{([^}]*)\}\s*" + name + ";", txt).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = []
+    for decl in body.split(";"):
+        for part in decl.split(","):
+            part = re.sub(r"\[\w*\]", "", part).strip()
+            if part:
+                names.append(re.findall(r"\w+", part)[-1])
+    return names
+
+
+@pytest.mark.parametrize("cname,pyname", [("mpk_options", "Options"), ("mpk_layer", "Layer"), ("mpk_dim3", "Dim3")])
+def test_binding_structs_mirror_the_header(cname, pyname):
+    """The ctypes structures passed through the C ABI list the header's members
+    in the header's order (a missing or reordered member shifts every later one)."""
+    fields = [f[0] for f in getattr(_lib, pyname)._fields_]
+    assert fields == _header_struct_fields(cname)
 
 
 GOLDEN = json.load(open(os.path.join(ROOT, "tests", "golden", "sm_split.json")))

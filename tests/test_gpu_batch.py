@@ -42,6 +42,33 @@ def _positions(R, seed):
     return np.array(sq.make_prompt_lengths(R, 0, 20, seed=seed).tolist(), np.int32)
 
 
+@pytest.mark.parametrize("R", [3, 8])
+def test_polled_inputs_and_published_rows_agree(weights, R):
+    """The projections' two ways of taking their inputs: rows their writers
+    publish in the shared-memory layout (default), or every tagged element
+    polled, normalised and split in the prologue (poll_inputs).  Both stay
+    within 1e-3 rel-L2 of the oracle in logits and every layer's residual
+    stream, and within 1e-3 of each other (the RMS factor scales the products
+    instead of the inputs, so they agree to rounding, not bit for bit)."""
+    w_cpu, w = weights
+    p0 = _positions(R, seed=R + 11)
+    P = int(p0.max())
+    kc, vc = sq.make_kv_prefill(SHAPE, R, S, P, seed=7)
+    tokens = sq.make_tokens(SHAPE, R, S, [S] * R, seed=8, teacher_forced=True)
+    iters = 3
+    ref, _, _, _ = oracle_teacher_forced(SHAPE, w_cpu, tokens, iters, _u16(kc), _u16(vc), step0=p0)
+    caps = []
+    for poll in (False, True):
+        dec = _build(w, R, k_cache=kc.cuda(), v_cache=vc.cuda(), poll_inputs=poll)
+        gpu, gtok, gstep = gpu_teacher_forced(dec, tokens, iters, step0=p0)
+        wl, wh = compare_captures(gpu, ref, logits_tol=1e-3, hidden_tol=1e-3)
+        print(f"R={R} poll_inputs={poll}: worst logits rel-L2 {wl:.2e}, hidden {wh:.2e}")
+        assert np.array_equal(gstep.numpy(), p0 + iters)
+        caps.append(gpu)
+        del dec
+    compare_captures(caps[0], caps[1], logits_tol=1e-3, hidden_tol=1e-3)
+
+
 @pytest.mark.parametrize("R", [2, 3, 8])
 def test_teacher_forced_batch(weights, R):
     """R requests at different positions (KV pre-filled below the largest):
