@@ -387,3 +387,32 @@ def test_decoder_matches_library_restatement(shape, mode):
     ref = _torch_reference(shape, w, toks[0], S - 1, mode)
     err = np.linalg.norm(np.stack(got) - ref) / np.linalg.norm(ref)
     assert err < 1e-9, err
+
+
+def test_decoder_requests_are_independent():
+    """Several requests decoded together (different prompt lengths, start and
+    end positions, one finishing while the others go on) give, request by
+    request, exactly what each gives decoded alone: tokens, final step, cache
+    rows and the logits of every iteration it was active.  Pins the oracle's
+    per-request bookkeeping (cache and token indexing by request, inactive
+    requests left untouched) that the batched GPU parity tests rely on."""
+    shape = qwen3.TINY
+    w = qwen3.make_weights(shape, seed=0)
+    dec = oracle.Decoder(shape, w)
+    S, R = 20, 3
+    toks = qwen3.make_tokens(shape, R, S, [5, 2, 8], seed=9).numpy().copy()
+    step0 = np.array([0, 1, 3], np.int32)
+    end = np.array([12, 6, 17], np.int32)
+    bt, bs, bk, bv, bcaps = dec.generate(toks, step0, end, capture=True)
+    assert np.array_equal(bs, end)
+    for r in range(R):
+        t, s, k, v, caps = dec.generate(toks[r:r + 1], step0[r:r + 1], end[r:r + 1], capture=True)
+        assert np.array_equal(bt[r], t[0]) and int(bs[r]) == int(s[0])
+        assert np.array_equal(bk[:, r], k[:, 0]) and np.array_equal(bv[:, r], v[:, 0])
+        n = int(end[r] - step0[r])
+        assert len(caps) == n
+        for i in range(n):
+            assert np.array_equal(bcaps[i][0][r], caps[i][0][0])
+            assert np.array_equal(bcaps[i][1][:, r], caps[i][1][:, 0])
+        # the cache rows past the request's last position are untouched
+        assert not bk[:, r, :, int(end[r]):].any()
