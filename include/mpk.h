@@ -341,15 +341,17 @@ MPK_API int mpk_timeline(mpk_ctx *ctx, uint64_t *out, int cap);
  *   logits_out device fp32 [num_requests, V] or NULL
  *   stream     cudaStream_t (NULL: legacy default stream); asynchronous.
  * Limits: 1 <= num_requests <= MPK_NOALLOC_MAX_REQUESTS, K a multiple of 8 up
- * to MPK_NOALLOC_MAX_K; larger sizes return MPK_ERR_INVALID_ARG / MPK_ERR_SHAPE
- * (message in mpk_noalloc_last_error()).
+ * to MPK_NOALLOC_MAX_K; larger sizes return MPK_ERR_INVALID_ARG / MPK_ERR_SHAPE,
+ * and eps must be positive and finite (else MPK_ERR_INVALID_ARG).  The message
+ * of a failed call is in mpk_noalloc_last_error() of the calling thread.
  * Scratch: a fixed __device__ array of 2 * MPK_NOALLOC_MAX_REQUESTS 64-bit
  * words (1 KiB) inside this library; every GPU that loads the library holds it
  * until the process exits.  Each call clears it on `stream` before use.  All
  * calls share it, so calls that overlap on the GPU (on different streams, or
  * from different threads) race and must be serialised by the caller.  The
  * first call on a device looks up the array's device address (set-up done once
- * per device, with that device current); make that first call before any
+ * per device and context, with that device current; a device whose context was
+ * reset gets a fresh lookup on its next call); make that first call before any
  * stream capture.  No cudaMalloc, cudaFree or allocating library routine is
  * called.
  */
@@ -359,7 +361,7 @@ MPK_API int mpk_lmhead_argmax_noalloc(const float *x, const uint16_t *norm_w, co
                                       int num_requests, int K, int V, float eps, int64_t *tokens_out,
                                       float *logits_out, void *stream);
 
-/* Message of the last failed mpk_lmhead_argmax_noalloc call ("" if none). */
+/* Message of this thread's last failed mpk_lmhead_argmax_noalloc call ("" if none). */
 MPK_API const char *mpk_noalloc_last_error(void);
 
 /* Free the context and every library-owned allocation. */

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -25,8 +26,6 @@ constexpr int kMaxDevices = 64;
 // [0, kMaxRequests): per-request maxima; [kMaxRequests, 2*kMaxRequests): arrival counters.
 static __device__ __align__(256) unsigned long long g_lmhead_scratch[2 * kMaxRequests];
 
-unsigned long long* g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
 
 __device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -105,28 +104,72 @@ __global__ void __launch_bounds__(kThreads) lmhead_argmax_noalloc_kernel(
   }
 }
 
-// Address of the scratch array on the current device, looked up once per
-// device (the symbol's host-side name is not a device address).
-cudaError_t scratch_on_current_device(unsigned long long** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_lmhead_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<unsigned long long*>(p);
+// Address of the scratch array in the current device's context.  The symbol's
+// host-side name is not a device address, so the address is looked up with
+// cudaGetSymbolAddress once per device and context: a context that was torn
+// down and created again (cudaDeviceReset, for instance) maps the array at a
+// new address, so the cache also keeps the id of the context it came from and
+// looks the address up again when the current context's id differs.
+typedef int (*CtxGetCurrentFn)(void**);
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);
+
+cudaError_t current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool resolved = false;
+  if (!resolved) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = cudaDriverEntryPointSymbolNotFound;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1);
+    if (e != cudaSuccess || q1 != cudaDriverEntryPointSuccess) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    e = cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2);
+    if (e != cudaSuccess || q2 != cudaDriverEntryPointSuccess) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    resolved = true;
   }
-  *out = g_scratch_addr[dev];
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0 || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  if (get_id(ctx, id) != 0) return cudaErrorDeviceUninitialized;
   return cudaSuccess;
 }
 
-char g_noalloc_err[256] = "";
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  unsigned long long* addr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+cudaError_t scratch_on_current_device(int dev, unsigned long long** out) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  // no context may be current yet (the lookup below creates the device's
+  // primary context); a missing id only means "look the address up"
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id) == cudaSuccess;
+  if (!have_id || g_scratch[dev].addr == nullptr || g_scratch[dev].ctx_id != id) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_lmhead_scratch);
+    if (e != cudaSuccess) return e;
+    e = current_context_id(&id);
+    g_scratch[dev].addr = static_cast<unsigned long long*>(p);
+    g_scratch[dev].ctx_id = e == cudaSuccess ? id : 0ull;
+    *out = g_scratch[dev].addr;
+    if (e != cudaSuccess) g_scratch[dev].addr = nullptr;  // no id to tie it to: look it up on every call
+    return cudaSuccess;
+  }
+  *out = g_scratch[dev].addr;
+  return cudaSuccess;
+}
+
+// per calling thread, so concurrent callers never see each other's message
+thread_local char g_noalloc_err[256] = "";
 
 int noalloc_fail(int code, const char* msg) {
   std::strncpy(g_noalloc_err, msg, sizeof(g_noalloc_err) - 1);
+  g_noalloc_err[sizeof(g_noalloc_err) - 1] = '\0';
   return code;
 }
 
@@ -146,17 +189,19 @@ MPK_API int mpk_lmhead_argmax_noalloc(const float* x, const uint16_t* norm_w, co
   if (V < 1) return noalloc_fail(MPK_ERR_SHAPE, "V must be positive");
   if (reinterpret_cast<uintptr_t>(w_lm) % 16 != 0)
     return noalloc_fail(MPK_ERR_INVALID_ARG, "w_lm must be 16-byte aligned");
-  if (!(eps > 0.f)) eps = 1e-6f;
+  if (!(eps > 0.f) || !(eps < INFINITY)) return noalloc_fail(MPK_ERR_INVALID_ARG, "eps must be positive and finite");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return noalloc_fail(MPK_ERR_CUDA, cudaGetErrorString(e));
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return noalloc_fail(MPK_ERR_CUDA, cudaGetErrorString(e));
   unsigned long long* scratch = nullptr;
-  cudaError_t e = scratch_on_current_device(&scratch);
+  e = scratch_on_current_device(dev, &scratch);
   if (e != cudaSuccess) return noalloc_fail(MPK_ERR_CUDA, cudaGetErrorString(e));
   // maxima and counters must start at zero; a memset allocates nothing
   e = cudaMemsetAsync(scratch, 0, sizeof(unsigned long long) * 2 * kMaxRequests, s);
   if (e != cudaSuccess) return noalloc_fail(MPK_ERR_CUDA, cudaGetErrorString(e));
-  int sms = 148, dev = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int nb = V < 2 * sms ? V : 2 * sms;
   const size_t smem = (size_t)K * sizeof(float);
   if (smem > 48 * 1024) {
