@@ -228,10 +228,13 @@ def barrier(pg, device=None):
 
 # ----------------------------------------------------------------------------- oracle timing
 
-def time_oracle(shape, w_cpu, tokens_cpu, budget_s: float, max_iters: int = 64, layer_sample=None):
-    """Time the CPU oracle on the first iterations of the same workload.  Returns
-    (ms per full token, iterations, threads, description)."""
+def time_oracle(shape, w_cpu, tokens_cpu, budget_s: float, max_iters: int = 64, layer_sample=None, kv=None,
+                step0: int = 0):
+    """Time the CPU oracle on the first iterations of the same workload (from
+    position step0, over the pre-filled bf16 caches kv = (K, V) when given).
+    Returns (ms per full token, iterations, threads, description)."""
     import numpy as np
+    import torch
     import oracle
     from synth import qwen3 as sq
 
@@ -246,8 +249,11 @@ def time_oracle(shape, w_cpu, tokens_cpu, budget_s: float, max_iters: int = 64, 
     dec = oracle.Decoder(sub_shape, sub_w)
     toks = tokens_cpu.numpy().copy()
     R, S = toks.shape
-    kc, vc = dec.new_cache(R, S)
-    step = np.zeros(R, np.int32)
+    if kv is None:
+        kc, vc = dec.new_cache(R, S)
+    else:
+        kc, vc = (np.ascontiguousarray(c[:sub_shape.layers].view(torch.int16).numpy().view(np.uint16)) for c in kv)
+    step = np.full(R, step0, np.int32)
     times = []
     t_start = time.perf_counter()
     while len(times) < max_iters:
@@ -257,10 +263,12 @@ def time_oracle(shape, w_cpu, tokens_cpu, budget_s: float, max_iters: int = 64, 
         if time.perf_counter() - t_start > budget_s:
             break
     ms = 1e3 * (sum(times) / len(times)) / frac
-    desc = (f"{len(times)} oracle decode iterations at positions 0..{len(times) - 1} of the same request "
+    first = step0
+    desc = (f"{len(times)} oracle decode iterations at positions {first}..{first + len(times) - 1} of the same request "
             f"({sub_shape.layers} of {shape.layers} layers + LM head, scaled by weight bytes x{1 / frac:.2f})"
             if frac < 1.0 else
-            f"{len(times)} full oracle decode iterations at positions 0..{len(times) - 1} of the same request")
+            f"{len(times)} full oracle decode iterations at positions {first}..{first + len(times) - 1} of the same "
+            f"request")
     return ms, len(times), oracle.num_threads(), desc
 
 
@@ -429,35 +437,65 @@ def main_batch(args):
         op_kind.per_layer = (dec.kernel.num_ops() - 2) // shape.layers
         timeline_stats = timeline_summary(tl, shape)
 
-    # end to end through the public API with host buffers: tokens in from pinned
-    # memory, prompts + the timed steps in one launch, tokens back to the host
+    op_ms = None
+    if args.op_by_op:
+        # the same timed iterations, one launch per operation
+        tok.copy_(tokens_cpu.to(dev))
+        step.copy_(p_end)
+        torch.cuda.synchronize(dev)
+        o0 = torch.cuda.Event(enable_timing=True)
+        o1 = torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
+        dec.run_op_by_op(step, tok, stop, stream)
+        o1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        op_ms = o0.elapsed_time(o1) / steps
+
+    # end to end through the public API with host buffers: the prompts are
+    # ingested in one launch (timed on its own); the decode window is H2D of
+    # tokens / step / step_end from pinned memory, the timed lock-step
+    # iterations in one launch and D2H of the tokens, reported per step.
     e2e = None
     if not args.no_e2e:
         host_tok = tokens_cpu.clone().pin_memory()
-        host_step = torch.zeros(R, dtype=torch.int32).pin_memory()
+        host_step0 = torch.zeros(R, dtype=torch.int32).pin_memory()
+        host_pend = (lens - 1).to(torch.int32).pin_memory()
         host_end = ((lens - 1) + steps).to(torch.int32).pin_memory()
         out_tok = torch.empty_like(host_tok).pin_memory()
         barrier(pg, dev)
         torch.cuda.synchronize(dev)
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
         tok.copy_(host_tok, non_blocking=True)
-        step.copy_(host_step, non_blocking=True)
+        step.copy_(host_step0, non_blocking=True)
+        stop.copy_(host_pend, non_blocking=True)
+        dec.run(step, tok, stop, stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        barrier(pg, dev)
+        ev[2].record(stream)
+        tok.copy_(host_tok, non_blocking=True)
+        step.copy_(host_pend, non_blocking=True)
         stop.copy_(host_end, non_blocking=True)
         dec.run(step, tok, stop, stream)
         out_tok.copy_(tok, non_blocking=True)
-        f1.record(stream)
+        ev[3].record(stream)
         torch.cuda.synchronize(dev)
         dec.kernel.check_status()
-        e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), dev)
+        prompt_ms = max_over_ranks(pg, ev[0].elapsed_time(ev[1]), dev)
+        e2e_ms = max_over_ranks(pg, ev[2].elapsed_time(ev[3]), dev)
         for r in range(R):
             assert torch.equal(out_tok[r, int(lens[r]):int(lens[r]) + steps], gen[r]), "e2e tokens differ"
         e2e = {"value": e2e_ms / steps, "unit": UNIT_BATCH,
                "h2d_bytes_per_step": (host_tok.numel() * 8 + 8 * R) / steps,
                "d2h_bytes_per_step": out_tok.numel() * 8 / steps,
-               "includes": "H2D of tokens/step/step_end, every request's prompt iterations + the timed "
-                           "iterations in one launch, D2H of tokens"}
+               "includes": f"H2D of tokens/step/step_end, {steps} lock-step decode iterations in one launch after "
+                           f"the prompts, D2H of tokens",
+               "prompt_ingestion_ms": prompt_ms,
+               "prompt_ingestion": "H2D of the prompts, each request's prompt as prefill-as-decode iterations in "
+                                   "one launch (longest prompt 512)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -492,6 +530,7 @@ def main_batch(args):
             "e2e": e2e,
             "gpu_launches": 1,
             "clocks": clocks,
+            "op_by_op_ms_per_step": op_ms,
             "timeline": timeline_stats,
             "setup_s": {"weights": round(t_gen, 1)},
         }
@@ -517,9 +556,10 @@ def main_long(args):
         raise SystemExit(f"--steps must be in 1..{LONG_GENERATED} and --warmup in 0..{LONG_GENERATED}")
     S = P + LONG_GENERATED + 1
     t0 = time.time()
-    w = {k: v.to(dev) for k, v in sq.make_weights(shape, seed=0).items()}
-    kc, vc = sq.make_kv_prefill(shape, 1, S, P, seed=11)
-    kc, vc = kc.to(dev), vc.to(dev)
+    w_cpu = sq.make_weights(shape, seed=0)
+    w = {k: v.to(dev) for k, v in w_cpu.items()}
+    kc_cpu, vc_cpu = sq.make_kv_prefill(shape, 1, S, P, seed=11)
+    kc, vc = kc_cpu.to(dev), vc_cpu.to(dev)
     t_gen = time.time() - t0
     tokens_cpu = sq.make_tokens(shape, 1, S, [P + 1], seed=12)
     ls = args.local_schedulers
@@ -565,6 +605,58 @@ def main_long(args):
             write_chrome_trace(tl, dec, args.timeline_out)
         op_kind.per_layer = (dec.kernel.num_ops() - 2) // shape.layers
         timeline_stats = timeline_summary(tl, shape)
+
+    op_ms = None
+    if args.op_by_op:
+        # the same timed iterations, one launch per operation
+        tok.copy_(tokens_cpu.to(dev))
+        step.fill_(P)
+        torch.cuda.synchronize(dev)
+        o0 = torch.cuda.Event(enable_timing=True)
+        o1 = torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
+        dec.run_op_by_op(step, tok, stop, stream)
+        o1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        op_ms = o0.elapsed_time(o1) / steps
+
+    # end to end through the public API with host buffers: H2D of tokens / step /
+    # step_end from pinned memory, the timed iterations in one launch over the
+    # resident pre-filled cache, D2H of the tokens; per generated token
+    e2e = None
+    if not args.no_e2e:
+        host_tok = tokens_cpu.clone().pin_memory()
+        host_step = torch.full((1,), P, dtype=torch.int32).pin_memory()
+        host_end = torch.full((1,), P + steps, dtype=torch.int32).pin_memory()
+        out_tok = torch.empty_like(host_tok).pin_memory()
+        barrier(pg, dev)
+        torch.cuda.synchronize(dev)
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        tok.copy_(host_tok, non_blocking=True)
+        step.copy_(host_step, non_blocking=True)
+        stop.copy_(host_end, non_blocking=True)
+        dec.run(step, tok, stop, stream)
+        out_tok.copy_(tok, non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), dev)
+        assert torch.equal(out_tok[0, P + 1:P + 1 + steps], gen), "e2e tokens differ from the timed run"
+        e2e = {"value": whole_job(e2e_ms, steps, world)[0], "unit": UNIT,
+               "h2d_bytes_per_step": (host_tok.numel() * 8 + 8) / steps,
+               "d2h_bytes_per_step": out_tok.numel() * 8 / steps,
+               "includes": f"H2D of tokens/step/step_end, {steps} decode iterations over the {P} cached positions "
+                           f"in one launch, D2H of tokens"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms_cpu, n, cores, desc = time_oracle(shape, w_cpu, tokens_cpu, args.cpu_budget_s, kv=(kc_cpu, vc_cpu),
+                                             step0=P)
+        cpu = {"value": ms_cpu, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": desc + f" over the {P} pre-filled cached positions"}
     if rank == 0:
         line = {
             "metric": METRIC_LONG, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
@@ -584,7 +676,7 @@ def main_long(args):
                          "traffic_source": "ncu dram bytes of a 2-iteration run scaled by algorithmic bytes",
                          "peak_kind": peak_kind, "algorithmic_bytes_per_launch": bytes_launch,
                          "launch_ms": ms_launch, "kernel": "mpk_persistent_split_kernel"},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": 1, "clocks": clocks,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 1, "clocks": clocks, "op_by_op_ms_per_token": op_ms,
             "timeline": timeline_stats,
             "setup_s": {"weights_and_kv": round(t_gen, 1)},
         }
@@ -675,41 +767,61 @@ def main():
         tok.copy_(tokens_cpu.to(dev))
         step.fill_(PROMPT - 1)
         torch.cuda.synchronize(dev)
-        a = time.perf_counter()
+        o0 = torch.cuda.Event(enable_timing=True)
+        o1 = torch.cuda.Event(enable_timing=True)
+        o0.record(stream)
         dec.run_op_by_op(step, tok, stop, stream)
+        o1.record(stream)
         torch.cuda.synchronize(dev)
-        op_ms = (time.perf_counter() - a) * 1e3 / args.steps
+        op_ms = o0.elapsed_time(o1) / args.steps
         dec.kernel.check_status()
 
-    # end to end through the public API with host buffers: prompt in from pinned
-    # memory, prompt + K generated tokens in one launch, tokens back to the host.
+    # end to end through the public API with host buffers.  Prompt ingestion
+    # (prefill as decode iterations) is one launch, timed on its own: H2D of the
+    # prompt, PROMPT - 1 iterations.  The decode window is the headline: H2D of
+    # tokens / step / step_end from pinned memory, the K generated tokens in one
+    # launch, D2H of the tokens; reported per generated token.
     e2e = None
     if not args.no_e2e:
         host_tok = tokens_cpu.clone().pin_memory()
-        host_step = torch.zeros(1, dtype=torch.int32).pin_memory()
+        host_step0 = torch.zeros(1, dtype=torch.int32).pin_memory()
+        host_pend = torch.full((1,), PROMPT - 1, dtype=torch.int32).pin_memory()
+        host_step = torch.full((1,), PROMPT - 1, dtype=torch.int32).pin_memory()
         host_end = torch.full((1,), PROMPT - 1 + args.steps, dtype=torch.int32).pin_memory()
         out_tok = torch.empty_like(host_tok).pin_memory()
         barrier(pg, dev)
         torch.cuda.synchronize(dev)
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record(stream)
+        tok.copy_(host_tok, non_blocking=True)
+        step.copy_(host_step0, non_blocking=True)
+        stop.copy_(host_pend, non_blocking=True)
+        dec.run(step, tok, stop, stream)
+        ev[1].record(stream)
+        torch.cuda.synchronize(dev)
+        dec.kernel.check_status()
+        barrier(pg, dev)
+        ev[2].record(stream)
         tok.copy_(host_tok, non_blocking=True)
         step.copy_(host_step, non_blocking=True)
         stop.copy_(host_end, non_blocking=True)
         dec.run(step, tok, stop, stream)
         out_tok.copy_(tok, non_blocking=True)
-        f1.record(stream)
+        ev[3].record(stream)
         torch.cuda.synchronize(dev)
         dec.kernel.check_status()
-        e2e_ms = max_over_ranks(pg, f0.elapsed_time(f1), dev)
+        prompt_ms = max_over_ranks(pg, ev[0].elapsed_time(ev[1]), dev)
+        e2e_ms = max_over_ranks(pg, ev[2].elapsed_time(ev[3]), dev)
         assert torch.equal(out_tok[0, PROMPT:PROMPT + args.steps], gen), "e2e tokens differ from the timed run"
         h2d = host_tok.numel() * 8 + 4 + 4
         d2h = out_tok.numel() * 8
         e2e = {"value": whole_job(e2e_ms, args.steps, world)[0], "unit": UNIT,
                "h2d_bytes_per_step": h2d / args.steps, "d2h_bytes_per_step": d2h / args.steps,
-               "includes": f"H2D of tokens/step/step_end, {PROMPT - 1} prompt iterations + {args.steps} decode "
-                           f"iterations in one launch, D2H of tokens"}
+               "includes": f"H2D of tokens/step/step_end, {args.steps} decode iterations in one launch after the "
+                           f"prompt, D2H of tokens",
+               "prompt_ingestion_ms": prompt_ms,
+               "prompt_ingestion": f"H2D of the {PROMPT}-token prompt, {PROMPT - 1} prefill-as-decode iterations "
+                                   f"in one launch"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -483,8 +483,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
             // terms, see batched_geometry).
             int ks = (op.K + MAX_K - 1) / MAX_K;
             while (ks <= op.K / 256 && (op.K % ks != 0 || (op.K / ks) % 256 != 0)) ++ks;
-            if (ks > op.K / 256)
-              return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d cannot be split", li, op.K);
+            if (ks > op.K / 256 || ks > MAX_KSPLIT)
+              return fail(c, MPK_ERR_UNSUPPORTED, "layer %d: reduction length %d cannot be split into at most %d "
+                          "segments", li, op.K, MAX_KSPLIT);
             if (ntasks % ks != 0)
               return fail(c, MPK_ERR_SHAPE,
                           "layer %d: reduction length %d is split into %d segments: grid_dim must give a multiple "

@@ -37,6 +37,7 @@ static_assert(MAX_K == MPK_MAX_GEMV_K, "the header states the input buffer lengt
 constexpr int MAX_NORM_K = 4096;            // longest RMSNorm input (held in registers)
 constexpr int MAX_XS = 1024;                // residual rows of a task preloaded to shared memory
 constexpr int MAX_SEG = 3;
+constexpr int MAX_KSPLIT = 8;               // reduction segments of one split residual projection
 constexpr int MAX_G = 8;                    // query heads per kv head
 constexpr int MAX_D = 128;                  // head dim
 constexpr int MAX_GCHUNK = 8;               // fused op: attention chunks per kv head (tasks 0.. of the group)

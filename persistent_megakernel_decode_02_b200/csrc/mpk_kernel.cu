@@ -209,6 +209,33 @@ __device__ __forceinline__ bool load_tagged(const Graph& g, const uint64_t* p, u
   return ok;
 }
 
+// A batch of tagged words, all loaded before any is looked at (so a prologue
+// costs one memory round trip, not one per load), settled until every word
+// that valid(u) selects carries `tag`.  While one is not current, that word
+// alone is polled until it is, then the whole batch is read again in one
+// round trip.  The batch is reloaded after every wait, so none of it stays
+// live across the waiting call.  addr(u) is the address of word u.  False on
+// abort or timeout.
+template <int N, typename Addr, typename Valid>
+__device__ __forceinline__ bool settle_tagged(const Graph& g, uint64_t (&w)[N], Addr addr, Valid valid, uint32_t tag,
+                                              int op, int worker, int iter) {
+  for (;;) {
+    int bad = -1;
+#pragma unroll
+    for (int u = 0; u < N; ++u)
+      if (valid(u) && word_tag(w[u]) != tag) bad = u;
+    if (bad < 0) return true;
+    const uint64_t x = poll_word(g, addr(bad), tag, op, worker, iter);
+    if (word_tag(x) != tag) {
+#pragma unroll
+      for (int u = 0; u < N; ++u) w[u] = 0ull;
+      return false;
+    }
+#pragma unroll
+    for (int u = 0; u < N; ++u) w[u] = valid(u) ? ld_tagged(addr(u)) : 0ull;
+  }
+}
+
 // ------------------------------------------------------------------ task geometry
 // Rows [row0, row1) of group g that task `task` computes (groups split the
 // tasks evenly; N is the row count of one group).
@@ -753,38 +780,65 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
   }
   if (KIND == TK_GEMV_RESID) {
     // the input (this task's segment of it) into shared memory once every
-    // element carries its writer's tag, the task's residual rows likewise
+    // element carries its writer's tag, the task's residual rows likewise;
+    // all loads are issued before any tag is looked at
+    constexpr int NC = MAX_K / (CONSUMER_THREADS * 4);
+    constexpr int NX = MAX_XS / CONSUMER_THREADS;
+    uint64_t aw[NC * 4], xw[NX];
+    const bool load_a = !reuse;
+    auto a_addr = [&](int u) { return op.a_in + koff + ((u / 4) * CONSUMER_THREADS + ctid) * 4 + (u % 4); };
+    auto a_valid = [&](int u) { return load_a && ((u / 4) * CONSUMER_THREADS + ctid) * 4 < K; };
+    auto x_addr = [&](int q) { return op.x_out + row0 + q * CONSUMER_THREADS + ctid; };
+    auto x_valid = [&](int q) { return xs_ok && q * CONSUMER_THREADS + ctid < nrows; };
 #pragma unroll
-    for (int c = 0; c < MAX_K / (CONSUMER_THREADS * 4); ++c) {
-      const int k = (c * CONSUMER_THREADS + ctid) * 4;
-      if (k < K && !reuse) {
-        float v[4];
-        pfail |= !load_tagged<4>(g, op.a_in + koff + k, atag, v, op.self, worker, (int)iter);
-        *reinterpret_cast<float4*>(hs + hperm(k)) = make_float4(v[0], v[1], v[2], v[3]);
+    for (int c = 0; c < NC; ++c)
+      if (a_valid(4 * c)) {
+        ld_tagged2(a_addr(4 * c), aw[4 * c], aw[4 * c + 1]);
+        ld_tagged2(a_addr(4 * c + 2), aw[4 * c + 2], aw[4 * c + 3]);
       }
+#pragma unroll
+    for (int q = 0; q < NX; ++q)
+      if (x_valid(q)) xw[q] = ld_tagged(x_addr(q));
+    pfail |= !settle_tagged(g, aw, a_addr, a_valid, atag, op.self, worker, (int)iter);
+    pfail |= !settle_tagged(g, xw, x_addr, x_valid, xtag, op.self, worker, (int)iter);
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const int k = (c * CONSUMER_THREADS + ctid) * 4;
+      if (a_valid(4 * c))
+        *reinterpret_cast<float4*>(hs + hperm(k)) = make_float4(word_value(aw[4 * c]), word_value(aw[4 * c + 1]),
+                                                                word_value(aw[4 * c + 2]), word_value(aw[4 * c + 3]));
     }
-    for (int j = ctid; xs_ok && j < nrows; j += CONSUMER_THREADS) {
-      float xv;
-      pfail |= !poll_tagged(g, op.x_out + row0 + j, ld_tagged(op.x_out + row0 + j), xtag, xv, op.self, worker,
-                            (int)iter);
-      sm.u.g.xs[j] = xv;
-    }
+#pragma unroll
+    for (int q = 0; q < NX; ++q)
+      if (x_valid(q)) sm.u.g.xs[q * CONSUMER_THREADS + ctid] = word_value(xw[q]);
   } else if (!reuse) {
     // RMSNorm: x and the norm weight are read once into registers, the
     // statistics are reduced in a fixed order.
     constexpr int NCH = MAX_NORM_K / (CONSUMER_THREADS * 8);
     float xr[NCH][8];
     uint4 wr[NCH];
+    uint64_t xw[NCH * 8];
+    auto x_addr = [&](int u) { return op.x + ((u / 8) * CONSUMER_THREADS + ctid) * 8 + (u % 8); };
+    auto x_valid = [&](int u) { return ((u / 8) * CONSUMER_THREADS + ctid) * 8 < K; };
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
       const int k = (c * CONSUMER_THREADS + ctid) * 8;
       if (k < K) wr[c] = __ldg(reinterpret_cast<const uint4*>(op.norm_w + k));
     }
+    // all of the task's x words issued before any is looked at
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
-      const int k = (c * CONSUMER_THREADS + ctid) * 8;
-      if (k < K) pfail |= !load_tagged<8>(g, op.x + k, xtag, xr[c], op.self, worker, (int)iter);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        if (x_valid(8 * c)) ld_tagged2(x_addr(8 * c + e), xw[8 * c + e], xw[8 * c + e + 1]);
+        else xw[8 * c + e] = xw[8 * c + e + 1] = 0ull;
+      }
     }
+    pfail |= !settle_tagged(g, xw, x_addr, x_valid, xtag, op.self, worker, (int)iter);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) xr[c][e] = word_value(xw[8 * c + e]);
     float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
@@ -915,14 +969,24 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
       bool ffail = false;
       for (int j = ctid; j < nrows; j += CONSUMER_THREADS) {
         const int row = row0 + j;
-        float sum = 0.f, xo = 0.f;
-        for (int k = 0; k < op.ksplit; ++k) {
-          const uint64_t* pk = op.kpart + (size_t)k * op.N + row;
-          float pv;
-          ffail |= !poll_tagged(g, pk, ld_tagged(pk), mytag, pv, op.self, worker, (int)iter);
-          sum = k == 0 ? pv : sum + pv;
-        }
-        ffail |= !poll_tagged(g, op.x_out + row, ld_tagged(op.x_out + row), xtag, xo, op.self, worker, (int)iter);
+        // every partial and the residual loaded before any tag is looked at
+        constexpr int MAXS = MAX_KSPLIT;
+        uint64_t pw[MAXS], xw[1];
+        auto p_addr = [&](int k) { return op.kpart + (size_t)k * op.N + row; };
+        auto p_valid = [&](int k) { return k < op.ksplit; };
+        auto x_addr = [&](int) { return op.x_out + row; };
+        auto x_valid = [](int) { return true; };
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k)
+          if (p_valid(k)) pw[k] = ld_tagged(p_addr(k));
+        xw[0] = ld_tagged(x_addr(0));
+        ffail |= !settle_tagged(g, pw, p_addr, p_valid, mytag, op.self, worker, (int)iter);
+        ffail |= !settle_tagged(g, xw, x_addr, x_valid, xtag, op.self, worker, (int)iter);
+        float sum = 0.f;
+#pragma unroll
+        for (int k = 0; k < MAXS; ++k)
+          if (p_valid(k)) sum = k == 0 ? word_value(pw[k]) : sum + word_value(pw[k]);
+        const float xo = word_value(xw[0]);
         const float nx = xo + sum;
         st_tagged(op.x_out + row, nx, mytag);
         if (capture && op.capture_slot >= 0 && g.cap_hidden != nullptr)
@@ -1296,24 +1360,16 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
     const uint64_t* pg = op.gpart + (size_t)j * nwords;
     bool mfail = false;
     consumer_sync();  // the chunk's own use of the scratch is over
-    for (int base = 0; base < nwords; base += 8 * CONSUMER_THREADS) {
-      uint64_t w[8];
+    constexpr int GW = (MAX_GCHUNK * (MAX_G / 2) * (MAX_D + 2) + CONSUMER_THREADS - 1) / CONSUMER_THREADS;
+    uint64_t w[GW];
+    auto g_addr = [&](int u) { return pg + u * CONSUMER_THREADS + ctid; };
+    auto g_valid = [&](int u) { return u * CONSUMER_THREADS + ctid < nwords; };
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int q = base + u * CONSUMER_THREADS + ctid;
-        w[u] = q < nwords ? ld_tagged(pg + q) : 0ull;
-      }
+    for (int u = 0; u < GW; ++u) w[u] = g_valid(u) ? ld_tagged(g_addr(u)) : 0ull;
+    mfail |= !settle_tagged(g, w, g_addr, g_valid, mytag, op.self, worker, (int)iter);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int q = base + u * CONSUMER_THREADS + ctid;
-        if (q < nwords) {
-          float v;
-          if (word_tag(w[u]) == mytag) v = word_value(w[u]);
-          else mfail |= !poll_tagged(g, pg + q, w[u], mytag, v, op.self, worker, (int)iter);
-          pv[q] = v;
-        }
-      }
-    }
+    for (int u = 0; u < GW; ++u)
+      if (g_valid(u)) pv[u * CONSUMER_THREADS + ctid] = word_value(w[u]);
     if (consumer_sync_or(mfail)) return false;
     for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
       const int hh = idx / D, i = idx % D;

@@ -1,9 +1,10 @@
-"""GEMV tasks with reduction length 4096 split the reduction across the eight
-consumer warps (each warp holds a slice of the input in registers; the
-per-warp partial dot products of a stage's rows are added in warp order).  A
-one-layer model with hidden size 4096 runs every GEMV kind through that path:
-against the oracle, with task splits that leave ragged last stages, against
-op-by-op execution, and against the row-per-warp path (block_dim 128)."""
+"""GEMV tasks with reduction length 4096 (the Qwen3-8B hidden size, the longest
+input the GEMV path keeps in shared memory): every consumer warp takes whole
+weight rows (two at a time, sharing each load of the fp32 input vector) from
+the weight stages.  A one-layer model with hidden size 4096 runs every GEMV
+kind through that path: against the oracle, with task splits that leave
+ragged last stages, against op-by-op execution, and with fewer consumer warps
+per task (block_dim 128)."""
 import pytest
 import torch
 

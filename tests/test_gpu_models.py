@@ -132,3 +132,19 @@ def test_qwen3_8b_batch8(qwen3_8b):
         rk = (rkc[:, r, :, a:a + 2].astype(np.uint32) << 16).view(np.float32)
         assert np.linalg.norm(gk - rk) <= 1e-2 * np.linalg.norm(rk)
     dec.kernel.close()
+
+
+def test_fused_attention_near_its_ceiling():
+    """The fused projections + attention operation at the top of its range
+    (4096 cached positions): an 8B-width, two-layer model over 4090 pre-filled
+    positions, so each kv head's eight chunks hold about 512 positions and the
+    attention loops run many rounds of loads.  Teacher-forced against the
+    oracle at positions 4090 and 4091."""
+    import dataclasses
+    from persistent_megakernel_decode_02_b200.qwen3 import FUSED_ATTENTION_MAX_SEQ
+
+    shape = dataclasses.replace(sq.QWEN3_8B, name="qwen3-8b-width-L2-V8192", layers=2, vocab=8192)
+    w_cpu = sq.make_weights(shape, seed=0)
+    w = to_cuda(w_cpu)
+    S = FUSED_ATTENTION_MAX_SEQ
+    _check(shape, w_cpu, w, S - 6, S, 2, fused_attention=True)
