@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-#define MPK_ABI_VERSION 2
+#define MPK_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MPK_API __attribute__((visibility("default")))
@@ -206,6 +206,20 @@ typedef struct {
                                <= 0 (default): published rows wherever the graph allows.
                                The RMSNorm factor then scales the input instead of the
                                products, so results agree to rounding, not bit for bit. */
+    int32_t prefill_tokens; /* T in 2..MPK_MAX_BATCH: a prefill graph.  Its activations
+                               have T rows, the columns of the tensor-core projections,
+                               and every iteration advances ONE request (tokens [1, S],
+                               step [1], KV cache [L, 1, Hkv, S, d], pred [1, S]) by T
+                               positions: column c consumes tokens[0, step + c], appends
+                               its K/V at step + c and attends to positions 0 .. step + c
+                               (the chunk's earlier positions from this iteration's k and
+                               v, the rest from the cache), so a prompt is ingested T
+                               tokens per iteration instead of one.  Column c's argmax
+                               goes to pred[0, step + c + 1] and to tokens[0, step + c +
+                               1] when that slot holds -1; step advances past the last
+                               active column.  A request's last chunk may be partial
+                               (step_end).  <= 1 (default): one position per request per
+                               iteration.                                                 */
 } mpk_options;
 
 /* Library build facts. */
@@ -275,8 +289,10 @@ MPK_API const char *mpk_warnings(mpk_ctx *ctx);
  * cudaStream_t; NULL = legacy default stream), asynchronously.  step: device
  * int32 [R]; tokens: device int64 [R,S] (R = num_requests, S = seq_length)
  * with -1 in slots to generate; step_end: device int32 [R] or NULL.  R must
- * equal the graph's request count and S-1 must not exceed the KV cache
- * length; an attached pred tensor must be [R,S].  Request r takes
+ * equal the graph's request count (a prefill graph: 1) and S-1 must not
+ * exceed the KV cache length; an attached pred tensor must be [R,S].  A
+ * prefill graph (mpk_options.prefill_tokens = T) advances its request by T
+ * positions per iteration, each position with the semantics below.  Request r takes
  * part in iterations while step[r] < min(step_end[r], S-1) (NULL: S-1); each
  * iteration consumes tokens[r, step[r]], appends K/V at that position and
  * advances step[r] by one ([EN] "How MPK Works": step and tokens are the meta

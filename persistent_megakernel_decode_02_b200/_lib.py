@@ -56,6 +56,7 @@ class Options(ctypes.Structure):
         ("dynamic_tasks", ctypes.c_int32),
         ("debug_stall_op", ctypes.c_int32),
         ("poll_inputs", ctypes.c_int32),
+        ("prefill_tokens", ctypes.c_int32),
     ]
 
 

@@ -76,6 +76,7 @@ struct mpk_ctx {
   Status* status_dev = nullptr;
   int32_t R = 0, S_cache = 0, V = 0, H = 0, L = 0;
   int32_t pred_S = 0;
+  int32_t prefill = 0;  // columns of a prefill graph (0: one position per request per iteration)
   std::string err, warnings;
   std::vector<std::pair<void*, size_t>> zero_each_run;  // tagged activations: versions restart at every run
   int capture_iter = -1;
@@ -400,6 +401,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (o.max_timeline <= 0) o.max_timeline = 1 << 20;
   if (o.prefetch_kb == 0) o.prefetch_kb = -1;
   c->opts = o;
+  // a prefill graph: its R columns are consecutive positions of one request,
+  // whose KV cache holds one request
+  const int PF = o.prefill_tokens > 1 ? o.prefill_tokens : 0;
 
   std::vector<OpDesc> ops(n_layers);
   int R = -1, H = -1, V = -1, L = -1, S = -1;
@@ -604,8 +608,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         SHAPE_CHECK(o->dims[1] == q->dims[1], "layer %d: o %s vs q %s", li, dims_str(o->dims).c_str(),
                     dims_str(q->dims).c_str());
         if (R < 0) R = (int)q->dims[0];
-        SHAPE_CHECK(q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R && kc->dims[1] == R,
-                    "layer %d: request count mismatch (graph %d)", li, R);
+        SHAPE_CHECK(q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R &&
+                        kc->dims[1] == (PF ? 1 : R),
+                    "layer %d: request count mismatch (graph %d%s)", li, R, PF ? ", prefill: one cached request" : "");
         SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range %lld", li, Ly.layer,
                     (long long)kc->dims[0]);
         const int G = Hq / Hkv;
@@ -1085,6 +1090,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (rc != MPK_OK) return rc;
   CUDA_OR_FAIL(c, cudaMemcpy(c->ops_dev, ops.data(), sizeof(OpDesc) * P, cudaMemcpyHostToDevice));
 
+  if (PF && (R != PF || R < 2 || R > MAX_BATCH))
+    return fail(c, MPK_ERR_SHAPE, "prefill_tokens = %d needs activations of that many rows (2..%d); the graph has %d",
+                PF, MAX_BATCH, R);
   Graph& g = c->graph;
   memset(&g, 0, sizeof(g));
   g.ops = c->ops_dev;
@@ -1123,6 +1131,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   c->H = H;
   c->L = g.L;
   c->pred_S = S;
+  c->prefill = PF;
+  g.prefill = PF ? 1 : 0;
   c->ops = ops;
   c->compiled = true;
   return MPK_OK;
@@ -1155,8 +1165,8 @@ static int prepare_run(mpk_ctx* c, int32_t* step, int64_t* tokens, const int32_t
 int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
             const int32_t* step_end, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (c && c->compiled && num_requests != c->R)
-    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->R);
+  if (c && c->compiled && num_requests != (c->prefill ? 1 : c->R))
+    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->prefill ? 1 : c->R);
   int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
   if (rc != MPK_OK) return rc;
   *(volatile int32_t*)c->abort_host = 0;
@@ -1168,20 +1178,24 @@ int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_
 int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
                      const int32_t* step_end, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (c && c->compiled && num_requests != c->R)
-    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->R);
+  const int nreq = c && c->compiled && c->prefill ? 1 : (c ? c->R : 0);
+  if (c && c->compiled && num_requests != nreq)
+    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, nreq);
   int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
   if (rc != MPK_OK) return rc;
   // The host needs the iteration count: read step / step_end.
-  std::vector<int32_t> st(c->R), se(c->R, (int32_t)(seq_len - 1));
-  CUDA_OR_FAIL(c, cudaMemcpyAsync(st.data(), step, sizeof(int32_t) * c->R, cudaMemcpyDeviceToHost, s));
+  std::vector<int32_t> st(nreq), se(nreq, (int32_t)(seq_len - 1));
+  CUDA_OR_FAIL(c, cudaMemcpyAsync(st.data(), step, sizeof(int32_t) * nreq, cudaMemcpyDeviceToHost, s));
   if (step_end)
-    CUDA_OR_FAIL(c, cudaMemcpyAsync(se.data(), step_end, sizeof(int32_t) * c->R, cudaMemcpyDeviceToHost, s));
+    CUDA_OR_FAIL(c, cudaMemcpyAsync(se.data(), step_end, sizeof(int32_t) * nreq, cudaMemcpyDeviceToHost, s));
   CUDA_OR_FAIL(c, cudaStreamSynchronize(s));
   int64_t n_iter = 0;
-  for (int r = 0; r < c->R; ++r) {
+  for (int r = 0; r < nreq; ++r) {
     const int64_t end = std::min<int64_t>(se[r], seq_len - 1);
-    if (st[r] >= 0 && st[r] < end) n_iter = std::max<int64_t>(n_iter, end - st[r]);
+    if (st[r] >= 0 && st[r] < end) {
+      const int64_t left = end - st[r];
+      n_iter = std::max<int64_t>(n_iter, c->prefill ? (left + c->R - 1) / c->R : left);
+    }
   }
   c->graph.op_by_op = 1;
   for (int64_t it = 0; it < n_iter; ++it)

@@ -182,10 +182,11 @@ struct Control {
   uint32_t ready;
   uint32_t n_iter;
   uint32_t pad[30];
-  // per request, read at the start of a run: step[r] and the last position it
-  // may reach, min(step_end[r], S - 1).  While a request is active its step
-  // advances by exactly one per iteration, so in iteration n it is
-  // step0[r] + n.
+  // per column, read at the start of a run: its position in the first
+  // iteration (step[r]; prefill: step[0] + r) and the last position it may
+  // reach, min(step_end, S - 1).  While a column is active its position
+  // advances by a fixed stride per iteration (1; prefill: the column count
+  // R), so in iteration n it is step0[r] + n * stride.
   int32_t step0[MAX_REQUESTS];
   int32_t stop[MAX_REQUESTS];
 };
@@ -196,6 +197,7 @@ struct Graph {
   int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
   int32_t batched;                  // 1: projections run on the tensor-core path (R >= 2)
   int32_t split_attn;               // 1: the graph has split-K attention operations
+  int32_t prefill;                  // 1: the R columns are R consecutive positions of request 0
   int32_t R, S, V, H, L;
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;

@@ -86,6 +86,8 @@ struct __align__(128) Smem {
   float bss[2][4][MAX_BATCH];                    // per block parity, epilogue warp, request: sums of squares
   unsigned long long bbest[4][MAX_BATCH];        // LM head: per epilogue warp and request (value, index) maxima
 };
+static_assert(NSTB < NSTAGES && 2 * MAX_BATCH * MAX_D * 2 <= STAGE_BYTES,
+              "a prefill attention task's k/v rows fit the stage the tensor-core path keeps for its inputs");
 static_assert((NSTAGES - NSTB) * STAGE_BYTES + sizeof(((Smem*)nullptr)->u) >= B_MAX_KBLOCKS * B_KBLOCK_BYTES,
               "the batch input rows fit in the stages the ring leaves free and the scratch after them");
 
@@ -281,19 +283,32 @@ __device__ __forceinline__ bool is_gemv(int kind) {
 // is active.
 __device__ __forceinline__ bool request_at(const Graph& g, int r, uint32_t iter, int& s) {
   const int s0 = __ldcg(&g.ctl->step0[r]);
-  s = s0 + (int)iter;
+  s = s0 + (int)iter * (g.prefill ? g.R : 1);
   return s0 >= 0 && s < __ldcg(&g.ctl->stop[r]);
 }
 
+// Request whose tokens, step, pred and KV cache column r uses (prefill: all
+// columns are positions of request 0).
+__device__ __forceinline__ int col_req(const Graph& g, int r) { return g.prefill ? 0 : r; }
+
 __device__ __forceinline__ bool request_active(const Graph& g, int r, int& s) {
-  s = __ldcg(g.step + r);
+  const int rq = col_req(g, r);
+  const int st = __ldcg(g.step + rq);
+  s = st + (g.prefill ? r : 0);
   int end = g.S - 1;
   if (g.step_end != nullptr) {
-    int e = __ldcg(g.step_end + r);
+    int e = __ldcg(g.step_end + rq);
     end = e < end ? e : end;
   }
-  return s >= 0 && s < end;
+  return st >= 0 && s < end;
 }
+
+// First position of the iteration's chunk of column r's request (column 0's
+// position): prefill columns r' < r hold positions chunk0 .. s - 1.
+__device__ __forceinline__ int chunk0(const Graph& g, int r, int s) { return s - (g.prefill ? r : 0); }
+
+// KV-cache requests of the graph (prefill: one).
+__device__ __forceinline__ int cache_reqs(const Graph& g) { return g.prefill ? 1 : g.R; }
 
 // Position and activity of request r in iteration `iter`: from the run-start
 // state in a persistent run, from `step` itself when every operation is its
@@ -394,26 +409,27 @@ __device__ __forceinline__ bool attn_slot(const Graph& g, const OpDesc& op, int 
   return r < g.R;
 }
 
-// Producer side of a split-K attention task: the cached positions of its
-// chunk, [lo, min(hi, s)), into the ring, PB positions of K then PB of V per
-// stage (1-D bulk copies), once the previous iteration's attention has
-// released the operation (so those positions are in the cache).  The consumer
-// takes exactly these stages.  False on abort or timeout.
 // Ring stages a split-K attention task takes (the producer issues them, the
-// consumer reads them): its chunk's cached positions in blocks of
+// consumer reads them): its chunk's cached positions, those below the
+// iteration's chunk start (s; prefill: column 0's position), in blocks of
 // STAGE_BYTES / (4 d).
 __device__ __forceinline__ uint32_t attn_stages(const Graph& g, const OpDesc& op, int task, uint32_t iter) {
   int r, c, Cr, s;
   if (!attn_slot(g, op, task / op.Hkv, iter, r, c, Cr) || !request_state(g, r, iter, s)) return 0u;
-  const int npos = s + 1;
+  const int npos = s + 1, sc0 = chunk0(g, r, s);
   const int lo = (int)(((long long)c * npos) / Cr);
   int hi = (int)(((long long)(c + 1) * npos) / Cr);
-  hi = hi < s ? hi : s;
+  hi = hi < sc0 ? hi : sc0;
   const int PB = STAGE_BYTES / (4 * op.d);
   return hi > lo ? (uint32_t)((hi - lo + PB - 1) / PB) : 0u;
 }
 
-// Not inlined, so it adds nothing to the producer loop's registers.
+// Producer side of a split-K attention task: the cached positions of its
+// chunk, [lo, min(hi, chunk start)), into the ring, PB positions of K then PB
+// of V per stage (1-D bulk copies), once the previous iteration's attention
+// has released the operation (so those positions are in the cache).  The
+// consumer takes exactly these stages.  False on abort or timeout.  Not
+// inlined, so it adds nothing to the producer loop's registers.
 __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
                                           uint32_t& pstage, int worker, uint64_t pol, int nr) {
   int r, c, Cr;
@@ -421,16 +437,16 @@ __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc
   const int j = task % op.Hkv;
   int s;
   if (!request_state(g, r, iter, s)) return true;
-  const int npos = s + 1;
+  const int npos = s + 1, sc0 = chunk0(g, r, s);
   const int lo = (int)(((long long)c * npos) / Cr);
   int hi = (int)(((long long)(c + 1) * npos) / Cr);
-  hi = hi < s ? hi : s;
+  hi = hi < sc0 ? hi : sc0;
   if (hi <= lo) return true;
   if (iter > 0 && !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 2,
                                 op.self, task, worker, (int)iter))
     return false;
   const int D = op.d, PB = STAGE_BYTES / (4 * D);
-  const size_t kvbase = ((((size_t)op.layer * g.R + r) * op.Hkv + j) * (size_t)op.S) * D;
+  const size_t kvbase = ((((size_t)op.layer * cache_reqs(g) + col_req(g, r)) * op.Hkv + j) * (size_t)op.S) * D;
   for (int p = lo; p < hi; p += PB) {
     const int n = min(PB, hi - p);
     const uint32_t slot = pstage % (uint32_t)nr;
@@ -693,22 +709,32 @@ __device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDes
                                            int mode, int cw, int lane, uint32_t iter, int worker);
 
 
-// The LM head's last task to arrive (sm.last) turns every active request's
+// The LM head's last task to arrive (sm.last) turns every active column's
 // maximum key into its next token: written to tokens[r, s+1] if that slot
-// holds -1, always to pred; step[r] advances; the keys are reset.
+// holds -1, always to pred; the request's step advances; the keys are reset.
+// A prefill graph's columns are positions of request 0: each column writes
+// its own prediction, the last active one advances step[0] (every column
+// reads the shared step before it changes).
 __device__ __forceinline__ void argmax_tokens(Smem& sm, const Graph& g, const OpDesc& op, uint32_t iter, int ctid) {
   if (!sm.last) return;
   __threadfence();
+  int s = 0, sn = 0;
+  bool act = false, next = false;
+  unsigned long long key = 0ull;
   if (ctid < g.R) {
-    const int rq = ctid;
-    int s;
-    if (request_state(g, rq, iter, s)) {
-      const unsigned long long key = atomicAdd(op.keys + rq, 0ull);
+    act = request_state(g, ctid, iter, s);
+    next = ctid + 1 < g.R && request_state(g, ctid + 1, iter, sn);
+    if (act) key = atomicAdd(op.keys + ctid, 0ull);
+  }
+  if (g.prefill) consumer_sync();
+  if (ctid < g.R) {
+    const int rq = ctid, row = col_req(g, rq);
+    if (act) {
       const int64_t nxt = (int64_t)argmax_key_index(key);
-      int64_t* trow = g.tokens + (size_t)rq * g.S;
+      int64_t* trow = g.tokens + (size_t)row * g.S;
       if (__ldcg(trow + s + 1) == -1) trow[s + 1] = nxt;
-      if (op.pred != nullptr) op.pred[(size_t)rq * g.S + s + 1] = nxt;
-      g.step[rq] = s + 1;
+      if (op.pred != nullptr) op.pred[(size_t)row * g.S + s + 1] = nxt;
+      if (!g.prefill || !next) g.step[row] = s + 1;
     }
     op.keys[rq] = 0ull;
   }
@@ -1077,7 +1103,15 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   const int ctid = cw * 32 + lane;
   const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
-  const size_t kvbase = ((((size_t)op.layer * g.R + r) * Hkv + j) * (size_t)op.S) * D;
+  const size_t kvbase = ((((size_t)op.layer * cache_reqs(g) + col_req(g, r)) * Hkv + j) * (size_t)op.S) * D;
+  // k and v (bf16, k normalised and rotated) of the positions the iteration
+  // itself produces: row 0 the task's own position (A.ks, A.vs); prefill: row
+  // c the position of column c of the chunk, in the ring stage that the
+  // tensor-core path keeps for its input rows (free while an attention task
+  // runs: every MMA of the previous projection task has completed)
+  const int own = g.prefill ? r : 0;
+  uint16_t* const KX = g.prefill ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) : A.ks;
+  uint16_t* const VX = g.prefill ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_BATCH * MAX_D : A.vs;
   const int CS = op.C;  // split op: chunk partials per (request, query head)
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * CS) * (D + 2);
   // Prologue rows: warp cw < G takes query head cw of the group, warp G the
@@ -1155,10 +1189,50 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       for (int e = 0; e < EL; ++e) {
         const int i = lane + 32 * e;
         if (prow < G) A.qs[prow * D + i] = x[e] * (LOG2E / sqrtf((float)D));
-        else if (prow == G) A.ks[i] = f32_to_bf16_rn(x[e]);
-        else A.vs[i] = f32_to_bf16_rn(x[e]);
+        else if (prow == G) KX[own * D + i] = f32_to_bf16_rn(x[e]);
+        else VX[own * D + i] = f32_to_bf16_rn(x[e]);
       }
     }
+    if (STREAMED && g.prefill) {
+      // the chunk's earlier positions this task attends to (columns below
+      // r, produced in this iteration and not read from the cache): their k
+      // (normalised, rotated at its own position) and v, one row per warp
+      const int sc0 = chunk0(g, r, s), a0 = lo > sc0 ? lo : sc0, b0 = hi < s ? hi : s;
+      for (int row = cw; row < 2 * (b0 - a0); row += CONSUMER_WARPS) {
+        const int pos = a0 + row / 2, rp = pos - sc0;
+        const bool isk = (row & 1) == 0;
+        const uint64_t* rs = (isk ? op.k : op.v) + (size_t)rp * Hkv * D + (size_t)j * D;
+        float y[EL];
+#pragma unroll
+        for (int e = 0; e < EL; ++e) {
+          const uint64_t w = ld_tagged(rs + lane + 32 * e);
+          if (word_tag(w) == intag) y[e] = word_value(w);
+          else afail |= !poll_tagged(g, rs + lane + 32 * e, w, intag, y[e], op.self, worker, (int)iter);
+        }
+        if (isk) {
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < EL; ++e) ss = fmaf(y[e], y[e], ss);
+          ss = warp_sum(ss);
+          const float rinv = 1.0f / sqrtf(ss / (float)D + op.eps);
+#pragma unroll
+          for (int e = 0; e < EL; ++e)
+            y[e] = y[e] * rinv * __uint_as_float((uint32_t)__ldg(op.kn_w + lane + 32 * e) << 16);
+          const float2* cs = op.rope + (size_t)pos * (D / 2);
+#pragma unroll
+          for (int e = 0; e < EL / 2; ++e) {
+            const float2 t = __ldg(cs + lane + 32 * e);
+            const float a = y[e], b = y[e + EL / 2];
+            y[e] = a * t.x - b * t.y;
+            y[e + EL / 2] = b * t.x + a * t.y;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < EL; ++e) (isk ? KX : VX)[rp * D + lane + 32 * e] = f32_to_bf16_rn(y[e]);
+      }
+    }
+    // the rows sit in memory the tensor cores' bulk copies rewrite later
+    if (g.prefill) fence_proxy_async_smem();
     if (consumer_sync_or(afail)) return false;
     // the cache append at s: by the chunk holding s, or in group mode by the
     // merging task (chunk 0), whose release after the merge covers it
@@ -1167,7 +1241,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
       uint16_t* dst = (which == 0 ? op.kc : op.vc) + kvbase + (size_t)s * D + q8 * 8;
-      const uint16_t* srcs = (which == 0 ? A.ks : A.vs) + q8 * 8;
+      const uint16_t* srcs = (which == 0 ? KX : VX) + own * D + q8 * 8;
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(srcs);
     }
 
@@ -1219,7 +1293,8 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       // this chunk, comes from shared memory.
       constexpr int PB = STAGE_BYTES / (4 * D);
       const int nr = g.batched ? NSTB : NSTAGES;
-      const int chi = hi < s ? hi : s;
+      const int sc0 = chunk0(g, r, s);
+      const int chi = hi < sc0 ? hi : sc0;  // cached positions, streamed
       bool sfail = false;
       for (int p0 = lo; p0 < chi; p0 += PB) {
         const int n = min(PB, chi - p0);
@@ -1259,10 +1334,16 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
         cstage = cs + 1u;
       }
       if (sfail) return false;
-      if (hi == npos && cw == 0) {
-        const uint4 kvs = grp == 0 ? *reinterpret_cast<const uint4*>(A.ks + sub * 8) : make_uint4(0, 0, 0, 0);
-        const uint4 vvs = grp == 0 ? *reinterpret_cast<const uint4*>(A.vs + sub * 8) : make_uint4(0, 0, 0, 0);
-        consume(kvs, vvs, grp == 0);
+      // the positions this iteration produced (s, and prefill: the chunk's
+      // earlier columns), from their rows in shared memory, PPW per warp
+      const int a0 = lo > sc0 ? lo : sc0, nin = hi - a0;
+      if (cw * PPW < nin) {
+        const int t = cw * PPW + grp;
+        const bool valid = t < nin;
+        const int rw = valid ? a0 - sc0 + t : 0;
+        const uint4 kvs = valid ? *reinterpret_cast<const uint4*>(KX + rw * D + sub * 8) : make_uint4(0, 0, 0, 0);
+        const uint4 vvs = valid ? *reinterpret_cast<const uint4*>(VX + rw * D + sub * 8) : make_uint4(0, 0, 0, 0);
+        consume(kvs, vvs, valid);
       }
     } else {
       const uint16_t* kg = op.kc + kvbase + sub * 8;
@@ -1474,7 +1555,7 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
     return true;
   }
   if (r < g.R) {
-    const int64_t tok = __ldcg(g.tokens + (size_t)r * g.S + s);
+    const int64_t tok = __ldcg(g.tokens + (size_t)col_req(g, r) * g.S + s);
     if (tok < 0 || tok >= g.V) {
       if (ctid == 0) record_error(g, -11 /*DEVICE*/, 8, -1, task, -1, (int)iter, (uint32_t)tok, (uint32_t)g.V);
       return true;
@@ -1830,13 +1911,17 @@ __device__ __forceinline__ void persistent_body(const Graph& g) {
   if ((int)blockIdx.x < g.sched_ctas) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       // iterations of this run: the furthest any request still has to go
+      // (prefill: request 0's remaining positions, R per iteration)
       uint32_t n_iter = 0;
       for (int r = 0; r < g.R; ++r) {
         int s;
         const bool act = request_active(g, r, s);
         int end = g.S - 1;
-        if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + r));
-        if (act) n_iter = max(n_iter, (uint32_t)(end - s));
+        if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + col_req(g, r)));
+        if (act) {
+          const uint32_t left = (uint32_t)(end - s);
+          n_iter = max(n_iter, g.prefill ? (left + (uint32_t)g.R - 1u) / (uint32_t)g.R : left);
+        }
         g.ctl->step0[r] = act ? s : -1;
         g.ctl->stop[r] = end;
       }

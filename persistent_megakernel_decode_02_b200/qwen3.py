@@ -192,15 +192,26 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
                   debug_stall_op: int = 0, dynamic_tasks: bool = False, tasks_per_worker: int = 2,
-                  poll_inputs: bool = False) -> Decoder:
+                  poll_inputs: bool = False, prefill_tokens: int = 0) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
     projection+attention operation for one request with up to
-    FUSED_ATTENTION_MAX_SEQ positions, split-K attention otherwise."""
+    FUSED_ATTENTION_MAX_SEQ positions, split-K attention otherwise.
+
+    prefill_tokens = T in 2..8 builds a prefill graph for one request
+    (requests = 1): every iteration ingests T consecutive prompt positions as
+    the T columns of the tensor-core projections (mpk_options.prefill_tokens).
+    Pass the decode graph's caches as k_cache / v_cache to continue decoding
+    from the prefilled state."""
     from . import _lib
 
     s = shape
+    cols = requests
+    if prefill_tokens > 1:
+        if requests != 1:
+            raise ValueError("a prefill graph serves one request")
+        cols = prefill_tokens
     if num_workers is None:
         num_workers = _lib.load().mpk_device_sm_count() - num_local_schedulers // 4
     mk = PersistentKernel(num_workers, num_local_schedulers, 0)
@@ -217,21 +228,22 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     pred = torch.full((requests, max_seq), -1, dtype=torch.int64, device=dev)
     mk.attach_input(pred, "pred")
     bufs = {
-        "x": mk.new_tensor((requests, s.hidden), FP32_TAGGED, "x"),
-        "q": mk.new_tensor((requests, s.q_dim), FP32_TAGGED, "q"),
-        "k": mk.new_tensor((requests, s.kv_dim), FP32_TAGGED, "k"),
-        "v": mk.new_tensor((requests, s.kv_dim), FP32_TAGGED, "v"),
-        "o": mk.new_tensor((requests, s.q_dim), FP32_TAGGED, "o"),
-        "a": mk.new_tensor((requests, s.intermediate), FP32_TAGGED, "a"),
+        "x": mk.new_tensor((cols, s.hidden), FP32_TAGGED, "x"),
+        "q": mk.new_tensor((cols, s.q_dim), FP32_TAGGED, "q"),
+        "k": mk.new_tensor((cols, s.kv_dim), FP32_TAGGED, "k"),
+        "v": mk.new_tensor((cols, s.kv_dim), FP32_TAGGED, "v"),
+        "o": mk.new_tensor((cols, s.q_dim), FP32_TAGGED, "o"),
+        "a": mk.new_tensor((cols, s.intermediate), FP32_TAGGED, "a"),
     }
     if attn_chunks is None:
-        attn_chunks = default_attn_chunks(s, requests, num_workers, max_seq)
+        attn_chunks = default_attn_chunks(s, cols, num_workers, max_seq)
     if fused_attention is None:
-        fused_attention = requests == 1 and max_seq <= FUSED_ATTENTION_MAX_SEQ
-    for op in layer_plan(s, requests, num_workers, attn_chunks, gemv_tasks, block_dim,
+        fused_attention = cols == 1 and max_seq <= FUSED_ATTENTION_MAX_SEQ
+    for op in layer_plan(s, cols, num_workers, attn_chunks, gemv_tasks, block_dim,
                          fused_attention=fused_attention, tasks_per_worker=tasks_per_worker if dynamic_tasks else 1):
         op = dict(op)
         getattr(mk, op.pop("method"))(**op)
     mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb,
-               debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks, poll_inputs=poll_inputs)
+               debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks, poll_inputs=poll_inputs,
+               prefill_tokens=prefill_tokens if prefill_tokens > 1 else 0)
     return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)

@@ -148,3 +148,50 @@ def test_fused_attention_near_its_ceiling():
     w = to_cuda(w_cpu)
     S = FUSED_ATTENTION_MAX_SEQ
     _check(shape, w_cpu, w, S - 6, S, 2, fused_attention=True)
+
+
+def _check_prefill(shape, w_cpu, w, P, T):
+    """One prefill iteration of T columns (positions P..P+T-1) over a seeded
+    pre-filled cache, per column against the oracle's per-position values."""
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    from tests.gpu_util import HIDDEN_TOL, LOGITS_TOL, rel_l2
+
+    S = P + T + 1
+    kc, vc = sq.make_kv_prefill(shape, 1, S, P, seed=41)
+    tokens = sq.make_tokens(shape, 1, S, [S], seed=42, teacher_forced=True)
+    pre = build_decoder(shape, w, requests=1, max_seq=S, prefill_tokens=T, k_cache=kc.cuda(), v_cache=vc.cuda())
+    lg = torch.full((T, shape.vocab), float("nan"), device="cuda")
+    hd = torch.full((shape.layers + 1, T, shape.hidden), float("nan"), device="cuda")
+    pre.kernel.set_capture(0, lg, hd)
+    step = torch.full((1,), P, dtype=torch.int32, device="cuda")
+    pre.run(step, tokens.cuda(), torch.full((1,), P + T, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    pre.kernel.check_status()
+    assert int(step.item()) == P + T
+    ref, _, rkc, _ = oracle_teacher_forced(shape, w_cpu, tokens, T, _u16(kc), _u16(vc), step0=P)
+    gl, gh = lg.double().cpu().numpy(), hd.double().cpu().numpy()
+    wl = wh = 0.0
+    for c in range(T):
+        rl, rh = ref[c]
+        e = rel_l2(gl[c], rl[0])
+        wl = max(wl, e)
+        assert e <= LOGITS_TOL, (c, e)
+        for layer in range(shape.layers + 1):
+            e = rel_l2(gh[layer, c], rh[layer, 0])
+            wh = max(wh, e)
+            assert e <= HIDDEN_TOL, (c, layer, e)
+    gk = pre.k_cache[:, :, :, P:P + T].float().cpu().numpy()
+    rk = (rkc[:, :, :, P:P + T].astype(np.uint32) << 16).view(np.float32)
+    assert np.linalg.norm(gk - rk) <= 1e-2 * np.linalg.norm(rk)
+    print(f"{shape.name} prefill T={T} at {P}: worst logits rel-L2 {wl:.2e}, hidden {wh:.2e}")
+    pre.kernel.close()
+
+
+def test_qwen3_0_6b_prefill(qwen3_0_6b):
+    w_cpu, w = qwen3_0_6b
+    _check_prefill(sq.QWEN3_0_6B, w_cpu, w, 31, 8)
+
+
+def test_qwen3_8b_prefill(qwen3_8b):
+    w_cpu, w = qwen3_8b
+    _check_prefill(sq.QWEN3_8B, w_cpu, w, 24, 8)
