@@ -394,11 +394,15 @@ def main_batch(args):
     dec = build_decoder(shape, w, requests=R, max_seq=S, num_workers=W, num_local_schedulers=ls,
                         attn_chunks=args.attn_chunks or None, sched_lookahead=args.lookahead,
                         profiling=args.profiling)
+    # the prompts' graph: PREFILL_TOKENS positions of one request per
+    # iteration, the requests one after another, on the decode graph's cache
+    pre = build_decoder(shape, w, requests=R, max_seq=S, num_workers=W, num_local_schedulers=ls,
+                        prefill_tokens=PREFILL_TOKENS, k_cache=dec.k_cache, v_cache=dec.v_cache)
     stream = torch.cuda.current_stream(dev)
     tok = tokens_cpu.to(dev)
     p_end = (lens - 1).to(torch.int32).to(dev)          # each request has consumed its prompt
     step = torch.zeros(R, dtype=torch.int32, device=dev)
-    dec.run(step, tok, p_end)                            # phase A: prompts (prefill-as-decode)
+    pre.run(step, tok, p_end)                            # phase A: the prompts
     dec.run(step, tok, p_end + args.warmup)              # warm-up iterations
     torch.cuda.synchronize(dev)
     dec.kernel.check_status()
@@ -454,8 +458,9 @@ def main_batch(args):
         op_ms = o0.elapsed_time(o1) / steps
 
     # end to end through the public API with host buffers: the prompts are
-    # ingested in one launch (timed on its own); the decode window is H2D of
-    # tokens / step / step_end from pinned memory, the timed lock-step
+    # ingested in one launch (timed on its own, through the prefill graph and
+    # for comparison as lock-step decode iterations); the decode window is H2D
+    # of tokens / step / step_end from pinned memory, the timed lock-step
     # iterations in one launch and D2H of the tokens, reported per step.
     e2e = None
     if not args.no_e2e:
@@ -466,27 +471,30 @@ def main_batch(args):
         out_tok = torch.empty_like(host_tok).pin_memory()
         barrier(pg, dev)
         torch.cuda.synchronize(dev)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        ev[0].record(stream)
-        tok.copy_(host_tok, non_blocking=True)
-        step.copy_(host_step0, non_blocking=True)
-        stop.copy_(host_pend, non_blocking=True)
-        dec.run(step, tok, stop, stream)
-        ev[1].record(stream)
-        torch.cuda.synchronize(dev)
-        dec.kernel.check_status()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        # ev[0..1]: prefill graph, ev[2..3]: lock-step decode (run first), ev[4..5]: decode window
+        for graph, (a, b) in ((dec, (2, 3)), (pre, (0, 1))):
+            ev[a].record(stream)
+            tok.copy_(host_tok, non_blocking=True)
+            step.copy_(host_step0, non_blocking=True)
+            stop.copy_(host_pend, non_blocking=True)
+            graph.run(step, tok, stop, stream)
+            ev[b].record(stream)
+            torch.cuda.synchronize(dev)
+            graph.kernel.check_status()
         barrier(pg, dev)
-        ev[2].record(stream)
+        ev[4].record(stream)
         tok.copy_(host_tok, non_blocking=True)
         step.copy_(host_pend, non_blocking=True)
         stop.copy_(host_end, non_blocking=True)
         dec.run(step, tok, stop, stream)
         out_tok.copy_(tok, non_blocking=True)
-        ev[3].record(stream)
+        ev[5].record(stream)
         torch.cuda.synchronize(dev)
         dec.kernel.check_status()
         prompt_ms = max_over_ranks(pg, ev[0].elapsed_time(ev[1]), dev)
-        e2e_ms = max_over_ranks(pg, ev[2].elapsed_time(ev[3]), dev)
+        prompt_decode_ms = max_over_ranks(pg, ev[2].elapsed_time(ev[3]), dev)
+        e2e_ms = max_over_ranks(pg, ev[4].elapsed_time(ev[5]), dev)
         for r in range(R):
             assert torch.equal(out_tok[r, int(lens[r]):int(lens[r]) + steps], gen[r]), "e2e tokens differ"
         e2e = {"value": e2e_ms / steps, "unit": UNIT_BATCH,
@@ -495,8 +503,10 @@ def main_batch(args):
                "includes": f"H2D of tokens/step/step_end, {steps} lock-step decode iterations in one launch after "
                            f"the prompts, D2H of tokens",
                "prompt_ingestion_ms": prompt_ms,
-               "prompt_ingestion": "H2D of the prompts, each request's prompt as prefill-as-decode iterations in "
-                                   "one launch (longest prompt 512)"}
+               "prompt_ingestion": f"H2D of the prompts, their {int((lens - 1).sum())} positions through the "
+                                   f"prefill graph ({PREFILL_TOKENS} positions of one request per iteration on the "
+                                   f"tensor cores, the requests one after another) in one launch",
+               "prompt_ingestion_ms_lock_step_decode": prompt_decode_ms}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -536,6 +546,7 @@ def main_batch(args):
             "setup_s": {"weights": round(t_gen, 1)},
         }
         print(json.dumps(line), flush=True)
+    pre.kernel.close()
     dec.kernel.close()
     if pg is not None:
         pg.destroy_process_group()

@@ -77,6 +77,7 @@ struct mpk_ctx {
   int32_t R = 0, S_cache = 0, V = 0, H = 0, L = 0;
   int32_t pred_S = 0;
   int32_t prefill = 0;  // columns of a prefill graph (0: one position per request per iteration)
+  int32_t Rq = 0;       // requests of tokens, step, pred and the KV cache (without prefill: R)
   std::string err, warnings;
   std::vector<std::pair<void*, size_t>> zero_each_run;  // tagged activations: versions restart at every run
   int capture_iter = -1;
@@ -202,9 +203,11 @@ int batched_geometry(mpk_ctx* c, int li, OpDesc& o, int R, const mpk_layer& Ly) 
   return MPK_OK;
 }
 
-// Tensor map of a bf16 [rows, K] row-major matrix for BM x BK tiles with
-// 128-byte swizzle (the layout the MMA's shared-memory descriptors describe).
-int make_weight_map(mpk_ctx* c, int li, CUtensorMap* m, const void* ptr, int64_t rows, int64_t K) {
+// Tensor map of a bf16 [rows, K] row-major matrix for box_rows x BK tiles
+// with 128-byte swizzle (the layout the MMA's shared-memory descriptors and the
+// attention's matrix loads expect).
+int make_weight_map(mpk_ctx* c, int li, CUtensorMap* m, const void* ptr, int64_t rows, int64_t K,
+                    int box_rows = BM) {
   static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
   if (!encode) {
     void* fn = nullptr;
@@ -216,7 +219,7 @@ int make_weight_map(mpk_ctx* c, int li, CUtensorMap* m, const void* ptr, int64_t
   }
   const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -401,12 +404,13 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (o.max_timeline <= 0) o.max_timeline = 1 << 20;
   if (o.prefetch_kb == 0) o.prefetch_kb = -1;
   c->opts = o;
-  // a prefill graph: its R columns are consecutive positions of one request,
-  // whose KV cache holds one request
+  // a prefill graph: its R columns are consecutive positions of one request
+  // of the KV cache, which may hold any number of requests (Rq)
   const int PF = o.prefill_tokens > 1 ? o.prefill_tokens : 0;
+  int Rq = -1;
 
   std::vector<OpDesc> ops(n_layers);
-  int R = -1, H = -1, V = -1, L = -1, S = -1;
+  int R = -1, H = -1, V = -1, L = -1, S = -1, pred_rows = -1;
   // attention workspace sizing
   size_t part_floats = 0, merge_u32 = 0, kpart_floats = 0, blk_u32 = 0, gpart_words = 0;
   std::vector<std::pair<int, size_t>> merge_off(n_layers, {0, 0});
@@ -534,6 +538,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
               NEED("outputs[0] (pred)", Ly.outputs[0], MPK_INT64, 2, &out);
               op.pred = (int64_t*)out->ptr;
               if (S < 0) S = (int)out->dims[1];
+              pred_rows = (int)out->dims[0];
             }
             if (V < 0) V = op.N;
             SHAPE_CHECK(op.N == V, "layer %d: LM head rows %d != vocabulary %d", li, op.N, V);
@@ -608,9 +613,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         SHAPE_CHECK(o->dims[1] == q->dims[1], "layer %d: o %s vs q %s", li, dims_str(o->dims).c_str(),
                     dims_str(q->dims).c_str());
         if (R < 0) R = (int)q->dims[0];
+        if (Rq < 0) Rq = (int)kc->dims[1];
         SHAPE_CHECK(q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R &&
-                        kc->dims[1] == (PF ? 1 : R),
-                    "layer %d: request count mismatch (graph %d%s)", li, R, PF ? ", prefill: one cached request" : "");
+                        kc->dims[1] == (PF ? Rq : R),
+                    "layer %d: request count mismatch (graph %d, cache %lld)", li, R, (long long)kc->dims[1]);
         SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range %lld", li, Ly.layer,
                     (long long)kc->dims[0]);
         const int G = Hq / Hkv;
@@ -676,6 +682,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
                     dims_str(wk->dims).c_str(), dims_str(wv->dims).c_str(), op.K, Hkv, d);
         SHAPE_CHECK(qn->dims[0] == d && kn->dims[0] == d, "layer %d: norm weights must have head_dim %d", li, d);
         if (R < 0) R = (int)x->dims[0];
+        if (Rq < 0) Rq = (int)kc->dims[1];
         SHAPE_CHECK(x->dims[0] == R && q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R &&
                         kc->dims[1] == R,
                     "layer %d: request count mismatch (graph %d)", li, R);
@@ -930,11 +937,26 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     rc = alloc(c, &bpart, sizeof(float) * bpart_floats);
     if (rc != MPK_OK) return rc;
   }
-  // tensor maps of the batched projections' weights (64-byte aligned device copies)
+  // tensor maps of the batched projections' weights and of the caches the
+  // split-K attention streams (64-byte aligned device copies)
   std::vector<CUtensorMap> tmaps;
-  std::vector<std::pair<int, int>> tmap_of;  // (op, slot): slot MAX_SEG = the up matrix
+  std::vector<std::pair<int, int>> tmap_of;  // (op, slot): slot MAX_SEG = the up matrix, -1 / -2: k / v cache
   for (int p = 0; p < P; ++p) {
     const OpDesc& op = ops[p];
+    if (op.kind == TK_ATTN) {
+      const int64_t rows = (int64_t)op.L * Rq * op.Hkv * op.S;
+      if (rows >= ((int64_t)1 << 31))
+        return fail(c, MPK_ERR_UNSUPPORTED, "op %d: a KV cache of %lld rows of d (at most 2^31 - 1)", p,
+                    (long long)rows);
+      for (int w = 0; w < 2; ++w) {
+        CUtensorMap m;
+        rc = make_weight_map(c, p, &m, w == 0 ? op.kc : op.vc, rows, op.d, STAGE_BYTES / (4 * op.d));
+        if (rc != MPK_OK) return rc;
+        tmaps.push_back(m);
+        tmap_of.push_back({p, -1 - w});
+      }
+      continue;
+    }
     if (!op.batched) continue;
     for (int sg = 0; sg <= MAX_SEG; ++sg) {
       const void* w = sg < MAX_SEG ? (sg < op.nseg ? op.W[sg] : nullptr)
@@ -955,7 +977,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     CUDA_OR_FAIL(c, cudaMemcpy(tm_dev, tmaps.data(), sizeof(CUtensorMap) * tmaps.size(), cudaMemcpyHostToDevice));
     for (size_t i = 0; i < tmap_of.size(); ++i) {
       OpDesc& op = ops[tmap_of[i].first];
-      if (tmap_of[i].second < MAX_SEG) op.tmap[tmap_of[i].second] = tm_dev + i;
+      const int slot = tmap_of[i].second;
+      if (slot == -1) op.tmap_kc = tm_dev + i;
+      else if (slot == -2) op.tmap_vc = tm_dev + i;
+      else if (slot < MAX_SEG) op.tmap[slot] = tm_dev + i;
       else op.tmap_up = tm_dev + i;
     }
   }
@@ -1093,6 +1118,11 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (PF && (R != PF || R < 2 || R > MAX_BATCH))
     return fail(c, MPK_ERR_SHAPE, "prefill_tokens = %d needs activations of that many rows (2..%d); the graph has %d",
                 PF, MAX_BATCH, R);
+  if (!PF || Rq < 1) Rq = R;
+  if (Rq > MAX_REQUESTS)
+    return fail(c, MPK_ERR_UNSUPPORTED, "%d cached requests (at most %d)", Rq, MAX_REQUESTS);
+  if (pred_rows >= 0 && pred_rows != Rq)
+    return fail(c, MPK_ERR_SHAPE, "pred has %d rows, the graph serves %d requests", pred_rows, Rq);
   Graph& g = c->graph;
   memset(&g, 0, sizeof(g));
   g.ops = c->ops_dev;
@@ -1132,7 +1162,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   c->L = g.L;
   c->pred_S = S;
   c->prefill = PF;
+  c->Rq = Rq;
   g.prefill = PF ? 1 : 0;
+  g.Rq = Rq;
   c->ops = ops;
   c->compiled = true;
   return MPK_OK;
@@ -1165,8 +1197,8 @@ static int prepare_run(mpk_ctx* c, int32_t* step, int64_t* tokens, const int32_t
 int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
             const int32_t* step_end, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (c && c->compiled && num_requests != (c->prefill ? 1 : c->R))
-    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->prefill ? 1 : c->R);
+  if (c && c->compiled && num_requests != c->Rq)
+    return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, c->Rq);
   int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
   if (rc != MPK_OK) return rc;
   *(volatile int32_t*)c->abort_host = 0;
@@ -1178,7 +1210,7 @@ int mpk_run(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_
 int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_requests, int64_t seq_len,
                      const int32_t* step_end, void* stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int nreq = c && c->compiled && c->prefill ? 1 : (c ? c->R : 0);
+  const int nreq = c && c->compiled ? c->Rq : 0;
   if (c && c->compiled && num_requests != nreq)
     return fail(c, MPK_ERR_SHAPE, "tokens has %d requests, the graph %d", num_requests, nreq);
   int rc = prepare_run(c, step, tokens, step_end, seq_len, s);
@@ -1194,7 +1226,8 @@ int mpk_run_op_by_op(mpk_ctx* c, int32_t* step, int64_t* tokens, int num_request
     const int64_t end = std::min<int64_t>(se[r], seq_len - 1);
     if (st[r] >= 0 && st[r] < end) {
       const int64_t left = end - st[r];
-      n_iter = std::max<int64_t>(n_iter, c->prefill ? (left + c->R - 1) / c->R : left);
+      // prefill: the requests one after another, R positions per iteration
+      n_iter = c->prefill ? n_iter + (left + c->R - 1) / c->R : std::max<int64_t>(n_iter, left);
     }
   }
   c->graph.op_by_op = 1;

@@ -113,6 +113,10 @@ struct OpDesc {
   const uint16_t* kn_w;
   uint16_t* kc;
   uint16_t* vc;
+  // split-K operation: tensor maps of the caches viewed as [L*R*Hkv*S rows, d]
+  // bf16, boxes of 64 elements x (STAGE_BYTES / (4 d)) rows, 128-byte swizzle
+  const void* tmap_kc;
+  const void* tmap_vc;
   float* part;                  // [R][Hq][C][d + 2]
   uint64_t* gpart;              // group mode: tagged chunk partials [Hkv][C][G][d + 2]
   int32_t group_sync;           // fused op: every task of a group attends to a chunk (tasks <= workers)
@@ -182,13 +186,15 @@ struct Control {
   uint32_t ready;
   uint32_t n_iter;
   uint32_t pad[30];
-  // per column, read at the start of a run: its position in the first
-  // iteration (step[r]; prefill: step[0] + r) and the last position it may
-  // reach, min(step_end, S - 1).  While a column is active its position
-  // advances by a fixed stride per iteration (1; prefill: the column count
-  // R), so in iteration n it is step0[r] + n * stride.
+  // per request, read at the start of a run: step[r] (-1: inactive) and the
+  // last position it may reach, min(step_end[r], S - 1).  While a request is
+  // active its step advances by exactly one per iteration, so in iteration n
+  // it is step0[r] + n.  A prefill graph serves its requests one after
+  // another, R positions per iteration; cum[q] is the number of iterations
+  // before request q's first (cum[Rq]: all of the run's).
   int32_t step0[MAX_REQUESTS];
   int32_t stop[MAX_REQUESTS];
+  uint32_t cum[MAX_REQUESTS + 1];
 };
 
 struct Graph {
@@ -197,7 +203,8 @@ struct Graph {
   int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
   int32_t batched;                  // 1: projections run on the tensor-core path (R >= 2)
   int32_t split_attn;               // 1: the graph has split-K attention operations
-  int32_t prefill;                  // 1: the R columns are R consecutive positions of request 0
+  int32_t prefill;                  // 1: the R columns are R consecutive positions of one request
+  int32_t Rq;                       // requests of tokens, step, pred and the KV cache (without prefill: R)
   int32_t R, S, V, H, L;
   int32_t num_workers, num_sched;   // scheduler warps
   int32_t sched_ctas;

@@ -278,44 +278,73 @@ __device__ __forceinline__ bool is_gemv(int kind) {
          kind == TK_NORM_GEMV_ARGMAX || kind == TK_QKV_ATTN;
 }
 
-// Position of request r in iteration `iter` of a persistent run (from the
-// run-start state, so nothing written during the run is read), and whether it
-// is active.
-__device__ __forceinline__ bool request_at(const Graph& g, int r, uint32_t iter, int& s) {
-  const int s0 = __ldcg(&g.ctl->step0[r]);
-  s = s0 + (int)iter * (g.prefill ? g.R : 1);
-  return s0 >= 0 && s < __ldcg(&g.ctl->stop[r]);
+// The position and request of column r in iteration `iter`, and whether it is
+// active.  Without prefill column r is request r, one position per
+// iteration.  A prefill graph ingests its requests one after another: the
+// iteration's request q is the one whose share of the run's iterations
+// (ceil(remaining positions / R) each, in request order) holds `iter`, and
+// column r is at q's position for that iteration plus r.
+// In a persistent run this comes from the run-start state (nothing written
+// during the run is read): per column (per request for prefill) the first
+// position and the last it may reach, and for prefill the iterations before
+// each request.
+__device__ __forceinline__ bool request_at(const Graph& g, int r, uint32_t iter, int& s, int& q) {
+  if (!g.prefill) {
+    q = r;
+    const int s0 = __ldcg(&g.ctl->step0[r]);
+    s = s0 + (int)iter;
+    return s0 >= 0 && s < __ldcg(&g.ctl->stop[r]);
+  }
+  q = 0;
+  for (int i = 1; i < g.Rq; ++i)
+    if (__ldcg(&g.ctl->cum[i]) <= iter) q = i;
+  const int s0 = __ldcg(&g.ctl->step0[q]);
+  s = s0 + (int)(iter - __ldcg(&g.ctl->cum[q])) * g.R + r;
+  return s0 >= 0 && s < __ldcg(&g.ctl->stop[q]);
 }
 
-// Request whose tokens, step, pred and KV cache column r uses (prefill: all
-// columns are positions of request 0).
-__device__ __forceinline__ int col_req(const Graph& g, int r) { return g.prefill ? 0 : r; }
-
-__device__ __forceinline__ bool request_active(const Graph& g, int r, int& s) {
-  const int rq = col_req(g, r);
-  const int st = __ldcg(g.step + rq);
-  s = st + (g.prefill ? r : 0);
-  int end = g.S - 1;
-  if (g.step_end != nullptr) {
-    int e = __ldcg(g.step_end + rq);
-    end = e < end ? e : end;
+// The same from `step` itself, when every operation is its own launch (the
+// launches order the updates): a prefill graph serves the first request
+// that still has positions to go.
+__device__ __forceinline__ bool request_active(const Graph& g, int r, int& s, int& q) {
+  auto last_pos = [&](int rq) {
+    int end = g.S - 1;
+    if (g.step_end != nullptr) {
+      const int e = __ldcg(g.step_end + rq);
+      end = e < end ? e : end;
+    }
+    return end;
+  };
+  if (!g.prefill) {
+    q = r;
+    s = __ldcg(g.step + r);
+    return s >= 0 && s < last_pos(r);
   }
-  return st >= 0 && s < end;
+  q = 0;
+  int st = -1;
+  for (int i = 0; i < g.Rq; ++i) {
+    const int si = __ldcg(g.step + i);
+    if (si >= 0 && si < last_pos(i)) {
+      q = i;
+      st = si;
+      break;
+    }
+  }
+  s = st + r;
+  return st >= 0 && s < last_pos(q);
+}
+
+__device__ __forceinline__ bool request_state(const Graph& g, int r, uint32_t iter, int& s, int& q) {
+  return g.op_by_op ? request_active(g, r, s, q) : request_at(g, r, iter, s, q);
+}
+__device__ __forceinline__ bool request_state(const Graph& g, int r, uint32_t iter, int& s) {
+  int q;
+  return request_state(g, r, iter, s, q);
 }
 
 // First position of the iteration's chunk of column r's request (column 0's
 // position): prefill columns r' < r hold positions chunk0 .. s - 1.
 __device__ __forceinline__ int chunk0(const Graph& g, int r, int s) { return s - (g.prefill ? r : 0); }
-
-// KV-cache requests of the graph (prefill: one).
-__device__ __forceinline__ int cache_reqs(const Graph& g) { return g.prefill ? 1 : g.R; }
-
-// Position and activity of request r in iteration `iter`: from the run-start
-// state in a persistent run, from `step` itself when every operation is its
-// own launch (the launches order the updates).
-__device__ __forceinline__ bool request_state(const Graph& g, int r, uint32_t iter, int& s) {
-  return g.op_by_op ? request_active(g, r, s) : request_at(g, r, iter, s);
-}
 
 // Locate global row `row` of a stacked multi-matrix operation.
 __device__ __forceinline__ int seg_of(const OpDesc& op, int row) {
@@ -425,9 +454,12 @@ __device__ __forceinline__ uint32_t attn_stages(const Graph& g, const OpDesc& op
 }
 
 // Producer side of a split-K attention task: the cached positions of its
-// chunk, [lo, min(hi, chunk start)), into the ring, PB positions of K then PB
-// of V per stage (1-D bulk copies), once the previous iteration's attention
-// has released the operation (so those positions are in the cache).  The
+// chunk, [lo, min(hi, chunk start)), into the ring, once the previous
+// iteration's attention has released the operation (so those positions are in
+// the cache).  A stage holds PB positions from p on: K in its first half, V in
+// the second, each as d/64 boxes of [PB rows][64] bf16 (2-D tensor copies with
+// 128-byte swizzle, box h holding dims 64h..64h+63).  The boxes always hold PB
+// rows: those past the chunk's last position are loaded but never used.  The
 // consumer takes exactly these stages.  False on abort or timeout.  Not
 // inlined, so it adds nothing to the producer loop's registers.
 __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
@@ -435,26 +467,32 @@ __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc
   int r, c, Cr;
   if (!attn_slot(g, op, task / op.Hkv, iter, r, c, Cr)) return true;
   const int j = task % op.Hkv;
-  int s;
-  if (!request_state(g, r, iter, s)) return true;
+  int s, q;
+  if (!request_state(g, r, iter, s, q)) return true;
   const int npos = s + 1, sc0 = chunk0(g, r, s);
   const int lo = (int)(((long long)c * npos) / Cr);
   int hi = (int)(((long long)(c + 1) * npos) / Cr);
   hi = hi < sc0 ? hi : sc0;
   if (hi <= lo) return true;
-  if (iter > 0 && !wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 2,
-                                op.self, task, worker, (int)iter))
-    return false;
+  if (iter > 0) {
+    if (!wait_counter(g, g.events + (size_t)op.out_event * EVENT_STRIDE, iter * (uint32_t)op.out_trigger, 2, op.self,
+                      task, worker, (int)iter))
+      return false;
+    // the cache rows were appended with ordinary stores: order them before
+    // this thread's tensor copies read them
+    fence_acq_rel_gpu();
+    fence_proxy_async_global();
+  }
   const int D = op.d, PB = STAGE_BYTES / (4 * D);
-  const size_t kvbase = ((((size_t)op.layer * cache_reqs(g) + col_req(g, r)) * op.Hkv + j) * (size_t)op.S) * D;
+  const int row0 = ((op.layer * g.Rq + q) * op.Hkv + j) * op.S;  // < 2^31 (checked on the host)
   for (int p = lo; p < hi; p += PB) {
-    const int n = min(PB, hi - p);
     const uint32_t slot = pstage % (uint32_t)nr;
     if (!wait_mbar(g, &sm.empty[slot], ((pstage / (uint32_t)nr) & 1u) ^ 1u, 3, worker)) return false;
-    const uint32_t bytes = (uint32_t)n * (uint32_t)D * 2u;
-    mbar_arrive_expect_tx(&sm.full[slot], 2u * bytes);
-    bulk_g2s(sm.ring[slot], op.kc + kvbase + (size_t)p * D, bytes, &sm.full[slot], pol);
-    bulk_g2s(sm.ring[slot] + (size_t)PB * D * 2, op.vc + kvbase + (size_t)p * D, bytes, &sm.full[slot], pol);
+    mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)STAGE_BYTES);
+    for (int h = 0; h < D / 64; ++h) {
+      tma_load_2d(sm.ring[slot] + h * PB * 128, op.tmap_kc, h * 64, row0 + p, &sm.full[slot], pol);
+      tma_load_2d(sm.ring[slot] + STAGE_BYTES / 2 + h * PB * 128, op.tmap_vc, h * 64, row0 + p, &sm.full[slot], pol);
+    }
     ++pstage;
   }
   return true;
@@ -712,23 +750,23 @@ __device__ __noinline__ bool attn_dispatch(Smem& sm, const Graph& g, const OpDes
 // The LM head's last task to arrive (sm.last) turns every active column's
 // maximum key into its next token: written to tokens[r, s+1] if that slot
 // holds -1, always to pred; the request's step advances; the keys are reset.
-// A prefill graph's columns are positions of request 0: each column writes
-// its own prediction, the last active one advances step[0] (every column
-// reads the shared step before it changes).
+// A prefill graph's columns are positions of one request: each column writes
+// its own prediction, the last active one advances that request's step
+// (every column reads the shared step before it changes).
 __device__ __forceinline__ void argmax_tokens(Smem& sm, const Graph& g, const OpDesc& op, uint32_t iter, int ctid) {
   if (!sm.last) return;
   __threadfence();
-  int s = 0, sn = 0;
+  int s = 0, sn = 0, row = 0, qn = 0;
   bool act = false, next = false;
   unsigned long long key = 0ull;
   if (ctid < g.R) {
-    act = request_state(g, ctid, iter, s);
-    next = ctid + 1 < g.R && request_state(g, ctid + 1, iter, sn);
+    act = request_state(g, ctid, iter, s, row);
+    next = ctid + 1 < g.R && request_state(g, ctid + 1, iter, sn, qn);
     if (act) key = atomicAdd(op.keys + ctid, 0ull);
   }
   if (g.prefill) consumer_sync();
   if (ctid < g.R) {
-    const int rq = ctid, row = col_req(g, rq);
+    const int rq = ctid;
     if (act) {
       const int64_t nxt = (int64_t)argmax_key_index(key);
       int64_t* trow = g.tokens + (size_t)row * g.S;
@@ -1079,6 +1117,191 @@ __device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32
   accn += bl;
 }
 
+// ------------------------------------------------------------------ attention on the tensor cores
+// The split-K operation's main loop: the chunk's cached positions arrive
+// through the ring (stages of PB positions, K then V, 128-byte swizzled boxes
+// of 64 dims), the positions the iteration itself produced are rows KX / VX in
+// shared memory (row a0r + t, nin of them).  Warp-level MMAs (m16n8k16, bf16
+// inputs, fp32 accumulation), one 16-position tile per warp and stage; warp w
+// takes tile w % T16 and dims d0 = 64 (w / T16) .. d0 + 63 of v:
+//  * scores S = Q K^T (16 x 16): A = the queries, rows 0..3 the bf16 part
+//    hi(q) of query heads 0..3, rows 4..7 the rest lo(q) = bf16(q - hi(q)),
+//    rows 8..15 zero; B = the tile's k rows.  Score of head h = row h + row
+//    h + 4 (lanes 16 apart): the products of the fp32 queries to ~16 bits;
+//  * online softmax in base 2 per head over the tile (the queries carry
+//    log2(e) / sqrt(d)), positions past the valid count masked;
+//  * O^T += V^T P^T (16 dims x 8 columns per MMA): A = the tile's v rows
+//    loaded transposed (zeroed past the valid count, where the rows may hold
+//    anything), B = the probabilities straight from the score fragments,
+//    column h the hi part and column h + 4 the lo part of head h.
+// The warp's (max, sum, output) go to A.wm / A.wacc for the block merge.
+template <int G, int D>
+__device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnScratch& A, int lo, int chi, int a0r,
+                                                int nin, const uint16_t* KX, const uint16_t* VX, int cw, int lane,
+                                                int worker, uint32_t& cstage) {
+  constexpr int PB = STAGE_BYTES / (4 * D);  // positions per stage
+  constexpr int T16 = PB / 16;               // tiles per stage
+  constexpr int KS = D / 16;                 // k-steps of the scores
+  static_assert(G <= 4 && (CONSUMER_WARPS / T16) * 64 == D && T16 * (CONSUMER_WARPS / T16) == CONSUMER_WARPS,
+                "one tile and 64 dims of v per warp");
+  const int ctid = cw * 32 + lane;
+  const int tile = cw % T16, d0 = (cw / T16) * 64;
+  const int gq = lane >> 2, tq = lane & 3, hq = gq & 3;
+  const bool lo_row = gq >= 4;
+  const uint32_t full_mask = 0xffffffffu;
+  // bf16 hi / lo part of x for this lane's row of the query / probability operand
+  auto part = [&](float x) -> uint32_t {
+    const uint16_t h = f32_to_bf16_rn(x);
+    return lo_row ? (uint32_t)f32_to_bf16_rn(x - __uint_as_float((uint32_t)h << 16)) : (uint32_t)h;
+  };
+  uint32_t qa[KS][2];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int d = 16 * ks + 8 * hf + 2 * tq;
+      const float x0 = hq < G ? A.qs[hq * D + d] : 0.f;
+      const float x1 = hq < G ? A.qs[hq * D + d + 1] : 0.f;
+      qa[ks][hf] = part(x0) | (part(x1) << 16);
+    }
+  }
+  // O^T fragments: dims d0 + 16 mt + gq (elements 0, 1) and + 8 (2, 3), columns 2 tq, 2 tq + 1
+  float o[4][4];
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+  float m = -INFINITY, l = 0.f;  // head hq's running max and this lane's share of its sum
+  const int src_a = 4 * ((2 * tq) & 3), src_b = 4 * ((2 * tq + 1) & 3);  // lanes holding the columns' heads
+
+  // one tile: kaddr(t, c) / vaddr(t, c) = shared address of the 16 bytes of
+  // dims 8c..8c+7 of the tile's row t; nv valid rows (1..16)
+  auto run_tile = [&](auto kaddr, auto vaddr, int nv) {
+    float sa[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sa[nt][e] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < KS / 2; ++kk) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kaddr(nt * 8 + (lane & 7), 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(sa[nt], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
+        mma_bf16_16816(sa[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
+      }
+    }
+    // this lane's positions: 2 tq, 2 tq + 1 (sa[0]) and 8 + 2 tq, 9 + 2 tq (sa[1])
+    float sc[4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float v = sa[nt][e] + __shfl_xor_sync(full_mask, sa[nt][e], 16);
+        sc[nt * 2 + e] = (nt * 8 + 2 * tq + e < nv) ? v : -INFINITY;
+      }
+    float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    mx = fmaxf(mx, __shfl_xor_sync(full_mask, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(full_mask, mx, 2));
+    const float mn = fmaxf(m, mx);   // finite: position 0 of the tile is valid
+    const float al = exp2f(m - mn);  // m = -inf -> 0
+    float p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = exp2f(sc[i] - mn);  // masked -> 0
+    l = fmaf(l, al, (p[0] + p[1]) + (p[2] + p[3]));
+    m = mn;
+    const float al_a = __shfl_sync(full_mask, al, src_a), al_b = __shfl_sync(full_mask, al, src_b);
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      o[mt][0] *= al_a;
+      o[mt][1] *= al_b;
+      o[mt][2] *= al_a;
+      o[mt][3] *= al_b;
+    }
+    const uint32_t pb0 = part(p[0]) | (part(p[1]) << 16);
+    const uint32_t pb1 = part(p[2]) | (part(p[3]) << 16);
+    const bool ragged = nv < 16;
+    auto keep = [&](uint32_t v, int t) -> uint32_t {
+      return (t < nv ? (v & 0xffffu) : 0u) | (t + 1 < nv ? (v & 0xffff0000u) : 0u);
+    };
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      // matrices: rows 0..7 / 8..15 of the tile (lanes 16..31 the second) x
+      // 8 dims at chunk c / c + 1 (lanes 8..15 and 24..31 the second)
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(vaddr((lane & 7) + ((lane >> 4) << 3), d0 / 8 + 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+      if (ragged) {
+        a0 = keep(a0, 2 * tq);
+        a1 = keep(a1, 2 * tq);
+        a2 = keep(a2, 8 + 2 * tq);
+        a3 = keep(a3, 8 + 2 * tq);
+      }
+      mma_bf16_16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+    }
+  };
+
+  const int nr = g.batched ? NSTB : NSTAGES;
+  bool sfail = false;
+  for (int p0 = lo; p0 < chi; p0 += PB) {
+    const int n = min(PB, chi - p0);
+    const uint32_t cs = cstage;
+    const uint32_t slot = cs % (uint32_t)nr;
+    bool okk = true;
+    if (ctid == 0) okk = wait_mbar(g, &sm.full[slot], (cs / (uint32_t)nr) & 1u, 3, worker);
+    if (consumer_sync_or(!okk)) {
+      sfail = true;
+      break;
+    }
+    const int nv = min(16, n - tile * 16);
+    if (nv > 0) {
+      const uint32_t kb = smem_u32(sm.ring[slot]) + (uint32_t)(tile * 16) * 128u;
+      // box c / 8, row t (128 bytes), 16-byte unit c % 8 swizzled by the row
+      // (boxes and tiles start on 1024-byte boundaries)
+      auto sw = [](int t, int c) -> uint32_t {
+        return (uint32_t)(c >> 3) * (uint32_t)(PB * 128) + (uint32_t)t * 128u + (uint32_t)(((c & 7) ^ (t & 7)) << 4);
+      };
+      run_tile([&](int t, int c) { return kb + sw(t, c); },
+               [&](int t, int c) { return kb + (uint32_t)(STAGE_BYTES / 2) + sw(t, c); }, nv);
+    }
+    // every warp is done with the stage: release it (the ring's empty
+    // barrier expects one arrival per consumer warp on the GEMV path, one on
+    // the tensor-core path)
+    consumer_sync();
+    if (ctid == 0) {
+      const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
+      for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[slot]);
+    }
+    cstage = cs + 1u;
+  }
+  if (sfail) return false;
+  if (tile == 0 && nin > 0) {
+    // the iteration's own rows (plain [row][d] bf16 layout; rows past nin
+    // read row a0r + nin - 1, then masked)
+    const uint32_t kx = smem_u32(KX), vx = smem_u32(VX);
+    auto rowp = [&](int t, int c) -> uint32_t { return (uint32_t)((a0r + min(t, nin - 1)) * D * 2 + c * 16); };
+    run_tile([&](int t, int c) { return kx + rowp(t, c); }, [&](int t, int c) { return vx + rowp(t, c); }, nin);
+  }
+  // the warp's partial: the head's sum over the lanes of its row, the output
+  // as hi column + lo column (lanes 2 apart)
+  l += __shfl_xor_sync(full_mask, l, 1);
+  l += __shfl_xor_sync(full_mask, l, 2);
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float ov = o[mt][e] + __shfl_xor_sync(full_mask, o[mt][e], 2);
+      const int h = 2 * tq + (e & 1), d = d0 + 16 * mt + gq + 8 * (e >> 1);
+      if (tq < 2 && h < G) A.wacc[cw][h * D + d] = ov;
+    }
+  }
+  if (!lo_row && hq < G && tq == 0) {
+    A.wm[cw][hq][0] = m;
+    A.wm[cw][hq][1] = l;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------ attention task
 // Attention of kv head j for request r at position s, over the positions
 // [c (s+1) / C, (c+1) (s+1) / C) of chunk c of C.  Prologue: RMSNorm over the
@@ -1094,7 +1317,10 @@ __device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32
 template <int G, int D, bool STREAMED>
 __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
                                           int mode, int cw, int lane, uint32_t iter, int worker, uint32_t cstage) {
-  const bool fused = mode == ATTN_GROUP;  // state fetched in the projections' prologue
+  // the fused operation (group mode, state fetched in the projections'
+  // prologue) reads the cache itself; the split-K operation streams it
+  constexpr bool fused = !STREAMED;
+  (void)mode;
   if (cw == 0 && lane == 0) sm.h_key = ~0ull;  // the attention scratch overlays the GEMV input vector
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
@@ -1103,15 +1329,16 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   const int ctid = cw * 32 + lane;
   const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
-  const size_t kvbase = ((((size_t)op.layer * cache_reqs(g) + col_req(g, r)) * Hkv + j) * (size_t)op.S) * D;
+  size_t kvbase = ((((size_t)op.layer * g.Rq + r) * Hkv + j) * (size_t)op.S) * D;  // set below for prefill
   // k and v (bf16, k normalised and rotated) of the positions the iteration
   // itself produces: row 0 the task's own position (A.ks, A.vs); prefill: row
   // c the position of column c of the chunk, in the ring stage that the
   // tensor-core path keeps for its input rows (free while an attention task
   // runs: every MMA of the previous projection task has completed)
-  const int own = g.prefill ? r : 0;
-  uint16_t* const KX = g.prefill ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) : A.ks;
-  uint16_t* const VX = g.prefill ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_BATCH * MAX_D : A.vs;
+  const bool pf = STREAMED && g.prefill;  // prefill graphs run split-K attention only
+  const int own = pf ? r : 0;
+  uint16_t* const KX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) : A.ks;
+  uint16_t* const VX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_BATCH * MAX_D : A.vs;
   const int CS = op.C;  // split op: chunk partials per (request, query head)
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * CS) * (D + 2);
   // Prologue rows: warp cw < G takes query head cw of the group, warp G the
@@ -1137,7 +1364,9 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
     s = sm.attn_s;
     active = s >= 0;
   } else {
-    active = request_state(g, r, iter, s);
+    int q;
+    active = request_state(g, r, iter, s, q);
+    kvbase = ((((size_t)op.layer * g.Rq + q) * Hkv + j) * (size_t)op.S) * D;
   }
   bool afail = false;
   if (active && prow < G + 2) {
@@ -1193,7 +1422,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
         else VX[own * D + i] = f32_to_bf16_rn(x[e]);
       }
     }
-    if (STREAMED && g.prefill) {
+    if (pf) {
       // the chunk's earlier positions this task attends to (columns below
       // r, produced in this iteration and not read from the cache): their k
       // (normalised, rotated at its own position) and v, one row per warp
@@ -1232,11 +1461,11 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       }
     }
     // the rows sit in memory the tensor cores' bulk copies rewrite later
-    if (g.prefill) fence_proxy_async_smem();
+    if (pf) fence_proxy_async_smem();
     if (consumer_sync_or(afail)) return false;
     // the cache append at s: by the chunk holding s, or in group mode by the
     // merging task (chunk 0), whose release after the merge covers it
-    if ((mode == ATTN_GROUP ? c == 0 : hi == npos) && ctid < D / 4) {
+    if ((fused ? c == 0 : hi == npos) && ctid < D / 4) {
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
@@ -1246,106 +1475,59 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
     }
 
     // ---- main loop
-    const int grp = lane / LP, sub = lane % LP;
-    float acc[G][8], m[G], l[G];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh) {
-      m[hh] = -INFINITY;
-      l[hh] = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
-    }
-    // one position's K/V (8 dims per lane) into the warp's online softmax
-    auto consume = [&](const uint4 kvu, const uint4 vvu, bool valid) {
-      const float kf[8] = {bf16_lo(kvu.x), bf16_hi(kvu.x), bf16_lo(kvu.y), bf16_hi(kvu.y),
-                           bf16_lo(kvu.z), bf16_hi(kvu.z), bf16_lo(kvu.w), bf16_hi(kvu.w)};
-      float sc[G];
+    if constexpr (STREAMED) {
+      // Split-K operation: the chunk's cached positions [lo, min(hi, chunk
+      // start)) arrive through the weight ring and run on the tensor cores;
+      // the positions this iteration produced (s, and prefill: the chunk's
+      // earlier columns) come from their rows in shared memory
+      const int sc0 = chunk0(g, r, s);
+      const int chi = hi < sc0 ? hi : sc0;
+      const int a0 = lo > sc0 ? lo : sc0;
+      if (!attn_stream_mma<G, D>(sm, g, A, lo, chi, a0 - sc0, hi - a0, KX, VX, cw, lane, worker, cstage))
+        return false;
+    } else {
+      // fused operation: the positions straight from the cache (and s from
+      // shared memory), LP lanes per position on the CUDA cores
+      const int grp = lane / LP, sub = lane % LP;
+      float acc[G][8], m[G], l[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
-        const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
-        float a = q0.x * kf[0];
-        a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
-        a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
+        m[hh] = -INFINITY;
+        l[hh] = 0.f;
 #pragma unroll
-        for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        sc[hh] = a;
+        for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
       }
-      if (valid) {
-        const float vf[8] = {bf16_lo(vvu.x), bf16_hi(vvu.x), bf16_lo(vvu.y), bf16_hi(vvu.y),
-                             bf16_lo(vvu.z), bf16_hi(vvu.z), bf16_lo(vvu.w), bf16_hi(vvu.w)};
+      // one position's K/V (8 dims per lane) into the warp's online softmax
+      auto consume = [&](const uint4 kvu, const uint4 vvu, bool valid) {
+        const float kf[8] = {bf16_lo(kvu.x), bf16_hi(kvu.x), bf16_lo(kvu.y), bf16_hi(kvu.y),
+                             bf16_lo(kvu.z), bf16_hi(kvu.z), bf16_lo(kvu.w), bf16_hi(kvu.w)};
+        float sc[G];
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          const float mn = fmaxf(m[hh], sc[hh]);
-          const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
-          const float p = exp2f(sc[hh] - mn);
-          l[hh] = l[hh] * al + p;
+          const float4 q0 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8);
+          const float4 q1 = *reinterpret_cast<const float4*>(A.qs + hh * D + sub * 8 + 4);
+          float a = q0.x * kf[0];
+          a = fmaf(q0.y, kf[1], a); a = fmaf(q0.z, kf[2], a); a = fmaf(q0.w, kf[3], a);
+          a = fmaf(q1.x, kf[4], a); a = fmaf(q1.y, kf[5], a); a = fmaf(q1.z, kf[6], a); a = fmaf(q1.w, kf[7], a);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
-          m[hh] = mn;
+          for (int o = 1; o < LP; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+          sc[hh] = a;
         }
-      }
-    };
-    if constexpr (STREAMED) {
-      // Split-K operation: the chunk's cached positions [lo, min(hi, s))
-      // arrive through the weight ring (the producer streams them with bulk
-      // copies, PB positions of K then of V per stage); position s, if in
-      // this chunk, comes from shared memory.
-      constexpr int PB = STAGE_BYTES / (4 * D);
-      const int nr = g.batched ? NSTB : NSTAGES;
-      const int sc0 = chunk0(g, r, s);
-      const int chi = hi < sc0 ? hi : sc0;  // cached positions, streamed
-      bool sfail = false;
-      for (int p0 = lo; p0 < chi; p0 += PB) {
-        const int n = min(PB, chi - p0);
-        const uint32_t cs = cstage;
-        const uint32_t slot = cs % (uint32_t)nr;
-        bool okk = true;
-        if (ctid == 0) okk = wait_mbar(g, &sm.full[slot], (cs / (uint32_t)nr) & 1u, 3, worker);
-        if (consumer_sync_or(!okk)) {
-          sfail = true;
-          break;
-        }
-        const uint16_t* Ks = reinterpret_cast<const uint16_t*>(sm.ring[slot]) + sub * 8;
-        const uint16_t* Vs = Ks + PB * D;
-        for (int b = cw * PPW; b < n; b += NSTEP * CONSUMER_WARPS * PPW) {
-          uint4 kv[NSTEP], vv[NSTEP];
+        if (valid) {
+          const float vf[8] = {bf16_lo(vvu.x), bf16_hi(vvu.x), bf16_lo(vvu.y), bf16_hi(vvu.y),
+                               bf16_lo(vvu.z), bf16_hi(vvu.z), bf16_lo(vvu.w), bf16_hi(vvu.w)};
 #pragma unroll
-          for (int u = 0; u < NSTEP; ++u) {
-            const int t = b + u * CONSUMER_WARPS * PPW + grp;
-            kv[u] = make_uint4(0, 0, 0, 0);
-            vv[u] = make_uint4(0, 0, 0, 0);
-            if (t < n) {
-              kv[u] = *reinterpret_cast<const uint4*>(Ks + (size_t)t * D);
-              vv[u] = *reinterpret_cast<const uint4*>(Vs + (size_t)t * D);
-            }
+          for (int hh = 0; hh < G; ++hh) {
+            const float mn = fmaxf(m[hh], sc[hh]);
+            const float al = exp2f(m[hh] - mn);  // m = -inf -> 0
+            const float p = exp2f(sc[hh] - mn);
+            l[hh] = l[hh] * al + p;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(p, vf[e], acc[hh][e] * al);
+            m[hh] = mn;
           }
-#pragma unroll
-          for (int u = 0; u < NSTEP; ++u) consume(kv[u], vv[u], b + u * CONSUMER_WARPS * PPW + grp < n);
         }
-        // every warp is done with the stage: release it (the ring's empty
-        // barrier expects one arrival per consumer warp on the GEMV path, one
-        // on the tensor-core path)
-        consumer_sync();
-        if (ctid == 0) {
-          const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
-          for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[slot]);
-        }
-        cstage = cs + 1u;
-      }
-      if (sfail) return false;
-      // the positions this iteration produced (s, and prefill: the chunk's
-      // earlier columns), from their rows in shared memory, PPW per warp
-      const int a0 = lo > sc0 ? lo : sc0, nin = hi - a0;
-      if (cw * PPW < nin) {
-        const int t = cw * PPW + grp;
-        const bool valid = t < nin;
-        const int rw = valid ? a0 - sc0 + t : 0;
-        const uint4 kvs = valid ? *reinterpret_cast<const uint4*>(KX + rw * D + sub * 8) : make_uint4(0, 0, 0, 0);
-        const uint4 vvs = valid ? *reinterpret_cast<const uint4*>(VX + rw * D + sub * 8) : make_uint4(0, 0, 0, 0);
-        consume(kvs, vvs, valid);
-      }
-    } else {
+      };
       const uint16_t* kg = op.kc + kvbase + sub * 8;
       const uint16_t* vg = op.vc + kvbase + sub * 8;
       for (int base = lo + cw * PPW; base < hi; base += NSTEP * CONSUMER_WARPS * PPW) {
@@ -1368,46 +1550,50 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
 #pragma unroll
         for (int u = 0; u < NSTEP; ++u) consume(kv[u], vv[u], base + u * CONSUMER_WARPS * PPW + grp < hi);
       }
-    }
-    // merge the position groups of the warp
+      // merge the position groups of the warp
 #pragma unroll
-    for (int off = LP; off < 32; off <<= 1) {
+      for (int off = LP; off < 32; off <<= 1) {
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const float mo = __shfl_xor_sync(0xffffffffu, m[hh], off);
-        const float lo_ = __shfl_xor_sync(0xffffffffu, l[hh], off);
-        const float mn = fmaxf(m[hh], mo);
-        const float a = (mn == -INFINITY) ? 0.f : exp2f(m[hh] - mn);
-        const float b = (mn == -INFINITY) ? 0.f : exp2f(mo - mn);
-        l[hh] = l[hh] * a + lo_ * b;
+        for (int hh = 0; hh < G; ++hh) {
+          const float mo = __shfl_xor_sync(0xffffffffu, m[hh], off);
+          const float lo_ = __shfl_xor_sync(0xffffffffu, l[hh], off);
+          const float mn = fmaxf(m[hh], mo);
+          const float a = (mn == -INFINITY) ? 0.f : exp2f(m[hh] - mn);
+          const float b = (mn == -INFINITY) ? 0.f : exp2f(mo - mn);
+          l[hh] = l[hh] * a + lo_ * b;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][e], off);
-          acc[hh][e] = acc[hh][e] * a + ao * b;
+          for (int e = 0; e < 8; ++e) {
+            const float ao = __shfl_xor_sync(0xffffffffu, acc[hh][e], off);
+            acc[hh][e] = acc[hh][e] * a + ao * b;
+          }
+          m[hh] = mn;
         }
-        m[hh] = mn;
       }
-    }
-    if (grp == 0) {
+      if (grp == 0) {
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
+        for (int hh = 0; hh < G; ++hh) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) A.wacc[cw][hh * D + sub * 8 + e] = acc[hh][e];
-        if (sub == 0) {
-          A.wm[cw][hh][0] = m[hh];
-          A.wm[cw][hh][1] = l[hh];
+          for (int e = 0; e < 8; ++e) A.wacc[cw][hh * D + sub * 8 + e] = acc[hh][e];
+          if (sub == 0) {
+            A.wm[cw][hh][0] = m[hh];
+            A.wm[cw][hh][1] = l[hh];
+          }
         }
       }
     }
     consumer_sync();
-    // merge the warps in fixed order -> this chunk's partial
+    // merge the warps in fixed order -> this chunk's partial.  Warps holding
+    // (head, dim i): every warp on the CUDA-core path; on the tensor-core
+    // path the NT warps whose 64 dims hold i (one per tile of a stage)
+    constexpr int NT = STREAMED ? STAGE_BYTES / (4 * D) / 16 : CONSUMER_WARPS;
     for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
       const int hh = idx / D, i = idx % D;
+      const int w0 = STREAMED ? (i / 64) * NT : 0;
       float M = -INFINITY;
-      for (int w = 0; w < CONSUMER_WARPS; ++w) M = fmaxf(M, A.wm[w][hh][0]);
+      for (int w = w0; w < w0 + NT; ++w) M = fmaxf(M, A.wm[w][hh][0]);
       float Ls = 0.f, Os = 0.f;
       if (M != -INFINITY) {
-        for (int w = 0; w < CONSUMER_WARPS; ++w) {
+        for (int w = w0; w < w0 + NT; ++w) {
           const float f = exp2f(A.wm[w][hh][0] - M);
           Ls = fmaf(A.wm[w][hh][1], f, Ls);
           Os = fmaf(A.wacc[w][hh * D + i], f, Os);
@@ -1534,8 +1720,8 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
 // ------------------------------------------------------------------ embedding task
 __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t iter, int ctid) {
   const int r = task;
-  int s;
-  if (r < g.R && !request_state(g, r, iter, s)) {
+  int s, q = 0;
+  if (r < g.R && !request_state(g, r, iter, s, q)) {
     // inactive request (several requests, this one done): x carries this
     // iteration's version with zeros, so every reader's wait ends; nothing
     // of it reaches the request's tokens or cache
@@ -1555,7 +1741,7 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
     return true;
   }
   if (r < g.R) {
-    const int64_t tok = __ldcg(g.tokens + (size_t)col_req(g, r) * g.S + s);
+    const int64_t tok = __ldcg(g.tokens + (size_t)q * g.S + s);
     if (tok < 0 || tok >= g.V) {
       if (ctid == 0) record_error(g, -11 /*DEVICE*/, 8, -1, task, -1, (int)iter, (uint32_t)tok, (uint32_t)g.V);
       return true;
@@ -1910,21 +2096,27 @@ __device__ __forceinline__ void persistent_body(const Graph& g) {
 
   if ((int)blockIdx.x < g.sched_ctas) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-      // iterations of this run: the furthest any request still has to go
-      // (prefill: request 0's remaining positions, R per iteration)
+      // iterations of this run: the furthest any request still has to go;
+      // prefill: every request's remaining positions, R per iteration, one
+      // request after another
       uint32_t n_iter = 0;
-      for (int r = 0; r < g.R; ++r) {
-        int s;
-        const bool act = request_active(g, r, s);
+      const int nq = g.prefill ? g.Rq : g.R;
+      for (int q = 0; q < nq; ++q) {
+        const int s = __ldcg(g.step + q);
         int end = g.S - 1;
-        if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + col_req(g, r)));
-        if (act) {
-          const uint32_t left = (uint32_t)(end - s);
-          n_iter = max(n_iter, g.prefill ? (left + (uint32_t)g.R - 1u) / (uint32_t)g.R : left);
+        if (g.step_end != nullptr) end = min(end, __ldcg(g.step_end + q));
+        const bool act = s >= 0 && s < end;
+        const uint32_t left = act ? (uint32_t)(end - s) : 0u;
+        if (g.prefill) {
+          g.ctl->cum[q] = n_iter;
+          n_iter += (left + (uint32_t)g.R - 1u) / (uint32_t)g.R;
+        } else {
+          n_iter = max(n_iter, left);
         }
-        g.ctl->step0[r] = act ? s : -1;
-        g.ctl->stop[r] = end;
+        g.ctl->step0[q] = act ? s : -1;
+        g.ctl->stop[q] = end;
       }
+      if (g.prefill) g.ctl->cum[nq] = n_iter;
       g.ctl->n_iter = n_iter;
       st_release(&g.ctl->ready, 1u);
     }

@@ -92,6 +92,35 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
       : "memory");
 }
 
+// ---------------------------------------------------------------- warp-level MMA (attention)
+// Four 8x8 bf16 matrices from shared memory: lanes 8i..8i+7 give the row
+// addresses (16 bytes each) of matrix i; matrix i lands in r_i, lane l holding
+// row l/4, elements 2(l%4) and 2(l%4)+1 (the lower index in the low half).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// The same, transposed: lane l holds elements (row 2(l%4), column l/4) and
+// (row 2(l%4)+1, column l/4) of each matrix.
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D += A B, A 16x16 bf16 (row-major fragments a0..a3: rows g / g+8 of lane
+// l = 4g + t, columns 2t.. and 2t+8..), B 16x8 bf16 (b0: rows 2t, 2t+1 of
+// column g; b1: rows 2t+8, 2t+9), D 16x8 fp32 (d0, d1: row g, columns 2t,
+// 2t+1; d2, d3: row g+8).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // ---------------------------------------------------------------- tensor memory and tcgen05 MMA
 // Columns of tensor memory one worker block allocates (a power of two >= 32):
 // all of it (one worker block per SM), as accumulator slots of 2 x 16 columns.

@@ -38,12 +38,13 @@ def reduction_split(K: int, max_k: int = _lib.MAX_GEMV_K) -> int:
 BATCH_BM, BATCH_BK, BATCH_MAX_KBLOCKS = 128, 64, 24
 # Task-size model used to choose the grid: a worker streams weights at about
 # its share of HBM bandwidth and pays a fixed cost per task, per extra pass
-# over the input rows, and (split reductions) for the finishing task's
-# partial-sum reduction.
+# over the input rows, and (split reductions) per partial sum that the
+# finishing task gathers and adds (measured on the 8B shape with 8 requests:
+# the o and down projections at 4 segments beat 9, 5.46 vs 5.89 ms/step).
 _WORKER_BYTES_PER_S = 43e9
 _TASK_OVERHEAD_S = 3e-6
 _PASS_OVERHEAD_S = 4e-6
-_SPLIT_OVERHEAD_S = 6e-6
+_SPLIT_PARTIAL_S = 1.5e-6
 BATCH_SLOTS = 16  # accumulator slots: row blocks a task may hold across passes
 
 
@@ -52,7 +53,7 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[i
     several requests: among segment counts s and, per number of rounds k of
     the workers, the largest run split gx <= row blocks with gx * s <= k *
     workers, the one with the least rounds x (largest task's weight bytes /
-    bandwidth + task, pass and split costs); fewer segments on ties.  A task
+    bandwidth + task, pass and per-partial split costs); fewer segments on ties.  A task
     longer than the input rows (passes) holds at most BATCH_SLOTS row blocks."""
     nb = -(-rows // BATCH_BM)
     nkb = K // BATCH_BK
@@ -67,7 +68,7 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[i
                 continue
             rounds = -(-(gx * s) // workers)
             t = rounds * (most * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S +
-                          (npass - 1) * _PASS_OVERHEAD_S) + (_SPLIT_OVERHEAD_S if s > 1 else 0.0)
+                          (npass - 1) * _PASS_OVERHEAD_S) + (s * _SPLIT_PARTIAL_S if s > 1 else 0.0)
             if best is None or t < best[0] * (1 - 1e-2):
                 best = (t, gx, s)
     return best[1], best[2]
@@ -199,18 +200,16 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     projection+attention operation for one request with up to
     FUSED_ATTENTION_MAX_SEQ positions, split-K attention otherwise.
 
-    prefill_tokens = T in 2..8 builds a prefill graph for one request
-    (requests = 1): every iteration ingests T consecutive prompt positions as
-    the T columns of the tensor-core projections (mpk_options.prefill_tokens).
-    Pass the decode graph's caches as k_cache / v_cache to continue decoding
-    from the prefilled state."""
+    prefill_tokens = T in 2..8 builds a prefill graph: every iteration ingests
+    T consecutive prompt positions of one request as the T columns of the
+    tensor-core projections (mpk_options.prefill_tokens), the requests one
+    after another.  Pass the decode graph's caches as k_cache / v_cache (and
+    the same `requests`) to continue decoding from the prefilled state."""
     from . import _lib
 
     s = shape
     cols = requests
     if prefill_tokens > 1:
-        if requests != 1:
-            raise ValueError("a prefill graph serves one request")
         cols = prefill_tokens
     if num_workers is None:
         num_workers = _lib.load().mpk_device_sm_count() - num_local_schedulers // 4

@@ -146,10 +146,11 @@ def test_batched_grid_rule():
                 if -(-nkb // gy) > BATCH_MAX_KBLOCKS:
                     assert -(-nb // gx) <= BATCH_SLOTS
     # the 8B plan for 144 workers: one round of tasks for the projections, the
-    # reductions split three or nine ways
+    # reductions split three or four ways
     assert batched_grid(6144, 4096, 144) == (48, 3)
     assert batched_grid(12288, 4096, 144, True) == (48, 3)
-    assert batched_grid(4096, 12288, 144) == (16, 9)
+    assert batched_grid(4096, 4096, 144) == (32, 4)
+    assert batched_grid(4096, 12288, 144) == (32, 4)
 
 
 def test_batched_layer_plan():

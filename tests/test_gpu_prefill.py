@@ -1,11 +1,12 @@
-"""Prompt ingestion by prefill graphs (mpk_options.prefill_tokens): T consecutive
-prompt positions of one request per iteration, as the T columns of the
-tensor-core projections, inside the same persistent kernel ("Mirage Persistent
-Kernel: Fusing Multi-GPU LLM Inference into One Kernel Launch", "How MPK
-Works": the `tokens` meta tensor holds the prompt; the runtime advances `step`).
+"""Prompt ingestion by prefill graphs (mpk_options.prefill_tokens): T
+consecutive prompt positions of one request per iteration, as the T columns
+of the tensor-core projections, the requests of the cache one after another,
+inside the same persistent kernel ("Mirage Persistent Kernel: Fusing
+Multi-GPU LLM Inference into One Kernel Launch", "How MPK Works": the
+`tokens` meta tensor holds the prompt; the runtime advances `step`).
 
-Each column at position p consumes tokens[0, p], appends its K/V at p and
-attends to positions 0..p: the chunk's earlier positions from this
+Each column at position p of request q consumes tokens[q, p], appends its K/V
+at p and attends to positions 0..p: the chunk's earlier positions from this
 iteration's k and v, the rest from the cache.  Checked against the CPU
 oracle, which ingests the prompt one position at a time: greedy tokens after
 a prefilled prompt are the oracle's, the per-column logits and residual
@@ -148,10 +149,99 @@ def test_prefill_op_by_op_bit_identical(weights):
         assert torch.equal(a, b)
 
 
-def test_prefill_rejects_a_cache_of_several_requests(weights):
+def test_prefill_several_requests_then_batched_decode(weights):
+    """A prefill graph over a KV cache of four requests ingests their prompts one
+    request after another (a one-token prompt has nothing to ingest, an
+    inactive request stays untouched), then the batched decode graph on the
+    same cache continues all of them: every generated token is the oracle's."""
+    w_cpu, w = weights
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    prompts = [19, 1, 7, 12]
+    R, T = len(prompts), 5
+    tokens = sq.make_tokens(SHAPE, R, S, prompts, seed=34)
+    dec = build_decoder(SHAPE, w, requests=R, max_seq=S)
+    pre = build_decoder(SHAPE, w, requests=R, max_seq=S, prefill_tokens=T, k_cache=dec.k_cache,
+                        v_cache=dec.v_cache)
+    tok = tokens.cuda()
+    step = torch.zeros(R, dtype=torch.int32, device="cuda")
+    p_end = torch.tensor([p - 1 for p in prompts], dtype=torch.int32, device="cuda")
+    pre.run(step, tok, p_end)
+    torch.cuda.synchronize()
+    pre.kernel.check_status()
+    assert step.cpu().tolist() == [p - 1 for p in prompts]
+    assert torch.equal(tok.cpu(), tokens)  # every slot the prefill reached holds a prompt token
+    dec.run(step, tok, torch.full((R,), S - 1, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    dec.kernel.check_status()
+    ref = oracle.Decoder(SHAPE, w_cpu)
+    out, st, rkc, _, _ = ref.generate(tokens.numpy(), np.zeros(R, np.int32), np.full(R, S - 1, np.int32))
+    assert step.cpu().tolist() == [S - 1] * R and st.tolist() == [S - 1] * R
+    got = tok.cpu().numpy()
+    assert np.array_equal(got, out), f"\n gpu    {got.tolist()}\n oracle {out.tolist()}"
+    gk = u16_to_f64(bf16_u16(dec.k_cache))
+    rk = u16_to_f64(rkc)
+    assert np.linalg.norm(gk - rk) <= 1e-2 * np.linalg.norm(rk)
+    pre.kernel.close()
+    dec.kernel.close()
+
+
+def test_prefill_skips_an_inactive_request(weights):
+    """step = -1 marks a request the run leaves alone: its step, tokens and
+    cache rows stay as they were while the others are prefilled."""
+    _, w = weights
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    R, T = 3, 4
+    tokens = sq.make_tokens(SHAPE, R, S, [PROMPT] * R, seed=35)
+    pre = build_decoder(SHAPE, w, requests=R, max_seq=S, prefill_tokens=T)
+    tok = tokens.cuda()
+    step = torch.tensor([0, -1, 0], dtype=torch.int32, device="cuda")
+    pre.run(step, tok, torch.full((R,), PROMPT - 1, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    pre.kernel.check_status()
+    assert step.cpu().tolist() == [PROMPT - 1, -1, PROMPT - 1]
+    assert torch.equal(tok.cpu(), tokens)
+    kc = pre.k_cache.cpu().float()
+    assert not bool(kc[:, 1].any()) and bool(kc[:, 0, :, :PROMPT - 1].any()) and bool(kc[:, 2, :, :PROMPT - 1].any())
+    assert not bool(kc[:, :, :, PROMPT - 1:].any())  # nothing past the ingested positions
+    assert bool((pre.pred.cpu()[1] == -1).all())
+    pre.kernel.close()
+
+
+def test_prefill_several_requests_op_by_op_bit_identical(weights):
+    _, w = weights
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    prompts = [9, 17, 4]
+    R = len(prompts)
+    tokens = sq.make_tokens(SHAPE, R, S, prompts, seed=36)
+    outs = []
+    for mode in ("run", "run_op_by_op"):
+        pre = build_decoder(SHAPE, w, requests=R, max_seq=S, prefill_tokens=6)
+        tok = tokens.cuda()
+        step = torch.zeros(R, dtype=torch.int32, device="cuda")
+        getattr(pre, mode)(step, tok, torch.tensor([p - 1 for p in prompts], dtype=torch.int32, device="cuda"))
+        torch.cuda.synchronize()
+        pre.kernel.check_status()
+        outs.append((step.cpu(), tok.cpu(), pre.pred.cpu(), pre.k_cache.cpu().view(torch.int16),
+                     pre.v_cache.cpu().view(torch.int16)))
+        pre.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_prefill_run_needs_every_cached_request(weights):
+    """A prefill graph over a cache of three requests takes tokens and step of
+    three rows: a run with one is a SHAPE error and the context stays usable."""
     from persistent_megakernel_decode_02_b200 import MpkError, build_decoder
     _, w = weights
-    kv = torch.zeros((SHAPE.layers, 2, SHAPE.kv_heads, S, SHAPE.head_dim), dtype=torch.bfloat16, device="cuda")
+    pre = build_decoder(SHAPE, w, requests=3, max_seq=S, prefill_tokens=4)
+    tok = sq.make_tokens(SHAPE, 1, S, [PROMPT], seed=37).cuda()
     with pytest.raises(MpkError) as e:
-        build_decoder(SHAPE, w, requests=1, max_seq=S, prefill_tokens=4, k_cache=kv, v_cache=kv.clone())
+        pre.run(torch.zeros(1, dtype=torch.int32, device="cuda"), tok)
     assert e.value.name == "SHAPE"
+    tok3 = sq.make_tokens(SHAPE, 3, S, [PROMPT] * 3, seed=37).cuda()
+    step = torch.zeros(3, dtype=torch.int32, device="cuda")
+    pre.run(step, tok3, torch.full((3,), 4, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    pre.kernel.check_status()
+    assert step.cpu().tolist() == [4, 4, 4]
+    pre.kernel.close()
