@@ -1318,9 +1318,10 @@ template <int G, int D, bool STREAMED>
 __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc& op, int j, int c, int C, int r,
                                           int mode, int cw, int lane, uint32_t iter, int worker, uint32_t cstage) {
   // the fused operation (group mode, state fetched in the projections'
-  // prologue) reads the cache itself; the split-K operation streams it
-  constexpr bool fused = !STREAMED;
-  (void)mode;
+  // prologue) reads the cache itself; the split-K operation streams it.  A
+  // run-time flag, although it follows STREAMED: measured, the compile-time
+  // form makes the fused operation's register allocation slower
+  const bool fused = mode == ATTN_GROUP;
   if (cw == 0 && lane == 0) sm.h_key = ~0ull;  // the attention scratch overlays the GEMV input vector
   constexpr int LP = D / 8;          // lanes per position
   constexpr int PPW = 32 / LP;       // positions per warp step
@@ -1335,7 +1336,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   // c the position of column c of the chunk, in the ring stage that the
   // tensor-core path keeps for its input rows (free while an attention task
   // runs: every MMA of the previous projection task has completed)
-  const bool pf = STREAMED && g.prefill;  // prefill graphs run split-K attention only
+  const bool pf = g.prefill;  // prefill graphs run split-K attention only
   const int own = pf ? r : 0;
   uint16_t* const KX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) : A.ks;
   uint16_t* const VX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_BATCH * MAX_D : A.vs;
@@ -1465,7 +1466,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
     if (consumer_sync_or(afail)) return false;
     // the cache append at s: by the chunk holding s, or in group mode by the
     // merging task (chunk 0), whose release after the merge covers it
-    if ((fused ? c == 0 : hi == npos) && ctid < D / 4) {
+    if ((mode == ATTN_GROUP ? c == 0 : hi == npos) && ctid < D / 4) {
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
