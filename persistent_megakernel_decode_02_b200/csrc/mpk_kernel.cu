@@ -1144,7 +1144,6 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
   constexpr int KS = D / 16;                 // k-steps of the scores
   static_assert(G <= 4 && (CONSUMER_WARPS / T16) * 64 == D && T16 * (CONSUMER_WARPS / T16) == CONSUMER_WARPS,
                 "one tile and 64 dims of v per warp");
-  const int ctid = cw * 32 + lane;
   const int tile = cw % T16, d0 = (cw / T16) * 64;
   const int gq = lane >> 2, tq = lane & 3, hq = gq & 3;
   const bool lo_row = gq >= 4;
@@ -1174,31 +1173,46 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
   float m = -INFINITY, l = 0.f;  // head hq's running max and this lane's share of its sum
   const int src_a = 4 * ((2 * tq) & 3), src_b = 4 * ((2 * tq + 1) & 3);  // lanes holding the columns' heads
 
-  // one tile: kaddr(t, c) / vaddr(t, c) = shared address of the 16 bytes of
-  // dims 8c..8c+7 of the tile's row t; nv valid rows (1..16)
-  auto run_tile = [&](auto kaddr, auto vaddr, int nv) {
-    float sa[2][4];
+  // The current tile: K rows at kb, V rows at vb, either a ring stage
+  // (swizzled boxes) or, for the iteration's own rows, plain [row][d] rows
+  // a0r.. (own > 0 of them; rows past them read the last, then masked).
+  // addr(base, t, c) = shared address of dims 8c..8c+7 of the tile's row t.
+  uint32_t kb = 0, vb = 0;
+  int own = 0;
+  auto addr = [&](uint32_t base, int t, int c) -> uint32_t {
+    if (own == 0)  // box c / 8, 128-byte row t, 16-byte unit c % 8 swizzled by the row
+      return base + (uint32_t)(c >> 3) * (uint32_t)(PB * 128) + (uint32_t)t * 128u +
+             (uint32_t)(((c & 7) ^ (t & 7)) << 4);
+    return base + (uint32_t)((a0r + min(t, own - 1)) * D * 2 + c * 16);
+  };
+  // one tile of nv valid rows (1..16)
+  auto run_tile = [&](int nv) {
+    // two accumulators per 8 positions (even / odd k-steps): shorter MMA chains
+    float sa[2][2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sa[nt][e] = 0.f;
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sa[nt][h][e] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < KS / 2; ++kk) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(kaddr(nt * 8 + (lane & 7), 4 * kk + (lane >> 3)), b0, b1, b2, b3);
-        mma_bf16_16816(sa[nt], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
-        mma_bf16_16816(sa[nt], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
+        ldsm_x4(addr(kb, nt * 8 + (lane & 7), 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+        mma_bf16_16816(sa[nt][0], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
+        mma_bf16_16816(sa[nt][1], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
       }
     }
-    // this lane's positions: 2 tq, 2 tq + 1 (sa[0]) and 8 + 2 tq, 9 + 2 tq (sa[1])
+    // this lane's positions: 2 tq, 2 tq + 1 (nt = 0) and 8 + 2 tq, 9 + 2 tq (nt = 1)
     float sc[4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float v = sa[nt][e] + __shfl_xor_sync(full_mask, sa[nt][e], 16);
+        const float x = sa[nt][0][e] + sa[nt][1][e];
+        const float v = x + __shfl_xor_sync(full_mask, x, 16);
         sc[nt * 2 + e] = (nt * 8 + 2 * tq + e < nv) ? v : -INFINITY;
       }
     float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
@@ -1230,7 +1244,7 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
       // matrices: rows 0..7 / 8..15 of the tile (lanes 16..31 the second) x
       // 8 dims at chunk c / c + 1 (lanes 8..15 and 24..31 the second)
       uint32_t a0, a1, a2, a3;
-      ldsm_x4_t(vaddr((lane & 7) + ((lane >> 4) << 3), d0 / 8 + 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
+      ldsm_x4_t(addr(vb, (lane & 7) + ((lane >> 4) << 3), d0 / 8 + 2 * mt + ((lane >> 3) & 1)), a0, a1, a2, a3);
       if (ragged) {
         a0 = keep(a0, 2 * tq);
         a1 = keep(a1, 2 * tq);
@@ -1241,6 +1255,11 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
     }
   };
 
+  // Stages: one elected thread waits (bounded), the block learns the outcome
+  // through the barrier; once every warp is done with its tile the stage is
+  // released (one arrival per consumer warp on the GEMV ring, one on the
+  // tensor-core ring).  Measured faster than per-warp waits and releases.
+  const bool elected = cw == 0 && lane == 0;
   const int nr = g.batched ? NSTB : NSTAGES;
   bool sfail = false;
   for (int p0 = lo; p0 < chi; p0 += PB) {
@@ -1248,39 +1267,31 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
     const uint32_t cs = cstage;
     const uint32_t slot = cs % (uint32_t)nr;
     bool okk = true;
-    if (ctid == 0) okk = wait_mbar(g, &sm.full[slot], (cs / (uint32_t)nr) & 1u, 3, worker);
+    if (elected) okk = wait_mbar(g, &sm.full[slot], (cs / (uint32_t)nr) & 1u, 3, worker);
     if (consumer_sync_or(!okk)) {
       sfail = true;
       break;
     }
     const int nv = min(16, n - tile * 16);
     if (nv > 0) {
-      const uint32_t kb = smem_u32(sm.ring[slot]) + (uint32_t)(tile * 16) * 128u;
-      // box c / 8, row t (128 bytes), 16-byte unit c % 8 swizzled by the row
-      // (boxes and tiles start on 1024-byte boundaries)
-      auto sw = [](int t, int c) -> uint32_t {
-        return (uint32_t)(c >> 3) * (uint32_t)(PB * 128) + (uint32_t)t * 128u + (uint32_t)(((c & 7) ^ (t & 7)) << 4);
-      };
-      run_tile([&](int t, int c) { return kb + sw(t, c); },
-               [&](int t, int c) { return kb + (uint32_t)(STAGE_BYTES / 2) + sw(t, c); }, nv);
+      kb = smem_u32(sm.ring[slot]) + (uint32_t)(tile * 16) * 128u;  // tiles start on 1024-byte boundaries
+      vb = kb + (uint32_t)(STAGE_BYTES / 2);
+      run_tile(nv);
     }
-    // every warp is done with the stage: release it (the ring's empty
-    // barrier expects one arrival per consumer warp on the GEMV path, one on
-    // the tensor-core path)
     consumer_sync();
-    if (ctid == 0) {
+    if (elected) {
       const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
       for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[slot]);
     }
     cstage = cs + 1u;
   }
-  if (sfail) return false;
+  if (consumer_sync_or(sfail)) return false;
   if (tile == 0 && nin > 0) {
-    // the iteration's own rows (plain [row][d] bf16 layout; rows past nin
-    // read row a0r + nin - 1, then masked)
-    const uint32_t kx = smem_u32(KX), vx = smem_u32(VX);
-    auto rowp = [&](int t, int c) -> uint32_t { return (uint32_t)((a0r + min(t, nin - 1)) * D * 2 + c * 16); };
-    run_tile([&](int t, int c) { return kx + rowp(t, c); }, [&](int t, int c) { return vx + rowp(t, c); }, nin);
+    // the iteration's own rows
+    own = nin;
+    kb = smem_u32(KX);
+    vb = smem_u32(VX);
+    run_tile(nin);
   }
   // the warp's partial: the head's sum over the lanes of its row, the output
   // as hi column + lo column (lanes 2 apart)
