@@ -42,6 +42,7 @@ struct AttnScratch {
   uint16_t vs[MAX_D];                            // this position's v (bf16)
   float wm[CONSUMER_WARPS][MAX_G][2];            // per-warp running (max, sum)
   float wacc[CONSUMER_WARPS][MAX_G * MAX_D / 2]; // per-warp unnormalised outputs
+  float4 xs[CONSUMER_WARPS * 32];                // tensor-core path: partial scores exchanged by a tile's two warps
 };
 static_assert(MAX_G * MAX_D / 2 >= 512, "attention scratch");
 static_assert(sizeof(AttnScratch) >= sizeof(float) * MAX_GCHUNK * (MAX_G / 2) * (MAX_D + 2),
@@ -1123,11 +1124,14 @@ __device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32
 // of 64 dims), the positions the iteration itself produced are rows KX / VX in
 // shared memory (row a0r + t, nin of them).  Warp-level MMAs (m16n8k16, bf16
 // inputs, fp32 accumulation), one 16-position tile per warp and stage; warp w
-// takes tile w % T16 and dims d0 = 64 (w / T16) .. d0 + 63 of v:
+// takes tile w % T16 and dims d0 = 64 (w / T16) .. d0 + 63 (d = 128: the
+// tile's two warps split the head dim):
 //  * scores S = Q K^T (16 x 16): A = the queries, rows 0..3 the bf16 part
 //    hi(q) of query heads 0..3, rows 4..7 the rest lo(q) = bf16(q - hi(q)),
 //    rows 8..15 zero; B = the tile's k rows.  Score of head h = row h + row
-//    h + 4 (lanes 16 apart): the products of the fp32 queries to ~16 bits;
+//    h + 4 (lanes 16 apart): the products of the fp32 queries to ~16 bits.
+//    With d = 128 each warp of the tile sums over its own 64 dims and the
+//    two add their halves through shared memory behind a two-warp barrier;
 //  * online softmax in base 2 per head over the tile (the queries carry
 //    log2(e) / sqrt(d)), positions past the valid count masked;
 //  * O^T += V^T P^T (16 dims x 8 columns per MMA): A = the tile's v rows
@@ -1153,12 +1157,17 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
     const uint16_t h = f32_to_bf16_rn(x);
     return lo_row ? (uint32_t)f32_to_bf16_rn(x - __uint_as_float((uint32_t)h << 16)) : (uint32_t)h;
   };
-  uint32_t qa[KS][2];
+  // with two warps per tile (d = 128) each computes the scores over its own
+  // 64 dims and the pair adds the halves through shared memory
+  constexpr bool PAIR = T16 * 2 == CONSUMER_WARPS;
+  constexpr int KSW = PAIR ? KS / 2 : KS;  // k-steps this warp takes
+  const int kd0 = PAIR ? d0 : 0;
+  uint32_t qa[KSW][2];
 #pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
+  for (int ks = 0; ks < KSW; ++ks) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int d = 16 * ks + 8 * hf + 2 * tq;
+      const int d = kd0 + 16 * ks + 8 * hf + 2 * tq;
       const float x0 = hq < G ? A.qs[hq * D + d] : 0.f;
       const float x1 = hq < G ? A.qs[hq * D + d + 1] : 0.f;
       qa[ks][hf] = part(x0) | (part(x1) << 16);
@@ -1196,14 +1205,25 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
 #pragma unroll
         for (int e = 0; e < 4; ++e) sa[nt][h][e] = 0.f;
 #pragma unroll
-    for (int kk = 0; kk < KS / 2; ++kk) {
+    for (int kk = 0; kk < KSW / 2; ++kk) {
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(addr(kb, nt * 8 + (lane & 7), 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+        ldsm_x4(addr(kb, nt * 8 + (lane & 7), kd0 / 8 + 4 * kk + (lane >> 3)), b0, b1, b2, b3);
         mma_bf16_16816(sa[nt][0], qa[2 * kk][0], 0u, qa[2 * kk][1], 0u, b0, b1);
         mma_bf16_16816(sa[nt][1], qa[2 * kk + 1][0], 0u, qa[2 * kk + 1][1], 0u, b2, b3);
       }
+    }
+    if (PAIR) {
+      float4* xs = A.xs;  // [warp][lane] partial scores (rows g)
+      xs[cw * 32 + lane] = make_float4(sa[0][0][0] + sa[0][1][0], sa[0][0][1] + sa[0][1][1],
+                                       sa[1][0][0] + sa[1][1][0], sa[1][0][1] + sa[1][1][1]);
+      named_sync(3 + tile, 64);  // the tile's two warps (barriers 0..2 serve the block and the epilogue)
+      const float4 ps = xs[(cw ^ T16) * 32 + lane];
+      sa[0][1][0] += ps.x;
+      sa[0][1][1] += ps.y;
+      sa[1][1][0] += ps.z;
+      sa[1][1][1] += ps.w;
     }
     // this lane's positions: 2 tq, 2 tq + 1 (nt = 0) and 8 + 2 tq, 9 + 2 tq (nt = 1)
     float sc[4];
@@ -1261,6 +1281,11 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
   // tensor-core ring).  Measured faster than per-warp waits and releases.
   const bool elected = cw == 0 && lane == 0;
   const int nr = g.batched ? NSTB : NSTAGES;
+  auto release = [&](uint32_t sl) {
+    const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
+    for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[sl]);
+  };
+  uint32_t prev = 0;
   bool sfail = false;
   for (int p0 = lo; p0 < chi; p0 += PB) {
     const int n = min(PB, chi - p0);
@@ -1272,20 +1297,19 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
       sfail = true;
       break;
     }
+    // every warp is past the previous stage: release it
+    if (elected && p0 > lo) release(prev);
     const int nv = min(16, n - tile * 16);
     if (nv > 0) {
       kb = smem_u32(sm.ring[slot]) + (uint32_t)(tile * 16) * 128u;  // tiles start on 1024-byte boundaries
       vb = kb + (uint32_t)(STAGE_BYTES / 2);
       run_tile(nv);
     }
-    consumer_sync();
-    if (elected) {
-      const int arrivals = g.batched ? 1 : CONSUMER_WARPS;
-      for (int a = 0; a < arrivals; ++a) mbar_arrive(&sm.empty[slot]);
-    }
+    prev = slot;
     cstage = cs + 1u;
   }
   if (consumer_sync_or(sfail)) return false;
+  if (elected && chi > lo) release(prev);
   if (tile == 0 && nin > 0) {
     // the iteration's own rows
     own = nin;

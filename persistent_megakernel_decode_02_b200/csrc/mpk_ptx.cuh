@@ -264,6 +264,11 @@ __device__ __forceinline__ uint32_t word_tag(uint64_t w) { return (uint32_t)(w >
 // of the tensor-core path).
 __device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 2, %0;" ::"r"(128) : "memory"); }
 
+// Named barrier `id` over `threads` threads (a multiple of 32).
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Named barrier 1 over the 256 consumer threads (the producer warp never joins).
 __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(256) : "memory");
