@@ -100,10 +100,11 @@ typedef enum {
      * inputs = q fp32 [R,Hq*d], k fp32 [R,Hkv*d], v fp32 [R,Hkv*d];
      * weights = q_norm bf16 [d], k_norm bf16 [d], k_cache, v_cache bf16
      * [L,R,Hkv,S,d]; outputs[0] = o fp32 [R,Hq*d].  layer selects the cache
-     * slice; rope_theta the RoPE base.  grid_dim = (Hkv, C, R): task
-     * (j, c, r) attends to chunk c of C of request r's positions (a split
-     * that never depends on the other requests); a request that is not active
-     * publishes zeros as its output. */
+     * slice; rope_theta the RoPE base.  grid_dim = (Hkv, C, R), C <= 256:
+     * task (j, c, r) attends to chunk c of C of request r's positions (a
+     * split that never depends on the other requests); a request that is not
+     * active publishes zeros as its output.  With a prefill graph the cache
+     * holds the graph's requests (Rq of them, dims[1]), R is the column count. */
     MPK_OP_ATTENTION = 3,
     /* x += W a.  inputs[0] = a fp32 [R,K]; weights[0] = W bf16 [N,K];
      * outputs[0] = x fp32 [R,N] (read and written in place).  When K exceeds
@@ -188,12 +189,14 @@ typedef struct {
     int32_t max_timeline;   /* timeline entries kept when profiling (<=0: 1<<20)         */
     int32_t prefetch_kb;    /* L2 prefetch distance per worker ahead of the shared-memory
                                weight ring, KiB (<=0: off)                                 */
-    int32_t dynamic_tasks;  /* > 0: the GEMV operations (all but the fused projections +
-                               attention) hand their tasks out through a shared counter:
-                               each worker claims the next task when its weight ring has
-                               room, so the work follows the workers that are ahead;
-                               <= 0 (default): fixed mapping, task t on worker
-                               (t + offset) % W.  Results are identical either way.     */
+    int32_t dynamic_tasks;  /* > 0: the one-request GEMV operations (all but the fused
+                               projections + attention) hand their tasks out through a
+                               shared counter: each worker claims the next task when its
+                               weight ring has room, so the work follows the workers that
+                               are ahead; <= 0 (default): fixed mapping, task t on worker
+                               (t + offset) % W.  The tensor-core projections over several
+                               requests are always claimed this way.  Results are
+                               identical either way.                                     */
     int32_t debug_stall_op; /* fault injection for tests: k > 0 makes operation k-1 wait
                                for an input nothing will produce (a version of the next
                                iteration, or one completion more than its dependency

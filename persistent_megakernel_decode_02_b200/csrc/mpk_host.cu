@@ -626,6 +626,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         const int gx = Ly.grid_dim.x, gy = Ly.grid_dim.y > 0 ? Ly.grid_dim.y : 1, gz = Ly.grid_dim.z > 0 ? Ly.grid_dim.z : 1;
         SHAPE_CHECK(gx == Hkv && gz == R, "layer %d: ATTENTION needs grid_dim = (kv_heads=%d, chunks, requests=%d)", li,
                     Hkv, R);
+        SHAPE_CHECK(gy >= 1 && gy <= MAX_SPLIT_CHUNKS, "layer %d: %d attention chunks (1..%d)", li, gy,
+                    MAX_SPLIT_CHUNKS);
         op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = gy;
         op.L = (int)kc->dims[0];
         op.S = (int)kc->dims[3];
@@ -829,15 +831,19 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       }
     }
   }
-  // Plain GEMV operations are claimed dynamically (tasks of an op are shared
-  // out by a counter, so workers that finish the previous op early take more);
-  // the fused projections+attention op keeps its fixed task-to-worker mapping
-  // (its group tasks wait on one another).
+  // Projections may be claimed dynamically: an op's tasks are shared out by a
+  // counter, so workers that finish the previous op early take them first and
+  // a worker that runs late takes fewer (or, with fewer tasks than workers,
+  // none).  The tensor-core projections over several requests always are (a
+  // late worker would otherwise stay late: the last segment task of a split
+  // reduction to arrive runs the row block's epilogue); the one-request GEMV
+  // operations when the options ask for it.  Attention keeps its fixed
+  // task-to-worker mapping (the fused op's group tasks wait on one another).
   for (int p = 0; p < P; ++p) {
     OpDesc& op = ops[p];
-    op.dynamic = (o.dynamic_tasks > 0) && !op.batched &&
-                 (op.kind == TK_NORM_GEMV || op.kind == TK_GEMV_RESID || op.kind == TK_NORM_GEMV_SILU ||
-                  op.kind == TK_NORM_GEMV_ARGMAX) ? 1 : 0;
+    const bool proj = op.kind == TK_NORM_GEMV || op.kind == TK_GEMV_RESID || op.kind == TK_NORM_GEMV_SILU ||
+                      op.kind == TK_NORM_GEMV_ARGMAX;
+    op.dynamic = proj && (op.batched || o.dynamic_tasks > 0) ? 1 : 0;
     if (op.dynamic && op.ntasks >= (int)TASK_CLAIM)
       return fail(c, MPK_ERR_INVALID_ARG, "layer %d: at most %u tasks", p, TASK_CLAIM - 1);
   }

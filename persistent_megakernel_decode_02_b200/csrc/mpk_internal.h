@@ -41,6 +41,7 @@ constexpr int MAX_KSPLIT = 8;               // reduction segments of one split r
 constexpr int MAX_G = 8;                    // query heads per kv head
 constexpr int MAX_D = 128;                  // head dim
 constexpr int MAX_GCHUNK = 8;               // fused op: attention chunks per kv head (tasks 0.. of the group)
+constexpr int MAX_SPLIT_CHUNKS = 256;       // split-K op: chunks per (request, kv head) (the merge's weights fit the scratch)
 constexpr int SCHED_WARPS_PER_SM = 4;
 
 // Tensor-core path (an operation over 2..MAX_BATCH requests): every

@@ -45,6 +45,8 @@ struct AttnScratch {
   float4 xs[CONSUMER_WARPS * 32];                // tensor-core path: partial scores exchanged by a tile's two warps
 };
 static_assert(MAX_G * MAX_D / 2 >= 512, "attention scratch");
+static_assert(CONSUMER_WARPS * (MAX_G * MAX_D / 2) >= 2 * (MAX_G / 2) * MAX_SPLIT_CHUNKS + MAX_G / 2,
+              "the split merge's chunk weights and sums fit the per-warp output scratch (G <= 4)");
 static_assert(sizeof(AttnScratch) >= sizeof(float) * MAX_GCHUNK * (MAX_G / 2) * (MAX_D + 2),
               "the group merge gathers every chunk partial of a kv head into the attention scratch");
 
@@ -1708,29 +1710,47 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   if (sm.last) {
     if (active) {
       __threadfence();
-      // one pass over the chunk partials, in chunk order (online rescaling)
+      // The chunk partials of the group's heads: first every chunk's (max,
+      // sum) into shared memory and, per head, the weights exp2(m_c - M) and
+      // the total sum; then each output element over the chunks in order,
+      // eight loads in flight at a time (not one dependent round trip per
+      // chunk).  The block merge's scratch is free again.
+      float* mw = A.wacc[0];  // [G][C] maxima, then weights; [G][C] sums; [G] totals
+      const int nml = G * C;
+      for (int u = ctid; u < nml; u += CONSUMER_THREADS) {
+        const float* p = pbase + ((size_t)(u / C) * CS + (u % C)) * (D + 2);
+        mw[u] = __ldcg(p);
+        mw[nml + u] = __ldcg(p + 1);
+      }
+      consumer_sync();
+      if (ctid < G) {
+        float M = -INFINITY, Ls = 0.f;
+        for (int cc = 0; cc < C; ++cc) M = fmaxf(M, mw[ctid * C + cc]);
+        for (int cc = 0; cc < C; ++cc) {
+          const float mc = mw[ctid * C + cc];
+          const float f = mc == -INFINITY ? 0.f : exp2f(mc - M);  // an empty chunk weighs 0
+          mw[ctid * C + cc] = f;
+          Ls = fmaf(mw[nml + ctid * C + cc], f, Ls);
+        }
+        mw[2 * nml + ctid] = Ls;
+      }
+      consumer_sync();
       for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
         const int hh = idx / D, i = idx % D;
-        const float* p = pbase + (size_t)hh * CS * (D + 2);
-        float M = -INFINITY, Ls = 0.f, Os = 0.f;
-#pragma unroll 4
-        for (int cc = 0; cc < C; ++cc) {
-          const float mc = __ldcg(p + (size_t)cc * (D + 2));
-          const float lc = __ldcg(p + (size_t)cc * (D + 2) + 1);
-          const float oc = __ldcg(p + (size_t)cc * (D + 2) + 2 + i);
-          if (mc == -INFINITY) continue;
-          if (mc > M) {
-            const float sc = exp2f(M - mc);  // M = -inf -> 0
-            Ls *= sc;
-            Os *= sc;
-            M = mc;
-          }
-          const float f = exp2f(mc - M);
-          Ls = fmaf(lc, f, Ls);
-          Os = fmaf(oc, f, Os);
+        const float* p = pbase + (size_t)hh * CS * (D + 2) + 2 + i;
+        const float* wgt = mw + hh * C;
+        float Os = 0.f;
+        for (int c0 = 0; c0 < C; c0 += 8) {
+          float ov[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) ov[u] = c0 + u < C ? __ldcg(p + (size_t)(c0 + u) * (D + 2)) : 0.f;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (c0 + u < C) Os = fmaf(ov[u], wgt[c0 + u], Os);
         }
-        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, Os / Ls, mytag);
-        if (op.xb_out != nullptr) publish_xb(op, (j * G + hh) * D + i, r, Os / Ls);
+        const float ov = Os / mw[2 * nml + hh];
+        st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, ov, mytag);
+        if (op.xb_out != nullptr) publish_xb(op, (j * G + hh) * D + i, r, ov);
       }
     } else {
       // an inactive request still publishes this iteration's version of its

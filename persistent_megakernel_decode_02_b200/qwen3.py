@@ -74,6 +74,21 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[i
     return best[1], best[2]
 
 
+def lm_head_grid(rows: int, K: int, workers: int) -> Tuple[int, int]:
+    """grid_dim of the LM head over several requests: no split of the
+    reduction (the argmax needs whole logits, and a split's last arrival runs
+    the epilogue late) and tasks for about five sixths of the workers, so the
+    workers that finish the last layer late claim none (measured on the 8B
+    shape with 8 requests: (120, 1) at 5.43 ms/step against 5.49 for the
+    batched_grid rule's (48, 3)).  Falls back to batched_grid when a task
+    would hold more row blocks than the accumulator slots."""
+    nb = -(-rows // BATCH_BM)
+    gx = max(1, min(nb, (workers * 5) // 6))
+    if -(-(K // BATCH_BK) // BATCH_MAX_KBLOCKS) > 1 and -(-nb // gx) > BATCH_SLOTS:
+        return batched_grid(rows, K, workers)
+    return gx, 1
+
+
 def batched_layer_plan(shape, requests: int, plan_workers: int, attn_chunks: int, block_dim: int = 0,
                        tied: Optional[bool] = None) -> List[dict]:
     """The fused-layer list for several requests: projections on the tensor
@@ -105,7 +120,7 @@ def batched_layer_plan(shape, requests: int, plan_workers: int, attn_chunks: int
                          capture_slot=l + 1))
     plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
                      weight_lm="embed_tokens" if tied else "lm_head", pred="pred",
-                     grid_dim=batched_grid(s.vocab, s.hidden, W), block_dim=block_dim, eps=s.eps))
+                     grid_dim=lm_head_grid(s.vocab, s.hidden, W), block_dim=block_dim, eps=s.eps))
     return plan
 
 

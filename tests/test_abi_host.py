@@ -130,7 +130,8 @@ def test_batched_grid_rule():
     header's geometry for every model shape and worker count: at most one task
     per row block and segment, at most one segment per K block, and a task
     whose segment needs passes holds at most the accumulator slots."""
-    from persistent_megakernel_decode_02_b200.qwen3 import BATCH_BM, BATCH_MAX_KBLOCKS, BATCH_SLOTS, batched_grid
+    from persistent_megakernel_decode_02_b200.qwen3 import (BATCH_BM, BATCH_MAX_KBLOCKS, BATCH_SLOTS, batched_grid,
+                                                            lm_head_grid)
     assert BATCH_BM == _header_define("MPK_BATCH_BM")
     assert BATCH_MAX_KBLOCKS * 64 == _header_define("MPK_BATCH_MAX_PASS_K")
     assert BATCH_SLOTS == _header_define("MPK_BATCH_SLOTS")
@@ -145,6 +146,14 @@ def test_batched_grid_rule():
                 assert 1 <= gx <= nb and 1 <= gy <= nkb
                 if -(-nkb // gy) > BATCH_MAX_KBLOCKS:
                     assert -(-nb // gx) <= BATCH_SLOTS
+        for W in (1, 7, 100, 144, 300):
+            gx, gy = lm_head_grid(shape.vocab, shape.hidden, W)
+            nb, nkb = -(-shape.vocab // BATCH_BM), shape.hidden // 64
+            assert 1 <= gx <= nb and 1 <= gy <= nkb
+            if -(-nkb // gy) > BATCH_MAX_KBLOCKS:
+                assert -(-nb // gx) <= BATCH_SLOTS
+    # the LM head: whole reductions, tasks for five sixths of the workers
+    assert lm_head_grid(151936, 4096, 144) == (120, 1)
     # the 8B plan for 144 workers: one round of tasks for the projections, the
     # reductions split three or four ways
     assert batched_grid(6144, 4096, 144) == (48, 3)

@@ -69,3 +69,38 @@ def test_split_attention_short_contexts():
     ref, _, _, _ = oracle_teacher_forced(shape, w_cpu, tokens, 20)
     compare_captures(gpu, ref)
     dec.kernel.close()
+
+
+def test_split_attention_more_chunks_than_workers():
+    """More chunk tasks than workers (several per worker, each streamed through
+    the ring after the previous one): the chunk partials are merged in chunk
+    order whoever computed them, so the result is bit-identical to op-by-op
+    execution (one block per task) and matches the oracle."""
+    from persistent_megakernel_decode_02_b200 import build_decoder
+    shape = sq.TINY
+    S = 300
+    w_cpu = sq.make_weights(shape, seed=0)
+    w = to_cuda(w_cpu)
+    p0 = np.array([230], np.int32)
+    kc, vc = sq.make_kv_prefill(shape, 1, S, int(p0.max()), seed=44)
+    tokens = sq.make_tokens(shape, 1, S, [S], seed=45, teacher_forced=True)
+    outs = []
+    for mode in ("run", "run_op_by_op"):
+        dec = build_decoder(shape, w, requests=1, max_seq=S, k_cache=kc.cuda(), v_cache=vc.cuda(),
+                            attn_chunks=100, fused_attention=False)
+        assert dec.kernel.num_workers < 100 * shape.kv_heads
+        tok = tokens.cuda()
+        step = torch.from_numpy(p0.copy()).cuda()
+        getattr(dec, mode)(step, tok, step + 4)
+        torch.cuda.synchronize()
+        dec.kernel.check_status()
+        outs.append((step.cpu(), dec.pred.cpu(), dec.k_cache.cpu().view(torch.int16)))
+        dec.kernel.close()
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+    dec = build_decoder(shape, w, requests=1, max_seq=S, k_cache=kc.cuda(), v_cache=vc.cuda(), attn_chunks=100,
+                        fused_attention=False)
+    gpu, _, _ = gpu_teacher_forced(dec, tokens, 3, step0=p0)
+    ref, _, _, _ = oracle_teacher_forced(shape, w_cpu, tokens, 3, _u16(kc), _u16(vc), step0=p0)
+    compare_captures(gpu, ref)
+    dec.kernel.close()
