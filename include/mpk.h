@@ -210,19 +210,21 @@ typedef struct {
                                The RMSNorm factor then scales the input instead of the
                                products, so results agree to rounding, not bit for bit. */
     int32_t prefill_tokens; /* T in 2..MPK_MAX_BATCH: a prefill graph.  Its activations
-                               have T rows, the columns of the tensor-core projections,
-                               and every iteration advances ONE request (tokens [1, S],
-                               step [1], KV cache [L, 1, Hkv, S, d], pred [1, S]) by T
-                               positions: column c consumes tokens[0, step + c], appends
-                               its K/V at step + c and attends to positions 0 .. step + c
-                               (the chunk's earlier positions from this iteration's k and
-                               v, the rest from the cache), so a prompt is ingested T
-                               tokens per iteration instead of one.  Column c's argmax
-                               goes to pred[0, step + c + 1] and to tokens[0, step + c +
-                               1] when that slot holds -1; step advances past the last
-                               active column.  A request's last chunk may be partial
-                               (step_end).  <= 1 (default): one position per request per
-                               iteration.                                                 */
+                               have T rows, the columns of the tensor-core projections;
+                               its KV cache [L, Rq, Hkv, S, d] holds Rq requests (tokens
+                               [Rq, S], step [Rq], pred [Rq, S]), served one after
+                               another in request order.  Every iteration advances ONE
+                               request q by T positions: column c consumes tokens[q,
+                               step[q] + c], appends its K/V there and attends to
+                               positions 0 .. step[q] + c (the chunk's earlier positions
+                               from this iteration's k and v, the rest from the cache),
+                               so a prompt is ingested T tokens per iteration instead of
+                               one.  Column c's argmax goes to pred[q, step[q] + c + 1]
+                               and to tokens[q, step[q] + c + 1] when that slot holds -1;
+                               step[q] advances past the last active column.  A
+                               request's last chunk may be partial (step_end); a request
+                               with step -1 is skipped.  <= 1 (default): one position
+                               per request per iteration.                                 */
 } mpk_options;
 
 /* Library build facts. */
@@ -292,10 +294,10 @@ MPK_API const char *mpk_warnings(mpk_ctx *ctx);
  * cudaStream_t; NULL = legacy default stream), asynchronously.  step: device
  * int32 [R]; tokens: device int64 [R,S] (R = num_requests, S = seq_length)
  * with -1 in slots to generate; step_end: device int32 [R] or NULL.  R must
- * equal the graph's request count (a prefill graph: 1) and S-1 must not
+ * equal the graph's request count (a prefill graph: its cache's) and S-1 must not
  * exceed the KV cache length; an attached pred tensor must be [R,S].  A
- * prefill graph (mpk_options.prefill_tokens = T) advances its request by T
- * positions per iteration, each position with the semantics below.  Request r takes
+ * prefill graph (mpk_options.prefill_tokens = T) advances one request at a
+ * time by T positions per iteration, each position with the semantics below.  Request r takes
  * part in iterations while step[r] < min(step_end[r], S-1) (NULL: S-1); each
  * iteration consumes tokens[r, step[r]], appends K/V at that position and
  * advances step[r] by one ([EN] "How MPK Works": step and tokens are the meta
