@@ -35,7 +35,7 @@
 extern "C" {
 #endif
 
-#define MPK_ABI_VERSION 3
+#define MPK_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MPK_API __attribute__((visibility("default")))
@@ -225,6 +225,18 @@ typedef struct {
                                request's last chunk may be partial (step_end); a request
                                with step -1 is skipped.  <= 1 (default): one position
                                per request per iteration.                                 */
+    int32_t kv_page_size;   /* > 0: paged KV caches for the ATTENTION operations.  The
+                               caches are [L, P, Hkv, kv_page_size, d] (P pages shared by
+                               all requests) and an MPK_INT32 tensor named "kv_pages",
+                               [R, max_pages], maps page i of request r (positions
+                               i * kv_page_size ..) to its page of the caches; the
+                               longest sequence is max_pages * kv_page_size positions.
+                               kv_page_size must be a multiple of 128.  A page index
+                               outside 0..P-1 ends the run with MPK_ERR_DEVICE (nothing
+                               is read or written there).  The fused projections +
+                               attention operation needs a contiguous cache
+                               (UNSUPPORTED otherwise).  <= 0 (default): contiguous
+                               caches [L, R, Hkv, S, d].                                  */
 } mpk_options;
 
 /* Library build facts. */

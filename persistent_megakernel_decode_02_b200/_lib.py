@@ -57,6 +57,7 @@ class Options(ctypes.Structure):
         ("debug_stall_op", ctypes.c_int32),
         ("poll_inputs", ctypes.c_int32),
         ("prefill_tokens", ctypes.c_int32),
+        ("kv_page_size", ctypes.c_int32),
     ]
 
 

@@ -408,6 +408,18 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   // of the KV cache, which may hold any number of requests (Rq)
   const int PF = o.prefill_tokens > 1 ? o.prefill_tokens : 0;
   int Rq = -1;
+  // paged KV caches: [L, pages, Hkv, PG, d] and the page table "kv_pages"
+  // [requests, max_pages] (int32)
+  const int PG = o.kv_page_size > 0 ? o.kv_page_size : 0;
+  const Tensor* kvp = nullptr;
+  if (PG) {
+    if (PG % 128 != 0)
+      return fail(c, MPK_ERR_INVALID_ARG, "kv_page_size %d is not a multiple of 128", PG);
+    int rc_ = need(c, -1, "page table", "kv_pages", MPK_INT32, 2, &kvp);
+    if (rc_ != MPK_OK) return rc_;
+    if (kvp->dims[0] < 1 || kvp->dims[1] < 1 || (int64_t)kvp->dims[1] * PG >= ((int64_t)1 << 31))
+      return fail(c, MPK_ERR_SHAPE, "kv_pages %s", dims_str(kvp->dims).c_str());
+  }
 
   std::vector<OpDesc> ops(n_layers);
   int R = -1, H = -1, V = -1, L = -1, S = -1, pred_rows = -1;
@@ -613,10 +625,15 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
         SHAPE_CHECK(o->dims[1] == q->dims[1], "layer %d: o %s vs q %s", li, dims_str(o->dims).c_str(),
                     dims_str(q->dims).c_str());
         if (R < 0) R = (int)q->dims[0];
-        if (Rq < 0) Rq = (int)kc->dims[1];
+        // requests of the cache: its second extent, or the page table's rows
+        const int64_t creq = PG ? kvp->dims[0] : kc->dims[1];
+        if (Rq < 0) Rq = (int)creq;
         SHAPE_CHECK(q->dims[0] == R && k->dims[0] == R && v->dims[0] == R && o->dims[0] == R &&
-                        kc->dims[1] == (PF ? Rq : R),
-                    "layer %d: request count mismatch (graph %d, cache %lld)", li, R, (long long)kc->dims[1]);
+                        creq == (PF ? Rq : R),
+                    "layer %d: request count mismatch (graph %d, cache %lld)", li, R, (long long)creq);
+        if (PG)
+          SHAPE_CHECK(kc->dims[3] == PG, "layer %d: paged caches %s need pages of kv_page_size = %d positions", li,
+                      dims_str(kc->dims).c_str(), PG);
         SHAPE_CHECK(Ly.layer >= 0 && Ly.layer < kc->dims[0], "layer %d: cache layer %d out of range %lld", li, Ly.layer,
                     (long long)kc->dims[0]);
         const int G = Hq / Hkv;
@@ -630,7 +647,13 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
                     MAX_SPLIT_CHUNKS);
         op.Hq = Hq; op.Hkv = Hkv; op.d = d; op.G = G; op.C = gy;
         op.L = (int)kc->dims[0];
-        op.S = (int)kc->dims[3];
+        op.S = PG ? (int)(kvp->dims[1] * PG) : (int)kc->dims[3];  // positions per request
+        if (PG) {
+          op.page = PG;
+          op.npages = (int)kc->dims[1];
+          op.max_pages = (int)kvp->dims[1];
+          op.kv_pages = (const int32_t*)kvp->ptr;
+        }
         op.layer = Ly.layer;
         op.q = (const uint64_t*)q->ptr; op.k = (const uint64_t*)k->ptr; op.v = (const uint64_t*)v->ptr;
         op.qn_w = (const uint16_t*)qn->ptr; op.kn_w = (const uint16_t*)kn->ptr;
@@ -656,6 +679,10 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       }
       case MPK_OP_RMSNORM_QKV_ATTENTION: {
         op.kind = TK_QKV_ATTN;
+        if (PG)
+          return fail(c, MPK_ERR_UNSUPPORTED,
+                      "layer %d: the fused projections + attention operation needs a contiguous KV cache (kv_page_size "
+                      "= 0); paged caches take RMSNORM_LINEAR + ATTENTION", li);
         const Tensor *x, *wn, *wq, *wk, *wv, *qn, *kn, *kc, *vc, *q, *k, *v, *o;
         NEED("inputs[0] (x)", Ly.inputs[0], MPK_FP32T, 2, &x);
         NEED("weights[0] (norm)", Ly.weights[0], MPK_BF16, 1, &wn);
@@ -950,7 +977,8 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   for (int p = 0; p < P; ++p) {
     const OpDesc& op = ops[p];
     if (op.kind == TK_ATTN) {
-      const int64_t rows = (int64_t)op.L * Rq * op.Hkv * op.S;
+      const int64_t rows = op.page > 0 ? (int64_t)op.L * op.npages * op.Hkv * op.page
+                                       : (int64_t)op.L * Rq * op.Hkv * op.S;
       if (rows >= ((int64_t)1 << 31))
         return fail(c, MPK_ERR_UNSUPPORTED, "op %d: a KV cache of %lld rows of d (at most 2^31 - 1)", p,
                     (long long)rows);
@@ -1262,8 +1290,8 @@ int mpk_status(mpk_ctx* c) {
   static const char* where[] = {"?", "worker dependency wait", "producer queue wait", "weight ring wait",
                                 "task fifo wait", "scheduler gate wait", "scheduler queue space wait", "start",
                                 "embedding token check", "task dispatch", "iteration boundary",
-                                "tagged input wait"};
-  const char* w = (st.where >= 0 && st.where < 12) ? where[st.where] : "?";
+                                "tagged input wait", "KV page table check"};
+  const char* w = (st.where >= 0 && st.where < 13) ? where[st.where] : "?";
   fail(c, st.code, "device status %d at %s: op %d task %d worker %d iter %d observed %u expected %u", st.code, w, st.op,
        st.task, st.worker, st.iter, st.observed, st.expected);
   return st.code;

@@ -114,10 +114,16 @@ struct OpDesc {
   const uint16_t* kn_w;
   uint16_t* kc;
   uint16_t* vc;
-  // split-K operation: tensor maps of the caches viewed as [L*R*Hkv*S rows, d]
-  // bf16, boxes of 64 elements x (STAGE_BYTES / (4 d)) rows, 128-byte swizzle
+  // split-K operation: tensor maps of the caches viewed as [rows, d] bf16
+  // (rows = L*R*Hkv*S, paged: L*npages*Hkv*page), boxes of 64 elements x
+  // (STAGE_BYTES / (4 d)) rows, 128-byte swizzle
   const void* tmap_kc;
   const void* tmap_vc;
+  // paged caches (split-K operation): page > 0 positions per page; the caches
+  // are [L][npages][Hkv][page][d] and position p of request q lives in page
+  // kv_pages[q * max_pages + p / page] at row p % page
+  const int32_t* kv_pages;
+  int32_t page, npages, max_pages;
   float* part;                  // [R][Hq][C][d + 2]
   uint64_t* gpart;              // group mode: tagged chunk partials [Hkv][C][G][d + 2]
   int32_t group_sync;           // fused op: every task of a group attends to a chunk (tasks <= workers)
@@ -177,7 +183,8 @@ struct OpDesc {
 
 struct Status {
   int32_t code;      // 0 ok, else negative mpk_error
-  int32_t where;     // 1 worker dep, 2 producer queue, 3 producer ring, 4 consumer fifo, 5 scheduler gate, 6 scheduler space, 7 start
+  int32_t where;     // 1 worker dep, 2 producer queue, 3 producer ring, 4 consumer fifo, 5 scheduler gate, 6 scheduler space, 7 start,
+                     // 8 token check, 9 task dispatch, 10 iteration boundary, 11 tagged input, 12 KV page check
   int32_t op, task, worker, iter;
   uint32_t observed, expected;
 };

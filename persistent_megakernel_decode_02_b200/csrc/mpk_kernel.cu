@@ -349,6 +349,38 @@ __device__ __forceinline__ bool request_state(const Graph& g, int r, uint32_t it
 // position): prefill columns r' < r hold positions chunk0 .. s - 1.
 __device__ __forceinline__ int chunk0(const Graph& g, int r, int s) { return s - (g.prefill ? r : 0); }
 
+// Row of the split-K operation's cache, viewed as [rows, d], that holds
+// position p of request q and kv head j; -1 when a paged cache's page table
+// names no page of the cache there (the caller records the error).
+__device__ __forceinline__ int kv_row(const Graph& g, const OpDesc& op, int q, int j, int p) {
+  if (op.page == 0) return ((op.layer * g.Rq + q) * op.Hkv + j) * op.S + p;
+  const int pg = __ldg(op.kv_pages + q * op.max_pages + p / op.page);
+  if (pg < 0 || pg >= op.npages) return -1;
+  return ((op.layer * op.npages + pg) * op.Hkv + j) * op.page + p % op.page;
+}
+
+// Positions [lo, hi) of chunk c of C of a split-K task over npos positions:
+// an even split; with a paged cache the inner boundaries are rounded down to a
+// multiple of the stage length PB, so that every stage but a chunk's last is
+// whole (the chunks still cover 0..npos-1 once, the last one ends at npos).
+__device__ __forceinline__ void chunk_bounds(const OpDesc& op, int c, int C, int npos, int& lo, int& hi) {
+  lo = (int)(((long long)c * npos) / C);
+  hi = (int)(((long long)(c + 1) * npos) / C);
+  if (op.page > 0) {
+    const int PB = STAGE_BYTES / (4 * op.d);
+    lo = lo / PB * PB;
+    if (c + 1 < C) hi = hi / PB * PB;
+  }
+}
+
+// End of the stage that starts at position p of a split-K chunk ending at
+// hi: PB positions on; with a paged cache up to the next multiple of PB (the
+// page size is a multiple of PB, so no stage straddles two pages).
+__device__ __forceinline__ int attn_stage_end(const OpDesc& op, int p, int hi, int PB) {
+  const int e = op.page > 0 ? (p / PB + 1) * PB : p + PB;
+  return e < hi ? e : hi;
+}
+
 // Locate global row `row` of a stacked multi-matrix operation.
 __device__ __forceinline__ int seg_of(const OpDesc& op, int row) {
   int s = 0;
@@ -449,11 +481,12 @@ __device__ __forceinline__ uint32_t attn_stages(const Graph& g, const OpDesc& op
   int r, c, Cr, s;
   if (!attn_slot(g, op, task / op.Hkv, iter, r, c, Cr) || !request_state(g, r, iter, s)) return 0u;
   const int npos = s + 1, sc0 = chunk0(g, r, s);
-  const int lo = (int)(((long long)c * npos) / Cr);
-  int hi = (int)(((long long)(c + 1) * npos) / Cr);
+  int lo, hi;
+  chunk_bounds(op, c, Cr, npos, lo, hi);
   hi = hi < sc0 ? hi : sc0;
   const int PB = STAGE_BYTES / (4 * op.d);
-  return hi > lo ? (uint32_t)((hi - lo + PB - 1) / PB) : 0u;
+  if (hi <= lo) return 0u;
+  return op.page > 0 ? (uint32_t)((hi - 1) / PB - lo / PB + 1) : (uint32_t)((hi - lo + PB - 1) / PB);
 }
 
 // Producer side of a split-K attention task: the cached positions of its
@@ -473,8 +506,8 @@ __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc
   int s, q;
   if (!request_state(g, r, iter, s, q)) return true;
   const int npos = s + 1, sc0 = chunk0(g, r, s);
-  const int lo = (int)(((long long)c * npos) / Cr);
-  int hi = (int)(((long long)(c + 1) * npos) / Cr);
+  int lo, hi;
+  chunk_bounds(op, c, Cr, npos, lo, hi);
   hi = hi < sc0 ? hi : sc0;
   if (hi <= lo) return true;
   if (iter > 0) {
@@ -487,14 +520,18 @@ __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc
     fence_proxy_async_global();
   }
   const int D = op.d, PB = STAGE_BYTES / (4 * D);
-  const int row0 = ((op.layer * g.Rq + q) * op.Hkv + j) * op.S;  // < 2^31 (checked on the host)
-  for (int p = lo; p < hi; p += PB) {
+  for (int p = lo; p < hi; p = attn_stage_end(op, p, hi, PB)) {
+    const int row = kv_row(g, op, q, j, p);  // rows < 2^31 (checked on the host)
+    if (row < 0) {
+      record_error(g, -11 /*DEVICE*/, 12, op.self, task, worker, (int)iter, (uint32_t)q, (uint32_t)p);
+      return false;
+    }
     const uint32_t slot = pstage % (uint32_t)nr;
     if (!wait_mbar(g, &sm.empty[slot], ((pstage / (uint32_t)nr) & 1u) ^ 1u, 3, worker)) return false;
     mbar_arrive_expect_tx(&sm.full[slot], (uint32_t)STAGE_BYTES);
     for (int h = 0; h < D / 64; ++h) {
-      tma_load_2d(sm.ring[slot] + h * PB * 128, op.tmap_kc, h * 64, row0 + p, &sm.full[slot], pol);
-      tma_load_2d(sm.ring[slot] + STAGE_BYTES / 2 + h * PB * 128, op.tmap_vc, h * 64, row0 + p, &sm.full[slot], pol);
+      tma_load_2d(sm.ring[slot] + h * PB * 128, op.tmap_kc, h * 64, row, &sm.full[slot], pol);
+      tma_load_2d(sm.ring[slot] + STAGE_BYTES / 2 + h * PB * 128, op.tmap_vc, h * 64, row, &sm.full[slot], pol);
     }
     ++pstage;
   }
@@ -1142,7 +1179,8 @@ __device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32
 //    column h the hi part and column h + 4 the lo part of head h.
 // The warp's (max, sum, output) go to A.wm / A.wacc for the block merge.
 template <int G, int D>
-__device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnScratch& A, int lo, int chi, int a0r,
+__device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, const OpDesc& op, AttnScratch& A, int lo,
+                                                int chi, int a0r,
                                                 int nin, const uint16_t* KX, const uint16_t* VX, int cw, int lane,
                                                 int worker, uint32_t& cstage) {
   constexpr int PB = STAGE_BYTES / (4 * D);  // positions per stage
@@ -1289,8 +1327,8 @@ __device__ __forceinline__ bool attn_stream_mma(Smem& sm, const Graph& g, AttnSc
   };
   uint32_t prev = 0;
   bool sfail = false;
-  for (int p0 = lo; p0 < chi; p0 += PB) {
-    const int n = min(PB, chi - p0);
+  for (int p0 = lo; p0 < chi; p0 = attn_stage_end(op, p0, chi, PB)) {
+    const int n = attn_stage_end(op, p0, chi, PB) - p0;
     const uint32_t cs = cstage;
     const uint32_t slot = cs % (uint32_t)nr;
     bool okk = true;
@@ -1367,7 +1405,8 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   const int ctid = cw * 32 + lane;
   const int Hkv = op.Hkv;
   AttnScratch& A = sm.u.a;
-  size_t kvbase = ((((size_t)op.layer * g.Rq + r) * Hkv + j) * (size_t)op.S) * D;  // set below for prefill
+  // the fused operation's cache rows (one request, contiguous cache)
+  size_t kvbase = ((((size_t)op.layer * g.Rq + r) * Hkv + j) * (size_t)op.S) * D;
   // k and v (bf16, k normalised and rotated) of the positions the iteration
   // itself produces: row 0 the task's own position (A.ks, A.vs); prefill: row
   // c the position of column c of the chunk, in the ring stage that the
@@ -1397,6 +1436,8 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   }
   int s;
   bool active;
+  bool afail = false;
+  size_t sdst = 0;  // element offset of position s in the caches (the append)
   if (fused) {
     // fused with the projections: state fetched in that task's prologue
     s = sm.attn_s;
@@ -1404,9 +1445,20 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   } else {
     int q;
     active = request_state(g, r, iter, s, q);
-    kvbase = ((((size_t)op.layer * g.Rq + q) * Hkv + j) * (size_t)op.S) * D;
+    if constexpr (STREAMED) {
+      if (active) {
+        const int row = kv_row(g, op, q, j, s);
+        if (row < 0) {
+          if (ctid == 0) record_error(g, -11 /*DEVICE*/, 12, op.self, -1, worker, (int)iter, (uint32_t)q, (uint32_t)s);
+          afail = true;
+        } else {
+          sdst = (size_t)row * D;
+        }
+      }
+    } else {
+      kvbase = ((((size_t)op.layer * g.Rq + q) * Hkv + j) * (size_t)op.S) * D;
+    }
   }
-  bool afail = false;
   if (active && prow < G + 2) {
     // q, k, v of this iteration (their tags), then the cache: positions below
     // s were appended by this operation's attention tasks of earlier
@@ -1424,8 +1476,13 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
 
   if (active) {
     const int npos = s + 1;
-    const int lo = (int)(((long long)c * npos) / C);
-    const int hi = (int)(((long long)(c + 1) * npos) / C);
+    int lo, hi;
+    if constexpr (STREAMED) {
+      chunk_bounds(op, c, C, npos, lo, hi);
+    } else {
+      lo = (int)(((long long)c * npos) / C);
+      hi = (int)(((long long)(c + 1) * npos) / C);
+    }
     if (prow < G + 2) {
       if (prow <= G) {
         float2 rc[EL / 2];
@@ -1507,7 +1564,9 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       // append k (first D/8 threads) and v (next D/8) at position s: 16 B each
       const int half = D / 8;
       const int which = ctid / half, q8 = ctid % half;
-      uint16_t* dst = (which == 0 ? op.kc : op.vc) + kvbase + (size_t)s * D + q8 * 8;
+      uint16_t* dst;
+      if constexpr (STREAMED) dst = (which == 0 ? op.kc : op.vc) + sdst + q8 * 8;
+      else dst = (which == 0 ? op.kc : op.vc) + kvbase + (size_t)s * D + q8 * 8;
       const uint16_t* srcs = (which == 0 ? KX : VX) + own * D + q8 * 8;
       *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(srcs);
     }
@@ -1521,7 +1580,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
       const int sc0 = chunk0(g, r, s);
       const int chi = hi < sc0 ? hi : sc0;
       const int a0 = lo > sc0 ? lo : sc0;
-      if (!attn_stream_mma<G, D>(sm, g, A, lo, chi, a0 - sc0, hi - a0, KX, VX, cw, lane, worker, cstage))
+      if (!attn_stream_mma<G, D>(sm, g, op, A, lo, chi, a0 - sc0, hi - a0, KX, VX, cw, lane, worker, cstage))
         return false;
     } else {
       // fused operation: the positions straight from the cache (and s from

@@ -186,11 +186,12 @@ class PersistentKernel:
     # ------------------------------------------------------------------ compile / run
     def compile(self, profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                 max_timeline: int = 0, prefetch_kb: int = 0, debug_stall_op: int = 0,
-                dynamic_tasks: bool = False, poll_inputs: bool = False, prefill_tokens: int = 0) -> str:
+                dynamic_tasks: bool = False, poll_inputs: bool = False, prefill_tokens: int = 0,
+                kv_page_size: int = 0) -> str:
         arr = (_lib.Layer * len(self._layers))(*self._layers)
         opts = _lib.Options(int(profiling), int(sched_lookahead), float(timeout_s), int(max_timeline),
                             int(prefetch_kb), 1 if dynamic_tasks else 0, int(debug_stall_op),
-                            1 if poll_inputs else 0, int(prefill_tokens))
+                            1 if poll_inputs else 0, int(prefill_tokens), int(kv_page_size))
         check(self._lib.mpk_compile(self._ctx, arr, len(self._layers), ctypes.byref(opts)), self._ctx)
         self._keep.append(arr)
         self.compiled = True

@@ -193,6 +193,7 @@ class Decoder:
     v_cache: torch.Tensor
     pred: torch.Tensor
     buffers: Dict[str, torch.Tensor]
+    kv_pages: Optional[torch.Tensor] = None  # paged caches: the page table
 
     def run(self, step, tokens, step_end=None, stream=None):
         self.kernel(step, tokens, step_end, stream)
@@ -208,7 +209,8 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
                   profiling: bool = False, sched_lookahead: int = 0, timeout_s: float = 0.0,
                   prefetch_kb: int = 0, fused_attention: Optional[bool] = None,
                   debug_stall_op: int = 0, dynamic_tasks: bool = False, tasks_per_worker: int = 2,
-                  poll_inputs: bool = False, prefill_tokens: int = 0) -> Decoder:
+                  poll_inputs: bool = False, prefill_tokens: int = 0, kv_page_size: int = 0,
+                  kv_pages: Optional[torch.Tensor] = None, num_pages: Optional[int] = None) -> Decoder:
     """Attach the weights (bf16 CUDA tensors keyed as in synth.qwen3), allocate the
     activations and compile the task graph.  max_seq = KV-cache positions = the
     tokens' row length (seq_length).  fused_attention: None picks the fused
@@ -219,7 +221,13 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
     T consecutive prompt positions of one request as the T columns of the
     tensor-core projections (mpk_options.prefill_tokens), the requests one
     after another.  Pass the decode graph's caches as k_cache / v_cache (and
-    the same `requests`) to continue decoding from the prefilled state."""
+    the same `requests`) to continue decoding from the prefilled state.
+
+    kv_page_size = P > 0 (a multiple of 128) makes the KV caches paged
+    (mpk_options.kv_page_size): k_cache / v_cache are [L, num_pages, Hkv, P, d]
+    and kv_pages (int32 [requests, ceil(max_seq / P)], default: request r's
+    pages r * max_pages ..) maps each request's logical pages to cache pages;
+    the attention is then the split-K operation."""
     from . import _lib
 
     s = shape
@@ -233,6 +241,17 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
         mk.attach_input(t, name)
     dev = next(iter(weights.values())).device
     kv_shape = (s.layers, requests, s.kv_heads, max_seq, s.head_dim)
+    if kv_page_size > 0:
+        if fused_attention:
+            raise ValueError("paged KV caches take the split-K attention operation")
+        fused_attention = False
+        max_pages = -(-max_seq // kv_page_size)
+        if kv_pages is None:
+            kv_pages = torch.arange(requests * max_pages, dtype=torch.int32, device=dev).view(requests, max_pages)
+        if num_pages is None:
+            num_pages = requests * max_pages
+        kv_shape = (s.layers, num_pages, s.kv_heads, kv_page_size, s.head_dim)
+        mk.attach_input(kv_pages, "kv_pages")
     if k_cache is None:
         k_cache = torch.zeros(kv_shape, dtype=torch.bfloat16, device=dev)
     if v_cache is None:
@@ -259,5 +278,5 @@ def build_decoder(shape, weights: Dict[str, torch.Tensor], requests: int, max_se
         getattr(mk, op.pop("method"))(**op)
     mk.compile(profiling=profiling, sched_lookahead=sched_lookahead, timeout_s=timeout_s, prefetch_kb=prefetch_kb,
                debug_stall_op=debug_stall_op, dynamic_tasks=dynamic_tasks, poll_inputs=poll_inputs,
-               prefill_tokens=prefill_tokens if prefill_tokens > 1 else 0)
-    return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs)
+               prefill_tokens=prefill_tokens if prefill_tokens > 1 else 0, kv_page_size=max(0, kv_page_size))
+    return Decoder(mk, s, requests, max_seq, k_cache, v_cache, pred, bufs, kv_pages)

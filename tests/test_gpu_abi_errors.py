@@ -73,7 +73,7 @@ def _graph(mk, w, drop=(), replace=None):
 def _compile_rc(mk):
     L = _lib()
     arr = (L.Layer * len(mk._layers))(*mk._layers)
-    opts = L.Options(0, 0, 0.0, 0, 0, 0, 0, 0)
+    opts = L.Options()
     return mk._lib.mpk_compile(mk._ctx, arr, len(mk._layers), ctypes.byref(opts))
 
 
