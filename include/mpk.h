@@ -162,13 +162,21 @@ typedef struct { int32_t x, y, z; } mpk_dim3;
  * With gy > 1 the last segment task of a row block to finish adds the partial
  * sums in segment order.  A task whose segment is longer than
  * MPK_BATCH_MAX_PASS_K runs it in passes and then holds at most
- * MPK_BATCH_SLOTS row blocks.  K must be a multiple of 64 and stacked
- * matrices start at multiples of MPK_BATCH_BM rows (MPK_ERR_UNSUPPORTED
- * otherwise); RMSNORM_QKV_ATTENTION takes one request. */
-#define MPK_MAX_BATCH 8
+ * MPK_BATCH_SLOTS row blocks.  Graphs of 9..MPK_MAX_BATCH requests run
+ * every contraction 16 requests wide (the weights are still read once per
+ * iteration); their limits are MPK_BATCH_WIDE_MAX_PASS_K and
+ * MPK_BATCH_WIDE_SLOTS.  K must be a multiple of 64 and stacked matrices
+ * start at multiples of MPK_BATCH_BM rows (MPK_ERR_UNSUPPORTED otherwise);
+ * RMSNORM_QKV_ATTENTION takes one request.  A prefill graph
+ * (mpk_options.prefill_tokens) takes at most MPK_MAX_PREFILL positions per
+ * iteration. */
+#define MPK_MAX_BATCH 16
+#define MPK_MAX_PREFILL 8
 #define MPK_BATCH_BM 128
 #define MPK_BATCH_MAX_PASS_K 1536
 #define MPK_BATCH_SLOTS 16
+#define MPK_BATCH_WIDE_MAX_PASS_K 768
+#define MPK_BATCH_WIDE_SLOTS 8
 typedef struct {
     int32_t op;                         /* mpk_op */
     const char *inputs[MPK_MAX_IO];
@@ -209,7 +217,7 @@ typedef struct {
                                <= 0 (default): published rows wherever the graph allows.
                                The RMSNorm factor then scales the input instead of the
                                products, so results agree to rounding, not bit for bit. */
-    int32_t prefill_tokens; /* T in 2..MPK_MAX_BATCH: a prefill graph.  Its activations
+    int32_t prefill_tokens; /* T in 2..MPK_MAX_PREFILL: a prefill graph.  Its activations
                                have T rows, the columns of the tensor-core projections;
                                its KV cache [L, Rq, Hkv, S, d] holds Rq requests (tokens
                                [Rq, S], step [Rq], pred [Rq, S]), served one after

@@ -12,10 +12,10 @@
 //  * consumers, prologue: the batch's input rows for the task's reduction
 //    segment (after RMSNorm for the norm operations) are split into bf16
 //    hi/lo pairs and written into the ring's remaining stages in the same
-//    swizzled K-major layout: K block b at b * B_KBLOCK_BYTES, the hi rows as
-//    one 8-row atom, the lo rows as the next; request r at 128 r inside an
-//    atom, its 16-byte chunk c at 16 (c ^ r);
-//  * one consumer thread issues the MMAs (M = BM weight rows, N = BN columns,
+//    swizzled K-major layout: K block b at b * KBLOCK_BYTES, the hi rows as
+//    BW / 8 eight-row atoms, the lo rows as as many more; request r's row at
+//    128 r, its 16-byte chunk c at 16 (c ^ (r mod 8));
+//  * one consumer thread issues the MMAs (M = BM weight rows, N = 2 BW columns,
 //    K = 16 per instruction) into a tensor-memory accumulator and commits each
 //    stage back to the producer;
 //  * the first consumer warpgroup reads the accumulator (lane = weight row,
@@ -38,10 +38,13 @@ __device__ __forceinline__ void btask(const OpDesc& op, int task, int& rb0, int&
   kb1 = (int)(((long long)(seg + 1) * op.nkb) / op.bsplit);
 }
 
-// A task's K blocks are processed in passes of at most B_MAX_KBLOCKS (the
+// A task's K blocks are processed in passes of at most MAX_KBLOCKS (the
 // input rows held in shared memory): passes of the task's row blocks
 // accumulate into one tensor-memory slot per block.
-__device__ __forceinline__ int bpasses(int nkbs) { return (nkbs + B_MAX_KBLOCKS - 1) / B_MAX_KBLOCKS; }
+template <int BW>
+__device__ __forceinline__ int bpasses(int nkbs) {
+  return (nkbs + BGeo<BW>::MAX_KBLOCKS - 1) / BGeo<BW>::MAX_KBLOCKS;
+}
 __device__ __forceinline__ void bpass(int kb0, int kb1, int npass, int ps, int& kp0, int& kp1) {
   kp0 = kb0 + (int)(((long long)ps * (kb1 - kb0)) / npass);
   kp1 = kb0 + (int)(((long long)(ps + 1) * (kb1 - kb0)) / npass);
@@ -54,10 +57,11 @@ __device__ __forceinline__ int bstages(const OpDesc& op, int nkbs) {
 }
 
 // Ring stages and accumulator slots a batched task takes.
+template <int BW>
 __device__ __forceinline__ void bgemm_counts(const OpDesc& op, int task, uint32_t& stages, uint32_t& blocks) {
   int rb0, rb1, kb0, kb1, seg;
   btask(op, task, rb0, rb1, kb0, kb1, seg);
-  const int npass = bpasses(kb1 - kb0);
+  const int npass = bpasses<BW>(kb1 - kb0);
   uint32_t st = 0;
   for (int ps = 0; ps < npass; ++ps) {
     int kp0, kp1;
@@ -70,12 +74,13 @@ __device__ __forceinline__ void bgemm_counts(const OpDesc& op, int task, uint32_
 
 // Producer side of a batched task: its weight tiles, stage by stage.  False on
 // abort or timeout.  t_issue (profiling) receives the first stage's issue time.
+template <int BW>
 __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
                          uint64_t pol, unsigned long long* t_issue) {
   int rb0, rb1, kb0, kb1, seg;
   btask(op, task, rb0, rb1, kb0, kb1, seg);
   const bool pair = op.kind == TK_NORM_GEMV_SILU;
-  const int npass = bpasses(kb1 - kb0);
+  const int npass = bpasses<BW>(kb1 - kb0);
   for (int ps = 0; ps < npass; ++ps) {
     int kp0, kp1;
     bpass(kb0, kb1, npass, ps, kp0, kp1);
@@ -106,24 +111,24 @@ __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, u
 // product with request r's input (gate/up: v gate, u up).  RESID leaves the
 // new residual values in nx (0 for rows past the end), for the block's sums
 // of squares.
-template <int KIND>
+template <int KIND, int BW>
 __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int row, const float* v, const float* u,
                                           uint32_t iter, uint32_t xtag, uint32_t mytag, bool capture,
-                                          unsigned long long (&best)[MAX_BATCH], float (&nx)[MAX_BATCH],
+                                          unsigned long long (&best)[BW], float (&nx)[BW],
                                           bool& fail, int worker) {
   const int R = g.R;
   if (KIND == TK_NORM_GEMV) {
     const int s = seg_of(op, row);
     const int local = row - op.seg_row0[s], ns = op.grp_rows[s];
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r)
+    for (int r = 0; r < BW; ++r)
       if (r < R) st_tagged(op.y[s] + (size_t)r * ns + local, v[r], mytag);
   } else if (KIND == TK_GEMV_RESID) {
-    uint64_t w[MAX_BATCH];
+    uint64_t w[BW];
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r) w[r] = r < R ? ld_tagged(op.x_out + (size_t)r * op.N + row) : 0ull;
+    for (int r = 0; r < BW; ++r) w[r] = r < R ? ld_tagged(op.x_out + (size_t)r * op.N + row) : 0ull;
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r) {
+    for (int r = 0; r < BW; ++r) {
       if (r < R) {
         uint64_t* p = op.x_out + (size_t)r * op.N + row;
         if (word_tag(w[r]) != xtag) {
@@ -138,7 +143,7 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
     }
   } else if (KIND == TK_NORM_GEMV_SILU) {
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r) {
+    for (int r = 0; r < BW; ++r) {
       if (r < R) {
         nx[r] = silu_f(v[r]) * u[r];
         st_tagged(op.a_out + (size_t)r * op.N + row, nx[r], mytag);
@@ -146,7 +151,7 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
     }
   } else {  // LM head
 #pragma unroll
-    for (int r = 0; r < MAX_BATCH; ++r) {
+    for (int r = 0; r < BW; ++r) {
       if (r < R) {
         const unsigned long long key = argmax_key(v[r], (uint32_t)row);
         best[r] = key > best[r] ? key : best[r];
@@ -157,17 +162,24 @@ __device__ __forceinline__ void bepilogue(const Graph& g, const OpDesc& op, int 
 }
 
 // Element k of request r's input row into the next projection's published
-// input rows: bf16 hi/lo of x (times w_next[k] when the next operation is an
-// RMSNorm) at row r (hi) and 8 + r (lo) of K block k / 64, 16-byte chunk
-// (k mod 64) / 8 swizzled by r.
+// input rows of batch width BW: bf16 hi/lo of x (times w_next[k] when the
+// next operation is an RMSNorm) at row r (hi) and BW + r (lo) of K block
+// k / 64, 16-byte chunk (k mod 64) / 8 swizzled by r mod 8.
+template <int BW>
 __device__ __forceinline__ void publish_xb(const OpDesc& op, int k, int r, float x) {
   const float h = op.xb_w != nullptr ? x * __uint_as_float((uint32_t)op.xb_w[k] << 16) : x;
   const uint16_t hi = f32_to_bf16_rn(h);
   const uint16_t lo = f32_to_bf16_rn(h - __uint_as_float((uint32_t)hi << 16));
-  uint16_t* blk = op.xb_out + (size_t)(k >> 6) * (B_KBLOCK_BYTES / 2);
-  const int off = r * BK + ((((k & 63) >> 3) ^ r) << 3) + (k & 7);
+  uint16_t* blk = op.xb_out + (size_t)(k >> 6) * (BGeo<BW>::KBLOCK_BYTES / 2);
+  const int off = r * BK + ((((k & 63) >> 3) ^ (r & 7)) << 3) + (k & 7);
   blk[off] = hi;
-  blk[MAX_BATCH * BK + off] = lo;
+  blk[BW * BK + off] = lo;
+}
+// The same for a writer outside the contractions (embedding, attention
+// merge), at the graph's batch width.
+__device__ __forceinline__ void publish_xb_g(const Graph& g, const OpDesc& op, int k, int r, float x) {
+  if (g.bw > 8) publish_xb<16>(op, k, r, x);
+  else publish_xb<8>(op, k, r, x);
 }
 
 // Two bf16 (bits) in one word, element k in the low half.
@@ -195,18 +207,19 @@ __device__ __forceinline__ void split8(const float (&v)[8], uint4& hi, uint4& lo
 //
 // Not inlined: the task gets its own register allocation, so neither its
 // arrays nor the attention's are spilled around the other.
-template <int KIND>
+template <int KIND, int BW>
 __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t iter,
                                         uint32_t cstage, uint32_t accn, int cw, int lane, int worker) {
   constexpr bool PAIR = KIND == TK_NORM_GEMV_SILU;
   constexpr bool NORM = KIND != TK_GEMV_RESID;
   constexpr int MMA_WARP = 4;
+  constexpr int BN = BGeo<BW>::BN, KBB = BGeo<BW>::KBLOCK_BYTES, NSLOT = BGeo<BW>::NSLOT;
   const int ctid = cw * 32 + lane;
   const int R = g.R;
   int rb0, rb1, kb0, kb1, seg;
   btask(op, task, rb0, rb1, kb0, kb1, seg);
   const int nblk = rb1 - rb0;
-  const int npass = bpasses(kb1 - kb0);
+  const int npass = bpasses<BW>(kb1 - kb0);
   const bool split = op.bsplit > 1;
   uint8_t* bsm = sm.ring[NSTB];
   const uint32_t xtag = vtag(g, iter, op.x_writer) + op.tag_skew;
@@ -218,21 +231,21 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
   const int nrows = op.N;
   // partial sums: [segment][row][PW] floats, PW = the requests' values (gate/up:
   // then the up values), so a thread moves its row with 16-byte accesses
-  constexpr int PW = PAIR ? 2 * MAX_BATCH : MAX_BATCH;
+  constexpr int PW = PAIR ? 2 * BW : BW;
   const size_t SEGW = (size_t)nrows * PW;
   bool fail = false;
-  unsigned long long best[MAX_BATCH];
+  unsigned long long best[BW];
 #pragma unroll
-  for (int r = 0; r < MAX_BATCH; ++r) best[r] = 0ull;
+  for (int r = 0; r < BW; ++r) best[r] = 0ull;
 
   // ---- RMSNorm factor of every request from the per-block sums of squares
-  // its writer published (warp r: request r, blocks in a fixed order)
+  // its writer published (warp w: requests w, w + 8, ..., blocks in a fixed order)
   if (NORM) {
     bool pfail = false;
-    if (cw < R) {
+    for (int rq = cw; rq < R; rq += CONSUMER_WARPS) {
       float ss = 0.f;
       for (int b = lane; b < op.xss_blocks; b += 32) {
-        const uint64_t* p = op.xss_in + (size_t)b * R + cw;
+        const uint64_t* p = op.xss_in + (size_t)b * R + rq;
         uint64_t w = ld_tagged(p);
         if (word_tag(w) != stag) {
           w = poll_word(g, p, stag, op.self, worker, (int)iter);
@@ -241,7 +254,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         ss += word_value(w);
       }
       ss = warp_sum(ss);
-      if (lane == 0) sm.brinv[cw] = 1.0f / sqrtf(ss / (float)op.K + op.eps);
+      if (lane == 0) sm.brinv[rq] = 1.0f / sqrtf(ss / (float)op.K + op.eps);
       if (op.xb_in != nullptr) __threadfence();  // acquire: the rows published before these sums
     }
     if (consumer_sync_or(pfail)) return false;
@@ -288,9 +301,9 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
       if (ctid == 0) {
         fence_acq_rel_gpu();
         fence_proxy_async_global();
-        const uint32_t bytes = (uint32_t)nkbs * (uint32_t)B_KBLOCK_BYTES;
+        const uint32_t bytes = (uint32_t)nkbs * (uint32_t)KBB;
         mbar_arrive_expect_tx(&sm.bload, bytes);
-        bulk_g2s(bsm, op.xb_in + (size_t)kp0 * (B_KBLOCK_BYTES / 2), bytes, &sm.bload, policy_evict_first());
+        bulk_g2s(bsm, op.xb_in + (size_t)kp0 * (KBB / 2), bytes, &sm.bload, policy_evict_first());
       }
       consumer_sync();
     } else {
@@ -299,7 +312,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
     {
       bool pfail = false;
       const int nch = nkbs * 8;  // 16-byte chunks per request row
-      const int total = MAX_BATCH * nch;
+      const int total = BW * nch;
       constexpr int FL = 2;
       for (int q0 = ctid; q0 < total; q0 += FL * CONSUMER_THREADS) {
         uint64_t w[FL][8];
@@ -342,9 +355,9 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
               }
               split8(v, hi, lo);
             }
-            uint8_t* dst = bsm + kbl * B_KBLOCK_BYTES + r * (BK * 2) + ((ch ^ r) << 4);
+            uint8_t* dst = bsm + kbl * KBB + r * (BK * 2) + ((ch ^ (r & 7)) << 4);
             *reinterpret_cast<uint4*>(dst) = hi;
-            *reinterpret_cast<uint4*>(dst + B_KBLOCK_BYTES / 2) = lo;
+            *reinterpret_cast<uint4*>(dst + KBB / 2) = lo;
           }
         }
       }
@@ -390,7 +403,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
             tc_fence_after_sync();
             const uint32_t a0 = smem_u32(sm.ring[rs]);
             if (PAIR) {
-              const uint32_t b0 = smem_u32(bsm) + (uint32_t)st * B_KBLOCK_BYTES;
+              const uint32_t b0 = smem_u32(bsm) + (uint32_t)st * KBB;
 #pragma unroll
               for (int kk = 0; kk < BK / 16; ++kk) {
                 const uint64_t bd = sw128_desc(b0 + kk * 32);
@@ -401,7 +414,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
             } else {
               const int nbox = min(2, nkbs - 2 * st);
               for (int b = 0; b < nbox; ++b) {
-                const uint32_t b0 = smem_u32(bsm) + (uint32_t)(2 * st + b) * B_KBLOCK_BYTES;
+                const uint32_t b0 = smem_u32(bsm) + (uint32_t)(2 * st + b) * KBB;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
                   mma_bf16_ss(dacc, sw128_desc(a0 + b * BOX_BYTES + kk * 32), sw128_desc(b0 + kk * 32), idesc,
@@ -427,20 +440,20 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         if (lane == 0) ok = wait_mbar(g, &sm.acc_full[slot], use & 1u, 3, worker);
         ok = __shfl_sync(0xffffffffu, ok, 0) != 0;
         tc_fence_after_sync();
-        float d[16], du[16];
+        float d[BN], du[BN];
         const uint32_t dacc = tmem + slot * (uint32_t)(2 * BN) + lanes;
-        tmem_ld16(dacc, d);
-        if (PAIR) tmem_ld16(dacc + BN, du);
+        tmem_ld_cols<BN>(dacc, d);
+        if (PAIR) tmem_ld_cols<BN>(dacc + BN, du);
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.acc_empty[slot]);
         fail |= !ok;
         // W hi + W lo per request (published rows: times the request's RMS factor)
-        float v[MAX_BATCH], u[MAX_BATCH], nx[MAX_BATCH];
+        float v[BW], u[BW], nx[BW];
 #pragma unroll
-        for (int r = 0; r < MAX_BATCH; ++r) {
-          v[r] = d[r] + d[MAX_BATCH + r];
-          u[r] = PAIR ? du[r] + du[MAX_BATCH + r] : 0.f;
+        for (int r = 0; r < BW; ++r) {
+          v[r] = d[r] + d[BW + r];
+          u[r] = PAIR ? du[r] + du[BW + r] : 0.f;
           if (NORM && published) {
             v[r] *= sm.brinv[r];
             u[r] *= sm.brinv[r];
@@ -452,11 +465,10 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         if (split) {
           if (ok && row < nrows) {
             float4* pp = reinterpret_cast<float4*>(op.bpart + (size_t)seg * SEGW + (size_t)row * PW);
-            pp[0] = make_float4(v[0], v[1], v[2], v[3]);
-            pp[1] = make_float4(v[4], v[5], v[6], v[7]);
-            if (PAIR) {
-              pp[2] = make_float4(u[0], u[1], u[2], u[3]);
-              pp[3] = make_float4(u[4], u[5], u[6], u[7]);
+#pragma unroll
+            for (int c4 = 0; c4 < BW / 4; ++c4) {
+              pp[c4] = make_float4(v[4 * c4], v[4 * c4 + 1], v[4 * c4 + 2], v[4 * c4 + 3]);
+              if (PAIR) pp[BW / 4 + c4] = make_float4(u[4 * c4], u[4 * c4 + 1], u[4 * c4 + 2], u[4 * c4 + 3]);
             }
           }
           // The last segment task of this row block to arrive adds the
@@ -487,9 +499,9 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
                 if (s0 + j < op.bsplit) {
                   const float* f = reinterpret_cast<const float*>(q[j]);
 #pragma unroll
-                  for (int r = 0; r < MAX_BATCH; ++r) {
+                  for (int r = 0; r < BW; ++r) {
                     v[r] = (s0 + j) == 0 ? f[r] : v[r] + f[r];
-                    if (PAIR) u[r] = (s0 + j) == 0 ? f[MAX_BATCH + r] : u[r] + f[MAX_BATCH + r];
+                    if (PAIR) u[r] = (s0 + j) == 0 ? f[BW + r] : u[r] + f[BW + r];
                   }
                 }
               }
@@ -498,11 +510,11 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
         }
         if (finish) {
           if (ok && row < nrows)
-            bepilogue<KIND>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
+            bepilogue<KIND, BW>(g, op, row, v, u, iter, xtag, mytag, capture, best, nx, fail, worker);
           if ((KIND == TK_GEMV_RESID || KIND == TK_NORM_GEMV_SILU) && op.xb_out != nullptr && row < nrows) {
 #pragma unroll
-            for (int r = 0; r < MAX_BATCH; ++r)
-              if (r < R) publish_xb(op, row, r, nx[r]);
+            for (int r = 0; r < BW; ++r)
+              if (r < R) publish_xb<BW>(op, row, r, nx[r]);
           }
           if (KIND == TK_NORM_GEMV_SILU && op.xb_out != nullptr) {
             // the row block's flag, after all its rows
@@ -516,7 +528,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
             // the block's sums of squares of the new x, per request: lanes,
             // then warps 0..3 in order
 #pragma unroll
-            for (int r = 0; r < MAX_BATCH; ++r) {
+            for (int r = 0; r < BW; ++r) {
               const float ssr = warp_sum(nx[r] * nx[r]);
               if (lane == 0) sm.bss[i & 1][cw][r] = ssr;
             }
@@ -541,7 +553,7 @@ __device__ __noinline__ bool bgemm_task(Smem& sm, const Graph& g, const OpDesc& 
     // task of the operation to arrive writes the tokens
     if (cw < 4) {
 #pragma unroll
-      for (int r = 0; r < MAX_BATCH; ++r) {
+      for (int r = 0; r < BW; ++r) {
         const unsigned long long b = warp_max_u64(best[r]);
         if (lane == 0) sm.bbest[cw][r] = b;
       }

@@ -192,13 +192,14 @@ int batched_geometry(mpk_ctx* c, int li, OpDesc& o, int R, const mpk_layer& Ly) 
                 o.nkb, BK);
   // a segment longer than the input buffer runs in passes, which keep every
   // row block of the task in its own tensor-memory accumulator slot
+  const int bw = batch_width(R), max_kblocks = b_max_kblocks(bw), nslot = b_nslot(bw);
   const int longest = (o.nkb + gy - 1) / gy;
   const int most_blocks = (o.nb + gx - 1) / gx;
-  if (longest > B_MAX_KBLOCKS && most_blocks > NSLOT)
+  if (longest > max_kblocks && most_blocks > nslot)
     return fail(c, MPK_ERR_SHAPE,
                 "layer %d: tasks of %d row blocks over %d elements of the reduction: a task longer than %d elements "
                 "takes at most %d row blocks (more tasks per segment, grid_dim.x, or more segments, grid_dim.y)",
-                li, most_blocks, longest * BK, B_MAX_KBLOCKS * BK, NSLOT);
+                li, most_blocks, longest * BK, max_kblocks * BK, nslot);
   o.dynamic = 0;
   return MPK_OK;
 }
@@ -930,7 +931,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
     bblk_off[p] = bblk_u32;
     bblk_u32 += (size_t)op.nb;
     bpart_off[p] = bpart_floats;
-    bpart_floats += (size_t)op.bsplit * op.N * MAX_BATCH * (op.kind == TK_NORM_GEMV_SILU ? 2 : 1);
+    bpart_floats += (size_t)op.bsplit * op.N * batch_width(R) * (op.kind == TK_NORM_GEMV_SILU ? 2 : 1);
   }
   const size_t o_bblk = take(sizeof(uint32_t) * (bblk_u32 ? bblk_u32 : 1));
   c->sync_bytes = off;
@@ -1071,7 +1072,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       if (q < 0) continue;
       uint16_t*& buf = xb[op.x_out];
       if (!buf) {
-        const size_t bytes = (size_t)((op.N + BK - 1) / BK) * B_KBLOCK_BYTES;
+        const size_t bytes = (size_t)((op.N + BK - 1) / BK) * b_kblock_bytes(batch_width(R));
         rc = alloc(c, &buf, bytes);
         if (rc != MPK_OK) return rc;
       }
@@ -1103,7 +1104,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
       if (wr.xb_out != nullptr || rd.K % BK != 0 || grp % BK != 0) continue;
       auto& e = ab[{rd.a_in, wr.kind}];
       if (!e.first) {
-        rc = alloc(c, &e.first, (size_t)(rd.K / BK) * B_KBLOCK_BYTES);
+        rc = alloc(c, &e.first, (size_t)(rd.K / BK) * b_kblock_bytes(batch_width(R)));
         if (rc != MPK_OK) return rc;
         rc = alloc(c, &e.second, nflags * sizeof(uint64_t));
         if (rc != MPK_OK) return rc;
@@ -1149,9 +1150,9 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   if (rc != MPK_OK) return rc;
   CUDA_OR_FAIL(c, cudaMemcpy(c->ops_dev, ops.data(), sizeof(OpDesc) * P, cudaMemcpyHostToDevice));
 
-  if (PF && (R != PF || R < 2 || R > MAX_BATCH))
+  if (PF && (R != PF || R < 2 || R > MAX_PREFILL))
     return fail(c, MPK_ERR_SHAPE, "prefill_tokens = %d needs activations of that many rows (2..%d); the graph has %d",
-                PF, MAX_BATCH, R);
+                PF, MAX_PREFILL, R);
   if (!PF || Rq < 1) Rq = R;
   if (Rq > MAX_REQUESTS)
     return fail(c, MPK_ERR_UNSUPPORTED, "%d cached requests (at most %d)", Rq, MAX_REQUESTS);
@@ -1162,6 +1163,7 @@ int mpk_compile(mpk_ctx* c, const mpk_layer* layers, int n_layers, const mpk_opt
   g.ops = c->ops_dev;
   g.nops = P;
   g.batched = R >= 2 ? 1 : 0;
+  g.bw = batch_width(R);
   g.split_attn = 0;
   for (int p = 0; p < P; ++p)
     if (ops[p].kind == TK_ATTN) g.split_attn = 1;

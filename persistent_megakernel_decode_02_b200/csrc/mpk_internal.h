@@ -46,26 +46,46 @@ constexpr int SCHED_WARPS_PER_SM = 4;
 
 // Tensor-core path (an operation over 2..MAX_BATCH requests): every
 // projection is a dense contraction [R, K] x W^T computed by tcgen05 MMAs of
-// M = BM weight rows x N = BN columns, K in blocks of BK elements.  The fp32
-// input of request r is split into two bf16 rows, hi = bf16(h) in column r and
-// lo = bf16(h - hi) in column MAX_BATCH + r, so one MMA yields W hi + W lo: the
+// M = BM weight rows x N columns, K in blocks of BK elements.  The fp32 input
+// of request r is split into two bf16 rows, hi = bf16(h) in column r and
+// lo = bf16(h - hi) in column BW + r, so one MMA yields W hi + W lo: the
 // contraction sees the input to about 16 significant bits, with the weights
-// exact.  Weights arrive as BM x BK tiles (TMA, 128-byte swizzle); the input
-// rows are held in the ring's last stages in the same layout; accumulators
-// live in tensor memory.
-constexpr int MAX_BATCH = 8;
+// exact.  BW, the batch width, is 8 for up to 8 requests and 16 for 9..16
+// (N = 2 BW = 16 or 32, both valid shapes for M = 128).  Weights arrive as
+// BM x BK tiles (TMA, 128-byte swizzle); the input rows are held in the ring's
+// last stages in the same layout (BW / 8 eight-row swizzle atoms of hi rows,
+// then as many of lo rows, per K block); accumulators live in tensor memory.
+constexpr int MAX_BATCH = 16;               // requests of one contraction
+constexpr int MAX_PREFILL = 8;              // positions of a prefill graph's iteration
 constexpr int BM = 128;                     // weight rows per MMA (tensor-memory lanes)
-constexpr int BN = 2 * MAX_BATCH;           // MMA N: hi columns, then lo columns (a valid shape for M = 128)
 constexpr int BK = 64;                      // K elements per tile row (128 bytes)
 constexpr int BOX_BYTES = BM * BK * 2;      // one weight tile: 16 KB
 constexpr int NSTB = 5;                     // weight stages of the ring in this mode
-constexpr int B_MAX_KBLOCKS = 24;           // longest reduction segment held for the inputs: 1536
-constexpr int B_KBLOCK_BYTES = BN * BK * 2; // the hi and lo rows of one K block: two 1 KB swizzle atoms
+constexpr int B_INPUT_BYTES = 49152;        // shared memory for one pass's input rows
+constexpr int B_TMEM_COLS = 512;            // tensor-memory columns of the accumulators
 static_assert(STAGE_BYTES == 2 * BOX_BYTES, "a weight stage holds two tiles");
-constexpr int NSLOT = 16;                   // accumulator slots of 2 BN tensor-memory columns (512 columns)
-static_assert(MAX_BATCH == 8, "one 8-row swizzle atom per half of the input columns");
-static_assert(MAX_BATCH == MPK_MAX_BATCH && BM == MPK_BATCH_BM && B_MAX_KBLOCKS * BK == MPK_BATCH_MAX_PASS_K &&
-                  NSLOT == MPK_BATCH_SLOTS,
+
+// Geometry of a contraction of batch width BW.
+template <int BW>
+struct BGeo {
+  static_assert(BW == 8 || BW == 16, "batch widths of whole 8-row swizzle atoms");
+  static constexpr int BN = 2 * BW;                          // MMA N: hi columns, then lo columns
+  static constexpr int KBLOCK_BYTES = BN * BK * 2;           // the hi and lo rows of one K block
+  static constexpr int MAX_KBLOCKS = B_INPUT_BYTES / KBLOCK_BYTES;  // longest reduction segment of a pass
+  static constexpr int NSLOT = B_TMEM_COLS / (2 * BN);       // accumulator slots of 2 BN columns
+};
+constexpr int NSLOT_MAX = BGeo<8>::NSLOT;
+__host__ __device__ constexpr int batch_width(int R) { return R > 8 ? 16 : 8; }
+__host__ __device__ constexpr int b_kblock_bytes(int bw) { return 4 * bw * BK; }
+__host__ __device__ constexpr int b_max_kblocks(int bw) { return B_INPUT_BYTES / b_kblock_bytes(bw); }
+__host__ __device__ constexpr int b_nslot(int bw) { return B_TMEM_COLS / (4 * bw); }
+static_assert(b_kblock_bytes(8) == BGeo<8>::KBLOCK_BYTES && b_kblock_bytes(16) == BGeo<16>::KBLOCK_BYTES &&
+                  b_max_kblocks(16) == BGeo<16>::MAX_KBLOCKS && b_nslot(16) == BGeo<16>::NSLOT,
+              "host and device geometry agree");
+static_assert(MAX_BATCH == MPK_MAX_BATCH && MAX_PREFILL == MPK_MAX_PREFILL && BM == MPK_BATCH_BM &&
+                  BGeo<8>::MAX_KBLOCKS * BK == MPK_BATCH_MAX_PASS_K && BGeo<8>::NSLOT == MPK_BATCH_SLOTS &&
+                  BGeo<16>::MAX_KBLOCKS * BK == MPK_BATCH_WIDE_MAX_PASS_K &&
+                  BGeo<16>::NSLOT == MPK_BATCH_WIDE_SLOTS,
               "the header states the batched geometry");
 
 enum TaskKind : int32_t {
@@ -156,7 +176,7 @@ struct OpDesc {
   int32_t ntb;                  // tasks per segment (grid_dim.x), each owning a run of row blocks
   const void* tmap[MAX_SEG];    // tensor maps of W[s] (device memory, 64-byte aligned)
   const void* tmap_up;          // SILU: tensor map of the up matrix
-  float* bpart;                 // bsplit > 1: partial sums [bsplit][N][MAX_BATCH] (gate/up: [..][2 MAX_BATCH])
+  float* bpart;                 // bsplit > 1: partial sums [bsplit][N][BW] (gate/up: [..][2 BW])
   // per-block sums of squares of x (batched graphs): EMBED and RESID publish
   // them for every BM-row block of the x they write, tagged [blocks][R]; the
   // RMSNorm operations read them instead of the whole of x
@@ -165,7 +185,7 @@ struct OpDesc {
   int32_t xss_blocks;
   // published input rows (batched graphs): the writer of a projection's input
   // also stores it as bf16 hi/lo in the swizzled layout of the shared-memory
-  // input buffer ([K/64 blocks][2 x 8 rows][64], 2 KB per block; rows past R
+  // input buffer ([K/64 blocks][2 x BW rows][64], 4 BW * 64 bytes per block; rows past R
   // zero) and the reader copies its K blocks with one bulk copy.  Writers of x
   // (EMBED, RESID) store x * w_norm of the next RMSNorm operation (xb_w) and
   // release the rows with the block's sums of squares; the reader applies the
@@ -210,6 +230,7 @@ struct Graph {
   int32_t nops;
   int32_t op_by_op;                 // 1: every operation is its own launch (mpk_run_op_by_op)
   int32_t batched;                  // 1: projections run on the tensor-core path (R >= 2)
+  int32_t bw;                       // batched: batch width of the contractions (8 or 16)
   int32_t split_attn;               // 1: the graph has split-K attention operations
   int32_t prefill;                  // 1: the R columns are R consecutive positions of one request
   int32_t Rq;                       // requests of tokens, step, pred and the KV cache (without prefill: R)

@@ -76,8 +76,8 @@ struct __align__(128) Smem {
   unsigned long long h_key;  // (iteration, op, segment) whose input vector hs holds (~0: none)
   float2 rope_row[MAX_D / 2];                    // its RoPE (cos, sin) row
   // tensor-core path
-  uint64_t acc_full[NSLOT];                      // accumulator slot b holds a finished row block
-  uint64_t acc_empty[NSLOT];                     // slot b has been read (one arrival per epilogue warp)
+  uint64_t acc_full[NSLOT_MAX];                  // accumulator slot b holds a finished row block
+  uint64_t acc_empty[NSLOT_MAX];                 // slot b has been read (one arrival per epilogue warp)
   uint64_t bfree;                                // the MMAs of a pass are done with the input rows
   uint32_t bfn;                                  // completed phases of bfree (read and advanced by consumer thread 0)
   uint64_t bload;                                // the published input rows of a pass have landed
@@ -89,9 +89,9 @@ struct __align__(128) Smem {
   float bss[2][4][MAX_BATCH];                    // per block parity, epilogue warp, request: sums of squares
   unsigned long long bbest[4][MAX_BATCH];        // LM head: per epilogue warp and request (value, index) maxima
 };
-static_assert(NSTB < NSTAGES && 2 * MAX_BATCH * MAX_D * 2 <= STAGE_BYTES,
+static_assert(NSTB < NSTAGES && 2 * MAX_PREFILL * MAX_D * 2 <= STAGE_BYTES,
               "a prefill attention task's k/v rows fit the stage the tensor-core path keeps for its inputs");
-static_assert((NSTAGES - NSTB) * STAGE_BYTES + sizeof(((Smem*)nullptr)->u) >= B_MAX_KBLOCKS * B_KBLOCK_BYTES,
+static_assert((NSTAGES - NSTB) * STAGE_BYTES + sizeof(((Smem*)nullptr)->u) >= B_INPUT_BYTES,
               "the batch input rows fit in the stages the ring leaves free and the scratch after them");
 
 // ------------------------------------------------------------------ status / waits
@@ -539,12 +539,14 @@ __device__ __noinline__ bool attn_produce(Smem& sm, const Graph& g, const OpDesc
 }
 
 // Producer side of a tensor-core (batched) task; defined with the batched path.
+template <int BW>
 __device__ bool bproduce(Smem& sm, const Graph& g, const OpDesc& op, int task, uint32_t& pstage, int worker,
                          uint64_t pol, unsigned long long* t_issue);
 
 // kSplit: the graph has split-K attention operations, whose K/V the producer
-// streams (kernels without them leave the code out entirely).
-template <bool kStandalone, bool kBatch, bool kSplit>
+// streams (kernels without them leave the code out entirely); BW: the batch
+// width of the tensor-core path.
+template <bool kStandalone, bool kBatch, bool kSplit, int BW>
 __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
   constexpr int NR = kBatch ? NSTB : NSTAGES;  // weight stages of the ring
   const uint64_t pol = policy_evict_first();
@@ -667,7 +669,7 @@ __device__ void producer_loop(Smem& sm, const Graph& g, int worker, uint32_t sa_
     }
     if (!is_gemv(op.kind)) continue;
     if constexpr (kBatch) {
-      if (!bproduce(sm, g, op, task, pstage, worker, pol, g.profiling ? &sm.fifo_t[f] : nullptr)) {
+      if (!bproduce<BW>(sm, g, op, task, pstage, worker, pol, g.profiling ? &sm.fifo_t[f] : nullptr)) {
         ok = false;
         break;
       }
@@ -1150,9 +1152,10 @@ __device__ bool gemv_task(Smem& sm, const Graph& g, const OpDesc& op, int task, 
 // ------------------------------------------------------------------ batched projections (tensor cores)
 #include "mpk_batch.cuh"
 
+template <int BW>
 __device__ __forceinline__ void bgemm_advance(const OpDesc& op, int task, uint32_t& cstage, uint32_t& accn) {
   uint32_t st, bl;
-  bgemm_counts(op, task, st, bl);
+  bgemm_counts<BW>(op, task, st, bl);
   cstage += st;
   accn += bl;
 }
@@ -1415,7 +1418,7 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
   const bool pf = g.prefill;  // prefill graphs run split-K attention only
   const int own = pf ? r : 0;
   uint16_t* const KX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) : A.ks;
-  uint16_t* const VX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_BATCH * MAX_D : A.vs;
+  uint16_t* const VX = pf ? reinterpret_cast<uint16_t*>(sm.ring[NSTB]) + MAX_PREFILL * MAX_D : A.vs;
   const int CS = op.C;  // split op: chunk partials per (request, query head)
   const float* pbase = op.part + (((size_t)r * op.Hq + (size_t)j * G) * CS) * (D + 2);
   // Prologue rows: warp cw < G takes query head cw of the group, warp G the
@@ -1809,14 +1812,14 @@ __device__ __forceinline__ bool attn_task(Smem& sm, const Graph& g, const OpDesc
         }
         const float ov = Os / mw[2 * nml + hh];
         st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)(j * G + hh) * D + i, ov, mytag);
-        if (op.xb_out != nullptr) publish_xb(op, (j * G + hh) * D + i, r, ov);
+        if (op.xb_out != nullptr) publish_xb_g(g, op, (j * G + hh) * D + i, r, ov);
       }
     } else {
       // an inactive request still publishes this iteration's version of its
       // output (zeros), which the next projection waits for
       for (int idx = ctid; idx < G * D; idx += CONSUMER_THREADS) {
         st_tagged(op.a_out + (size_t)r * op.Hq * D + (size_t)j * G * D + idx, 0.f, mytag);
-        if (op.xb_out != nullptr) publish_xb(op, j * G * D + idx, r, 0.f);
+        if (op.xb_out != nullptr) publish_xb_g(g, op, j * G * D + idx, r, 0.f);
       }
     }
     consumer_sync();
@@ -1846,7 +1849,7 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
       const int cw = ctid >> 5, lane = ctid & 31;
       for (int b = cw; b < op.xss_blocks; b += CONSUMER_WARPS) {
         if (op.xb_out != nullptr) {
-          for (int i = b * BM + lane; i < min(op.N, (b + 1) * BM); i += 32) publish_xb(op, i, r, 0.f);
+          for (int i = b * BM + lane; i < min(op.N, (b + 1) * BM); i += 32) publish_xb_g(g, op, i, r, 0.f);
           __threadfence();
         }
         __syncwarp();
@@ -1892,8 +1895,8 @@ __device__ bool embed_task(const Graph& g, const OpDesc& op, int task, uint32_t 
           ss = e0 * e0 + e1 * e1 + e2 * e2 + e3 * e3;
           if (op.xb_out != nullptr) {
             // the rows the next RMSNorm operation reads, before the sums
-            publish_xb(op, i, r, e0); publish_xb(op, i + 1, r, e1);
-            publish_xb(op, i + 2, r, e2); publish_xb(op, i + 3, r, e3);
+            publish_xb_g(g, op, i, r, e0); publish_xb_g(g, op, i + 1, r, e1);
+            publish_xb_g(g, op, i + 2, r, e2); publish_xb_g(g, op, i + 3, r, e3);
           }
         }
         if (op.xb_out != nullptr) __threadfence();
@@ -1954,7 +1957,7 @@ __device__ __noinline__ int attn_split_task(Smem& sm, const Graph& g, const OpDe
   return ok ? (int)attn_stages(g, op, task, iter) : -1;
 }
 
-template <bool kStandalone, bool kBatch, bool kSplit>
+template <bool kStandalone, bool kBatch, bool kSplit, int BW>
 __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int lane) {
   const int ctid = cw * 32 + lane;
   uint32_t fpos = 0, cstage = 0, accn = 0;
@@ -2002,19 +2005,19 @@ __device__ void consumer_loop(Smem& sm, const Graph& g, int worker, int cw, int 
     if constexpr (kBatch) {
       switch (op.kind) {
         case TK_EMBED: ok = embed_task(g, op, task, iter, ctid); break;
-        case TK_NORM_GEMV: ok = bgemm_task<TK_NORM_GEMV>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
-          bgemm_advance(op, task, cstage, accn); break;
+        case TK_NORM_GEMV: ok = bgemm_task<TK_NORM_GEMV, BW>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance<BW>(op, task, cstage, accn); break;
         case TK_GEMV_RESID:
-          ok = bgemm_task<TK_GEMV_RESID>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
-          bgemm_advance(op, task, cstage, accn);
+          ok = bgemm_task<TK_GEMV_RESID, BW>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance<BW>(op, task, cstage, accn);
           break;
         case TK_NORM_GEMV_SILU:
-          ok = bgemm_task<TK_NORM_GEMV_SILU>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
-          bgemm_advance(op, task, cstage, accn);
+          ok = bgemm_task<TK_NORM_GEMV_SILU, BW>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance<BW>(op, task, cstage, accn);
           break;
         case TK_NORM_GEMV_ARGMAX:
-          ok = bgemm_task<TK_NORM_GEMV_ARGMAX>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
-          bgemm_advance(op, task, cstage, accn);
+          ok = bgemm_task<TK_NORM_GEMV_ARGMAX, BW>(sm, g, op, task, iter, cstage, accn, cw, lane, worker);
+          bgemm_advance<BW>(op, task, cstage, accn);
           break;
         case TK_ATTN: {
           const int n = attn_split_task(sm, g, op, task, iter, cw, lane, worker, cstage);
@@ -2144,7 +2147,7 @@ __device__ __forceinline__ void init_barriers(Smem& sm) {
     mbar_init(&sm.full[i], 1);
     mbar_init(&sm.empty[i], kBatch ? 1 : CONSUMER_WARPS);
   }
-  for (int i = 0; i < NSLOT; ++i) {
+  for (int i = 0; i < NSLOT_MAX; ++i) {
     mbar_init(&sm.acc_full[i], 1);
     mbar_init(&sm.acc_empty[i], 4);
   }
@@ -2174,7 +2177,7 @@ __device__ __forceinline__ Smem& smem_layout(uint8_t* raw) {
 // A worker block: barriers (and, on the tensor-core path, the accumulator's
 // tensor memory, allocated by consumer warp 0 and released by it after the
 // last task, once no MMA is in flight), then the producer and consumer roles.
-template <bool kStandalone, bool kBatch, bool kSplit>
+template <bool kStandalone, bool kBatch, bool kSplit, int BW = 8>
 __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worker, uint32_t sa_iter, int sa_op) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) init_barriers<kBatch>(sm);
@@ -2184,11 +2187,11 @@ __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worke
   if (kBatch) tc_fence_after_sync();
   if (warp < PRODUCER_WARPS) {
     regs_dec<PRODUCER_REGS>();
-    if (warp == 0 && lane == 0) producer_loop<kStandalone, kBatch, kSplit>(sm, g, worker, sa_iter, sa_op);
+    if (warp == 0 && lane == 0) producer_loop<kStandalone, kBatch, kSplit, BW>(sm, g, worker, sa_iter, sa_op);
     return;
   }
   regs_inc<CONSUMER_REGS>();
-  consumer_loop<kStandalone, kBatch, kSplit>(sm, g, worker, warp - PRODUCER_WARPS, lane);
+  consumer_loop<kStandalone, kBatch, kSplit, BW>(sm, g, worker, warp - PRODUCER_WARPS, lane);
   if (kBatch) {
     // the MMA-issuing thread waits (bounded) until none of its MMAs is outstanding
     if (warp == PRODUCER_WARPS + 4 && lane == 0) {
@@ -2205,7 +2208,7 @@ __device__ __forceinline__ void worker_block(Smem& sm, const Graph& g, int worke
   }
 }
 
-template <bool kBatch, bool kSplit>
+template <bool kBatch, bool kSplit, int BW = 8>
 __device__ __forceinline__ void persistent_body(const Graph& g) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -2241,12 +2244,13 @@ __device__ __forceinline__ void persistent_body(const Graph& g) {
     }
     return;
   }
-  worker_block<false, kBatch, kSplit>(smem_layout(smem_raw), g, blockIdx.x - g.sched_ctas, 0, 0);
+  worker_block<false, kBatch, kSplit, BW>(smem_layout(smem_raw), g, blockIdx.x - g.sched_ctas, 0, 0);
 }
 
 // Kernels: one request without split-K attention (the fused projections +
 // attention operation), one request with it (long contexts), several requests
-// (tensor-core projections, split-K attention).
+// (tensor-core projections, split-K attention): up to 8, and 9..16 (batch
+// width 16).
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_kernel(const Graph g) {
   persistent_body<false, false>(g);
 }
@@ -2254,7 +2258,10 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_sp
   persistent_body<false, true>(g);
 }
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_batch_kernel(const Graph g) {
-  persistent_body<true, true>(g);
+  persistent_body<true, true, 8>(g);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_persistent_batch16_kernel(const Graph g) {
+  persistent_body<true, true, 16>(g);
 }
 
 // One operation of one iteration as an ordinary launch: block b runs task b.
@@ -2267,16 +2274,21 @@ extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_split_kern
 }
 extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_batch_kernel(const Graph g, int op,
                                                                                   uint32_t iter) {
-  worker_block<true, true, true>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+  worker_block<true, true, true, 8>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
+}
+extern "C" __global__ void __launch_bounds__(BLOCK_THREADS, 1) mpk_op_batch16_kernel(const Graph g, int op,
+                                                                                    uint32_t iter) {
+  worker_block<true, true, true, 16>(smem_layout(smem_raw), g, blockIdx.x, iter, op);
 }
 
 // ------------------------------------------------------------------ host-side launch helpers
 size_t kernel_smem_bytes() { return SMEM_BYTES; }
 
 cudaError_t prepare_kernels() {
-  const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_split_kernel,
-                      (const void*)mpk_persistent_batch_kernel, (const void*)mpk_op_kernel,
-                      (const void*)mpk_op_split_kernel, (const void*)mpk_op_batch_kernel};
+  const void* ks[] = {(const void*)mpk_persistent_kernel,  (const void*)mpk_persistent_split_kernel,
+                      (const void*)mpk_persistent_batch_kernel, (const void*)mpk_persistent_batch16_kernel,
+                      (const void*)mpk_op_kernel, (const void*)mpk_op_split_kernel,
+                      (const void*)mpk_op_batch_kernel, (const void*)mpk_op_batch16_kernel};
   for (const void* k : ks) {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -2286,7 +2298,7 @@ cudaError_t prepare_kernels() {
 
 cudaError_t max_blocks_per_sm(int* n) {
   const void* ks[] = {(const void*)mpk_persistent_kernel, (const void*)mpk_persistent_split_kernel,
-                      (const void*)mpk_persistent_batch_kernel};
+                      (const void*)mpk_persistent_batch_kernel, (const void*)mpk_persistent_batch16_kernel};
   int m = 1 << 30;
   for (const void* k : ks) {
     int a = 0;
@@ -2300,7 +2312,8 @@ cudaError_t max_blocks_per_sm(int* n) {
 
 cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream) {
   void* args[] = {const_cast<Graph*>(&g)};
-  const void* k = g.batched ? (const void*)mpk_persistent_batch_kernel
+  const void* k = g.batched ? (g.bw > 8 ? (const void*)mpk_persistent_batch16_kernel
+                                        : (const void*)mpk_persistent_batch_kernel)
                   : g.split_attn ? (const void*)mpk_persistent_split_kernel : (const void*)mpk_persistent_kernel;
   return cudaLaunchCooperativeKernel(k, dim3(grid), dim3(BLOCK_THREADS), args, SMEM_BYTES, stream);
 }
@@ -2308,7 +2321,7 @@ cudaError_t launch_persistent(const Graph& g, int grid, cudaStream_t stream) {
 // An operation whose tasks wait on one another (group mode) is launched
 // cooperatively, so all of its blocks are resident together.
 cudaError_t launch_op(const Graph& g, int op, int ntasks, uint32_t iter, bool cooperative, cudaStream_t stream) {
-  const void* k = g.batched ? (const void*)mpk_op_batch_kernel
+  const void* k = g.batched ? (g.bw > 8 ? (const void*)mpk_op_batch16_kernel : (const void*)mpk_op_batch_kernel)
                   : g.split_attn ? (const void*)mpk_op_split_kernel : (const void*)mpk_op_kernel;
   void* args[] = {const_cast<Graph*>(&g), &op, &iter};
   if (cooperative)

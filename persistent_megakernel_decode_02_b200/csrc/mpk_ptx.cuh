@@ -204,6 +204,14 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// NC consecutive accumulator columns (NC a multiple of 16), 16 at a time.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, float (&v)[NC]) {
+  static_assert(NC % 16 == 0, "whole 16-column loads");
+#pragma unroll
+  for (int c = 0; c < NC / 16; ++c) tmem_ld16(taddr + 16u * (uint32_t)c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+}
+
 // ---------------------------------------------------------------- scoped accesses
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
   uint32_t v;

@@ -46,25 +46,37 @@ _TASK_OVERHEAD_S = 3e-6
 _PASS_OVERHEAD_S = 4e-6
 _SPLIT_PARTIAL_S = 1.5e-6
 BATCH_SLOTS = 16  # accumulator slots: row blocks a task may hold across passes
+# Graphs of 9..16 requests run every contraction 16 requests wide: the input
+# rows of a K block take twice the shared memory and an accumulator twice the
+# tensor-memory columns, so a pass holds half the K blocks and half the slots.
+MAX_BATCH = 16
+BATCH_WIDE_MAX_KBLOCKS, BATCH_WIDE_SLOTS = 12, 8
 
 
-def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[int, int]:
+def batch_limits(requests: int) -> Tuple[int, int]:
+    """(K blocks per pass, accumulator slots) of a contraction over `requests`."""
+    return (BATCH_WIDE_MAX_KBLOCKS, BATCH_WIDE_SLOTS) if requests > 8 else (BATCH_MAX_KBLOCKS, BATCH_SLOTS)
+
+
+def batched_grid(rows: int, K: int, workers: int, pair: bool = False, requests: int = 8) -> Tuple[int, int]:
     """grid_dim (tasks per reduction segment, segments) of a projection over
     several requests: among segment counts s and, per number of rounds k of
     the workers, the largest run split gx <= row blocks with gx * s <= k *
     workers, the one with the least rounds x (largest task's weight bytes /
     bandwidth + task, pass and per-partial split costs); fewer segments on ties.  A task
-    longer than the input rows (passes) holds at most BATCH_SLOTS row blocks."""
+    longer than the input rows (passes) holds at most the accumulator slots'
+    row blocks (batch_limits)."""
+    max_kblocks, slots = batch_limits(requests)
     nb = -(-rows // BATCH_BM)
     nkb = K // BATCH_BK
     block_bytes = BATCH_BM * K * 2 * (2 if pair else 1)
     best = None
     for s in range(1, min(nkb, 16) + 1):
-        npass = -(-(-(-nkb // s)) // BATCH_MAX_KBLOCKS)
+        npass = -(-(-(-nkb // s)) // max_kblocks)
         for k in range(1, 5):
             gx = max(1, min(nb, (k * workers) // s))
             most = -(-nb // gx)
-            if npass > 1 and most > BATCH_SLOTS:
+            if npass > 1 and most > slots:
                 continue
             rounds = -(-(gx * s) // workers)
             t = rounds * (most * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S +
@@ -74,7 +86,7 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False) -> Tuple[i
     return best[1], best[2]
 
 
-def lm_head_grid(rows: int, K: int, workers: int) -> Tuple[int, int]:
+def lm_head_grid(rows: int, K: int, workers: int, requests: int = 8) -> Tuple[int, int]:
     """grid_dim of the LM head over several requests: no split of the
     reduction (the argmax needs whole logits, and a split's last arrival runs
     the epilogue late) and tasks for about five sixths of the workers, so the
@@ -82,10 +94,11 @@ def lm_head_grid(rows: int, K: int, workers: int) -> Tuple[int, int]:
     shape with 8 requests: (120, 1) at 5.43 ms/step against 5.49 for the
     batched_grid rule's (48, 3)).  Falls back to batched_grid when a task
     would hold more row blocks than the accumulator slots."""
+    max_kblocks, slots = batch_limits(requests)
     nb = -(-rows // BATCH_BM)
     gx = max(1, min(nb, (workers * 5) // 6))
-    if -(-(K // BATCH_BK) // BATCH_MAX_KBLOCKS) > 1 and -(-nb // gx) > BATCH_SLOTS:
-        return batched_grid(rows, K, workers)
+    if -(-(K // BATCH_BK) // max_kblocks) > 1 and -(-nb // gx) > slots:
+        return batched_grid(rows, K, workers, requests=requests)
     return gx, 1
 
 
@@ -103,24 +116,24 @@ def batched_layer_plan(shape, requests: int, plan_workers: int, attn_chunks: int
         p = f"layers.{l}."
         plan.append(dict(method="rmsnorm_linear_layer", input="x", weight_norm=p + "input_layernorm",
                          weight_linear=[p + "q_proj", p + "k_proj", p + "v_proj"], output=["q", "k", "v"],
-                         grid_dim=batched_grid(s.q_dim + 2 * s.kv_dim, s.hidden, W), block_dim=block_dim, eps=s.eps))
+                         grid_dim=batched_grid(s.q_dim + 2 * s.kv_dim, s.hidden, W, requests=requests), block_dim=block_dim, eps=s.eps))
         plan.append(dict(method="attention_layer", q="q", k="k", v="v", q_norm=p + "q_norm",
                          k_norm=p + "k_norm", k_cache="k_cache", v_cache="v_cache", output="o", layer=l,
                          grid_dim=(s.kv_heads, attn_chunks, requests), block_dim=block_dim, eps=s.eps,
                          rope_theta=s.rope_theta))
         plan.append(dict(method="linear_residual_layer", input="o", weight=p + "o_proj", residual="x",
-                         grid_dim=batched_grid(s.hidden, s.q_dim, W), block_dim=block_dim))
+                         grid_dim=batched_grid(s.hidden, s.q_dim, W, requests=requests), block_dim=block_dim))
         plan.append(dict(method="rmsnorm_linear_silu_mul_layer", input="x",
                          weight_norm=p + "post_attention_layernorm", weight_gate=p + "gate_proj",
                          weight_up=p + "up_proj", output="a",
-                         grid_dim=batched_grid(s.intermediate, s.hidden, W, pair=True), block_dim=block_dim,
+                         grid_dim=batched_grid(s.intermediate, s.hidden, W, pair=True, requests=requests), block_dim=block_dim,
                          eps=s.eps))
         plan.append(dict(method="linear_residual_layer", input="a", weight=p + "down_proj", residual="x",
-                         grid_dim=batched_grid(s.hidden, s.intermediate, W), block_dim=block_dim,
+                         grid_dim=batched_grid(s.hidden, s.intermediate, W, requests=requests), block_dim=block_dim,
                          capture_slot=l + 1))
     plan.append(dict(method="rmsnorm_lmhead_argmax_layer", input="x", weight_norm="norm",
                      weight_lm="embed_tokens" if tied else "lm_head", pred="pred",
-                     grid_dim=lm_head_grid(s.vocab, s.hidden, W), block_dim=block_dim, eps=s.eps))
+                     grid_dim=lm_head_grid(s.vocab, s.hidden, W, requests=requests), block_dim=block_dim, eps=s.eps))
     return plan
 
 

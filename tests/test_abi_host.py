@@ -154,6 +154,23 @@ def test_batched_grid_rule():
                 assert -(-nb // gx) <= BATCH_SLOTS
     # the LM head: whole reductions, tasks for five sixths of the workers
     assert lm_head_grid(151936, 4096, 144) == (120, 1)
+    # 9..16 requests: contractions 16 wide, half the K blocks per pass and
+    # half the accumulator slots
+    from persistent_megakernel_decode_02_b200.qwen3 import (BATCH_WIDE_MAX_KBLOCKS, BATCH_WIDE_SLOTS, MAX_BATCH,
+                                                            batch_limits)
+    assert MAX_BATCH == _header_define("MPK_MAX_BATCH")
+    assert BATCH_WIDE_MAX_KBLOCKS * 64 == _header_define("MPK_BATCH_WIDE_MAX_PASS_K")
+    assert BATCH_WIDE_SLOTS == _header_define("MPK_BATCH_WIDE_SLOTS")
+    assert batch_limits(8) == (BATCH_MAX_KBLOCKS, BATCH_SLOTS) and batch_limits(9) == (12, 8)
+    for shape in (sq.TINY, sq.QWEN3_0_6B, sq.QWEN3_8B):
+        for rows, K, pair in [(shape.intermediate, shape.hidden, True), (shape.hidden, shape.intermediate, False),
+                              (shape.vocab, shape.hidden, False)]:
+            for W in (1, 7, 144):
+                for gx, gy in (batched_grid(rows, K, W, pair, requests=16), lm_head_grid(rows, K, W, requests=16)):
+                    nb, nkb = -(-rows // BATCH_BM), K // 64
+                    assert 1 <= gx <= nb and 1 <= gy <= nkb
+                    if -(-nkb // gy) > BATCH_WIDE_MAX_KBLOCKS:
+                        assert -(-nb // gx) <= BATCH_WIDE_SLOTS
     # the 8B plan for 144 workers: one round of tasks for the projections, the
     # reductions split three or four ways
     assert batched_grid(6144, 4096, 144) == (48, 3)

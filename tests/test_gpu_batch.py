@@ -270,7 +270,7 @@ def test_reduction_passes_and_splits(wide_weights, monkeypatch, down_grid, gu_gr
     grids = {(WIDE.hidden, WIDE.intermediate, False): down_grid, (WIDE.intermediate, WIDE.hidden, True): gu_grid,
              (WIDE.vocab, WIDE.hidden, False): lm_grid}
     orig = q3.batched_grid
-    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, w, pair=False: grids.get((rows, K, pair)) or
+    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, w, pair=False, **kw: grids.get((rows, K, pair)) or
                         orig(rows, K, w, pair))
     w_cpu, w = wide_weights
     R = 4
@@ -298,7 +298,7 @@ def test_too_many_blocks_for_passes_is_rejected(wide_weights, monkeypatch):
     shape = sq.Qwen3Shape("tiny-long", 1, 2048, 4, 2, 64, 4096, 1024, tied=False)
     w = to_cuda(sq.make_weights(shape, seed=5))
     orig = q3.batched_grid
-    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, wk, pair=False: (1, 1) if pair else orig(rows, K, wk, pair))
+    monkeypatch.setattr(q3, "batched_grid", lambda rows, K, wk, pair=False, **kw: (1, 1) if pair else orig(rows, K, wk, pair))
     with pytest.raises(MpkError, match="at most 16 row blocks"):
         build_decoder(shape, w, requests=2, max_seq=16)
 
