@@ -23,6 +23,8 @@ tokens each.  The prompts are ingested first (untimed, one decode iteration
 per prompt token), then 256 lock-step iterations (every request one token per
 iteration, each at its own position) run in ONE timed launch; a step is one
 such iteration, reported in ms/step.  The projections run on the tensor cores.
+--requests R (2..16) runs the same workload with R requests (9..16: every
+contraction 16 requests wide).
 
 --workload long measures one request over a KV cache pre-filled with 32768
 positions (seeded N(0,1) bf16): 128 greedy iterations in one timed launch.
@@ -64,6 +66,7 @@ def parse():
     p.add_argument("--workload", choices=["batch1", "batch8", "long"], default="batch1",
                    help="batch1: one request, 39-token prompt + 512 tokens (default); batch8: 8 requests; "
                         "long: one request over 32768 pre-filled positions")
+    p.add_argument("--requests", type=int, default=0, help="batch8 workload: requests (2..16, default 8)")
     p.add_argument("--steps", type=int, default=0, help="timed steps (default: 512 for batch1, 256 for batch8)")
     p.add_argument("--warmup", type=int, default=8)
     p.add_argument("--impl", choices=["mpk", "reference"], default="mpk")
@@ -379,7 +382,10 @@ def main_batch(args):
     from persistent_megakernel_decode_02_b200 import build_decoder, load
 
     shape = sized_shape(sq, args)
-    R, S, G = BATCH, BATCH_SEQ, BATCH_GENERATED
+    R, S, G = args.requests or BATCH, BATCH_SEQ, BATCH_GENERATED
+    if not 2 <= R <= 16:
+        raise SystemExit("--requests must be in 2..16")
+    kname = "mpk_persistent_batch_kernel" if R <= 8 else "mpk_persistent_batch16_kernel"
     steps = args.steps
     if not (1 <= steps <= G and 0 <= args.warmup <= G):
         raise SystemExit(f"--steps must be in 1..{G} and --warmup in 0..{G}")
@@ -516,7 +522,7 @@ def main_batch(args):
 
     if rank == 0:
         line = {
-            "metric": METRIC_BATCH, "value": ms_per_step, "unit": UNIT_BATCH, "n_gpus": world, "steps": steps,
+            "metric": METRIC_BATCH.replace("8 requests", f"{R} requests"), "value": ms_per_step, "unit": UNIT_BATCH, "n_gpus": world, "steps": steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {
@@ -531,12 +537,11 @@ def main_batch(args):
             "tokens_per_s": tokens_per_s,
             "hbm_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "traffic": (None if traffic_ratio("mpk_persistent_batch_kernel") is None
-                                     else traffic_ratio("mpk_persistent_batch_kernel") * bytes_launch),
+                         "traffic": (None if traffic_ratio(kname) is None else traffic_ratio(kname) * bytes_launch),
                          "traffic_source": "ncu dram bytes of a 4-layer case scaled by algorithmic bytes",
                          "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": bytes_launch, "launch_ms": ms_launch,
-                         "kernel": "mpk_persistent_batch_kernel"},
+                         "kernel": kname},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 1,

@@ -92,12 +92,20 @@ def lm_head_grid(rows: int, K: int, workers: int, requests: int = 8) -> Tuple[in
     the epilogue late) and tasks for about five sixths of the workers, so the
     workers that finish the last layer late claim none (measured on the 8B
     shape with 8 requests: (120, 1) at 5.43 ms/step against 5.49 for the
-    batched_grid rule's (48, 3)).  Falls back to batched_grid when a task
-    would hold more row blocks than the accumulator slots."""
+    batched_grid rule's (48, 3)).  When a task would hold more row blocks
+    than the accumulator slots, the fewest tasks that fit them (up to two per
+    worker), else batched_grid."""
     max_kblocks, slots = batch_limits(requests)
     nb = -(-rows // BATCH_BM)
     gx = max(1, min(nb, (workers * 5) // 6))
     if -(-(K // BATCH_BK) // max_kblocks) > 1 and -(-nb // gx) > slots:
+        # a task whose reduction runs in passes holds at most `slots` row
+        # blocks: the fewest whole-reduction tasks that fit (measured on the 8B
+        # shape with 16 requests: 160 such tasks at 8.63 ms/step against 8.76
+        # for batched_grid's six-way split)
+        gx = -(-nb // slots)
+        if gx <= 2 * workers:
+            return gx, 1
         return batched_grid(rows, K, workers, requests=requests)
     return gx, 1
 
