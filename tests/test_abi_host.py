@@ -193,3 +193,30 @@ def test_batched_layer_plan():
             assert p["grid_dim"] == (s.kv_heads, 2, 8)
         else:
             assert isinstance(p["grid_dim"], tuple) and len(p["grid_dim"]) == 2
+
+
+def test_wide_batched_layer_plan():
+    """16 requests: the projections' grids follow the 16-wide limits (a task
+    whose segment exceeds 12 K blocks holds at most 8 row blocks), the LM head
+    runs whole reductions in tasks that fit the slots, the embedding and the
+    attention grids carry the 16 requests."""
+    from persistent_megakernel_decode_02_b200.qwen3 import BATCH_WIDE_MAX_KBLOCKS, BATCH_WIDE_SLOTS
+    s = sq.QWEN3_8B
+    plan = layer_plan(s, requests=16, num_workers=144, attn_chunks=1)
+    assert plan[0]["grid_dim"] == 16
+    rows_k = {"rmsnorm_linear_layer": (s.q_dim + 2 * s.kv_dim, s.hidden),
+              "rmsnorm_linear_silu_mul_layer": (s.intermediate, s.hidden),
+              "rmsnorm_lmhead_argmax_layer": (s.vocab, s.hidden)}
+    for p in plan[1:]:
+        m = p["method"]
+        if m == "attention_layer":
+            assert p["grid_dim"] == (s.kv_heads, 1, 16)
+            continue
+        gx, gy = p["grid_dim"]
+        rows, K = rows_k.get(m) or ((s.hidden, s.q_dim) if p["input"] == "o" else (s.hidden, s.intermediate))
+        nb, nkb = -(-rows // 128), K // 64
+        assert 1 <= gx <= nb and 1 <= gy <= nkb
+        if -(-nkb // gy) > BATCH_WIDE_MAX_KBLOCKS:
+            assert -(-nb // gx) <= BATCH_WIDE_SLOTS
+        if m == "rmsnorm_lmhead_argmax_layer":
+            assert (gx, gy) == (-(-nb // BATCH_WIDE_SLOTS), 1)
