@@ -67,6 +67,11 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False, requests: 
     longer than the input rows (passes) holds at most the accumulator slots'
     row blocks (batch_limits)."""
     max_kblocks, slots = batch_limits(requests)
+    # a partial sum holds one value per request of the batch width (8 or 16):
+    # at width 16 it costs twice as much (measured on the 8B shape with 16
+    # requests: o and down projections in 3 and 4 segments, 8.18 ms/step,
+    # against 4 and 9 at the width-8 cost, 8.62)
+    partial_s = _SPLIT_PARTIAL_S * (2 if requests > 8 else 1)
     nb = -(-rows // BATCH_BM)
     nkb = K // BATCH_BK
     block_bytes = BATCH_BM * K * 2 * (2 if pair else 1)
@@ -80,7 +85,7 @@ def batched_grid(rows: int, K: int, workers: int, pair: bool = False, requests: 
                 continue
             rounds = -(-(gx * s) // workers)
             t = rounds * (most * block_bytes / s / _WORKER_BYTES_PER_S + _TASK_OVERHEAD_S +
-                          (npass - 1) * _PASS_OVERHEAD_S) + (s * _SPLIT_PARTIAL_S if s > 1 else 0.0)
+                          (npass - 1) * _PASS_OVERHEAD_S) + (s * partial_s if s > 1 else 0.0)
             if best is None or t < best[0] * (1 - 1e-2):
                 best = (t, gx, s)
     return best[1], best[2]

@@ -177,6 +177,10 @@ def test_batched_grid_rule():
     assert batched_grid(12288, 4096, 144, True) == (48, 3)
     assert batched_grid(4096, 4096, 144) == (32, 4)
     assert batched_grid(4096, 12288, 144) == (32, 4)
+    # 16 requests: partial sums of 16 values cost twice as much, fewer segments
+    assert batched_grid(4096, 4096, 144, requests=16) == (32, 3)
+    assert batched_grid(4096, 12288, 144, requests=16) == (32, 4)
+    assert lm_head_grid(151936, 4096, 144, requests=16) == (149, 1)
 
 
 def test_batched_layer_plan():
