@@ -389,20 +389,26 @@ def test_decoder_matches_library_restatement(shape, mode):
     assert err < 1e-9, err
 
 
-def test_decoder_requests_are_independent():
+@pytest.mark.parametrize("R", [3, 16])
+def test_decoder_requests_are_independent(R):
     """Several requests decoded together (different prompt lengths, start and
-    end positions, one finishing while the others go on) give, request by
+    end positions, some finishing while the others go on) give, request by
     request, exactly what each gives decoded alone: tokens, final step, cache
     rows and the logits of every iteration it was active.  Pins the oracle's
     per-request bookkeeping (cache and token indexing by request, inactive
-    requests left untouched) that the batched GPU parity tests rely on."""
+    requests left untouched) that the batched GPU parity tests rely on, up to
+    the 16 requests of the widest contraction."""
     shape = qwen3.TINY
     w = qwen3.make_weights(shape, seed=0)
     dec = oracle.Decoder(shape, w)
-    S, R = 20, 3
-    toks = qwen3.make_tokens(shape, R, S, [5, 2, 8], seed=9).numpy().copy()
-    step0 = np.array([0, 1, 3], np.int32)
-    end = np.array([12, 6, 17], np.int32)
+    S = 20
+    if R == 3:
+        lens, step0, end = [5, 2, 8], np.array([0, 1, 3], np.int32), np.array([12, 6, 17], np.int32)
+    else:
+        lens = [2 + (5 * r) % 9 for r in range(R)]
+        step0 = np.array([min(r % 4, lens[r] - 1) for r in range(R)], np.int32)  # each starts on a prompt token
+        end = np.array([8 + (7 * r) % 11 for r in range(R)], np.int32)
+    toks = qwen3.make_tokens(shape, R, S, lens, seed=9).numpy().copy()
     bt, bs, bk, bv, bcaps = dec.generate(toks, step0, end, capture=True)
     assert np.array_equal(bs, end)
     for r in range(R):
