@@ -60,7 +60,7 @@ PREFILL_TOKENS = 8  # prompt positions per prefill iteration (the tensor-core pa
 METRIC_LONG = "decode ms/token (Qwen3-8B-shape, batch 1, 32768 cached positions) and HBM GB/s vs ~8 TB/s peak"
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--workload", choices=["batch1", "batch8", "long"], default="batch1",
@@ -88,7 +88,9 @@ def parse():
     p.add_argument("--attention", choices=["auto", "fused", "split"], default="auto")
     p.add_argument("--layers", type=int, default=0, help="override the layer count (profiling cases)")
     p.add_argument("--vocab", type=int, default=0, help="override the vocabulary (profiling cases)")
-    args = p.parse_args()
+    args = p.parse_args(argv)
+    if args.requests and not 2 <= args.requests <= 16:
+        p.error("--requests must be in 2..16")
     if not args.steps:
         args.steps = {"batch1": GENERATED, "batch8": BATCH_GENERATED, "long": LONG_GENERATED}[args.workload]
     return args

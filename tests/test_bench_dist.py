@@ -83,3 +83,16 @@ def test_whole_job_single_rank():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.whole_job(20.0, 10, 1) == pytest.approx((2.0, 500.0))
+
+
+def test_requests_option_is_checked_before_any_gpu_work():
+    """--requests outside 2..16 is refused while parsing the arguments; inside
+    it, the batch workload takes it (default 8)."""
+    import bench
+    with pytest.raises(SystemExit):
+        bench.parse(["--workload", "batch8", "--requests", "17"])
+    with pytest.raises(SystemExit):
+        bench.parse(["--workload", "batch8", "--requests", "1"])
+    a = bench.parse(["--workload", "batch8", "--requests", "16"])
+    assert a.requests == 16 and a.steps == bench.BATCH_GENERATED
+    assert bench.parse(["--workload", "batch8"]).requests == 0
