@@ -165,7 +165,8 @@ typedef struct { int32_t x, y, z; } mpk_dim3;
  * MPK_BATCH_SLOTS row blocks.  Graphs of 9..MPK_MAX_BATCH requests run
  * every contraction 16 requests wide (the weights are still read once per
  * iteration); their limits are MPK_BATCH_WIDE_MAX_PASS_K and
- * MPK_BATCH_WIDE_SLOTS.  K must be a multiple of 64 and stacked matrices
+ * MPK_BATCH_WIDE_SLOTS; more requests fail mpk_compile with
+ * MPK_ERR_UNSUPPORTED.  K must be a multiple of 64 and stacked matrices
  * start at multiples of MPK_BATCH_BM rows (MPK_ERR_UNSUPPORTED otherwise);
  * RMSNORM_QKV_ATTENTION takes one request.  A prefill graph
  * (mpk_options.prefill_tokens) takes at most MPK_MAX_PREFILL positions per
